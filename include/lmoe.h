@@ -1,0 +1,169 @@
+/*
+ * lmoe.h -- C ABI of the B200 (sm_100a) Stable-LatentMoE layer with Quantile Balancing.
+ *
+ * The layer (forward pass, per token t of x[T,d]):
+ *   r_t   = 1/sqrt(mean_j x_tj^2 + eps);  x_hat = g * x * r_t                      (RMSNorm)
+ *   h     = x_hat W_down^T                      width d -> latent l              (width separation)
+ *   s     = sigmoid(h W_router^T + c)           fp32 router scores [T,E]
+ *   sel   = top-k of u = s + b                  larger u first, ties to the lower expert index
+ *   g_i   = s_sel_i / sum_j s_sel_j             unbiased, renormalised gate weights
+ *   o_i   = SwiGLU_{sel_i}(h)                   routed experts in width l (SwiGLU stands in for SiTU-GLU)
+ *   y     = (sum_i g_i o_i) W_up^T + SwiGLU_shared(x_hat)
+ * and Quantile Balancing (QB), a delayed bias update:
+ *   q_e   = (1 - k/E) quantile of column e of s, from a 4096-bin histogram over [0,1]
+ *   b_e  <- b_e - beta (u_e - mean_e u_e),  u_e = q_e + b_e   (quantile of the biased column;
+ *                                                             LMOE_QB_LITERAL: u_e = q_e)
+ * Sources: "KimiK3MoE架构轻量化复刻演示上线,12个交互模块详解StableLatentMoE设计逻辑"
+ * (tech.news18a.com): Tab 1 (width separation, shared/routed dual path), Tab 2 Figure 2
+ * (QB load balance, histogram quantile), Tab 3 (forward contract), Tab 5 (RMSNorm),
+ * Tab 8-11 (QB: bias only reroutes, normalised weights, delayed, mean-centred, frozen at
+ * inference), Tab 12 (SiTU-GLU, whose formula the page does not give).
+ * "免费电子书:Pretraining a Mini Kimi K3" (g.15386.cn), capsules 20 and 25: experts as
+ * batched matmuls over their tokens, no silent fallback when the dispatch buffer overflows.
+ *
+ * Conventions for every call:
+ *  - Pointers named *_dev are CUDA device pointers; *_host are host pointers (pinned memory
+ *    gives truly asynchronous copies).  The caller owns every pointer it passes.
+ *  - Matrices are row-major.  Weights use the (out, in) layout of a linear layer.
+ *  - Every call only enqueues work on `stream` (a cudaStream_t; NULL = legacy default stream)
+ *    and returns, except lmoe_create (returns after enqueuing its copies), lmoe_get_status
+ *    and lmoe_destroy, which synchronise.  Calls on one handle are not thread-safe.
+ *  - Calls return 0 (LMOE_OK) or a negative LMOE_E* code; nothing is thrown across the ABI.
+ *    There is no fallback: a shape the kernels do not support returns LMOE_EUNSUPPORTED.
+ *  - Faults found on the device (NaN score, an index out of range, a pipeline wait that gave
+ *    up) set bits of a device status word that lmoe_get_status reads; no kernel traps.
+ */
+#ifndef LMOE_H
+#define LMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* return codes */
+#define LMOE_OK 0
+#define LMOE_EINVAL (-1)        /* bad argument: null pointer, shape, T > max_tokens, nbins != 4096 */
+#define LMOE_ENOMEM (-2)        /* a device or pinned allocation failed */
+#define LMOE_ECUDA (-3)         /* a CUDA call or kernel launch failed */
+#define LMOE_EUNSUPPORTED (-4)  /* valid shape that these kernels do not implement */
+#define LMOE_EDEVICE (-5)       /* not an sm_100 device */
+
+/* lmoe_config.dtype: storage and arithmetic type of activations and of all weights except the
+ * router (always fp32).  BF16 runs the GEMMs on tcgen05 tensor cores with fp32 accumulation;
+ * F32 runs them as fp32 FFMA (tensor-core tf32 would not meet fp32 accuracy). */
+#define LMOE_F32 0
+#define LMOE_BF16 1
+
+/* lmoe_forward flags */
+#define LMOE_RECORD_STATS 1u    /* add this forward's scores to the QB histogram (training);
+                                   without it the forward leaves the QB state untouched */
+/* lmoe_qb_update flags */
+#define LMOE_QB_LITERAL 1u      /* u_e = q_e (quantile of the unbiased column) */
+
+/* device status bits (lmoe_get_status) */
+#define LMOE_STATUS_NAN_SCORE 1u   /* a router score was NaN; it was never selected */
+#define LMOE_STATUS_WATCHDOG 2u    /* a pipeline wait gave up after its time limit */
+#define LMOE_STATUS_BAD_INDEX 4u   /* an expert index or permuted row was out of range */
+
+#define LMOE_NBINS 4096
+
+typedef struct lmoe_handle lmoe_handle;
+
+typedef struct {
+  int32_t d;          /* backbone width; multiple of 64 */
+  int32_t l;          /* latent width; multiple of 64 */
+  int32_t E;          /* routed experts; multiple of 64 for BF16, of 32 for F32; <= 1024 */
+  int32_t k;          /* experts per token, 1 <= k <= min(E, 32) */
+  int32_t h;          /* routed-expert SwiGLU hidden width; multiple of 64 */
+  int32_t hs;         /* shared-expert SwiGLU hidden width; multiple of 64; 0 = no shared expert */
+  int32_t dtype;      /* LMOE_F32 or LMOE_BF16 */
+  int32_t nbins;      /* QB histogram bins; must be LMOE_NBINS */
+  float rms_eps;      /* RMSNorm epsilon (1e-6) */
+  int32_t max_tokens; /* largest T any forward will pass; sizes the workspace */
+} lmoe_config;
+
+/* Weights, all device pointers, row-major (out, in).  "dtype" means lmoe_config.dtype.
+ * They are repacked into the handle: the caller may free them once lmoe_create returned
+ * and `stream` has synchronised. */
+typedef struct {
+  const void *rms_gain;      /* [d] dtype, or NULL for all ones */
+  const void *w_down;        /* [l, d] dtype */
+  const float *w_router;     /* [E, l] fp32 */
+  const float *router_bias;  /* [E] fp32 column offsets c, or NULL for zeros */
+  const void *w1;            /* [E, h, l] dtype, SwiGLU gate projection of each expert */
+  const void *w3;            /* [E, h, l] dtype, SwiGLU linear projection */
+  const void *w2;            /* [E, l, h] dtype, SwiGLU output projection */
+  const void *w_up;          /* [d, l] dtype */
+  const void *ws1;           /* [hs, d] dtype (ignored when hs == 0) */
+  const void *ws3;           /* [hs, d] dtype */
+  const void *ws2;           /* [d, hs] dtype */
+} lmoe_weights;
+
+/* Validates cfg, repacks the weights (gain folded into W_down and the shared expert, gate and
+ * linear projections interleaved, [W_up | Ws2] concatenated along K), allocates the workspace
+ * for max_tokens and sets b = 0 and an empty histogram.  On error *out is NULL and nothing is
+ * leaked. */
+int lmoe_create(const lmoe_config *cfg, const lmoe_weights *w, void *stream, lmoe_handle **out);
+
+/* Releases every device allocation of the handle (synchronises the device first). */
+int lmoe_destroy(lmoe_handle *h);
+
+/* Bytes of device memory lmoe_create allocates for cfg (repacked weights + workspace + state). */
+int lmoe_workspace_bytes(const lmoe_config *cfg, size_t *bytes);
+
+/* One forward pass: y_dev[T,d] (dtype) from x_dev[T,d] (dtype), 0 <= T <= max_tokens.
+ * T == 0 is a no-op.  x and y must not overlap and must be 16-byte aligned.  With
+ * LMOE_RECORD_STATS the scores are added to the QB histogram and T to its token count. */
+int lmoe_forward(lmoe_handle *h, const void *x_dev, void *y_dev, int32_t T, uint32_t flags,
+                 void *stream);
+
+/* The same forward with host buffers: copies x_host to the device, runs lmoe_forward into a
+ * handle-owned buffer and copies the result to y_host, all enqueued on `stream`.  y_host is
+ * valid after the stream synchronises. */
+int lmoe_forward_host(lmoe_handle *h, const void *x_host, void *y_host, int32_t T,
+                      uint32_t flags, void *stream);
+
+/* Quantile Balancing step from everything recorded since the last update (N = the sum of T of
+ * those forwards): m = ceil((E-k) N / E) (exact integer), q_e = histogram estimate of the m-th
+ * smallest score of expert e, b updated as above with step `beta`; then the histogram and N are
+ * cleared.  With N == 0 the bias is left unchanged.  Delayed: it changes only later forwards. */
+int lmoe_qb_update(lmoe_handle *h, float beta, uint32_t flags, void *stream);
+
+/* Routing stage on caller-given scores: runs biased top-k, gates, counts, offsets, the stable
+ * permutation and (with LMOE_RECORD_STATS) the histogram on scores_dev[T,E] fp32, exactly as
+ * lmoe_forward does after its router.  For stage-level checks. */
+int lmoe_route_scores(lmoe_handle *h, const float *scores_dev, int32_t T, uint32_t flags,
+                      void *stream);
+
+/* Copies the last forward's routing into caller buffers (any may be NULL), all device:
+ *  idx [T,k] int32 (rank order), gates [T,k] fp32, scores [T,E] fp32, counts [E] int32,
+ *  offsets [E+1] int32, perm [T*k] int32 (permuted row -> token; expert ascending, then token
+ *  ascending), inv [T*k] int32 ((token, slot) -> permuted row). */
+int lmoe_get_routing(lmoe_handle *h, int32_t *idx, float *gates, float *scores, int32_t *counts,
+                     int32_t *offsets, int32_t *perm, int32_t *inv, void *stream);
+
+/* QB state: bias b [E] fp32 (device), histogram [E, 4096] uint32 and token count N (int64),
+ * all device pointers. */
+int lmoe_get_bias(lmoe_handle *h, float *b_dev, void *stream);
+int lmoe_set_bias(lmoe_handle *h, const float *b_dev, void *stream);
+int lmoe_get_hist(lmoe_handle *h, uint32_t *hist_dev, int64_t *ntok_dev, void *stream);
+int lmoe_set_hist(lmoe_handle *h, const uint32_t *hist_dev, const int64_t *ntok_dev, void *stream);
+
+/* Synchronises the device, then returns the status word in *status and clears it. */
+int lmoe_get_status(lmoe_handle *h, uint32_t *status);
+
+/* Static text for a return code. */
+const char *lmoe_strerror(int code);
+
+/* Check of the tensor-core GEMM engine on its own: C[M,N] (fp32) = A[M,K] B[N,K]^T with
+ * A, B bf16 device buffers, K and N multiples of 64, row pitches equal to K.  For tests. */
+int lmoe_gemm_bf16(const void *a_dev, const void *b_dev, float *c_dev, int32_t M, int32_t N,
+                   int32_t K, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LMOE_H */

@@ -1,0 +1,247 @@
+"""Python binding of liblmoe.so, the B200 Stable-LatentMoE layer with Quantile Balancing.
+
+Argument marshalling only: every step of the layer runs in the CUDA kernels behind the C ABI
+(include/lmoe.h).  torch supplies device memory and streams.  If the library is not built the
+import of the binding still works, but the first call raises: there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, c_float, c_int, c_int32, c_size_t, c_uint32, c_void_p
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblmoe.so")
+
+F32, BF16 = 0, 1
+RECORD_STATS = 1
+QB_LITERAL = 1
+STATUS_NAN_SCORE, STATUS_WATCHDOG, STATUS_BAD_INDEX = 1, 2, 4
+NBINS = 4096
+
+EXPORTED = (
+    "lmoe_create", "lmoe_destroy", "lmoe_workspace_bytes", "lmoe_forward", "lmoe_forward_host",
+    "lmoe_qb_update", "lmoe_route_scores", "lmoe_get_routing", "lmoe_get_bias", "lmoe_set_bias",
+    "lmoe_get_hist", "lmoe_set_hist", "lmoe_get_status", "lmoe_strerror", "lmoe_gemm_bf16",
+)
+
+
+class LmoeError(RuntimeError):
+    pass
+
+
+class lmoe_config(ctypes.Structure):
+    _fields_ = [("d", c_int32), ("l", c_int32), ("E", c_int32), ("k", c_int32), ("h", c_int32),
+                ("hs", c_int32), ("dtype", c_int32), ("nbins", c_int32), ("rms_eps", c_float),
+                ("max_tokens", c_int32)]
+
+
+class lmoe_weights(ctypes.Structure):
+    _fields_ = [(n, c_void_p) for n in ("rms_gain", "w_down", "w_router", "router_bias", "w1", "w3",
+                                         "w2", "w_up", "ws1", "ws3", "ws2")]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise LmoeError(f"{LIB_PATH} is missing: build it with `python -m latent_routing_quantile_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, u32 = c_void_p, c_int32, c_uint32
+        sig = {
+            "lmoe_create": [POINTER(lmoe_config), POINTER(lmoe_weights), vp, POINTER(vp)],
+            "lmoe_destroy": [vp],
+            "lmoe_workspace_bytes": [POINTER(lmoe_config), POINTER(c_size_t)],
+            "lmoe_forward": [vp, vp, vp, i32, u32, vp],
+            "lmoe_forward_host": [vp, vp, vp, i32, u32, vp],
+            "lmoe_qb_update": [vp, c_float, u32, vp],
+            "lmoe_route_scores": [vp, vp, i32, u32, vp],
+            "lmoe_get_routing": [vp, vp, vp, vp, vp, vp, vp, vp, vp],
+            "lmoe_get_bias": [vp, vp, vp],
+            "lmoe_set_bias": [vp, vp, vp],
+            "lmoe_get_hist": [vp, vp, vp, vp],
+            "lmoe_set_hist": [vp, vp, vp, vp],
+            "lmoe_get_status": [vp, POINTER(u32)],
+            "lmoe_gemm_bf16": [vp, vp, vp, i32, i32, i32, vp],
+        }
+        for name, args in sig.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = c_int
+        L.lmoe_strerror.argtypes = [c_int]
+        L.lmoe_strerror.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise LmoeError(f"{what}: {lib().lmoe_strerror(rc).decode()} ({rc})")
+
+
+def _ptr(t):
+    return None if t is None else c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return c_void_p(s.cuda_stream)
+
+
+def _dev(t: torch.Tensor, dtype=None, shape=None, name="tensor"):
+    if not t.is_cuda or not t.is_contiguous():
+        raise LmoeError(f"{name} must be a contiguous CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise LmoeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise LmoeError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+class Layer:
+    """One LatentMoE layer handle (lmoe_create ... lmoe_destroy).
+
+    weights: dict of CUDA tensors named as in lmoe_weights (rms_gain, w_down, w_router,
+    router_bias, w1, w3, w2, w_up, ws1, ws3, ws2), layouts (out, in).
+    """
+
+    def __init__(self, d, l, E, k, h, hs, dtype, max_tokens, weights, rms_eps=1e-6, stream=None):
+        self.cfg = lmoe_config(d, l, E, k, h, hs, dtype, NBINS, rms_eps, max_tokens)
+        self.dtype = torch.float32 if dtype == F32 else torch.bfloat16
+        dt = self.dtype
+        shapes = {"rms_gain": ((d,), dt), "w_down": ((l, d), dt), "w_router": ((E, l), torch.float32),
+                  "router_bias": ((E,), torch.float32), "w1": ((E, h, l), dt), "w3": ((E, h, l), dt),
+                  "w2": ((E, l, h), dt), "w_up": ((d, l), dt)}
+        if hs:
+            shapes.update({"ws1": ((hs, d), dt), "ws3": ((hs, d), dt), "ws2": ((d, hs), dt)})
+        w = lmoe_weights()
+        for name, (shape, tdt) in shapes.items():
+            t = weights.get(name)
+            if t is not None:
+                _dev(t, tdt, shape, name)
+                setattr(w, name, t.data_ptr())
+        self._keep = dict(weights)
+        self.handle = c_void_p()
+        _check(lib().lmoe_create(ctypes.byref(self.cfg), ctypes.byref(w), _stream(stream),
+                                 ctypes.byref(self.handle)), "lmoe_create")
+        (torch.cuda.current_stream() if stream is None else stream).synchronize()
+        self._keep = None
+        self.last_T = 0
+
+    # ---------------------------------------------------------------- forward
+    def forward(self, x, y=None, record_stats=False, stream=None):
+        T = x.shape[0]
+        _dev(x, self.dtype, (T, self.cfg.d), "x")
+        if y is None:
+            y = torch.empty_like(x)
+        _dev(y, self.dtype, (T, self.cfg.d), "y")
+        _check(lib().lmoe_forward(self.handle, _ptr(x), _ptr(y), T, RECORD_STATS if record_stats else 0,
+                                  _stream(stream)), "lmoe_forward")
+        self.last_T = T
+        return y
+
+    def forward_host(self, x_host, y_host, record_stats=False, stream=None):
+        """Host tensors (pinned for asynchronous copies); y_host is valid after the stream syncs."""
+        T = x_host.shape[0]
+        if x_host.is_cuda or y_host.is_cuda or x_host.dtype != self.dtype or y_host.dtype != self.dtype:
+            raise LmoeError("forward_host takes host tensors of the layer dtype")
+        _check(lib().lmoe_forward_host(self.handle, c_void_p(x_host.data_ptr()), c_void_p(y_host.data_ptr()), T,
+                                       RECORD_STATS if record_stats else 0, _stream(stream)),
+               "lmoe_forward_host")
+        self.last_T = T
+        return y_host
+
+    def route_scores(self, scores, record_stats=False, stream=None):
+        T = scores.shape[0]
+        _dev(scores, torch.float32, (T, self.cfg.E), "scores")
+        _check(lib().lmoe_route_scores(self.handle, _ptr(scores), T, RECORD_STATS if record_stats else 0,
+                                       _stream(stream)), "lmoe_route_scores")
+        self.last_T = T
+
+    def qb_update(self, beta, literal=False, stream=None):
+        _check(lib().lmoe_qb_update(self.handle, float(beta), QB_LITERAL if literal else 0, _stream(stream)),
+               "lmoe_qb_update")
+
+    # ---------------------------------------------------------------- introspection
+    def routing(self, stream=None):
+        T, k, E = self.last_T, self.cfg.k, self.cfg.E
+        dev = torch.device("cuda")
+        out = dict(idx=torch.empty((T, k), dtype=torch.int32, device=dev),
+                   gates=torch.empty((T, k), dtype=torch.float32, device=dev),
+                   scores=torch.empty((T, E), dtype=torch.float32, device=dev),
+                   counts=torch.empty(E, dtype=torch.int32, device=dev),
+                   offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+                   perm=torch.empty(T * k, dtype=torch.int32, device=dev),
+                   inv=torch.empty(T * k, dtype=torch.int32, device=dev))
+        _check(lib().lmoe_get_routing(self.handle, *(_ptr(out[n]) for n in
+                                                     ("idx", "gates", "scores", "counts", "offsets", "perm", "inv")),
+                                      _stream(stream)), "lmoe_get_routing")
+        return out
+
+    def bias(self, stream=None):
+        b = torch.empty(self.cfg.E, dtype=torch.float32, device="cuda")
+        _check(lib().lmoe_get_bias(self.handle, _ptr(b), _stream(stream)), "lmoe_get_bias")
+        return b
+
+    def set_bias(self, b, stream=None):
+        _dev(b, torch.float32, (self.cfg.E,), "b")
+        _check(lib().lmoe_set_bias(self.handle, _ptr(b), _stream(stream)), "lmoe_set_bias")
+
+    def hist(self, stream=None):
+        hist = torch.empty((self.cfg.E, NBINS), dtype=torch.int32, device="cuda")
+        n = torch.empty(1, dtype=torch.int64, device="cuda")
+        _check(lib().lmoe_get_hist(self.handle, _ptr(hist), _ptr(n), _stream(stream)), "lmoe_get_hist")
+        return hist, n
+
+    def set_hist(self, hist, ntok, stream=None):
+        _dev(hist, torch.int32, (self.cfg.E, NBINS), "hist")
+        _dev(ntok, torch.int64, (1,), "ntok")
+        _check(lib().lmoe_set_hist(self.handle, _ptr(hist), _ptr(ntok), _stream(stream)), "lmoe_set_hist")
+
+    def status(self) -> int:
+        v = c_uint32(0)
+        _check(lib().lmoe_get_status(self.handle, ctypes.byref(v)), "lmoe_get_status")
+        return v.value
+
+    def close(self):
+        if self.handle:
+            _check(lib().lmoe_destroy(self.handle), "lmoe_destroy")
+            self.handle = c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def workspace_bytes(d, l, E, k, h, hs, dtype, max_tokens, rms_eps=1e-6) -> int:
+    cfg = lmoe_config(d, l, E, k, h, hs, dtype, NBINS, rms_eps, max_tokens)
+    n = c_size_t(0)
+    _check(lib().lmoe_workspace_bytes(ctypes.byref(cfg), ctypes.byref(n)), "lmoe_workspace_bytes")
+    return n.value
+
+
+def gemm_bf16(a, b, stream=None):
+    """C = A B^T on the tensor-core engine (fp32 result), for checks of the engine itself."""
+    M, K = a.shape
+    N = b.shape[0]
+    _dev(a, torch.bfloat16, (M, K), "a")
+    _dev(b, torch.bfloat16, (N, K), "b")
+    c = torch.empty((M, N), dtype=torch.float32, device=a.device)
+    _check(lib().lmoe_gemm_bf16(_ptr(a), _ptr(b), _ptr(c), M, N, K, _stream(stream)), "lmoe_gemm_bf16")
+    return c
+
+
+def layer_from_weights(shape, weights_cpu: dict, max_tokens=None, device="cuda", stream=None) -> Layer:
+    """Creates a Layer from the CPU weight dict of the seeded generator (copied to the device)."""
+    w = {n: t.to(device) for n, t in weights_cpu.items()}
+    return Layer(shape.d, shape.l, shape.E, shape.k, shape.h, shape.hs,
+                 F32 if shape.dtype == "f32" else BF16, max_tokens or shape.T, w,
+                 rms_eps=shape.rms_eps, stream=stream)

@@ -1,0 +1,774 @@
+// Host side of the C ABI declared in include/lmoe.h: validation, weight repacking, workspace,
+// tensor maps, and the launch sequence of one forward.  Nothing here synchronises inside a
+// forward; every launch goes to the caller's stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "common.cuh"
+#include "route.cuh"
+#include "simt_gemm.cuh"
+#include "tc_gemm.cuh"
+
+using namespace lmoe;
+
+namespace {
+
+// ------------------------------------------------------------------ tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// bf16 matrix [rows, cols] with row pitch `pitch` elements; box = 64 columns x box_rows rows,
+// 128-byte swizzle (the layout the MMA descriptors expect).
+bool make_map(CUtensorMap* m, const void* base, long long rows, long long cols, long long pitch, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  if (((uintptr_t)base & 15) || ((pitch * 2) & 15) || rows <= 0 || cols <= 0) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(pitch * 2)};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int pick_bn(int n) { return n % 256 == 0 ? 256 : (n % 128 == 0 ? 128 : 64); }
+
+template <int BN, int EPI>
+cudaError_t launch_tc_t(const TcParams& p, int grid, cudaStream_t st) {
+  auto kern = tc_gemm_kernel<BN, EPI>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<BN>::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, 192, TcCfg<BN>::kSmemBytes, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <int EPI>
+cudaError_t launch_tc_e(const TcParams& p, int bn, int grid, cudaStream_t st) {
+  switch (bn) {
+    case 256: return launch_tc_t<256, EPI>(p, grid, st);
+    case 128: return launch_tc_t<128, EPI>(p, grid, st);
+    default:
+      if constexpr (EPI == EPI_SWIGLU) return cudaErrorInvalidValue;
+      else return launch_tc_t<64, EPI>(p, grid, st);
+  }
+}
+
+cudaError_t launch_tc(const TcParams& p, int epi, int bn, int grid, cudaStream_t st) {
+  switch (epi) {
+    case EPI_F32: return launch_tc_e<EPI_F32>(p, bn, grid, st);
+    case EPI_BF16: return launch_tc_e<EPI_BF16>(p, bn, grid, st);
+    case EPI_SWIGLU: return launch_tc_e<EPI_SWIGLU>(p, bn, grid, st);
+    case EPI_DOWN3: return launch_tc_e<EPI_DOWN3>(p, bn, grid, st);
+    default: return launch_tc_e<EPI_ROUTER>(p, bn, grid, st);
+  }
+}
+
+template <int NJ>
+cudaError_t launch_topk_t(const float* s, const float* b, int T, int E, int k, int* idx, float* gates, int* rank,
+                          int* blkcnt, int* counts, uint32_t* status, cudaStream_t st) {
+  const int nblk = (T + kTokBlock - 1) / kTokBlock;
+  topk_kernel<NJ><<<nblk, 256, E * 4 * sizeof(uint32_t), st>>>(s, b, T, E, k, idx, gates, rank, blkcnt, counts,
+                                                               status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_topk(const float* s, const float* b, int T, int E, int k, int* idx, float* gates, int* rank,
+                        int* blkcnt, int* counts, uint32_t* status, cudaStream_t st) {
+  const int nj = (E + 31) / 32;
+  if (nj <= 1) return launch_topk_t<1>(s, b, T, E, k, idx, gates, rank, blkcnt, counts, status, st);
+  if (nj <= 2) return launch_topk_t<2>(s, b, T, E, k, idx, gates, rank, blkcnt, counts, status, st);
+  if (nj <= 4) return launch_topk_t<4>(s, b, T, E, k, idx, gates, rank, blkcnt, counts, status, st);
+  if (nj <= 8) return launch_topk_t<8>(s, b, T, E, k, idx, gates, rank, blkcnt, counts, status, st);
+  if (nj <= 16) return launch_topk_t<16>(s, b, T, E, k, idx, gates, rank, blkcnt, counts, status, st);
+  return launch_topk_t<32>(s, b, T, E, k, idx, gates, rank, blkcnt, counts, status, st);
+}
+
+template <int EPI>
+cudaError_t launch_simt(const SimtParams& p, int mtiles, cudaStream_t st) {
+  dim3 grid(p.N / 32, mtiles);
+  simt_gemm_kernel<EPI><<<grid, 256, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+}  // namespace
+
+// ---------------------------------------------------------------------- handle
+struct lmoe_handle {
+  lmoe_config cfg;
+  int device = 0, sms = 148;
+  size_t es = 2;  // bytes per activation element
+  bool bf = true;
+  bool unit_gain = true;
+  int nblk_max = 0, max_mtiles = 0, hist_g = 1;
+  uint8_t* arena = nullptr;
+  size_t arena_bytes = 0;
+  // repacked weights
+  void* w_down = nullptr;   // bf16 [l, d] or [l, 2d] (hi|lo); f32 [l, d]
+  void* w_r = nullptr;      // bf16 [E, 3l] (hi|mid|lo); f32 [E, l]
+  float* c = nullptr;       // [E]
+  void* ws13 = nullptr;     // bf16 [2hs, d] interleaved; f32: ws1 [hs, d]
+  void* ws3f = nullptr;     // f32 only: ws3 [hs, d]
+  void* w13 = nullptr;      // bf16 [E, 2h, l] interleaved; f32: w1 [E, h, l]
+  void* w3f = nullptr;      // f32 only: w3 [E, h, l]
+  void* w2 = nullptr;       // [E, l, h]
+  void* wy = nullptr;       // [d, l + hs]
+  // workspace
+  float* r = nullptr;
+  void* hx = nullptr;       // bf16 [Tm, 3l] (hi|mid|lo of h); f32 [Tm, l]
+  float* s = nullptr;
+  int *idx = nullptr, *rank = nullptr, *blkcnt = nullptr, *blkbase = nullptr, *counts = nullptr;
+  int *offsets = nullptr, *num_mtiles = nullptr, *perm = nullptr, *inv = nullptr;
+  float* gates = nullptr;
+  int2* mtiles = nullptr;
+  void *a_perm = nullptr, *act = nullptr, *o = nullptr, *z = nullptr, *a_s = nullptr;
+  void *x_stage = nullptr, *y_stage = nullptr;
+  // state
+  float* bias = nullptr;
+  uint32_t* hist = nullptr;
+  long long* ntok = nullptr;
+  uint32_t* status = nullptr;
+  double* u = nullptr;
+  int last_T = 0;
+  // tensor maps (bf16)
+  CUtensorMap tm_hx, tm_wr, tm_wdown, tm_ws13, tm_aperm, tm_w13, tm_act, tm_w2, tm_z, tm_as, tm_wy;
+  int bn_down = 256, bn_r = 256, bn_s1 = 256, bn_e1 = 256, bn_e2 = 256, bn_y = 256;
+};
+
+namespace {
+
+struct Arena {
+  size_t off = 0;
+  std::vector<std::pair<void**, size_t>> items;
+  void add(void** p, size_t bytes) {
+    items.push_back({p, off});
+    off += align_up(bytes ? bytes : 1, 1024);
+  }
+};
+
+void plan_layout(lmoe_handle* h, Arena& a) {
+  const lmoe_config& c = h->cfg;
+  const size_t es = h->es;
+  const size_t Tm = c.max_tokens, TK = (size_t)c.max_tokens * c.k;
+  const size_t d = c.d, l = c.l, E = c.E, hh = c.h, hs = c.hs;
+  // weights
+  a.add(&h->w_down, (h->bf && !h->unit_gain ? 2 : 1) * l * d * es);
+  a.add(&h->w_r, h->bf ? E * 3 * l * 2 : E * l * 4);
+  a.add((void**)&h->c, E * 4);
+  if (hs) {
+    a.add(&h->ws13, 2 * hs * d * es);
+    if (!h->bf) a.add(&h->ws3f, hs * d * es);
+  }
+  a.add(&h->w13, 2 * E * hh * l * es);
+  if (!h->bf) a.add(&h->w3f, E * hh * l * es);
+  a.add(&h->w2, E * l * hh * es);
+  a.add(&h->wy, d * (l + hs) * es);
+  // workspace
+  a.add((void**)&h->r, Tm * 4);
+  a.add(&h->hx, h->bf ? Tm * 3 * l * 2 : Tm * l * 4);
+  a.add((void**)&h->s, Tm * E * 4);
+  a.add((void**)&h->idx, TK * 4);
+  a.add((void**)&h->gates, TK * 4);
+  a.add((void**)&h->rank, TK * 4);
+  a.add((void**)&h->blkcnt, (size_t)h->nblk_max * E * 4);
+  a.add((void**)&h->blkbase, (size_t)h->nblk_max * E * 4);
+  a.add((void**)&h->counts, E * 4);
+  a.add((void**)&h->offsets, (E + 1) * 4);
+  a.add((void**)&h->num_mtiles, 4);
+  a.add((void**)&h->mtiles, (size_t)h->max_mtiles * 8);
+  a.add((void**)&h->perm, TK * 4);
+  a.add((void**)&h->inv, TK * 4);
+  a.add(&h->a_perm, TK * l * es);
+  a.add(&h->act, TK * hh * es);
+  a.add(&h->o, TK * l * es);
+  a.add(&h->z, Tm * l * es);
+  if (hs) a.add(&h->a_s, Tm * hs * es);
+  a.add(&h->x_stage, Tm * d * es);
+  a.add(&h->y_stage, Tm * d * es);
+  // state
+  a.add((void**)&h->bias, E * 4);
+  a.add((void**)&h->hist, E * LMOE_NBINS * 4);
+  a.add((void**)&h->ntok, 8);
+  a.add((void**)&h->status, 4);
+  a.add((void**)&h->u, E * 8);
+}
+
+int validate(const lmoe_config* c) {
+  if (!c) return LMOE_EINVAL;
+  if (c->d <= 0 || c->l <= 0 || c->E <= 0 || c->k <= 0 || c->h <= 0 || c->hs < 0 || c->max_tokens <= 0)
+    return LMOE_EINVAL;
+  if (c->k > c->E || c->nbins != LMOE_NBINS || !(c->rms_eps >= 0.f)) return LMOE_EINVAL;
+  if (c->dtype != LMOE_F32 && c->dtype != LMOE_BF16) return LMOE_EINVAL;
+  if (c->d % 64 || c->l % 64 || c->h % 64 || c->hs % 64) return LMOE_EUNSUPPORTED;
+  if (c->k > 32 || c->E > 1024) return LMOE_EUNSUPPORTED;
+  if (c->dtype == LMOE_BF16 && c->E % 64) return LMOE_EUNSUPPORTED;
+  if (c->dtype == LMOE_F32 && c->E % 32) return LMOE_EUNSUPPORTED;
+  if ((long long)c->max_tokens * c->k > (1LL << 30)) return LMOE_EUNSUPPORTED;
+  return LMOE_OK;
+}
+
+#define CK(x)                                 \
+  do {                                        \
+    if ((x) != cudaSuccess) return LMOE_ECUDA; \
+  } while (0)
+
+int grid_1d(long long n, int threads) {
+  long long b = (n + threads - 1) / threads;
+  return (int)(b > 65535 * 16 ? 65535 * 16 : (b < 1 ? 1 : b));
+}
+
+int build_maps(lmoe_handle* h) {
+  const lmoe_config& c = h->cfg;
+  const long long Tm = c.max_tokens, TK = (long long)c.max_tokens * c.k;
+  const long long d = c.d, l = c.l, E = c.E, hh = c.h, hs = c.hs;
+  h->bn_down = pick_bn(c.l);
+  h->bn_r = pick_bn(c.E);
+  h->bn_s1 = pick_bn(2 * c.hs) == 64 ? 128 : pick_bn(2 * c.hs);
+  h->bn_e1 = (2 * c.h) % 256 == 0 ? 256 : 128;
+  h->bn_e2 = pick_bn(c.l);
+  h->bn_y = pick_bn(c.d);
+  bool ok = true;
+  ok &= make_map(&h->tm_hx, h->hx, Tm, 3 * l, 3 * l, 128);
+  ok &= make_map(&h->tm_wr, h->w_r, E, 3 * l, 3 * l, h->bn_r);
+  const long long wdk = h->unit_gain ? d : 2 * d;
+  ok &= make_map(&h->tm_wdown, h->w_down, l, wdk, wdk, h->bn_down);
+  if (hs) ok &= make_map(&h->tm_ws13, h->ws13, 2 * hs, d, d, h->bn_s1);
+  ok &= make_map(&h->tm_aperm, h->a_perm, TK, l, l, 128);
+  ok &= make_map(&h->tm_w13, h->w13, E * 2 * hh, l, l, h->bn_e1);
+  ok &= make_map(&h->tm_act, h->act, TK, hh, hh, 128);
+  ok &= make_map(&h->tm_w2, h->w2, E * l, hh, hh, h->bn_e2);
+  ok &= make_map(&h->tm_z, h->z, Tm, l, l, 128);
+  if (hs) ok &= make_map(&h->tm_as, h->a_s, Tm, hs, hs, 128);
+  ok &= make_map(&h->tm_wy, h->wy, d, l + hs, l + hs, h->bn_y);
+  return ok ? LMOE_OK : LMOE_ECUDA;
+}
+
+TcParams tc_base(lmoe_handle* h) {
+  TcParams p;
+  memset(&p, 0, sizeof(p));
+  p.status = h->status;
+  return p;
+}
+
+// ---- stages shared by lmoe_forward and lmoe_route_scores
+int route_from_scores(lmoe_handle* h, int T, uint32_t flags, cudaStream_t st) {
+  const lmoe_config& c = h->cfg;
+  const int nblk = (T + kTokBlock - 1) / kTokBlock;
+  CK(cudaMemsetAsync(h->counts, 0, c.E * sizeof(int), st));
+  CK(launch_topk(h->s, h->bias, T, c.E, c.k, h->idx, h->gates, h->rank, h->blkcnt, h->counts, h->status, st));
+  plan_kernel<<<(c.E + 31) / 32, 1024, 0, st>>>(h->counts, h->blkcnt, nblk, c.E, h->offsets, h->blkbase,
+                                                  h->mtiles, h->num_mtiles);
+  CK(cudaGetLastError());
+  const int pairs = T * c.k;
+  if (h->bf) {
+    gather_kernel<bf16><<<(pairs + 7) / 8, 256, 0, st>>>((const bf16*)h->hx, 3 * c.l, c.l, h->idx, h->rank,
+                                                         h->blkbase, T, c.E, c.k, h->perm, h->inv,
+                                                         (bf16*)h->a_perm, h->status);
+  } else {
+    gather_kernel<float><<<(pairs + 7) / 8, 256, 0, st>>>((const float*)h->hx, c.l, c.l, h->idx, h->rank,
+                                                          h->blkbase, T, c.E, c.k, h->perm, h->inv,
+                                                          (float*)h->a_perm, h->status);
+  }
+  CK(cudaGetLastError());
+  if (flags & LMOE_RECORD_STATS) {
+    const int G = h->hist_g;
+    CK(cudaFuncSetAttribute(hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                            G * LMOE_NBINS * (int)sizeof(uint32_t)));
+    hist_kernel<<<(c.E + G - 1) / G, 1024, G * LMOE_NBINS * sizeof(uint32_t), st>>>(h->s, T, c.E, G, h->hist,
+                                                                                   h->ntok);
+    CK(cudaGetLastError());
+  }
+  h->last_T = T;
+  return LMOE_OK;
+}
+
+int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, cudaStream_t st) {
+  const lmoe_config& c = h->cfg;
+  const int mt = (T + 127) / 128;
+  CUtensorMap tm_x;
+  if (!make_map(&tm_x, x, T, c.d, c.d, 128)) return LMOE_EINVAL;
+  rms_kernel<bf16><<<(T + 7) / 8, 256, 0, st>>>((const bf16*)x, T, c.d, c.rms_eps, h->r);
+  CK(cudaGetLastError());
+  // h = r * (x Wdown^T), stored as hi | mid | lo bf16 parts
+  {
+    TcParams p = tc_base(h);
+    p.tmA[0] = tm_x;
+    p.tmA[1] = tm_x;
+    p.tmB = h->tm_wdown;
+    p.nseg = h->unit_gain ? 1 : 2;
+    p.seg[0] = {0, 0, 0, c.d / 64};
+    p.seg[1] = {0, 0, c.d, c.d / 64};
+    p.M = T;
+    p.n_tiles = c.l / h->bn_down;
+    p.out = h->hx;
+    p.ldo = 3 * c.l;
+    p.split = c.l;
+    p.row_scale = h->r;
+    CK(launch_tc(p, EPI_DOWN3, h->bn_down, std::min(mt * p.n_tiles, h->sms), st));
+  }
+  // s = sigmoid(h Wr^T + c) from six bf16 x bf16 products of the hi/mid/lo parts
+  {
+    TcParams p = tc_base(h);
+    p.tmA[0] = h->tm_hx;
+    p.tmA[1] = h->tm_hx;
+    p.tmB = h->tm_wr;
+    const int L = c.l, nk = c.l / 64;
+    p.nseg = 6;
+    p.seg[0] = {0, L, L, nk};      // mid * mid
+    p.seg[1] = {0, 2 * L, 0, nk};  // lo * hi
+    p.seg[2] = {0, 0, 2 * L, nk};  // hi * lo
+    p.seg[3] = {0, L, 0, nk};      // mid * hi
+    p.seg[4] = {0, 0, L, nk};      // hi * mid
+    p.seg[5] = {0, 0, 0, nk};      // hi * hi
+    p.M = T;
+    p.n_tiles = c.E / h->bn_r;
+    p.out = h->s;
+    p.ldo = c.E;
+    p.col_bias = h->c;
+    CK(launch_tc(p, EPI_ROUTER, h->bn_r, std::min(mt * p.n_tiles, h->sms), st));
+  }
+  int rc = route_from_scores(h, T, flags, st);
+  if (rc) return rc;
+  // shared expert, first half: a_s = silu(r x Ws1^T) * (r x Ws3^T)
+  if (c.hs) {
+    TcParams p = tc_base(h);
+    p.tmA[0] = tm_x;
+    p.tmA[1] = tm_x;
+    p.tmB = h->tm_ws13;
+    p.nseg = 1;
+    p.seg[0] = {0, 0, 0, c.d / 64};
+    p.M = T;
+    p.n_tiles = 2 * c.hs / h->bn_s1;
+    p.out = h->a_s;
+    p.ldo = c.hs;
+    p.row_scale = h->r;
+    CK(launch_tc(p, EPI_SWIGLU, h->bn_s1, std::min(mt * p.n_tiles, h->sms), st));
+  }
+  // routed experts, grouped over the permuted rows
+  {
+    TcParams p = tc_base(h);
+    p.tmA[0] = h->tm_aperm;
+    p.tmA[1] = h->tm_aperm;
+    p.tmB = h->tm_w13;
+    p.nseg = 1;
+    p.seg[0] = {0, 0, 0, c.l / 64};
+    p.grouped = 1;
+    p.n_tiles = 2 * c.h / h->bn_e1;
+    p.mtile_table = h->mtiles;
+    p.num_mtiles = h->num_mtiles;
+    p.seg_off = h->offsets;
+    p.b_rows_per_group = 2 * c.h;
+    p.out = h->act;
+    p.ldo = c.h;
+    CK(launch_tc(p, EPI_SWIGLU, h->bn_e1, h->sms, st));
+  }
+  {
+    TcParams p = tc_base(h);
+    p.tmA[0] = h->tm_act;
+    p.tmA[1] = h->tm_act;
+    p.tmB = h->tm_w2;
+    p.nseg = 1;
+    p.seg[0] = {0, 0, 0, c.h / 64};
+    p.grouped = 1;
+    p.n_tiles = c.l / h->bn_e2;
+    p.mtile_table = h->mtiles;
+    p.num_mtiles = h->num_mtiles;
+    p.seg_off = h->offsets;
+    p.b_rows_per_group = c.l;
+    p.out = h->o;
+    p.ldo = c.l;
+    CK(launch_tc(p, EPI_BF16, h->bn_e2, h->sms, st));
+  }
+  combine_kernel<bf16><<<(T + 7) / 8, 256, 0, st>>>((const bf16*)h->o, h->gates, h->inv, T, c.k, c.l,
+                                                    (bf16*)h->z);
+  CK(cudaGetLastError());
+  // y = [z | a_s] [W_up | Ws2]^T
+  {
+    TcParams p = tc_base(h);
+    p.tmA[0] = h->tm_z;
+    p.tmA[1] = c.hs ? h->tm_as : h->tm_z;
+    p.tmB = h->tm_wy;
+    p.nseg = c.hs ? 2 : 1;
+    p.seg[0] = {0, 0, 0, c.l / 64};
+    p.seg[1] = {1, 0, c.l, c.hs / 64};
+    p.M = T;
+    p.n_tiles = c.d / h->bn_y;
+    p.out = y;
+    p.ldo = c.d;
+    CK(launch_tc(p, EPI_BF16, h->bn_y, std::min(mt * p.n_tiles, h->sms), st));
+  }
+  return LMOE_OK;
+}
+
+int forward_f32(lmoe_handle* h, const void* xv, void* yv, int T, uint32_t flags, cudaStream_t st) {
+  const lmoe_config& c = h->cfg;
+  const float* x = (const float*)xv;
+  const int mt = (T + 127) / 128;
+  rms_kernel<float><<<(T + 7) / 8, 256, 0, st>>>(x, T, c.d, c.rms_eps, h->r);
+  CK(cudaGetLastError());
+  SimtParams b;
+  memset(&b, 0, sizeof(b));
+  b.status = h->status;
+  {  // h = r * (x Wdown'^T)
+    SimtParams p = b;
+    p.A0 = x; p.lda0 = c.d; p.K0 = c.d; p.a_rows = T;
+    p.B0 = (const float*)h->w_down; p.ldb = c.d;
+    p.M = T; p.N = c.l;
+    p.out = (float*)h->hx; p.ldo = c.l; p.row_scale = h->r;
+    CK(launch_simt<SE_STORE>(p, mt, st));
+  }
+  {  // s = sigmoid(h Wr^T + c)
+    SimtParams p = b;
+    p.A0 = (const float*)h->hx; p.lda0 = c.l; p.K0 = c.l; p.a_rows = T;
+    p.B0 = (const float*)h->w_r; p.ldb = c.l;
+    p.M = T; p.N = c.E;
+    p.out = h->s; p.ldo = c.E; p.col_bias = h->c;
+    CK(launch_simt<SE_ROUTER>(p, mt, st));
+  }
+  int rc = route_from_scores(h, T, flags, st);
+  if (rc) return rc;
+  if (c.hs) {  // a_s = silu(r x Ws1'^T) * (r x Ws3'^T)
+    SimtParams p = b;
+    p.A0 = x; p.lda0 = c.d; p.K0 = c.d; p.a_rows = T;
+    p.B0 = (const float*)h->ws13; p.B1 = (const float*)h->ws3f; p.ldb = c.d;
+    p.M = T; p.N = c.hs;
+    p.out = (float*)h->a_s; p.ldo = c.hs; p.row_scale = h->r;
+    CK(launch_simt<SE_SWIGLU>(p, mt, st));
+  }
+  const int gm = (T * c.k + 127) / 128 + c.E;
+  {  // act = silu(A W1_e^T) * (A W3_e^T)
+    SimtParams p = b;
+    p.A0 = (const float*)h->a_perm; p.lda0 = c.l; p.K0 = c.l; p.a_rows = T * c.k;
+    p.B0 = (const float*)h->w13; p.B1 = (const float*)h->w3f; p.ldb = c.l;
+    p.b_group_stride = (long long)c.h * c.l;
+    p.N = c.h; p.grouped = 1;
+    p.mtile_table = h->mtiles; p.num_mtiles = h->num_mtiles; p.seg_off = h->offsets;
+    p.out = (float*)h->act; p.ldo = c.h;
+    CK(launch_simt<SE_SWIGLU>(p, gm, st));
+  }
+  {  // o = act W2_e^T
+    SimtParams p = b;
+    p.A0 = (const float*)h->act; p.lda0 = c.h; p.K0 = c.h; p.a_rows = T * c.k;
+    p.B0 = (const float*)h->w2; p.ldb = c.h;
+    p.b_group_stride = (long long)c.l * c.h;
+    p.N = c.l; p.grouped = 1;
+    p.mtile_table = h->mtiles; p.num_mtiles = h->num_mtiles; p.seg_off = h->offsets;
+    p.out = (float*)h->o; p.ldo = c.l;
+    CK(launch_simt<SE_STORE>(p, gm, st));
+  }
+  combine_kernel<float><<<(T + 7) / 8, 256, 0, st>>>((const float*)h->o, h->gates, h->inv, T, c.k, c.l,
+                                                     (float*)h->z);
+  CK(cudaGetLastError());
+  {  // y = [z | a_s] [W_up | Ws2]^T
+    SimtParams p = b;
+    p.A0 = (const float*)h->z; p.lda0 = c.l; p.K0 = c.l;
+    p.A1 = (const float*)h->a_s; p.lda1 = c.hs; p.K1 = c.hs; p.a_rows = T;
+    p.B0 = (const float*)h->wy; p.ldb = c.l + c.hs;
+    p.M = T; p.N = c.d;
+    p.out = (float*)yv; p.ldo = c.d;
+    CK(launch_simt<SE_STORE>(p, mt, st));
+  }
+  return LMOE_OK;
+}
+
+int repack(lmoe_handle* h, const lmoe_weights* w, cudaStream_t st) {
+  const lmoe_config& c = h->cfg;
+  const long long d = c.d, l = c.l, E = c.E, hh = c.h, hs = c.hs;
+  const int TPB = 256;
+  if (h->bf) {
+    const bf16* g = h->unit_gain ? nullptr : (const bf16*)w->rms_gain;
+    if (h->unit_gain)
+      fold_gain_kernel<bf16><<<grid_1d(l * d, TPB), TPB, 0, st>>>((const bf16*)w->w_down, nullptr, l, d,
+                                                                  (bf16*)h->w_down, d, 0);
+    else
+      fold_gain_split_kernel<<<grid_1d(l * d, TPB), TPB, 0, st>>>((const bf16*)w->w_down, g, l, d,
+                                                                  (bf16*)h->w_down);
+    split3_kernel<<<grid_1d(E * l, TPB), TPB, 0, st>>>(w->w_router, E, l, (bf16*)h->w_r);
+    if (hs)
+      interleave_kernel<bf16><<<grid_1d(hs * d, TPB), TPB, 0, st>>>((const bf16*)w->ws1, (const bf16*)w->ws3, g, 1,
+                                                                    hs, d, (bf16*)h->ws13);
+    interleave_kernel<bf16><<<grid_1d(E * hh * l, TPB), TPB, 0, st>>>((const bf16*)w->w1, (const bf16*)w->w3,
+                                                                      nullptr, E, hh, l, (bf16*)h->w13);
+    CK(cudaMemcpyAsync(h->w2, w->w2, E * l * hh * 2, cudaMemcpyDeviceToDevice, st));
+    fold_gain_kernel<bf16><<<grid_1d(d * l, TPB), TPB, 0, st>>>((const bf16*)w->w_up, nullptr, d, l,
+                                                                (bf16*)h->wy, l + hs, 0);
+    if (hs)
+      fold_gain_kernel<bf16><<<grid_1d(d * hs, TPB), TPB, 0, st>>>((const bf16*)w->ws2, nullptr, d, hs,
+                                                                   (bf16*)h->wy, l + hs, l);
+  } else {
+    const float* g = (const float*)w->rms_gain;
+    fold_gain_kernel<float><<<grid_1d(l * d, TPB), TPB, 0, st>>>((const float*)w->w_down, g, l, d,
+                                                                 (float*)h->w_down, d, 0);
+    CK(cudaMemcpyAsync(h->w_r, w->w_router, E * l * 4, cudaMemcpyDeviceToDevice, st));
+    if (hs) {
+      fold_gain_kernel<float><<<grid_1d(hs * d, TPB), TPB, 0, st>>>((const float*)w->ws1, g, hs, d,
+                                                                    (float*)h->ws13, d, 0);
+      fold_gain_kernel<float><<<grid_1d(hs * d, TPB), TPB, 0, st>>>((const float*)w->ws3, g, hs, d,
+                                                                    (float*)h->ws3f, d, 0);
+    }
+    CK(cudaMemcpyAsync(h->w13, w->w1, E * hh * l * 4, cudaMemcpyDeviceToDevice, st));
+    CK(cudaMemcpyAsync(h->w3f, w->w3, E * hh * l * 4, cudaMemcpyDeviceToDevice, st));
+    CK(cudaMemcpyAsync(h->w2, w->w2, E * l * hh * 4, cudaMemcpyDeviceToDevice, st));
+    fold_gain_kernel<float><<<grid_1d(d * l, TPB), TPB, 0, st>>>((const float*)w->w_up, nullptr, d, l,
+                                                                 (float*)h->wy, l + hs, 0);
+    if (hs)
+      fold_gain_kernel<float><<<grid_1d(d * hs, TPB), TPB, 0, st>>>((const float*)w->ws2, nullptr, d, hs,
+                                                                    (float*)h->wy, l + hs, l);
+  }
+  CK(cudaGetLastError());
+  if (w->router_bias)
+    CK(cudaMemcpyAsync(h->c, w->router_bias, E * 4, cudaMemcpyDeviceToDevice, st));
+  else
+    CK(cudaMemsetAsync(h->c, 0, E * 4, st));
+  return LMOE_OK;
+}
+
+bool gain_is_unit(const lmoe_config& c, const void* g) {
+  if (!g) return true;
+  const size_t es = c.dtype == LMOE_BF16 ? 2 : 4;
+  std::vector<uint8_t> buf(c.d * es);
+  if (cudaMemcpy(buf.data(), g, buf.size(), cudaMemcpyDeviceToHost) != cudaSuccess) return false;
+  for (int j = 0; j < c.d; ++j) {
+    if (es == 2) {
+      uint16_t v;
+      memcpy(&v, &buf[j * 2], 2);
+      if (v != 0x3F80) return false;
+    } else {
+      float v;
+      memcpy(&v, &buf[j * 4], 4);
+      if (v != 1.0f) return false;
+    }
+  }
+  return true;
+}
+
+}  // namespace
+
+// ======================================================================= C ABI
+extern "C" {
+
+const char* lmoe_strerror(int code) {
+  switch (code) {
+    case LMOE_OK: return "ok";
+    case LMOE_EINVAL: return "invalid argument";
+    case LMOE_ENOMEM: return "out of device memory";
+    case LMOE_ECUDA: return "CUDA error";
+    case LMOE_EUNSUPPORTED: return "unsupported shape";
+    case LMOE_EDEVICE: return "device is not sm_100";
+    default: return "unknown error";
+  }
+}
+
+static void size_handle(lmoe_handle* h, const lmoe_config* cfg) {
+  h->cfg = *cfg;
+  h->bf = cfg->dtype == LMOE_BF16;
+  h->es = h->bf ? 2 : 4;
+  h->nblk_max = (cfg->max_tokens + kTokBlock - 1) / kTokBlock;
+  h->max_mtiles = (int)(((long long)cfg->max_tokens * cfg->k + kTileRows - 1) / kTileRows) + cfg->E;
+  int g = (cfg->E + 147) / 148;
+  h->hist_g = g < 1 ? 1 : (g > 12 ? 12 : g);
+}
+
+int lmoe_workspace_bytes(const lmoe_config* cfg, size_t* bytes) {
+  int rc = validate(cfg);
+  if (rc) return rc;
+  if (!bytes) return LMOE_EINVAL;
+  lmoe_handle h;
+  size_handle(&h, cfg);
+  h.unit_gain = false;  // upper bound
+  Arena a;
+  plan_layout(&h, a);
+  *bytes = a.off;
+  return LMOE_OK;
+}
+
+int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, void* stream, lmoe_handle** out) {
+  if (!out) return LMOE_EINVAL;
+  *out = nullptr;
+  int rc = validate(cfg);
+  if (rc) return rc;
+  if (!w || !w->w_down || !w->w_router || !w->w1 || !w->w3 || !w->w2 || !w->w_up) return LMOE_EINVAL;
+  if (cfg->hs && (!w->ws1 || !w->ws3 || !w->ws2)) return LMOE_EINVAL;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LMOE_ECUDA;
+  int major = 0, sms = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (major != 10) return LMOE_EDEVICE;
+  lmoe_handle* h = new (std::nothrow) lmoe_handle();
+  if (!h) return LMOE_ENOMEM;
+  size_handle(h, cfg);
+  h->device = dev;
+  h->sms = sms;
+  h->unit_gain = gain_is_unit(*cfg, w->rms_gain);
+  Arena a;
+  plan_layout(h, a);
+  if (cudaMalloc(&h->arena, a.off) != cudaSuccess) {
+    cudaGetLastError();
+    delete h;
+    return LMOE_ENOMEM;
+  }
+  h->arena_bytes = a.off;
+  for (auto& it : a.items) *it.first = h->arena + it.second;
+  cudaStream_t st = (cudaStream_t)stream;
+  rc = repack(h, w, st);
+  if (!rc && cudaMemsetAsync(h->bias, 0, cfg->E * 4, st) != cudaSuccess) rc = LMOE_ECUDA;
+  if (!rc && cudaMemsetAsync(h->hist, 0, (size_t)cfg->E * LMOE_NBINS * 4, st) != cudaSuccess) rc = LMOE_ECUDA;
+  if (!rc && cudaMemsetAsync(h->ntok, 0, 8, st) != cudaSuccess) rc = LMOE_ECUDA;
+  if (!rc && cudaMemsetAsync(h->status, 0, 4, st) != cudaSuccess) rc = LMOE_ECUDA;
+  if (!rc && h->bf) rc = build_maps(h);
+  if (rc) {
+    cudaStreamSynchronize(st);
+    cudaFree(h->arena);
+    delete h;
+    return rc;
+  }
+  *out = h;
+  return LMOE_OK;
+}
+
+int lmoe_destroy(lmoe_handle* h) {
+  if (!h) return LMOE_EINVAL;
+  cudaDeviceSynchronize();
+  cudaFree(h->arena);
+  delete h;
+  return LMOE_OK;
+}
+
+int lmoe_forward(lmoe_handle* h, const void* x, void* y, int32_t T, uint32_t flags, void* stream) {
+  if (!h || T < 0 || T > h->cfg.max_tokens) return LMOE_EINVAL;
+  if (T == 0) return LMOE_OK;
+  if (!x || !y || ((uintptr_t)x & 15) || ((uintptr_t)y & 15)) return LMOE_EINVAL;
+  const size_t bytes = (size_t)T * h->cfg.d * h->es;
+  if ((const char*)x < (const char*)y + bytes && (const char*)y < (const char*)x + bytes) return LMOE_EINVAL;
+  cudaStream_t st = (cudaStream_t)stream;
+  return h->bf ? forward_bf16(h, x, y, T, flags, st) : forward_f32(h, x, y, T, flags, st);
+}
+
+int lmoe_forward_host(lmoe_handle* h, const void* x_host, void* y_host, int32_t T, uint32_t flags, void* stream) {
+  if (!h || !x_host || !y_host || T < 0 || T > h->cfg.max_tokens) return LMOE_EINVAL;
+  if (T == 0) return LMOE_OK;
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t bytes = (size_t)T * h->cfg.d * h->es;
+  CK(cudaMemcpyAsync(h->x_stage, x_host, bytes, cudaMemcpyHostToDevice, st));
+  int rc = lmoe_forward(h, h->x_stage, h->y_stage, T, flags, stream);
+  if (rc) return rc;
+  CK(cudaMemcpyAsync(y_host, h->y_stage, bytes, cudaMemcpyDeviceToHost, st));
+  return LMOE_OK;
+}
+
+int lmoe_route_scores(lmoe_handle* h, const float* scores, int32_t T, uint32_t flags, void* stream) {
+  if (!h || !scores || T < 0 || T > h->cfg.max_tokens) return LMOE_EINVAL;
+  if (T == 0) return LMOE_OK;
+  cudaStream_t st = (cudaStream_t)stream;
+  CK(cudaMemcpyAsync(h->s, scores, (size_t)T * h->cfg.E * 4, cudaMemcpyDeviceToDevice, st));
+  return route_from_scores(h, T, flags, st);
+}
+
+int lmoe_qb_update(lmoe_handle* h, float beta, uint32_t flags, void* stream) {
+  if (!h || !(beta == beta)) return LMOE_EINVAL;
+  cudaStream_t st = (cudaStream_t)stream;
+  qb_quantile_kernel<<<h->cfg.E, 256, 0, st>>>(h->hist, h->ntok, h->bias, h->cfg.E, h->cfg.k,
+                                                (flags & LMOE_QB_LITERAL) ? 1 : 0, h->u, h->status);
+  CK(cudaGetLastError());
+  qb_apply_kernel<<<1, 1024, 0, st>>>(h->bias, h->ntok, h->u, h->cfg.E, beta);
+  CK(cudaGetLastError());
+  return LMOE_OK;
+}
+
+int lmoe_get_routing(lmoe_handle* h, int32_t* idx, float* gates, float* scores, int32_t* counts, int32_t* offsets,
+                     int32_t* perm, int32_t* inv, void* stream) {
+  if (!h) return LMOE_EINVAL;
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t T = h->last_T, k = h->cfg.k, E = h->cfg.E;
+  auto cp = [&](void* dst, const void* src, size_t bytes) {
+    return dst && bytes ? cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, st) : cudaSuccess;
+  };
+  CK(cp(idx, h->idx, T * k * 4));
+  CK(cp(gates, h->gates, T * k * 4));
+  CK(cp(scores, h->s, T * E * 4));
+  CK(cp(counts, h->counts, E * 4));
+  CK(cp(offsets, h->offsets, (E + 1) * 4));
+  CK(cp(perm, h->perm, T * k * 4));
+  CK(cp(inv, h->inv, T * k * 4));
+  return LMOE_OK;
+}
+
+int lmoe_get_bias(lmoe_handle* h, float* b, void* stream) {
+  if (!h || !b) return LMOE_EINVAL;
+  CK(cudaMemcpyAsync(b, h->bias, h->cfg.E * 4, cudaMemcpyDeviceToDevice, (cudaStream_t)stream));
+  return LMOE_OK;
+}
+
+int lmoe_set_bias(lmoe_handle* h, const float* b, void* stream) {
+  if (!h || !b) return LMOE_EINVAL;
+  CK(cudaMemcpyAsync(h->bias, b, h->cfg.E * 4, cudaMemcpyDeviceToDevice, (cudaStream_t)stream));
+  return LMOE_OK;
+}
+
+int lmoe_get_hist(lmoe_handle* h, uint32_t* hist, int64_t* ntok, void* stream) {
+  if (!h) return LMOE_EINVAL;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (hist) CK(cudaMemcpyAsync(hist, h->hist, (size_t)h->cfg.E * LMOE_NBINS * 4, cudaMemcpyDeviceToDevice, st));
+  if (ntok) CK(cudaMemcpyAsync(ntok, h->ntok, 8, cudaMemcpyDeviceToDevice, st));
+  return LMOE_OK;
+}
+
+int lmoe_set_hist(lmoe_handle* h, const uint32_t* hist, const int64_t* ntok, void* stream) {
+  if (!h || !hist || !ntok) return LMOE_EINVAL;
+  cudaStream_t st = (cudaStream_t)stream;
+  CK(cudaMemcpyAsync(h->hist, hist, (size_t)h->cfg.E * LMOE_NBINS * 4, cudaMemcpyDeviceToDevice, st));
+  CK(cudaMemcpyAsync(h->ntok, ntok, 8, cudaMemcpyDeviceToDevice, st));
+  return LMOE_OK;
+}
+
+int lmoe_get_status(lmoe_handle* h, uint32_t* status) {
+  if (!h || !status) return LMOE_EINVAL;
+  CK(cudaDeviceSynchronize());
+  CK(cudaMemcpy(status, h->status, 4, cudaMemcpyDeviceToHost));
+  CK(cudaMemset(h->status, 0, 4));
+  return LMOE_OK;
+}
+
+int lmoe_gemm_bf16(const void* a, const void* b, float* c, int32_t M, int32_t N, int32_t K, void* stream) {
+  if (!a || !b || !c || M <= 0 || N <= 0 || K <= 0 || N % 64 || K % 64) return LMOE_EINVAL;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int bn = pick_bn(N);
+  TcParams p;
+  memset(&p, 0, sizeof(p));
+  if (!make_map(&p.tmA[0], a, M, K, K, 128) || !make_map(&p.tmB, b, N, K, K, bn)) return LMOE_EINVAL;
+  p.tmA[1] = p.tmA[0];
+  p.nseg = 1;
+  p.seg[0] = {0, 0, 0, K / 64};
+  p.M = M;
+  p.n_tiles = N / bn;
+  p.out = c;
+  p.ldo = N;
+  const int tiles = ((M + 127) / 128) * p.n_tiles;
+  CK(launch_tc(p, EPI_F32, bn, tiles < sms ? tiles : sms, (cudaStream_t)stream));
+  return LMOE_OK;
+}
+
+}  // extern "C"

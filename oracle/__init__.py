@@ -36,7 +36,8 @@ histogram over [0, 1] for the QB quantile.
 Readings where the pages are silent (each also listed in the design notes):
   * QB quantile is the type-1 (inverse empirical CDF) quantile at rank
     m = ceil((E - k) * N / E), computed in exact integer arithmetic.
-  * Bin rule min(floor(s * 4096), 4095); the estimate interpolates linearly
+  * Bin rule min(floor(s * 4096), 4095) on the fp32 score (the layer keeps s in
+    fp32, so the bin is decided in that precision); the estimate interpolates linearly
     inside the bin where the cumulative count first reaches m, so
     |estimate - exact| <= 1/4096.
   * The update uses the quantile of the biased column s + b, which is
@@ -238,8 +239,13 @@ def stable_permutation(idx: np.ndarray, E: int):
 # --------------------------------------------------------------------------
 
 def score_bins(s: np.ndarray, nbins: int = NBINS) -> np.ndarray:
-    """Bin of each score on [0, 1]: min(floor(s * nbins), nbins - 1)."""
-    return np.minimum(np.floor(s * nbins), nbins - 1).astype(np.int64)
+    """Bin of each score on [0, 1]: min(floor(s * nbins), nbins - 1).
+
+    The layer keeps its router scores in fp32, so the bin (an integer decided by a float) is
+    taken on the score rounded to fp32, the precision the layer fixes for s.
+    """
+    s32 = np.asarray(s, dtype=np.float32).astype(np.float64)
+    return np.minimum(np.floor(s32 * nbins), nbins - 1).astype(np.int64)
 
 
 def score_histogram(s: np.ndarray, nbins: int = NBINS) -> np.ndarray:

@@ -294,7 +294,7 @@ def test_histogram_quantile_within_one_bin_of_exact(case):
         s = 0.5 + rng.random((N, E)) / 8192
     else:
         s = np.floor(rng.random((N, E)) * 4097) / 4096
-    s = np.clip(s, 0, 1)
+    s = np.clip(s, 0, 1).astype(np.float32).astype(np.float64)  # bins are taken on fp32 scores
     hist = oracle.score_histogram(s)
     m = oracle.quantile_rank(N, k, E)
     for e in range(E):
@@ -336,7 +336,7 @@ def test_qb_single_step_at_beta_one():
     b1 = oracle.qb_update(b, hist, N, k, 1.0)
     m = oracle.quantile_rank(N, k, E)
     level = np.array([oracle.exact_quantile(s[:, e] + b1[e], m) for e in range(E)])
-    assert level.max() - level.min() <= 2 / 4096 + 1e-12
+    assert level.max() - level.min() <= 2 / 4096 + 1e-7  # + fp32 rounding of the binned scores
     before = oracle.load_ratio(oracle.expert_counts(oracle.biased_topk(s, b, k), E))
     after = oracle.load_ratio(oracle.expert_counts(oracle.biased_topk(s, b1, k), E))
     assert after < before / 3
