@@ -1,0 +1,418 @@
+#!/usr/bin/env python
+"""Throughput of the Stable-LatentMoE layer step on B200s, one JSON line on rank 0.
+
+A step is one pass of the whole hot path over one batch of synthetic tokens already resident
+in HBM: lmoe_forward with QB statistics recorded (RMSNorm, latent down-projection, sigmoid
+router, biased top-k and gates, histogram, dispatch plan and permutation, routed SwiGLU
+experts, shared SwiGLU expert, combine, up-projection), then lmoe_qb_update.  With N > 1 ranks
+every rank runs its own tokens (weak scaling) and the ranks sum their QB histograms with one
+NCCL all-reduce before the update, so every rank keeps the same bias.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mini_replica] [--tokens T]
+    python bench.py --impl reference ...   # the CPU oracle on the host cores, same metric
+
+Timing: W untimed steps, then K steps each bracketed by CUDA events on the launching stream,
+with a 256 MiB write between steps (outside the events) to flush the 126 MB L2; barrier and
+synchronize on both sides; the per-step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "LatentMoE layer fwd tokens/s on 1 B200; % BF16 tensor peak; router/permute GB/s"
+UNIT = "tokens/s"
+BETA = 0.01
+FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return p, "measured (MEASURED_PEAKS.json)"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def csrc_digest() -> str:
+    d = os.path.join(ROOT, "latent_routing_quantile_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(d)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(d, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def stage_work(shape, T):
+    """Algorithmic FLOPs and HBM bytes of one launch of each stage on T tokens (bf16 storage)."""
+    d, l, E, k, h, hs = shape.d, shape.l, shape.E, shape.k, shape.h, shape.hs
+    w = 2 if shape.dtype == "bf16" else 4
+    TK = T * k
+    nblk = (T + 127) // 128
+    return {
+        "rms": (0, T * w * d + 4 * T),
+        "down_proj": (2 * T * d * l, T * w * d + l * d * w + 4 * T * l),
+        "router": (2 * T * l * E, 4 * T * l + 4 * E * l + 4 * T * E),
+        "topk": (0, 4 * T * E + 12 * TK),
+        "plan": (0, 3 * 4 * nblk * E),
+        "gather": (0, TK * (2 * w * l + 8)),
+        "hist": (0, 4 * T * E),
+        "shared_swiglu": (4 * T * d * hs, T * w * d + 2 * hs * d * w + T * w * hs),
+        "expert_swiglu": (4 * TK * l * h, TK * w * l + 2 * E * h * l * w + TK * w * h),
+        "expert_down": (2 * TK * h * l, TK * w * h + E * l * h * w + TK * w * l),
+        "combine": (0, TK * (w * l + 8) + T * w * l),
+        "up_proj": (2 * T * d * (l + hs), T * w * (l + hs) + d * (l + hs) * w + T * w * d),
+        "qb_quantile": (0, 2 * E * 4096 * 4),
+        "qb_apply": (0, 16 * E),
+    }
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while the timed region runs."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples, self.reasons = [], 0
+        self.period = period_s
+        self.stop_ev = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.hnd = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.hnd, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        while not self.stop_ev.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.hnd, self.nv.NVML_CLOCK_SM))
+                self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.hnd)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.th = threading.Thread(target=self._run, daemon=True)
+            self.th.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self.stop_ev.set()
+            self.th.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "samples": len(self.samples),
+                "reasons": sorted(n for b, n in self.REASONS.items() if self.reasons & b)}
+
+
+# ----------------------------------------------------------------------------------------- ours
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import datagen
+    import latent_routing_quantile_b200 as lq
+
+    torch.cuda.set_device(local_rank)
+    shape = datagen.WORKLOADS[args.workload]
+    if args.tokens:
+        shape = shape.with_tokens(args.tokens)
+    T = shape.T
+    w = datagen.layer_weights(shape)
+    x_cpu = datagen.tokens(shape, seed=shape.seed + 1000 * rank)
+    layer = lq.layer_from_weights(shape, w)
+    stream = torch.cuda.current_stream()
+    x = x_cpu.cuda()
+    y = torch.empty_like(x)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+
+    hist_buf = torch.empty((shape.E, lq.NBINS), dtype=torch.int32, device="cuda")
+    ntok_buf = torch.empty(1, dtype=torch.int64, device="cuda")
+
+    def step():
+        layer.forward(x, y, record_stats=True)
+        if world > 1:  # the one exchange step: sum the QB statistics of all ranks
+            hist, n = layer.hist()
+            dist.all_reduce(hist)
+            dist.all_reduce(n)
+            layer.set_hist(hist, n)
+        layer.qb_update(BETA)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    barrier()
+    # ---------------- timed region
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    launches0 = layer.launches()
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        barrier()
+    launches = layer.launches() - launches0
+    ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / args.steps
+    # per-stage times: the same K steps again with an event before every stage (eager launches;
+    # the timed region above replays each call as one CUDA graph)
+    layer.profile(True)
+    layer.profile_read()
+    barrier()
+    for i in range(args.steps):
+        flush.zero_()
+        step()
+    barrier()
+    stage_ms, nfwd = layer.profile_read()
+    layer.profile(False)
+    ms_t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    assert layer.status() == 0, "device status word set during the bench"
+
+    # ---------------- end to end through the host-buffer entry point
+    e2e_steps = max(3, min(args.steps, 50))
+    xh = x_cpu.pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+
+    def step_host():
+        layer.forward_host(xh, yh, record_stats=True)
+        if world > 1:
+            hist, n = layer.hist()
+            dist.all_reduce(hist)
+            dist.all_reduce(n)
+            layer.set_hist(hist, n)
+        layer.qb_update(BETA)
+
+    for _ in range(3):
+        flush.zero_()
+        step_host()
+    barrier()
+    es = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+    ee = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+    for i in range(e2e_steps):
+        flush.zero_()
+        es[i].record(stream)
+        step_host()
+        ee[i].record(stream)
+    barrier()
+    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(es, ee)) / e2e_steps
+    e2e_t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+    e2e_ms = float(e2e_t.item())
+    layer.close()
+
+    if rank != 0:
+        return None
+    peaks, peak_src = load_peaks()
+    work = stage_work(shape, T)
+    per_launch = {n: stage_ms[n] / max(1, nfwd) for n in stage_ms}
+    step_stage_ms = sum(per_launch.values())
+    kernels = {}
+    for n, t in per_launch.items():
+        fl, by = work[n]
+        t_s = t / 1e3
+        if t_s <= 0:
+            continue
+        t_tensor = fl / (peaks["bf16_tflops"] * 1e12) if fl else 0.0
+        t_hbm = by / (peaks["hbm_gbs"] * 1e9)
+        bound = "tensor" if t_tensor >= t_hbm else "hbm"
+        kernels[n] = {"ms": round(t, 5), "share": round(t / step_stage_ms, 4), "bound": bound,
+                      "tflops": round(fl / t_s / 1e12, 2), "gbs": round(by / t_s / 1e9, 1),
+                      "frac": round(max(t_tensor, t_hbm) / t_s, 4)}
+    dom = max(kernels, key=lambda n: kernels[n]["ms"])
+    kd = kernels[dom]
+    fl, by = work[dom]
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        tj = json.load(open(tpath))
+        ent = tj.get("kernels", {}).get(dom)
+        if ent and tj.get("csrc_digest") == csrc_digest() and tj.get("workload") == shape.name:
+            traffic = ent["dram_bytes_per_launch"]
+    if kd["bound"] == "tensor":
+        roof = {"bound": "tensor", "achieved": kd["tflops"], "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": kd["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
+    roof.update({"traffic": traffic, "kernel": dom, "algorithmic_flops": fl, "algorithmic_bytes": by,
+                 "peak_source": f"{peak_src}, burst"})
+    gemm = [n for n in work if work[n][0] > 0]
+    gemm_flops = sum(work[n][0] for n in gemm)
+    rp = ["router", "topk", "plan", "gather"]
+    rp_bytes = sum(work[n][1] for n in rp)
+    rp_ms = sum(per_launch[n] for n in rp)
+    value = T * world / (ms_max / 1e3)
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_max, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": shape.dtype, "data": "synthetic (seeded; x ~ N(0,1), weights ~ N(0,1/fan_in))",
+        "config": {"workload": shape.name, "T": T, "d": shape.d, "l": shape.l, "E": shape.E, "k": shape.k,
+                   "h": shape.h, "hs": shape.hs, "tokens_per_gpu": T, "global_tokens": T * world,
+                   "step": "forward with QB statistics + QB update", "beta": BETA,
+                   "l2": "flushed between steps (256 MiB write outside the timed events)",
+                   "parallelism": f"dp{world}" + (" (histogram all-reduce)" if world > 1 else "")},
+        "e2e": {"value": round(T * world / (e2e_ms / 1e3), 1), "unit": UNIT, "ms_per_step": round(e2e_ms, 5),
+                "h2d_bytes_per_step": T * shape.d * (2 if shape.dtype == "bf16" else 4),
+                "d2h_bytes_per_step": T * shape.d * (2 if shape.dtype == "bf16" else 4),
+                "api": "lmoe_forward_host + lmoe_qb_update, pinned host buffers"},
+        "gpu_launches": launches,
+        "kernel_timing": "CUDA events before every stage on the launching stream, in a second pass of the "
+                         "same K steps with eager launches (the timed region replays each call as a CUDA graph)",
+        "roofline": roof,
+        "tensor_peak_frac_step": round(gemm_flops / (ms_max / 1e3) / (peaks["bf16_tflops"] * 1e12), 4),
+        "router_permute_gbs": round(rp_bytes / (rp_ms / 1e3) / 1e9, 1) if rp_ms > 0 else None,
+        "kernels": kernels,
+        "clocks": clk.summary(),
+    }
+    return out
+
+
+# ------------------------------------------------------------------------------ CPU oracle legs
+def oracle_step_time(shape, w, x_sample, b):
+    """One oracle pass (layer forward + QB update) over the sample; returns seconds."""
+    import numpy as np
+
+    import oracle
+    t0 = time.perf_counter()
+    out = oracle.layer_forward(x_sample, w, b, shape.k, shape.rms_eps)
+    oracle.qb_update(b, oracle.score_histogram(out["s"]), x_sample.shape[0], shape.k, BETA)
+    return time.perf_counter() - t0
+
+
+def blas_threads():
+    try:
+        import threadpoolctl
+        n = [p["num_threads"] for p in threadpoolctl.threadpool_info() if p.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(shape, budget_s=15.0):
+    import numpy as np
+
+    import datagen
+    w = datagen.layer_weights(shape)
+    b = np.zeros(shape.E)
+    S = 128
+    x = datagen.tokens(shape, rows=range(S))
+    t = oracle_step_time(shape, w, x, b)
+    S = int(min(shape.T, max(S, S * budget_s / max(t, 1e-3) / 2)))
+    x = datagen.tokens(shape, rows=range(S))
+    t = oracle_step_time(shape, w, x, b)
+    return {"value": round(S / t, 2), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"first {S} tokens of the {shape.name} workload: float64 numpy layer forward + QB update, "
+                      f"{t:.1f} s", "seconds": round(t, 2)}
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return None
+    import numpy as np
+
+    import datagen
+    shape = datagen.WORKLOADS[args.workload]
+    if args.tokens:
+        shape = shape.with_tokens(args.tokens)
+    w = datagen.layer_weights(shape)
+    b = np.zeros(shape.E)
+    S0 = 64
+    t0 = oracle_step_time(shape, w, datagen.tokens(shape, rows=range(S0)), b)
+    # size the per-step sample so that warm-up + timed steps take about 90 s of host time
+    per_step = 90.0 / max(1, args.steps + args.warmup)
+    S = int(min(shape.T, max(16, S0 * per_step / max(t0, 1e-3))))
+    x = datagen.tokens(shape, rows=range(S))
+    for _ in range(args.warmup):
+        oracle_step_time(shape, w, x, b)
+    ts = [oracle_step_time(shape, w, x, b) for _ in range(args.steps)]
+    sec = sum(ts) / len(ts)
+    value = S / sec
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (same seeded workload)",
+        "config": {"workload": shape.name, "T": shape.T, "d": shape.d, "l": shape.l, "E": shape.E, "k": shape.k,
+                   "h": shape.h, "hs": shape.hs, "sample_tokens_per_step": S},
+        "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"first {S} tokens of {shape.name} per step: float64 numpy forward + QB update"},
+        "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mini_replica")
+    ap.add_argument("--tokens", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        out = run_reference(args, rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+
+    import datetime
+
+    import torch.distributed as dist
+    if world > 1:
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=__import__("torch").device("cuda", local_rank))
+    try:
+        out = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+    if out is not None:
+        if world == 1 and not args.no_cpu_baseline:
+            import datagen
+            shape = datagen.WORKLOADS[args.workload]
+            if args.tokens:
+                shape = shape.with_tokens(args.tokens)
+            out["cpu_baseline"] = cpu_baseline(shape)
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

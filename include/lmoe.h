@@ -155,6 +155,20 @@ int lmoe_set_hist(lmoe_handle *h, const uint32_t *hist_dev, const int64_t *ntok_
 /* Synchronises the device, then returns the status word in *status and clears it. */
 int lmoe_get_status(lmoe_handle *h, uint32_t *status);
 
+/* Measurement support.  With profiling enabled, every lmoe_forward, lmoe_route_scores and
+ * lmoe_qb_update records a CUDA event on its stream before each of its stages and after the last
+ * (at most 4096 calls between two reads; later calls go unrecorded).  lmoe_profile_read
+ * synchronises the device, stores in ms[i] (n >= 14) the time of stage i summed over the recorded
+ * calls, the number of recorded forwards in *calls, and forgets the records.  Stage i is named by
+ * lmoe_stage_name(i): rms, down_proj, router, topk, plan, gather, hist, shared_swiglu,
+ * expert_swiglu, expert_down, combine, up_proj, qb_quantile, qb_apply. */
+int lmoe_profile_enable(lmoe_handle *h, int32_t enable);
+int lmoe_profile_read(lmoe_handle *h, float *ms, int32_t n, int32_t *calls);
+const char *lmoe_stage_name(int32_t i);
+
+/* Number of kernels the handle has launched since it was created. */
+int lmoe_launch_count(lmoe_handle *h, int64_t *n);
+
 /* Static text for a return code. */
 const char *lmoe_strerror(int code);
 

@@ -25,7 +25,9 @@ EXPORTED = (
     "lmoe_create", "lmoe_destroy", "lmoe_workspace_bytes", "lmoe_forward", "lmoe_forward_host",
     "lmoe_qb_update", "lmoe_route_scores", "lmoe_get_routing", "lmoe_get_bias", "lmoe_set_bias",
     "lmoe_get_hist", "lmoe_set_hist", "lmoe_get_status", "lmoe_strerror", "lmoe_gemm_bf16",
+    "lmoe_profile_enable", "lmoe_profile_read", "lmoe_stage_name", "lmoe_launch_count",
 )
+NUM_STAGES = 14
 
 
 class LmoeError(RuntimeError):
@@ -69,6 +71,9 @@ def lib() -> ctypes.CDLL:
             "lmoe_set_hist": [vp, vp, vp, vp],
             "lmoe_get_status": [vp, POINTER(u32)],
             "lmoe_gemm_bf16": [vp, vp, vp, i32, i32, i32, vp],
+            "lmoe_profile_enable": [vp, i32],
+            "lmoe_profile_read": [vp, POINTER(c_float), i32, POINTER(i32)],
+            "lmoe_launch_count": [vp, POINTER(ctypes.c_int64)],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -76,6 +81,8 @@ def lib() -> ctypes.CDLL:
             f.restype = c_int
         L.lmoe_strerror.argtypes = [c_int]
         L.lmoe_strerror.restype = ctypes.c_char_p
+        L.lmoe_stage_name.argtypes = [c_int32]
+        L.lmoe_stage_name.restype = ctypes.c_char_p
         _lib = L
     return _lib
 
@@ -204,6 +211,21 @@ class Layer:
         _dev(ntok, torch.int64, (1,), "ntok")
         _check(lib().lmoe_set_hist(self.handle, _ptr(hist), _ptr(ntok), _stream(stream)), "lmoe_set_hist")
 
+    def profile(self, enable: bool = True):
+        _check(lib().lmoe_profile_enable(self.handle, 1 if enable else 0), "lmoe_profile_enable")
+
+    def profile_read(self):
+        """(per-stage milliseconds summed over the recorded calls, number of recorded forwards)."""
+        ms = (c_float * NUM_STAGES)()
+        calls = c_int32(0)
+        _check(lib().lmoe_profile_read(self.handle, ms, NUM_STAGES, ctypes.byref(calls)), "lmoe_profile_read")
+        return {stage_name(i): ms[i] for i in range(NUM_STAGES)}, calls.value
+
+    def launches(self) -> int:
+        n = ctypes.c_int64(0)
+        _check(lib().lmoe_launch_count(self.handle, ctypes.byref(n)), "lmoe_launch_count")
+        return n.value
+
     def status(self) -> int:
         v = c_uint32(0)
         _check(lib().lmoe_get_status(self.handle, ctypes.byref(v)), "lmoe_get_status")
@@ -219,6 +241,10 @@ class Layer:
             self.close()
         except Exception:
             pass
+
+
+def stage_name(i: int) -> str:
+    return lib().lmoe_stage_name(i).decode()
 
 
 def workspace_bytes(d, l, E, k, h, hs, dtype, max_tokens, rms_eps=1e-6) -> int:

@@ -52,12 +52,37 @@ bool make_map(CUtensorMap* m, const void* base, long long rows, long long cols, 
 
 int pick_bn(int n) { return n % 256 == 0 ? 256 : (n % 128 == 0 ? 128 : 64); }
 
+// Tile width for a non-grouped GEMM of M rows and N columns: the widest that divides N and still
+// gives every SM a tile (min_bn = 128 for the SwiGLU epilogue, whose column groups are 128 wide).
+int pick_bn_for(long long M, int N, int sms, int min_bn) {
+  const long long mt = (M + 127) / 128;
+  for (int bn = 256; bn >= min_bn; bn >>= 1)
+    if (N % bn == 0 && mt * (N / bn) >= sms) return bn;
+  for (int bn = min_bn; bn <= 256; bn <<= 1)
+    if (N % bn == 0) return bn;
+  return min_bn;
+}
+
+// Raises a kernel's dynamic shared-memory limit once per device; `done` is the caller's own
+// per-kernel flag word (one bit per device).
+template <typename K>
+cudaError_t ensure_smem_attr(K kern, int bytes, unsigned& done) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const unsigned bit = 1u << (dev & 31);
+  if (done & bit) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done |= bit;
+  return e;
+}
+
 template <int BN, int EPI>
 cudaError_t launch_tc_t(const TcParams& p, int grid, cudaStream_t st) {
   auto kern = tc_gemm_kernel<BN, EPI>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<BN>::kSmemBytes);
+  static unsigned done = 0;
+  cudaError_t e = ensure_smem_attr(kern, TcCfg<BN>::kSmemBytes, done);
   if (e != cudaSuccess) return e;
-  kern<<<grid, 192, TcCfg<BN>::kSmemBytes, st>>>(p);
+  kern<<<grid, kTcThreads, TcCfg<BN>::kSmemBytes, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -82,24 +107,39 @@ cudaError_t launch_tc(const TcParams& p, int epi, int bn, int grid, cudaStream_t
   }
 }
 
+struct TopkArgs {
+  const float* s;
+  const float* b;
+  int T, E, k;
+  int *idx, *rank, *blkcnt, *counts;
+  float* gates;
+  uint16_t* bins;
+  int ld_bins;
+  uint32_t* status;
+};
+
 template <int NJ>
-cudaError_t launch_topk_t(const float* s, const float* b, int T, int E, int k, int* idx, float* gates, int* rank,
-                          int* blkcnt, int* counts, uint32_t* status, cudaStream_t st) {
-  const int nblk = (T + kTokBlock - 1) / kTokBlock;
-  topk_kernel<NJ><<<nblk, 256, E * 4 * sizeof(uint32_t), st>>>(s, b, T, E, k, idx, gates, rank, blkcnt, counts,
-                                                               status);
+cudaError_t launch_topk_t(const TopkArgs& a, cudaStream_t st) {
+  const int nblk = (a.T + kTokBlock - 1) / kTokBlock;
+  const size_t smem = a.E * sizeof(uint32_t) + (a.bins ? (size_t)a.E * kTokBlock * sizeof(uint16_t) : 0);
+  if (smem > 48 * 1024) {
+    static unsigned done = 0;
+    cudaError_t e = ensure_smem_attr(topk_kernel<NJ>, 64 * 1024 + 4 * 1024 + 1024, done);
+    if (e != cudaSuccess) return e;
+  }
+  topk_kernel<NJ><<<nblk, 256, smem, st>>>(a.s, a.b, a.T, a.E, a.k, a.idx, a.gates, a.rank, a.blkcnt, a.counts,
+                                           a.bins, a.ld_bins, a.status);
   return cudaGetLastError();
 }
 
-cudaError_t launch_topk(const float* s, const float* b, int T, int E, int k, int* idx, float* gates, int* rank,
-                        int* blkcnt, int* counts, uint32_t* status, cudaStream_t st) {
-  const int nj = (E + 31) / 32;
-  if (nj <= 1) return launch_topk_t<1>(s, b, T, E, k, idx, gates, rank, blkcnt, counts, status, st);
-  if (nj <= 2) return launch_topk_t<2>(s, b, T, E, k, idx, gates, rank, blkcnt, counts, status, st);
-  if (nj <= 4) return launch_topk_t<4>(s, b, T, E, k, idx, gates, rank, blkcnt, counts, status, st);
-  if (nj <= 8) return launch_topk_t<8>(s, b, T, E, k, idx, gates, rank, blkcnt, counts, status, st);
-  if (nj <= 16) return launch_topk_t<16>(s, b, T, E, k, idx, gates, rank, blkcnt, counts, status, st);
-  return launch_topk_t<32>(s, b, T, E, k, idx, gates, rank, blkcnt, counts, status, st);
+cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st) {
+  const int nj = (a.E + 31) / 32;
+  if (nj <= 1) return launch_topk_t<1>(a, st);
+  if (nj <= 2) return launch_topk_t<2>(a, st);
+  if (nj <= 4) return launch_topk_t<4>(a, st);
+  if (nj <= 8) return launch_topk_t<8>(a, st);
+  if (nj <= 16) return launch_topk_t<16>(a, st);
+  return launch_topk_t<32>(a, st);
 }
 
 template <int EPI>
@@ -111,6 +151,47 @@ cudaError_t launch_simt(const SimtParams& p, int mtiles, cudaStream_t st) {
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// Stages timed by the optional per-stage profiler (lmoe_profile_enable).
+enum Stage : int {
+  ST_RMS = 0, ST_DOWN, ST_ROUTER, ST_TOPK, ST_PLAN, ST_GATHER, ST_HIST, ST_SHARED, ST_EXPERT1, ST_EXPERT2,
+  ST_COMBINE, ST_UP, ST_QB_QUANTILE, ST_QB_APPLY, ST_COUNT
+};
+const char* const kStageNames[ST_COUNT] = {
+    "rms", "down_proj", "router", "topk", "plan", "gather", "hist", "shared_swiglu", "expert_swiglu",
+    "expert_down", "combine", "up_proj", "qb_quantile", "qb_apply"};
+constexpr int kProfRecords = 4096;
+
+// One cached CUDA graph of a call with fixed arguments (see lmoe_forward).
+struct GraphCache {
+  cudaGraphExec_t exec = nullptr;
+  const void* x = nullptr;
+  void* y = nullptr;
+  int T = -1;
+  uint32_t flags = 0;
+  float beta = 0.f;
+  int seen = 0;
+  long long kernels = 0;
+  bool same(const void* x_, void* y_, int T_, uint32_t f_, float b_) const {
+    return x == x_ && y == y_ && T == T_ && flags == f_ && beta == b_;
+  }
+  void reset(const void* x_, void* y_, int T_, uint32_t f_, float b_) {
+    if (exec) cudaGraphExecDestroy(exec);
+    exec = nullptr;
+    x = x_;
+    y = y_;
+    T = T_;
+    flags = f_;
+    beta = b_;
+    seen = 0;
+    kernels = 0;
+  }
+};
+
+struct ProfRecord {
+  int first, n;                 // stages [first, first + n)
+  cudaEvent_t ev[ST_COUNT + 1];  // ev[i] marks the start of stage first + i; ev[n] the end
+};
+
 }  // namespace
 
 // ---------------------------------------------------------------------- handle
@@ -120,7 +201,7 @@ struct lmoe_handle {
   size_t es = 2;  // bytes per activation element
   bool bf = true;
   bool unit_gain = true;
-  int nblk_max = 0, max_mtiles = 0, hist_g = 1;
+  int nblk_max = 0, max_mtiles = 0, ld_bins = 0;
   uint8_t* arena = nullptr;
   size_t arena_bytes = 0;
   // repacked weights
@@ -137,6 +218,7 @@ struct lmoe_handle {
   float* r = nullptr;
   void* hx = nullptr;       // bf16 [Tm, 3l] (hi|mid|lo of h); f32 [Tm, l]
   float* s = nullptr;
+  uint16_t* bins = nullptr;  // [E, ld_bins] histogram bin of every score, expert-major
   int *idx = nullptr, *rank = nullptr, *blkcnt = nullptr, *blkbase = nullptr, *counts = nullptr;
   int *offsets = nullptr, *num_mtiles = nullptr, *perm = nullptr, *inv = nullptr;
   float* gates = nullptr;
@@ -151,8 +233,19 @@ struct lmoe_handle {
   double* u = nullptr;
   int last_T = 0;
   // tensor maps (bf16)
-  CUtensorMap tm_hx, tm_wr, tm_wdown, tm_ws13, tm_aperm, tm_w13, tm_act, tm_w2, tm_z, tm_as, tm_wy;
-  int bn_down = 256, bn_r = 256, bn_s1 = 256, bn_e1 = 256, bn_e2 = 256, bn_y = 256;
+  // weight maps of the non-grouped GEMMs exist for each tile width 64/128/256 that divides N
+  CUtensorMap tm_hx, tm_aperm, tm_w13, tm_act, tm_w2, tm_z, tm_as;
+  CUtensorMap tm_wr[3], tm_wdown[3], tm_ws13[3], tm_wy[3];
+  int bn_e1 = 256, bn_e2 = 256;
+  // launch counter and optional per-stage profiler
+  long long launches = 0;
+  bool profiling = false;
+  std::vector<ProfRecord> prof;
+  int prof_used = 0;
+  ProfRecord* cur = nullptr;
+  // graph replay of repeated calls
+  cudaStream_t cap = nullptr;
+  GraphCache g_fwd, g_qb;
 };
 
 namespace {
@@ -187,6 +280,7 @@ void plan_layout(lmoe_handle* h, Arena& a) {
   a.add((void**)&h->r, Tm * 4);
   a.add(&h->hx, h->bf ? Tm * 3 * l * 2 : Tm * l * 4);
   a.add((void**)&h->s, Tm * E * 4);
+  a.add((void**)&h->bins, (size_t)h->ld_bins * E * 2);
   a.add((void**)&h->idx, TK * 4);
   a.add((void**)&h->gates, TK * 4);
   a.add((void**)&h->rank, TK * 4);
@@ -237,30 +331,57 @@ int grid_1d(long long n, int threads) {
   return (int)(b > 65535 * 16 ? 65535 * 16 : (b < 1 ? 1 : b));
 }
 
+int bn_index(int bn) { return bn == 64 ? 0 : (bn == 128 ? 1 : 2); }
+
+// Maps of one weight matrix [rows, cols] for every tile width that divides rows.
+bool make_weight_maps(CUtensorMap (&m)[3], const void* base, long long rows, long long cols) {
+  bool ok = true;
+  for (int bn = 64; bn <= 256; bn <<= 1)
+    if (rows % bn == 0) ok &= make_map(&m[bn_index(bn)], base, rows, cols, cols, bn);
+  return ok;
+}
+
 int build_maps(lmoe_handle* h) {
   const lmoe_config& c = h->cfg;
   const long long Tm = c.max_tokens, TK = (long long)c.max_tokens * c.k;
   const long long d = c.d, l = c.l, E = c.E, hh = c.h, hs = c.hs;
-  h->bn_down = pick_bn(c.l);
-  h->bn_r = pick_bn(c.E);
-  h->bn_s1 = pick_bn(2 * c.hs) == 64 ? 128 : pick_bn(2 * c.hs);
   h->bn_e1 = (2 * c.h) % 256 == 0 ? 256 : 128;
   h->bn_e2 = pick_bn(c.l);
-  h->bn_y = pick_bn(c.d);
   bool ok = true;
   ok &= make_map(&h->tm_hx, h->hx, Tm, 3 * l, 3 * l, 128);
-  ok &= make_map(&h->tm_wr, h->w_r, E, 3 * l, 3 * l, h->bn_r);
-  const long long wdk = h->unit_gain ? d : 2 * d;
-  ok &= make_map(&h->tm_wdown, h->w_down, l, wdk, wdk, h->bn_down);
-  if (hs) ok &= make_map(&h->tm_ws13, h->ws13, 2 * hs, d, d, h->bn_s1);
+  ok &= make_weight_maps(h->tm_wr, h->w_r, E, 3 * l);
+  ok &= make_weight_maps(h->tm_wdown, h->w_down, l, h->unit_gain ? d : 2 * d);
+  if (hs) ok &= make_weight_maps(h->tm_ws13, h->ws13, 2 * hs, d);
   ok &= make_map(&h->tm_aperm, h->a_perm, TK, l, l, 128);
   ok &= make_map(&h->tm_w13, h->w13, E * 2 * hh, l, l, h->bn_e1);
   ok &= make_map(&h->tm_act, h->act, TK, hh, hh, 128);
   ok &= make_map(&h->tm_w2, h->w2, E * l, hh, hh, h->bn_e2);
   ok &= make_map(&h->tm_z, h->z, Tm, l, l, 128);
   if (hs) ok &= make_map(&h->tm_as, h->a_s, Tm, hs, hs, 128);
-  ok &= make_map(&h->tm_wy, h->wy, d, l + hs, l + hs, h->bn_y);
+  ok &= make_weight_maps(h->tm_wy, h->wy, d, l + hs);
   return ok ? LMOE_OK : LMOE_ECUDA;
+}
+
+// Profiler: opens a record for stages [first, first + n) of one call, marks stage starts, closes.
+void prof_open(lmoe_handle* h, int first, int n) {
+  h->cur = nullptr;
+  if (!h->profiling || h->prof_used >= kProfRecords) return;
+  if ((int)h->prof.size() <= h->prof_used) {
+    ProfRecord r;
+    r.first = r.n = 0;
+    for (auto& e : r.ev) cudaEventCreate(&e);
+    h->prof.push_back(r);
+  }
+  h->cur = &h->prof[h->prof_used++];
+  h->cur->first = first;
+  h->cur->n = n;
+}
+void mark(lmoe_handle* h, int stage, cudaStream_t st) {
+  if (h->cur) cudaEventRecord(h->cur->ev[stage - h->cur->first], st);
+}
+void prof_close(lmoe_handle* h, cudaStream_t st) {
+  if (h->cur) cudaEventRecord(h->cur->ev[h->cur->n], st);
+  h->cur = nullptr;
 }
 
 TcParams tc_base(lmoe_handle* h) {
@@ -274,12 +395,17 @@ TcParams tc_base(lmoe_handle* h) {
 int route_from_scores(lmoe_handle* h, int T, uint32_t flags, cudaStream_t st) {
   const lmoe_config& c = h->cfg;
   const int nblk = (T + kTokBlock - 1) / kTokBlock;
+  mark(h, ST_TOPK, st);
   CK(cudaMemsetAsync(h->counts, 0, c.E * sizeof(int), st));
-  CK(launch_topk(h->s, h->bias, T, c.E, c.k, h->idx, h->gates, h->rank, h->blkcnt, h->counts, h->status, st));
+  TopkArgs ta{h->s, h->bias, T, c.E, c.k, h->idx, h->rank, h->blkcnt, h->counts, h->gates,
+              (flags & LMOE_RECORD_STATS) ? h->bins : nullptr, h->ld_bins, h->status};
+  CK(launch_topk(ta, st));
+  mark(h, ST_PLAN, st);
   plan_kernel<<<(c.E + 31) / 32, 1024, 0, st>>>(h->counts, h->blkcnt, nblk, c.E, h->offsets, h->blkbase,
                                                   h->mtiles, h->num_mtiles);
   CK(cudaGetLastError());
   const int pairs = T * c.k;
+  mark(h, ST_GATHER, st);
   if (h->bf) {
     gather_kernel<bf16><<<(pairs + 7) / 8, 256, 0, st>>>((const bf16*)h->hx, 3 * c.l, c.l, h->idx, h->rank,
                                                          h->blkbase, T, c.E, c.k, h->perm, h->inv,
@@ -290,13 +416,12 @@ int route_from_scores(lmoe_handle* h, int T, uint32_t flags, cudaStream_t st) {
                                                           (float*)h->a_perm, h->status);
   }
   CK(cudaGetLastError());
+  mark(h, ST_HIST, st);
+  h->launches += 3;
   if (flags & LMOE_RECORD_STATS) {
-    const int G = h->hist_g;
-    CK(cudaFuncSetAttribute(hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                            G * LMOE_NBINS * (int)sizeof(uint32_t)));
-    hist_kernel<<<(c.E + G - 1) / G, 1024, G * LMOE_NBINS * sizeof(uint32_t), st>>>(h->s, T, c.E, G, h->hist,
-                                                                                   h->ntok);
+    hist_kernel<<<c.E, 512, 0, st>>>(h->bins, h->ld_bins, T, h->hist, h->ntok);
     CK(cudaGetLastError());
+    h->launches += 1;
   }
   h->last_T = T;
   return LMOE_OK;
@@ -307,31 +432,36 @@ int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, 
   const int mt = (T + 127) / 128;
   CUtensorMap tm_x;
   if (!make_map(&tm_x, x, T, c.d, c.d, 128)) return LMOE_EINVAL;
+  mark(h, ST_RMS, st);
   rms_kernel<bf16><<<(T + 7) / 8, 256, 0, st>>>((const bf16*)x, T, c.d, c.rms_eps, h->r);
   CK(cudaGetLastError());
   // h = r * (x Wdown^T), stored as hi | mid | lo bf16 parts
+  mark(h, ST_DOWN, st);
   {
     TcParams p = tc_base(h);
     p.tmA[0] = tm_x;
     p.tmA[1] = tm_x;
-    p.tmB = h->tm_wdown;
+    const int bn = pick_bn_for(T, c.l, h->sms, 64);
+    p.tmB = h->tm_wdown[bn_index(bn)];
     p.nseg = h->unit_gain ? 1 : 2;
     p.seg[0] = {0, 0, 0, c.d / 64};
     p.seg[1] = {0, 0, c.d, c.d / 64};
     p.M = T;
-    p.n_tiles = c.l / h->bn_down;
+    p.n_tiles = c.l / bn;
     p.out = h->hx;
     p.ldo = 3 * c.l;
     p.split = c.l;
     p.row_scale = h->r;
-    CK(launch_tc(p, EPI_DOWN3, h->bn_down, std::min(mt * p.n_tiles, h->sms), st));
+    CK(launch_tc(p, EPI_DOWN3, bn, std::min(mt * p.n_tiles, h->sms), st));
   }
   // s = sigmoid(h Wr^T + c) from six bf16 x bf16 products of the hi/mid/lo parts
+  mark(h, ST_ROUTER, st);
   {
     TcParams p = tc_base(h);
     p.tmA[0] = h->tm_hx;
     p.tmA[1] = h->tm_hx;
-    p.tmB = h->tm_wr;
+    const int bn = pick_bn_for(T, c.E, h->sms, 64);
+    p.tmB = h->tm_wr[bn_index(bn)];
     const int L = c.l, nk = c.l / 64;
     p.nseg = 6;
     p.seg[0] = {0, L, L, nk};      // mid * mid
@@ -341,30 +471,33 @@ int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, 
     p.seg[4] = {0, 0, L, nk};      // hi * mid
     p.seg[5] = {0, 0, 0, nk};      // hi * hi
     p.M = T;
-    p.n_tiles = c.E / h->bn_r;
+    p.n_tiles = c.E / bn;
     p.out = h->s;
     p.ldo = c.E;
     p.col_bias = h->c;
-    CK(launch_tc(p, EPI_ROUTER, h->bn_r, std::min(mt * p.n_tiles, h->sms), st));
+    CK(launch_tc(p, EPI_ROUTER, bn, std::min(mt * p.n_tiles, h->sms), st));
   }
   int rc = route_from_scores(h, T, flags, st);
   if (rc) return rc;
   // shared expert, first half: a_s = silu(r x Ws1^T) * (r x Ws3^T)
+  mark(h, ST_SHARED, st);
   if (c.hs) {
     TcParams p = tc_base(h);
     p.tmA[0] = tm_x;
     p.tmA[1] = tm_x;
-    p.tmB = h->tm_ws13;
+    const int bn = pick_bn_for(T, 2 * c.hs, h->sms, 128);
+    p.tmB = h->tm_ws13[bn_index(bn)];
     p.nseg = 1;
     p.seg[0] = {0, 0, 0, c.d / 64};
     p.M = T;
-    p.n_tiles = 2 * c.hs / h->bn_s1;
+    p.n_tiles = 2 * c.hs / bn;
     p.out = h->a_s;
     p.ldo = c.hs;
     p.row_scale = h->r;
-    CK(launch_tc(p, EPI_SWIGLU, h->bn_s1, std::min(mt * p.n_tiles, h->sms), st));
+    CK(launch_tc(p, EPI_SWIGLU, bn, std::min(mt * p.n_tiles, h->sms), st));
   }
   // routed experts, grouped over the permuted rows
+  mark(h, ST_EXPERT1, st);
   {
     TcParams p = tc_base(h);
     p.tmA[0] = h->tm_aperm;
@@ -382,6 +515,7 @@ int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, 
     p.ldo = c.h;
     CK(launch_tc(p, EPI_SWIGLU, h->bn_e1, h->sms, st));
   }
+  mark(h, ST_EXPERT2, st);
   {
     TcParams p = tc_base(h);
     p.tmA[0] = h->tm_act;
@@ -399,24 +533,28 @@ int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, 
     p.ldo = c.l;
     CK(launch_tc(p, EPI_BF16, h->bn_e2, h->sms, st));
   }
+  mark(h, ST_COMBINE, st);
   combine_kernel<bf16><<<(T + 7) / 8, 256, 0, st>>>((const bf16*)h->o, h->gates, h->inv, T, c.k, c.l,
                                                     (bf16*)h->z);
   CK(cudaGetLastError());
   // y = [z | a_s] [W_up | Ws2]^T
+  mark(h, ST_UP, st);
   {
     TcParams p = tc_base(h);
     p.tmA[0] = h->tm_z;
     p.tmA[1] = c.hs ? h->tm_as : h->tm_z;
-    p.tmB = h->tm_wy;
+    const int bn = pick_bn_for(T, c.d, h->sms, 64);
+    p.tmB = h->tm_wy[bn_index(bn)];
     p.nseg = c.hs ? 2 : 1;
     p.seg[0] = {0, 0, 0, c.l / 64};
     p.seg[1] = {1, 0, c.l, c.hs / 64};
     p.M = T;
-    p.n_tiles = c.d / h->bn_y;
+    p.n_tiles = c.d / bn;
     p.out = y;
     p.ldo = c.d;
-    CK(launch_tc(p, EPI_BF16, h->bn_y, std::min(mt * p.n_tiles, h->sms), st));
+    CK(launch_tc(p, EPI_BF16, bn, std::min(mt * p.n_tiles, h->sms), st));
   }
+  h->launches += 4 + (c.hs ? 2 : 1) + 2;
   return LMOE_OK;
 }
 
@@ -424,11 +562,13 @@ int forward_f32(lmoe_handle* h, const void* xv, void* yv, int T, uint32_t flags,
   const lmoe_config& c = h->cfg;
   const float* x = (const float*)xv;
   const int mt = (T + 127) / 128;
+  mark(h, ST_RMS, st);
   rms_kernel<float><<<(T + 7) / 8, 256, 0, st>>>(x, T, c.d, c.rms_eps, h->r);
   CK(cudaGetLastError());
   SimtParams b;
   memset(&b, 0, sizeof(b));
   b.status = h->status;
+  mark(h, ST_DOWN, st);
   {  // h = r * (x Wdown'^T)
     SimtParams p = b;
     p.A0 = x; p.lda0 = c.d; p.K0 = c.d; p.a_rows = T;
@@ -437,6 +577,7 @@ int forward_f32(lmoe_handle* h, const void* xv, void* yv, int T, uint32_t flags,
     p.out = (float*)h->hx; p.ldo = c.l; p.row_scale = h->r;
     CK(launch_simt<SE_STORE>(p, mt, st));
   }
+  mark(h, ST_ROUTER, st);
   {  // s = sigmoid(h Wr^T + c)
     SimtParams p = b;
     p.A0 = (const float*)h->hx; p.lda0 = c.l; p.K0 = c.l; p.a_rows = T;
@@ -447,6 +588,7 @@ int forward_f32(lmoe_handle* h, const void* xv, void* yv, int T, uint32_t flags,
   }
   int rc = route_from_scores(h, T, flags, st);
   if (rc) return rc;
+  mark(h, ST_SHARED, st);
   if (c.hs) {  // a_s = silu(r x Ws1'^T) * (r x Ws3'^T)
     SimtParams p = b;
     p.A0 = x; p.lda0 = c.d; p.K0 = c.d; p.a_rows = T;
@@ -456,6 +598,7 @@ int forward_f32(lmoe_handle* h, const void* xv, void* yv, int T, uint32_t flags,
     CK(launch_simt<SE_SWIGLU>(p, mt, st));
   }
   const int gm = (T * c.k + 127) / 128 + c.E;
+  mark(h, ST_EXPERT1, st);
   {  // act = silu(A W1_e^T) * (A W3_e^T)
     SimtParams p = b;
     p.A0 = (const float*)h->a_perm; p.lda0 = c.l; p.K0 = c.l; p.a_rows = T * c.k;
@@ -466,6 +609,7 @@ int forward_f32(lmoe_handle* h, const void* xv, void* yv, int T, uint32_t flags,
     p.out = (float*)h->act; p.ldo = c.h;
     CK(launch_simt<SE_SWIGLU>(p, gm, st));
   }
+  mark(h, ST_EXPERT2, st);
   {  // o = act W2_e^T
     SimtParams p = b;
     p.A0 = (const float*)h->act; p.lda0 = c.h; p.K0 = c.h; p.a_rows = T * c.k;
@@ -476,9 +620,11 @@ int forward_f32(lmoe_handle* h, const void* xv, void* yv, int T, uint32_t flags,
     p.out = (float*)h->o; p.ldo = c.l;
     CK(launch_simt<SE_STORE>(p, gm, st));
   }
+  mark(h, ST_COMBINE, st);
   combine_kernel<float><<<(T + 7) / 8, 256, 0, st>>>((const float*)h->o, h->gates, h->inv, T, c.k, c.l,
                                                      (float*)h->z);
   CK(cudaGetLastError());
+  mark(h, ST_UP, st);
   {  // y = [z | a_s] [W_up | Ws2]^T
     SimtParams p = b;
     p.A0 = (const float*)h->z; p.lda0 = c.l; p.K0 = c.l;
@@ -488,6 +634,7 @@ int forward_f32(lmoe_handle* h, const void* xv, void* yv, int T, uint32_t flags,
     p.out = (float*)yv; p.ldo = c.d;
     CK(launch_simt<SE_STORE>(p, mt, st));
   }
+  h->launches += 4 + (c.hs ? 2 : 1) + 2;
   return LMOE_OK;
 }
 
@@ -562,6 +709,49 @@ bool gain_is_unit(const lmoe_config& c, const void* g) {
   return true;
 }
 
+// Runs `body(stream)` through the handle's graph cache.  The first call with a new argument key
+// runs eagerly on the caller's stream; a repeat of the same key is captured once on the handle's
+// private stream into an executable graph, which every later repeat replays on the caller's
+// stream.  Eager whenever profiling is on or the caller's stream is itself being captured.
+template <typename F>
+int run_cached(lmoe_handle* h, GraphCache& g, const void* x, void* y, int T, uint32_t flags, float beta,
+               cudaStream_t st, F body) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (h->profiling || cudaStreamIsCapturing(st, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) {
+    return body(st);
+  }
+  if (!g.same(x, y, T, flags, beta)) g.reset(x, y, T, flags, beta);
+  if (g.exec) {
+    CK(cudaGraphLaunch(g.exec, st));
+    h->launches += g.kernels;
+    return LMOE_OK;
+  }
+  if (g.seen == 0) {
+    g.seen = 1;
+    return body(st);
+  }
+  const long long before = h->launches;
+  cudaGraph_t graph = nullptr;
+  CK(cudaStreamBeginCapture(h->cap, cudaStreamCaptureModeThreadLocal));
+  int rc = body(h->cap);
+  cudaError_t ce = cudaStreamEndCapture(h->cap, &graph);
+  if (rc != LMOE_OK || ce != cudaSuccess) {
+    if (graph) cudaGraphDestroy(graph);
+    cudaGetLastError();
+    h->launches = before;
+    return rc != LMOE_OK ? rc : LMOE_ECUDA;
+  }
+  ce = cudaGraphInstantiate(&g.exec, graph, 0);
+  cudaGraphDestroy(graph);
+  if (ce != cudaSuccess) {
+    g.exec = nullptr;
+    return LMOE_ECUDA;
+  }
+  g.kernels = h->launches - before;
+  CK(cudaGraphLaunch(g.exec, st));
+  return LMOE_OK;
+}
+
 }  // namespace
 
 // ======================================================================= C ABI
@@ -585,8 +775,7 @@ static void size_handle(lmoe_handle* h, const lmoe_config* cfg) {
   h->es = h->bf ? 2 : 4;
   h->nblk_max = (cfg->max_tokens + kTokBlock - 1) / kTokBlock;
   h->max_mtiles = (int)(((long long)cfg->max_tokens * cfg->k + kTileRows - 1) / kTileRows) + cfg->E;
-  int g = (cfg->E + 147) / 148;
-  h->hist_g = g < 1 ? 1 : (g > 12 ? 12 : g);
+  h->ld_bins = (cfg->max_tokens + 31) / 32 * 32;
 }
 
 int lmoe_workspace_bytes(const lmoe_config* cfg, size_t* bytes) {
@@ -637,6 +826,7 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, void* stream, lmo
   if (!rc && cudaMemsetAsync(h->ntok, 0, 8, st) != cudaSuccess) rc = LMOE_ECUDA;
   if (!rc && cudaMemsetAsync(h->status, 0, 4, st) != cudaSuccess) rc = LMOE_ECUDA;
   if (!rc && h->bf) rc = build_maps(h);
+  if (!rc && cudaStreamCreateWithFlags(&h->cap, cudaStreamNonBlocking) != cudaSuccess) rc = LMOE_ECUDA;
   if (rc) {
     cudaStreamSynchronize(st);
     cudaFree(h->arena);
@@ -650,6 +840,11 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, void* stream, lmo
 int lmoe_destroy(lmoe_handle* h) {
   if (!h) return LMOE_EINVAL;
   cudaDeviceSynchronize();
+  for (auto& r : h->prof)
+    for (auto& e : r.ev) cudaEventDestroy(e);
+  h->g_fwd.reset(nullptr, nullptr, -1, 0, 0.f);
+  h->g_qb.reset(nullptr, nullptr, -1, 0, 0.f);
+  if (h->cap) cudaStreamDestroy(h->cap);
   cudaFree(h->arena);
   delete h;
   return LMOE_OK;
@@ -662,7 +857,13 @@ int lmoe_forward(lmoe_handle* h, const void* x, void* y, int32_t T, uint32_t fla
   const size_t bytes = (size_t)T * h->cfg.d * h->es;
   if ((const char*)x < (const char*)y + bytes && (const char*)y < (const char*)x + bytes) return LMOE_EINVAL;
   cudaStream_t st = (cudaStream_t)stream;
-  return h->bf ? forward_bf16(h, x, y, T, flags, st) : forward_f32(h, x, y, T, flags, st);
+  h->last_T = T;
+  return run_cached(h, h->g_fwd, x, y, T, flags, 0.f, st, [&](cudaStream_t s) {
+    prof_open(h, ST_RMS, ST_UP - ST_RMS + 1);
+    int rc = h->bf ? forward_bf16(h, x, y, T, flags, s) : forward_f32(h, x, y, T, flags, s);
+    prof_close(h, s);
+    return rc;
+  });
 }
 
 int lmoe_forward_host(lmoe_handle* h, const void* x_host, void* y_host, int32_t T, uint32_t flags, void* stream) {
@@ -682,18 +883,28 @@ int lmoe_route_scores(lmoe_handle* h, const float* scores, int32_t T, uint32_t f
   if (T == 0) return LMOE_OK;
   cudaStream_t st = (cudaStream_t)stream;
   CK(cudaMemcpyAsync(h->s, scores, (size_t)T * h->cfg.E * 4, cudaMemcpyDeviceToDevice, st));
-  return route_from_scores(h, T, flags, st);
+  prof_open(h, ST_TOPK, ST_HIST - ST_TOPK + 1);
+  int rc = route_from_scores(h, T, flags, st);
+  prof_close(h, st);
+  return rc;
 }
 
 int lmoe_qb_update(lmoe_handle* h, float beta, uint32_t flags, void* stream) {
   if (!h || !(beta == beta)) return LMOE_EINVAL;
   cudaStream_t st = (cudaStream_t)stream;
-  qb_quantile_kernel<<<h->cfg.E, 256, 0, st>>>(h->hist, h->ntok, h->bias, h->cfg.E, h->cfg.k,
-                                                (flags & LMOE_QB_LITERAL) ? 1 : 0, h->u, h->status);
-  CK(cudaGetLastError());
-  qb_apply_kernel<<<1, 1024, 0, st>>>(h->bias, h->ntok, h->u, h->cfg.E, beta);
-  CK(cudaGetLastError());
-  return LMOE_OK;
+  return run_cached(h, h->g_qb, nullptr, nullptr, 0, flags, beta, st, [&](cudaStream_t s) {
+    prof_open(h, ST_QB_QUANTILE, 2);
+    mark(h, ST_QB_QUANTILE, s);
+    qb_quantile_kernel<<<h->cfg.E, 256, 0, s>>>(h->hist, h->ntok, h->bias, h->cfg.E, h->cfg.k,
+                                                 (flags & LMOE_QB_LITERAL) ? 1 : 0, h->u, h->status);
+    CK(cudaGetLastError());
+    mark(h, ST_QB_APPLY, s);
+    qb_apply_kernel<<<1, 1024, 0, s>>>(h->bias, h->ntok, h->u, h->cfg.E, beta);
+    CK(cudaGetLastError());
+    prof_close(h, s);
+    h->launches += 2;
+    return LMOE_OK;
+  });
 }
 
 int lmoe_get_routing(lmoe_handle* h, int32_t* idx, float* gates, float* scores, int32_t* counts, int32_t* offsets,
@@ -747,6 +958,39 @@ int lmoe_get_status(lmoe_handle* h, uint32_t* status) {
   CK(cudaDeviceSynchronize());
   CK(cudaMemcpy(status, h->status, 4, cudaMemcpyDeviceToHost));
   CK(cudaMemset(h->status, 0, 4));
+  return LMOE_OK;
+}
+
+int lmoe_profile_enable(lmoe_handle* h, int32_t enable) {
+  if (!h) return LMOE_EINVAL;
+  h->profiling = enable != 0;
+  return LMOE_OK;
+}
+
+int lmoe_profile_read(lmoe_handle* h, float* ms, int32_t n, int32_t* calls) {
+  if (!h || !ms || n < ST_COUNT) return LMOE_EINVAL;
+  CK(cudaDeviceSynchronize());
+  for (int i = 0; i < ST_COUNT; ++i) ms[i] = 0.f;
+  int forwards = 0;
+  for (int r = 0; r < h->prof_used; ++r) {
+    const ProfRecord& pr = h->prof[r];
+    if (pr.first == ST_RMS) ++forwards;
+    for (int i = 0; i < pr.n; ++i) {
+      float t = 0.f;
+      if (cudaEventElapsedTime(&t, pr.ev[i], pr.ev[i + 1]) == cudaSuccess) ms[pr.first + i] += t;
+    }
+  }
+  if (calls) *calls = forwards;
+  h->prof_used = 0;
+  cudaGetLastError();
+  return LMOE_OK;
+}
+
+const char* lmoe_stage_name(int32_t i) { return (i >= 0 && i < ST_COUNT) ? kStageNames[i] : nullptr; }
+
+int lmoe_launch_count(lmoe_handle* h, int64_t* n) {
+  if (!h || !n) return LMOE_EINVAL;
+  *n = h->launches;
   return LMOE_OK;
 }
 

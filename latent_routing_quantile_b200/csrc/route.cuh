@@ -9,7 +9,7 @@
 
 namespace lmoe {
 
-constexpr int kTokBlock = 128;     // tokens per routing block: a rank bitmask is 4 words
+constexpr int kTokBlock = 32;      // tokens per routing block: one rank-mask word per expert
 constexpr int kTileRows = 128;     // rows per grouped-GEMM M-tile
 constexpr unsigned kFull = 0xffffffffu;
 
@@ -38,22 +38,36 @@ __global__ void __launch_bounds__(256) rms_kernel(const T* __restrict__ x, int n
 }
 
 // --------------------------------------------------------------------------- top-k
-// One warp per token, 16 tokens per warp, kTokBlock tokens per block.  k rounds of a warp
-// arg-max of u = s + b over the experts not yet taken; order: larger u, then lower index.
-// Gates are the chosen unbiased s divided by their sum.  Each choice sets the token's bit in
-// the expert's shared bitmask; a token's rank inside the block for expert e is the number of
-// set bits below its own, which gives a stable (token-ascending) order without atomics on the
-// order.  Per-block counts go to blkcnt and are summed into counts.
+// Order-preserving map of a float to uint32 (larger float -> larger key); 0 is kept free to mark
+// taken or absent experts and 1 for a NaN score, which ranks below every number.
+__device__ __forceinline__ uint32_t order_key(float f) {
+  if (f != f) return 1u;
+  if (f == 0.f) f = 0.f;  // -0 and +0 compare equal, so give them one key
+  const uint32_t b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// One warp per token, 4 tokens per warp, kTokBlock = 32 tokens per block.  Lane L holds the
+// scores of experts L, L+32, ...  k rounds of: local best (larger key, then lower index), warp
+// max of the keys (redux), warp min of the expert index among the lanes holding that key (redux),
+// broadcast of its unbiased score.  This is top-k of u = s + b in fp32 with ties to the lower
+// expert index.  Gates are the chosen s over their sum.  Each choice sets the token's bit in the
+// expert's shared mask; the token's rank inside the block for that expert is the number of set
+// bits below it, so the permutation is stable (token ascending) with no order-dependent atomics.
+// With bins != null it also stores each score's histogram bin, min(floor(s * 4096), 4095) as
+// uint16, expert-major (bins[e * ld_bins + t]) for the histogram kernel.
 template <int NJ>
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ s, const float* __restrict__ bias,
                                                    int ntok, int E, int k, int* __restrict__ idx,
                                                    float* __restrict__ gates, int* __restrict__ rank,
                                                    int* __restrict__ blkcnt, int* __restrict__ counts,
-                                                   uint32_t* status) {
-  extern __shared__ uint32_t mask[];  // [E][4]
+                                                   uint16_t* __restrict__ bins, int ld_bins, uint32_t* status) {
+  extern __shared__ uint32_t smem_topk[];
+  uint32_t* mask = smem_topk;                                          // [E]
+  uint16_t* sbins = reinterpret_cast<uint16_t*>(smem_topk + E);        // [E][32]
   const int blk = blockIdx.x, t0 = blk * kTokBlock;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int i = threadIdx.x; i < E * 4; i += blockDim.x) mask[i] = 0;
+  for (int i = threadIdx.x; i < E; i += blockDim.x) mask[i] = 0;
   float bj[NJ];
 #pragma unroll
   for (int j = 0; j < NJ; ++j) {
@@ -62,90 +76,88 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ s, 
   }
   __syncthreads();
 
+  constexpr int TPW = kTokBlock / 8;  // tokens per warp
+  int sel_q[TPW];
   bool nan = false;
-  for (int q = 0; q < kTokBlock / 8; ++q) {
-    const int t = t0 + warp * (kTokBlock / 8) + q;
+#pragma unroll
+  for (int q = 0; q < TPW; ++q) {
+    sel_q[q] = -1;
+    const int tl = warp * TPW + q, t = t0 + tl;
     if (t >= ntok) break;
-    float u[NJ], sv[NJ];
-    uint32_t taken = 0;
+    uint32_t key[NJ];
+    float sv[NJ];
 #pragma unroll
     for (int j = 0; j < NJ; ++j) {
       const int e = j * 32 + lane;
       if (e < E) {
         const float v = s[(size_t)t * E + e];
-        if (v != v) {
-          nan = true;
-          u[j] = -INFINITY;
-          sv[j] = 0.f;
-        } else {
-          u[j] = v + bj[j];
-          sv[j] = v;
-        }
+        nan |= (v != v);
+        sv[j] = (v == v) ? v : 0.f;
+        key[j] = order_key(v + bj[j]);
+        if (bins) sbins[e * kTokBlock + tl] = (uint16_t)(v >= 0.f ? min((int)(v * (float)LMOE_NBINS), LMOE_NBINS - 1) : 0);
       } else {
-        u[j] = -INFINITY;
         sv[j] = 0.f;
-        taken |= 1u << j;
+        key[j] = 0u;
       }
     }
     int my_sel = -1;
     float my_s = 0.f;
     for (int i = 0; i < k; ++i) {
-      float bu = 0.f, bs = 0.f;
-      int be = INT_MAX;
+      uint32_t bk = 0u;
+      uint32_t be = 0xffffffffu;
+      float bs = 0.f;
 #pragma unroll
       for (int j = 0; j < NJ; ++j) {
-        if (!((taken >> j) & 1u) && (be == INT_MAX || u[j] > bu)) {
-          bu = u[j];
-          be = j * 32 + lane;
+        if (key[j] > bk) {
+          bk = key[j];
+          be = (uint32_t)(j * 32 + lane);
           bs = sv[j];
         }
       }
+      const uint32_t wmax = __reduce_max_sync(kFull, bk);
+      const uint32_t emin = __reduce_min_sync(kFull, bk == wmax ? be : 0xffffffffu);
+      const float es = __shfl_sync(kFull, bs, (int)(emin & 31u));
 #pragma unroll
-      for (int off = 16; off; off >>= 1) {
-        const float ou = __shfl_xor_sync(kFull, bu, off);
-        const int oe = __shfl_xor_sync(kFull, be, off);
-        const float os = __shfl_xor_sync(kFull, bs, off);
-        if (oe != INT_MAX && (be == INT_MAX || ou > bu || (ou == bu && oe < be))) {
-          bu = ou;
-          be = oe;
-          bs = os;
-        }
-      }
-      if ((be & 31) == lane) taken |= 1u << (be >> 5);
+      for (int j = 0; j < NJ; ++j)
+        if ((uint32_t)(j * 32 + lane) == emin) key[j] = 0u;
       if (lane == i) {
-        my_sel = be;
-        my_s = bs;
+        my_sel = (int)emin;
+        my_s = es;
       }
     }
     float ssum = lane < k ? my_s : 0.f;
 #pragma unroll
     for (int off = 16; off; off >>= 1) ssum += __shfl_xor_sync(kFull, ssum, off);
     if (lane < k) {
+      if (my_sel < 0 || my_sel >= E) {
+        set_status(status, LMOE_STATUS_BAD_INDEX);
+        my_sel = 0;
+      }
       idx[(size_t)t * k + lane] = my_sel;
       gates[(size_t)t * k + lane] = my_s / ssum;
-      const int tl = t - t0;
-      atomicOr(&mask[my_sel * 4 + (tl >> 5)], 1u << (tl & 31));
+      atomicOr(&mask[my_sel], 1u << tl);
     }
+    sel_q[q] = my_sel;
   }
   if (nan) set_status(status, LMOE_STATUS_NAN_SCORE);
   __syncthreads();
 
-  for (int q = 0; q < kTokBlock / 8; ++q) {
-    const int t = t0 + warp * (kTokBlock / 8) + q;
+#pragma unroll
+  for (int q = 0; q < TPW; ++q) {
+    const int tl = warp * TPW + q, t = t0 + tl;
     if (t >= ntok) break;
-    if (lane < k) {
-      const int e = idx[(size_t)t * k + lane];
-      const int tl = t - t0, w = tl >> 5;
-      int r = __popc(mask[e * 4 + w] & ((1u << (tl & 31)) - 1u));
-      for (int ww = 0; ww < w; ++ww) r += __popc(mask[e * 4 + ww]);
-      rank[(size_t)t * k + lane] = r;
-    }
+    if (lane < k) rank[(size_t)t * k + lane] = __popc(mask[sel_q[q]] & ((1u << tl) - 1u));
   }
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    const int c = __popc(mask[e * 4]) + __popc(mask[e * 4 + 1]) + __popc(mask[e * 4 + 2]) +
-                  __popc(mask[e * 4 + 3]);
+    const int c = __popc(mask[e]);
     blkcnt[(size_t)blk * E + e] = c;
     if (c) atomicAdd(&counts[e], c);
+  }
+  if (bins) {
+    // expert-major store: one warp writes 32 tokens (64 bytes) of one expert per step
+    const int nt = min(kTokBlock, ntok - t0);
+    for (int e = warp; e < E; e += 8)
+      if (lane < nt) bins[(size_t)e * ld_bins + t0 + lane] = sbins[e * kTokBlock + lane];
   }
 }
 
@@ -254,29 +266,35 @@ __global__ void __launch_bounds__(256) gather_kernel(const T* __restrict__ src, 
 }
 
 // --------------------------------------------------------------------------- QB histogram
-// Each block owns G experts' 4096 bins in shared memory, reads their columns of s over all
-// tokens, then adds its bins into the global histogram (no other block touches those rows).
-// bin = min(floor(s * 4096), 4095); a NaN score counts in bin 0 (and was flagged by top-k).
-__global__ void __launch_bounds__(1024) hist_kernel(const float* __restrict__ s, int ntok, int E, int G,
-                                                    uint32_t* __restrict__ hist, long long* ntok_acc) {
-  extern __shared__ uint32_t sh[];  // [G][4096]
-  const int e0 = blockIdx.x * G, g_count = min(G, E - e0);
-  for (int i = threadIdx.x; i < g_count * LMOE_NBINS; i += blockDim.x) sh[i] = 0;
+// Block per expert: counts that expert's uint16 bins (written expert-major by the top-k kernel)
+// in a shared 4096-bin histogram, then adds it into the expert's global row, which no other
+// block touches.  Block 0 adds T to the recorded token count.
+__global__ void __launch_bounds__(512) hist_kernel(const uint16_t* __restrict__ bins, int ld_bins, int ntok,
+                                                   uint32_t* __restrict__ hist, long long* ntok_acc) {
+  __shared__ uint32_t sh[LMOE_NBINS];
+  const int e = blockIdx.x;
+  for (int i = threadIdx.x; i < LMOE_NBINS; i += blockDim.x) sh[i] = 0;
   __syncthreads();
-  const long long n = (long long)ntok * g_count;
-  for (long long p = threadIdx.x; p < n; p += blockDim.x) {
-    const int t = (int)(p / g_count), g = (int)(p - (long long)t * g_count);
-    const float v = s[(size_t)t * E + e0 + g];
-    const int bin = v >= 0.f ? min((int)(v * (float)LMOE_NBINS), LMOE_NBINS - 1) : 0;
-    atomicAdd(&sh[g * LMOE_NBINS + bin], 1u);
+  const uint16_t* row = bins + (size_t)e * ld_bins;
+  const int nvec = ntok / 8;  // ld_bins is a multiple of 32, so rows are 16-byte aligned
+  const uint4* row4 = reinterpret_cast<const uint4*>(row);
+  for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+    const uint4 q = row4[v];
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      atomicAdd(&sh[w[j] & 0xFFFFu], 1u);
+      atomicAdd(&sh[w[j] >> 16], 1u);
+    }
   }
+  for (int t = nvec * 8 + threadIdx.x; t < ntok; t += blockDim.x) atomicAdd(&sh[row[t]], 1u);
   __syncthreads();
-  uint32_t* hrow = hist + (size_t)e0 * LMOE_NBINS;
-  for (int i = threadIdx.x; i < g_count * LMOE_NBINS; i += blockDim.x) {
+  uint32_t* hrow = hist + (size_t)e * LMOE_NBINS;
+  for (int i = threadIdx.x; i < LMOE_NBINS; i += blockDim.x) {
     const uint32_t v = sh[i];
     if (v) hrow[i] += v;
   }
-  if (blockIdx.x == 0 && threadIdx.x == 0) *ntok_acc += ntok;
+  if (e == 0 && threadIdx.x == 0) *ntok_acc += ntok;
 }
 
 // --------------------------------------------------------------------------- combine

@@ -1,9 +1,11 @@
 // Persistent tcgen05 GEMM for sm_100a: C[M, N] = A[M, K] * B[N, K]^T, A and B bf16 K-major,
 // fp32 accumulation in tensor memory (TMEM), with the layer's epilogues fused.
 //
-// CTA = 6 warps: warp 0 issues TMA loads into a STAGES-deep shared-memory ring, warp 1 issues
-// tcgen05.mma (one thread) into one of two TMEM accumulators, warps 2-5 drain the other
-// accumulator (tcgen05.ld) through the epilogue while the next tile is multiplied.  Tiles are
+// CTA = 10 warps: warp 0 issues TMA loads into a STAGES-deep shared-memory ring, warp 1 issues
+// tcgen05.mma (one thread) into one of two TMEM accumulators, warps 2-9 drain the other
+// accumulator (tcgen05.ld) through the epilogue while the next tile is multiplied.  Two
+// epilogue warps share each TMEM lane quarter and split its columns, so the element-wise
+// epilogue math keeps pace with the tensor core.  Tiles are
 // 128 x BN, K steps of 64 (one 128-byte swizzle atom).  The grid is at most one CTA per SM and
 // walks the tile list with a stride of gridDim.x.
 //
@@ -93,8 +95,11 @@ __device__ __forceinline__ int tc_num_tiles(const TcParams& p) {
   return mt * p.n_tiles;
 }
 
+constexpr int kEpiWarps = 8;
+constexpr int kTcThreads = 64 + 32 * kEpiWarps;
+
 template <int BN, int EPI>
-__global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__ TcParams p) {
+__global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_constant__ TcParams p) {
   using C = TcCfg<BN>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -116,7 +121,7 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 4);
+      mbar_init(&tempty[i], kEpiWarps);
     }
     mbar_init(drain, 1);
     *abort = 0;
@@ -167,13 +172,8 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
       }
       if (!ok) {
         // let every load this thread issued land before the CTA's shared memory is released
-        for (int i = 0; i < S; ++i) {
-          if (!((armed >> i) & 1u)) continue;
-          unsigned long long t0 = global_timer_ns();
-          while (!mbar_try_wait(&full[i], (armed_parity >> i) & 1u) &&
-                 global_timer_ns() - t0 < kWaitLimitNs) {
-          }
-        }
+        for (int i = 0; i < S; ++i)
+          if ((armed >> i) & 1u) mbar_drain(&full[i], (armed_parity >> i) & 1u);
       }
     }
   } else if (warp == 1) {
@@ -221,14 +221,13 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
       if (!ok) {
         // wait (bounded) for the MMAs already issued before TMEM is released
         tc_commit(drain);
-        unsigned long long t0 = global_timer_ns();
-        while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
-        }
+        mbar_drain(drain, 0);
       }
     }
   } else {
-    // ---------------- epilogue warps 2..5: TMEM lane quarter (warp % 4)
+    // ---------------- epilogue warps 2..9: TMEM lane quarter (warp % 4), column half (warp-2)/4
     const int wq = warp & 3;
+    const int half_id = (warp - 2) >> 2;
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int acc = it & 1;
@@ -244,49 +243,45 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
       const float rs = (p.row_scale != nullptr && valid) ? p.row_scale[row] : 1.0f;
 
       if constexpr (EPI == EPI_SWIGLU) {
+        // item i = (group g = i / 2, part = i % 2): gate columns g*128 + part*32 .. +31, linear
+        // columns 64 further; items alternate between the two warps of a lane quarter
 #pragma unroll 1
-        for (int g = 0; g < BN / 128; ++g) {
-#pragma unroll 1
-          for (int half = 0; half < 2; ++half) {
-            uint32_t gv[32], uv[32];
-            tmem_ld32(tbase + g * 128 + half * 32, gv);
-            tmem_ld32(tbase + g * 128 + 64 + half * 32, uv);
-            tc_wait_ld();
-            if (valid) {
-              bf16* o = reinterpret_cast<bf16*>(p.out) + (size_t)row * p.ldo + (ti.n0 >> 1) +
-                        g * 64 + half * 32;
-              uint32_t pk[16];
+        for (int item = half_id; item < BN / 64; item += 2) {
+          const int g = item >> 1, part = item & 1;
+          uint32_t gv[32], uv[32];
+          tmem_ld32(tbase + g * 128 + part * 32, gv);
+          tmem_ld32(tbase + g * 128 + 64 + part * 32, uv);
+          tc_wait_ld();
+          if (valid) {
+            bf16* o = reinterpret_cast<bf16*>(p.out) + (size_t)row * p.ldo + (ti.n0 >> 1) + g * 64 + part * 32;
+            uint32_t pk[16];
 #pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                float g0 = __uint_as_float(gv[2 * j]) * rs, g1 = __uint_as_float(gv[2 * j + 1]) * rs;
-                float u0 = __uint_as_float(uv[2 * j]) * rs, u1 = __uint_as_float(uv[2 * j + 1]) * rs;
-                pk[j] = pack_bf16x2(siluf(g0) * u0, siluf(g1) * u1);
-              }
-              uint4* o4 = reinterpret_cast<uint4*>(o);
-#pragma unroll
-              for (int j = 0; j < 4; ++j)
-                o4[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+            for (int j = 0; j < 16; ++j) {
+              const float g0 = __uint_as_float(gv[2 * j]) * rs, g1 = __uint_as_float(gv[2 * j + 1]) * rs;
+              const float u0 = __uint_as_float(uv[2 * j]) * rs, u1 = __uint_as_float(uv[2 * j + 1]) * rs;
+              pk[j] = pack_bf16x2(silu_fast(g0) * u0, silu_fast(g1) * u1);
             }
+            uint4* o4 = reinterpret_cast<uint4*>(o);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) o4[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
           }
         }
       } else {
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = half_id; c < BN / 32; c += 2) {
           uint32_t v[32];
           tmem_ld32(tbase + c * 32, v);
           tc_wait_ld();
           if (!valid) continue;
           const int col = ti.n0 + c * 32;
           if constexpr (EPI == EPI_F32) {
-            float4* o4 = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) +
-                                                   (size_t)row * p.ldo + col);
+            float4* o4 = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + (size_t)row * p.ldo + col);
 #pragma unroll
             for (int j = 0; j < 8; ++j)
               o4[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
                                   __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
           } else if constexpr (EPI == EPI_BF16) {
-            uint4* o4 = reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(p.out) +
-                                                 (size_t)row * p.ldo + col);
+            uint4* o4 = reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(p.out) + (size_t)row * p.ldo + col);
 #pragma unroll
             for (int j = 0; j < 4; ++j)
               o4[j] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * j]), __uint_as_float(v[8 * j + 1])),
@@ -299,11 +294,11 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
             uint32_t hi[16], mid[16], lo[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-              float a0 = __uint_as_float(v[2 * j]) * rs, a1 = __uint_as_float(v[2 * j + 1]) * rs;
-              bf16 h0 = __float2bfloat16_rn(a0), h1 = __float2bfloat16_rn(a1);
-              float r0 = a0 - __bfloat162float(h0), r1 = a1 - __bfloat162float(h1);
-              bf16 m0 = __float2bfloat16_rn(r0), m1 = __float2bfloat16_rn(r1);
-              float q0 = r0 - __bfloat162float(m0), q1 = r1 - __bfloat162float(m1);
+              const float a0 = __uint_as_float(v[2 * j]) * rs, a1 = __uint_as_float(v[2 * j + 1]) * rs;
+              const bf16 h0 = __float2bfloat16_rn(a0), h1 = __float2bfloat16_rn(a1);
+              const float r0 = a0 - __bfloat162float(h0), r1 = a1 - __bfloat162float(h1);
+              const bf16 m0 = __float2bfloat16_rn(r0), m1 = __float2bfloat16_rn(r1);
+              const float q0 = r0 - __bfloat162float(m0), q1 = r1 - __bfloat162float(m1);
               __nv_bfloat162 ph = __halves2bfloat162(h0, h1), pm = __halves2bfloat162(m0, m1);
               hi[j] = *reinterpret_cast<uint32_t*>(&ph);
               mid[j] = *reinterpret_cast<uint32_t*>(&pm);
@@ -319,18 +314,19 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
               ol[j] = make_uint4(lo[4 * j], lo[4 * j + 1], lo[4 * j + 2], lo[4 * j + 3]);
             }
           } else if constexpr (EPI == EPI_ROUTER) {
-            float* o = reinterpret_cast<float*>(p.out) + (size_t)row * p.ldo + col;
-            float4* o4 = reinterpret_cast<float4*>(o);
+            float4* o4 = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + (size_t)row * p.ldo + col);
+            const float4* cb4 = reinterpret_cast<const float4*>(p.col_bias + col);
             bool nan = false;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-              float s4[4];
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                s4[q] = sigmoidf_acc(__uint_as_float(v[4 * j + q]) + p.col_bias[col + 4 * j + q]);
-                nan |= (s4[q] != s4[q]);
-              }
-              o4[j] = make_float4(s4[0], s4[1], s4[2], s4[3]);
+              const float4 cb = cb4[j];
+              float4 o;
+              o.x = sigmoidf_acc(__uint_as_float(v[4 * j]) + cb.x);
+              o.y = sigmoidf_acc(__uint_as_float(v[4 * j + 1]) + cb.y);
+              o.z = sigmoidf_acc(__uint_as_float(v[4 * j + 2]) + cb.z);
+              o.w = sigmoidf_acc(__uint_as_float(v[4 * j + 3]) + cb.w);
+              nan |= (o.x != o.x) | (o.y != o.y) | (o.z != o.z) | (o.w != o.w);
+              o4[j] = o;
             }
             if (nan) set_status(p.status, LMOE_STATUS_NAN_SCORE);
           }

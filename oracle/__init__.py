@@ -114,6 +114,16 @@ def topk_gap(s: np.ndarray, b: np.ndarray, k: int) -> np.ndarray:
     return u[:, k - 1] - u[:, k]
 
 
+def topk_order_gap(s: np.ndarray, b: np.ndarray, k: int) -> np.ndarray:
+    """Per token, the smallest margin between consecutive biased scores among the top k+1
+    (the top k when k == E): how close the rank order of the chosen experts is to a tie."""
+    E = s.shape[1]
+    u = np.sort(s + b[None, :], axis=1)[:, ::-1][:, :min(k + 1, E)]
+    if u.shape[1] < 2:
+        return np.full(s.shape[0], np.inf)
+    return np.min(u[:, :-1] - u[:, 1:], axis=1)
+
+
 def gate_weights(s: np.ndarray, idx: np.ndarray) -> np.ndarray:
     """g_i = s_{sel_i} / sum_j s_{sel_j}: unbiased scores of the chosen experts, renormalised.
 
@@ -185,7 +195,7 @@ def layer_forward(x, w: dict, b, k: int, eps: float = 1e-6) -> dict:
     if "ws1" in w:
         y = y + shared_expert(x_hat, f64(w["ws1"]), f64(w["ws3"]), f64(w["ws2"]))
     return dict(r=rms_reciprocal(x, eps), h=h, s=s, idx=idx, gates=g, gap=topk_gap(s, b, k),
-                o=o, z=z, y=y)
+                order_gap=topk_order_gap(s, b, k), o=o, z=z, y=y)
 
 
 def layer_routing(x, w: dict, b, k: int, eps: float = 1e-6) -> dict:
@@ -196,7 +206,8 @@ def layer_routing(x, w: dict, b, k: int, eps: float = 1e-6) -> dict:
     h = latent_down(x_hat, f64(w["w_down"]))
     s = router_scores(h, f64(w["w_router"]), f64(w["router_bias"]))
     idx = biased_topk(s, b, k)
-    return dict(h=h, s=s, idx=idx, gates=gate_weights(s, idx), gap=topk_gap(s, b, k))
+    return dict(h=h, s=s, idx=idx, gates=gate_weights(s, idx), gap=topk_gap(s, b, k),
+                order_gap=topk_order_gap(s, b, k))
 
 
 # --------------------------------------------------------------------------

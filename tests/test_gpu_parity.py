@@ -37,10 +37,21 @@ def normwise(y, ref):
     return float(np.max(np.abs(y - ref)) / np.max(np.abs(ref)))
 
 
-def check_routing(gpu_idx, ora_idx, gap):
-    """Returns the mismatch fraction; asserts every mismatch is a near-tie and the fraction < 1e-4."""
-    mism = (gpu_idx != ora_idx).any(1)
-    assert not (mism & ~(gap < NEAR_TIE)).any(), "a token that is not a near-tie was routed differently"
+def routing_mismatches(gpu_idx, ora, slack=0.0):
+    """Tokens whose chosen set differs from the oracle's, and tokens with the same set in another
+    rank order.  Asserts each set difference sits on a near-tie at the k / k+1 boundary and each
+    order difference on a near-tie among the top k+1; returns (set_diff, order_diff) masks."""
+    set_diff = (np.sort(gpu_idx, 1) != np.sort(ora["idx"], 1)).any(1)
+    order_diff = (gpu_idx != ora["idx"]).any(1) & ~set_diff
+    assert not (set_diff & ~(ora["gap"] < NEAR_TIE + slack)).any(), "a chosen set differs off a near-tie"
+    assert not (order_diff & ~(ora["order_gap"] < NEAR_TIE + slack)).any(), "a rank order differs off a near-tie"
+    return set_diff, order_diff
+
+
+def check_routing(gpu_idx, ora):
+    """Every mismatch is a near-tie, and mismatched tokens are under 1e-4 of all tokens."""
+    set_diff, order_diff = routing_mismatches(gpu_idx, ora)
+    mism = set_diff | order_diff
     frac = float(mism.mean())
     assert mism.sum() <= int(1e-4 * len(mism)), f"mismatch fraction {frac}"
     return frac
@@ -163,7 +174,7 @@ def run_layer_check(shape, w, x, b=None, sample=None, record=True):
     s_gpu = r["scores"].cpu().numpy()
     s_err = float(np.max(np.abs(s_gpu - ro["s"])))
     assert s_err < 2e-6, f"router scores off by {s_err}"
-    frac = check_routing(r["idx"].cpu().numpy(), ro["idx"], ro["gap"])
+    frac = check_routing(r["idx"].cpu().numpy(), ro)
     check_permutation(r, T, k, E)
     rows = np.arange(T) if sample is None else sample
     xs = x[torch.from_numpy(rows)]
@@ -211,6 +222,13 @@ def test_forward_host_and_determinism():
     layer = make_layer(shape, w)
     y1 = layer.forward(x.cuda())
     y2 = layer.forward(x.cuda())
+    # repeated calls with the same buffers: eager, then captured, then replayed as a CUDA graph
+    xd, yd = x.cuda(), torch.empty_like(y1)
+    for _ in range(4):
+        yd.zero_()
+        layer.forward(xd, yd)
+        torch.cuda.synchronize()
+        assert torch.equal(yd, y1)
     xh = x.pin_memory()
     yh = torch.empty_like(xh).pin_memory()
     layer.forward_host(xh, yh)
@@ -235,13 +253,13 @@ def test_mini_replica_full_size():
 
 
 def test_qb_skewed_router_run():
-    """50 forward + QB steps on the skewed router, GPU and oracle each following their own bias.
+    """50 forward + QB-update steps on the skewed router, with the bias teacher-forced.
 
-    The two bias trajectories can drift apart by at most the histogram resolution: each side's
-    quantile estimate lies within one bin (1/4096) of the exact quantile of its own scores, and
-    the scores agree to ~1e-6, so |b_gpu - b_oracle| stays below 2/4096 (each update contracts
-    the earlier difference by 1 - beta).  A token may then route differently only if its oracle
-    margin is below 1e-5 plus twice the measured bias difference.
+    Each step starts both sides from the same fp32 bias (the oracle's, set into the layer), so
+    routing is compared with identical state at every step.  The GPU's own update of that bias
+    from its histogram is compared with the oracle's update from the oracle's histogram: they
+    differ only where a score sits on a bin edge, by at most beta * 2/4096.  The load ratio is
+    tracked from the GPU counts and must fall from >= 3.5 to near the demo's 1.5.
     """
     shape = datagen.WORKLOADS["qb_skewed"]
     a = json.load(open(os.path.join(GOLDEN, "qb_skew_offset.json")))["a"]
@@ -249,32 +267,31 @@ def test_qb_skewed_router_run():
     c[0] = a
     w = datagen.layer_weights(shape, router_offsets=c)
     layer = make_layer(shape, w)
-    b_ora = np.zeros(shape.E)
-    ratios, qerr, berr, mism = [], [], [], []
+    b = np.zeros(shape.E, dtype=np.float32)
+    ratios, qerr, berr, nmism = [], [], [], 0
     for step in range(shape.steps):
-        db = float(np.max(np.abs(layer.bias().cpu().numpy() - b_ora)))
-        berr.append(db)
-        assert db <= 2 / 4096, (step, db)
+        layer.set_bias(torch.from_numpy(b).cuda())
         x = datagen.tokens(shape, seed=shape.seed + step)
         layer.forward(x.cuda(), record_stats=True)
         r = layer.routing()
-        torch.cuda.synchronize()
-        ro = oracle.layer_routing(x, w, b_ora, shape.k, shape.rms_eps)
-        diff = (r["idx"].cpu().numpy() != ro["idx"]).any(1)
-        assert not (diff & ~(ro["gap"] < NEAR_TIE + 2 * db)).any(), (step, db)
-        mism.append(float(diff.mean()))
-        cnt = r["counts"].cpu().numpy()
-        ratios.append(oracle.load_ratio(cnt))
+        layer.qb_update(shape.beta)
+        b_gpu = layer.bias().cpu().numpy()
+        ro = oracle.layer_routing(x, w, b.astype(np.float64), shape.k, shape.rms_eps)
+        set_diff, order_diff = routing_mismatches(r["idx"].cpu().numpy(), ro)
+        nmism += int((set_diff | order_diff).sum())
+        ratios.append(oracle.load_ratio(r["counts"].cpu().numpy()))
         hist_o = oracle.score_histogram(ro["s"])
         m = oracle.quantile_rank(shape.T, shape.k, shape.E)
         qerr.append(max(abs(oracle.histogram_quantile(hist_o[e], m) - oracle.exact_quantile(ro["s"][:, e], m))
                         for e in range(shape.E)))
-        layer.qb_update(shape.beta)
-        b_ora = oracle.qb_update(b_ora, hist_o, shape.T, shape.k, shape.beta)
+        b_new = oracle.qb_update(b.astype(np.float64), hist_o, shape.T, shape.k, shape.beta)
+        berr.append(float(np.max(np.abs(b_gpu - b_new))))
+        b = b_new.astype(np.float32)
+    frac = nmism / (shape.T * shape.steps)
     print("qb_skewed", json.dumps(dict(ratio_first=ratios[0], ratio_last=ratios[-1], ratios=ratios,
-                                       max_q_err=max(qerr), max_bias_diff=max(berr),
-                                       max_mismatch_frac=max(mism), mean_mismatch_frac=float(np.mean(mism)))))
-    assert mism[0] <= 1e-4  # same bias (zero) on both sides at step 0
+                                       max_q_err=max(qerr), max_update_diff=max(berr), mismatch_frac=frac)))
+    assert nmism <= 1e-4 * shape.T * shape.steps
+    assert max(berr) <= shape.beta * 2 / 4096 + 1e-6
     assert ratios[0] >= 3.5 and ratios[-1] < 2.0
     assert max(qerr) <= 1 / 4096 + 1e-7
     layer.close()

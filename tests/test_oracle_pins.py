@@ -68,6 +68,7 @@ def test_worked_example_closed_forms():
     assert out["idx"].tolist() == [[0, 1], [0, 3]]
     np.testing.assert_allclose(out["gates"], [[0.5, 0.5], [15 / 31, 16 / 31]], rtol=1e-14)
     np.testing.assert_allclose(out["gap"], [0.2, 0.05], rtol=1e-12)
+    np.testing.assert_allclose(out["order_gap"], [0.0, 0.05], atol=1e-15)  # token 0: exact tie
     # routed: silu(ln m) = ln m * m/(m+1); act = silu(a_e) * h[1]; o = act * [1, e+1]
     za0 = 0.5 * (ln(2) * 2 / 3 * 0.5) + 0.5 * (ln(3) * 3 / 4 * 0.5)
     zb0 = 0.5 * (ln(2) * 2 / 3 * 0.5) + 0.5 * 2 * (ln(3) * 3 / 4 * 0.5)
