@@ -148,15 +148,11 @@ def run_ours(args, rank, world, local_rank):
     y = torch.empty_like(x)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
 
-    hist_buf = torch.empty((shape.E, lq.NBINS), dtype=torch.int32, device="cuda")
-    ntok_buf = torch.empty(1, dtype=torch.int64, device="cuda")
-
     def step():
         layer.forward(x, y, record_stats=True)
         if world > 1:  # the one exchange step: sum the QB statistics of all ranks
             hist, n = layer.hist()
-            dist.all_reduce(hist)
-            dist.all_reduce(n)
+            lq.sum_qb_statistics(hist, n)
             layer.set_hist(hist, n)
         layer.qb_update(BETA)
 
@@ -209,8 +205,7 @@ def run_ours(args, rank, world, local_rank):
         layer.forward_host(xh, yh, record_stats=True)
         if world > 1:
             hist, n = layer.hist()
-            dist.all_reduce(hist)
-            dist.all_reduce(n)
+            lq.sum_qb_statistics(hist, n)
             layer.set_hist(hist, n)
         layer.qb_update(BETA)
 

@@ -265,6 +265,16 @@ def gemm_bf16(a, b, stream=None):
     return c
 
 
+def sum_qb_statistics(hist, ntok, group=None):
+    """The data-parallel exchange step of QB: sums the integer histograms [E, 4096] and token
+    counts of all ranks in place (torch.distributed all-reduce), so every rank then applies the
+    same bias update as one device that saw every token."""
+    import torch.distributed as dist
+    dist.all_reduce(hist, group=group)
+    dist.all_reduce(ntok, group=group)
+    return hist, ntok
+
+
 def layer_from_weights(shape, weights_cpu: dict, max_tokens=None, device="cuda", stream=None) -> Layer:
     """Creates a Layer from the CPU weight dict of the seeded generator (copied to the device)."""
     w = {n: t.to(device) for n, t in weights_cpu.items()}
