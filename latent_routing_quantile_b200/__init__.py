@@ -26,6 +26,7 @@ EXPORTED = (
     "lmoe_qb_update", "lmoe_route_scores", "lmoe_get_routing", "lmoe_get_bias", "lmoe_set_bias",
     "lmoe_get_hist", "lmoe_set_hist", "lmoe_get_status", "lmoe_strerror", "lmoe_gemm_bf16",
     "lmoe_profile_enable", "lmoe_profile_read", "lmoe_stage_name", "lmoe_launch_count",
+    "lmoe_route_noalloc",
 )
 NUM_STAGES = 14
 
@@ -74,6 +75,7 @@ def lib() -> ctypes.CDLL:
             "lmoe_profile_enable": [vp, i32],
             "lmoe_profile_read": [vp, POINTER(c_float), i32, POINTER(i32)],
             "lmoe_launch_count": [vp, POINTER(ctypes.c_int64)],
+            "lmoe_route_noalloc": [vp, vp, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -273,6 +275,27 @@ def sum_qb_statistics(hist, ntok, group=None):
     dist.all_reduce(hist, group=group)
     dist.all_reduce(ntok, group=group)
     return hist, ntok
+
+
+def route_noalloc(scores, bias, k, out=None, stream=None):
+    """Routing of fp32 scores [T, E] with bias [E] through lmoe_route_noalloc, which allocates no
+    device memory (its scratch is a static array in the library).  `out` may pass preallocated
+    buffers (idx, gates, counts, offsets, perm, inv); missing ones are allocated here by torch."""
+    T, E = scores.shape
+    _dev(scores, torch.float32, (T, E), "scores")
+    _dev(bias, torch.float32, (E,), "bias")
+    dev = scores.device
+    shapes = dict(idx=((T, k), torch.int32), gates=((T, k), torch.float32), counts=((E,), torch.int32),
+                  offsets=((E + 1,), torch.int32), perm=((T * k,), torch.int32), inv=((T * k,), torch.int32))
+    out = dict(out or {})
+    for n, (shp, dt) in shapes.items():
+        if n not in out:
+            out[n] = torch.empty(shp, dtype=dt, device=dev)
+        _dev(out[n], dt, shp, n)
+    _check(lib().lmoe_route_noalloc(_ptr(scores), _ptr(bias), T, E, k,
+                                    *(_ptr(out[n]) for n in ("idx", "gates", "counts", "offsets", "perm", "inv")),
+                                    _stream(stream)), "lmoe_route_noalloc")
+    return out
 
 
 def layer_from_weights(shape, weights_cpu: dict, max_tokens=None, device="cuda", stream=None) -> Layer:

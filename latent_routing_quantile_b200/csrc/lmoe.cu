@@ -6,6 +6,7 @@
 
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -1012,6 +1013,83 @@ int lmoe_gemm_bf16(const void* a, const void* b, float* c, int32_t M, int32_t N,
   p.ldo = N;
   const int tiles = ((M + 127) / 128) * p.n_tiles;
   CK(launch_tc(p, EPI_F32, bn, tiles < sms ? tiles : sms, (cudaStream_t)stream));
+  return LMOE_OK;
+}
+
+// ---------------------------------------------------------------- routing without allocation
+// Scratch of lmoe_route_noalloc: a fixed device array in this library's image.  Every GPU that
+// loads the library holds it until the process exits.  Its name is only a host-side stand-in;
+// kernels get its device address, taken once per device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[LMOE_NOALLOC_SCRATCH_BYTES];
+
+static size_t noalloc_bytes(long long T, long long E, long long k, size_t* off_rank, size_t* off_cnt,
+                            size_t* off_base, size_t* off_tiles, size_t* off_ntiles) {
+  const long long nblk = (T + kTokBlock - 1) / kTokBlock;
+  const long long mtiles = (T * k + kTileRows - 1) / kTileRows + E;
+  size_t o = 0;
+  *off_rank = o;
+  o += align_up((size_t)(T * k) * 4, 256);
+  *off_cnt = o;
+  o += align_up((size_t)(nblk * E) * 4, 256);
+  *off_base = o;
+  o += align_up((size_t)(nblk * E) * 4, 256);
+  *off_tiles = o;
+  o += align_up((size_t)mtiles * 8, 256);
+  *off_ntiles = o;
+  o += 256;
+  return o;
+}
+
+int lmoe_route_noalloc(const float* scores, const float* bias, int32_t T, int32_t E, int32_t k, int32_t* idx,
+                       float* gates, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
+                       void* stream) {
+  if (!scores || !bias || !idx || !gates || !counts || !offsets || !perm || !inv) return LMOE_EINVAL;
+  if (T < 0 || E <= 0 || E > 1024 || k <= 0 || k > E || k > 32) return LMOE_EINVAL;
+  size_t o_rank, o_cnt, o_base, o_tiles, o_ntiles;
+  if (noalloc_bytes(T, E, k, &o_rank, &o_cnt, &o_base, &o_tiles, &o_ntiles) > LMOE_NOALLOC_SCRATCH_BYTES)
+    return LMOE_EUNSUPPORTED;
+  // set-up, once per device: the device address of the scratch array
+  static std::mutex mu;
+  static unsigned char* base_of[64] = {};
+  int dev = 0;
+  CK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return LMOE_EDEVICE;
+  unsigned char* base;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!base_of[dev]) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+        cudaGetLastError();
+        return LMOE_ECUDA;
+      }
+      base_of[dev] = static_cast<unsigned char*>(p);
+    }
+    base = base_of[dev];
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  CK(cudaMemsetAsync(counts, 0, (size_t)E * sizeof(int32_t), st));  // summed with atomics
+  if (T == 0) {
+    CK(cudaMemsetAsync(offsets, 0, (size_t)(E + 1) * sizeof(int32_t), st));
+    return LMOE_OK;
+  }
+  int* rank = reinterpret_cast<int*>(base + o_rank);
+  int* blkcnt = reinterpret_cast<int*>(base + o_cnt);
+  int* blkbase = reinterpret_cast<int*>(base + o_base);
+  int2* tiles = reinterpret_cast<int2*>(base + o_tiles);
+  int* ntiles = reinterpret_cast<int*>(base + o_ntiles);
+  uint32_t* status = reinterpret_cast<uint32_t*>(base + o_ntiles + 128);
+  // every scratch word is written before it is read, except the status word
+  CK(cudaMemsetAsync(status, 0, sizeof(uint32_t), st));
+  TopkArgs ta{scores, bias, T, E, k, idx, rank, blkcnt, counts, gates, nullptr, 0, status};
+  CK(launch_topk(ta, st));
+  const int nblk = (T + kTokBlock - 1) / kTokBlock;
+  plan_kernel<<<(E + 31) / 32, 1024, 0, st>>>(counts, blkcnt, nblk, E, offsets, blkbase, tiles, ntiles);
+  CK(cudaGetLastError());
+  const int pairs = T * k;
+  gather_kernel<float><<<(pairs + 7) / 8, 256, 0, st>>>(nullptr, 0, 0, idx, rank, blkbase, T, E, k, perm, inv,
+                                                        nullptr, status);
+  CK(cudaGetLastError());
   return LMOE_OK;
 }
 
