@@ -73,8 +73,7 @@ def stage_work(shape, T):
         "expert_down": (2 * TK * h * l, TK * w * h + E * l * h * w + TK * w * l),
         "combine": (0, TK * (w * l + 8) + T * w * l),
         "up_proj": (2 * T * d * (l + hs), T * w * (l + hs) + d * (l + hs) * w + T * w * d),
-        "qb_quantile": (0, 2 * E * 4096 * 4),
-        "qb_apply": (0, 16 * E),
+        "qb_update": (0, 2 * E * 4096 * 4 + 16 * E),
     }
 
 

@@ -158,10 +158,10 @@ int lmoe_get_status(lmoe_handle *h, uint32_t *status);
 /* Measurement support.  With profiling enabled, every lmoe_forward, lmoe_route_scores and
  * lmoe_qb_update records a CUDA event on its stream before each of its stages and after the last
  * (at most 4096 calls between two reads; later calls go unrecorded).  lmoe_profile_read
- * synchronises the device, stores in ms[i] (n >= 14) the time of stage i summed over the recorded
+ * synchronises the device, stores in ms[i] (n >= 13) the time of stage i summed over the recorded
  * calls, the number of recorded forwards in *calls, and forgets the records.  Stage i is named by
  * lmoe_stage_name(i): rms, down_proj, router, topk, plan, gather, hist, shared_swiglu,
- * expert_swiglu, expert_down, combine, up_proj, qb_quantile, qb_apply. */
+ * expert_swiglu, expert_down, combine, up_proj, qb_update. */
 int lmoe_profile_enable(lmoe_handle *h, int32_t enable);
 int lmoe_profile_read(lmoe_handle *h, float *ms, int32_t n, int32_t *calls);
 const char *lmoe_stage_name(int32_t i);

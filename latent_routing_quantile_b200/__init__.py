@@ -28,7 +28,7 @@ EXPORTED = (
     "lmoe_profile_enable", "lmoe_profile_read", "lmoe_stage_name", "lmoe_launch_count",
     "lmoe_route_noalloc",
 )
-NUM_STAGES = 14
+NUM_STAGES = 13
 
 
 class LmoeError(RuntimeError):

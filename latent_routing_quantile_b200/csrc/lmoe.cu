@@ -122,7 +122,7 @@ struct TopkArgs {
 template <int NJ>
 cudaError_t launch_topk_t(const TopkArgs& a, cudaStream_t st) {
   const int nblk = (a.T + kTokBlock - 1) / kTokBlock;
-  const size_t smem = a.E * sizeof(uint32_t) + (a.bins ? (size_t)a.E * kTokBlock * sizeof(uint16_t) : 0);
+  const size_t smem = a.E * sizeof(uint32_t) + (a.bins ? (size_t)(a.E + 2) * kTokBlock * sizeof(uint16_t) : 0);
   if (smem > 48 * 1024) {
     static unsigned done = 0;
     cudaError_t e = ensure_smem_attr(topk_kernel<NJ>, 64 * 1024 + 4 * 1024 + 1024, done);
@@ -155,11 +155,11 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 // Stages timed by the optional per-stage profiler (lmoe_profile_enable).
 enum Stage : int {
   ST_RMS = 0, ST_DOWN, ST_ROUTER, ST_TOPK, ST_PLAN, ST_GATHER, ST_HIST, ST_SHARED, ST_EXPERT1, ST_EXPERT2,
-  ST_COMBINE, ST_UP, ST_QB_QUANTILE, ST_QB_APPLY, ST_COUNT
+  ST_COMBINE, ST_UP, ST_QB_UPDATE, ST_COUNT
 };
 const char* const kStageNames[ST_COUNT] = {
     "rms", "down_proj", "router", "topk", "plan", "gather", "hist", "shared_swiglu", "expert_swiglu",
-    "expert_down", "combine", "up_proj", "qb_quantile", "qb_apply"};
+    "expert_down", "combine", "up_proj", "qb_update"};
 constexpr int kProfRecords = 4096;
 
 // One cached CUDA graph of a call with fixed arguments (see lmoe_forward).
@@ -232,6 +232,7 @@ struct lmoe_handle {
   long long* ntok = nullptr;
   uint32_t* status = nullptr;
   double* u = nullptr;
+  unsigned int* qb_done = nullptr;  // block counter of the QB update kernel (zero between calls)
   int last_T = 0;
   // tensor maps (bf16)
   // weight maps of the non-grouped GEMMs exist for each tile width 64/128/256 that divides N
@@ -306,6 +307,7 @@ void plan_layout(lmoe_handle* h, Arena& a) {
   a.add((void**)&h->ntok, 8);
   a.add((void**)&h->status, 4);
   a.add((void**)&h->u, E * 8);
+  a.add((void**)&h->qb_done, 4);
 }
 
 int validate(const lmoe_config* c) {
@@ -826,6 +828,7 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, void* stream, lmo
   if (!rc && cudaMemsetAsync(h->hist, 0, (size_t)cfg->E * LMOE_NBINS * 4, st) != cudaSuccess) rc = LMOE_ECUDA;
   if (!rc && cudaMemsetAsync(h->ntok, 0, 8, st) != cudaSuccess) rc = LMOE_ECUDA;
   if (!rc && cudaMemsetAsync(h->status, 0, 4, st) != cudaSuccess) rc = LMOE_ECUDA;
+  if (!rc && cudaMemsetAsync(h->qb_done, 0, 4, st) != cudaSuccess) rc = LMOE_ECUDA;
   if (!rc && h->bf) rc = build_maps(h);
   if (!rc && cudaStreamCreateWithFlags(&h->cap, cudaStreamNonBlocking) != cudaSuccess) rc = LMOE_ECUDA;
   if (rc) {
@@ -894,16 +897,14 @@ int lmoe_qb_update(lmoe_handle* h, float beta, uint32_t flags, void* stream) {
   if (!h || !(beta == beta)) return LMOE_EINVAL;
   cudaStream_t st = (cudaStream_t)stream;
   return run_cached(h, h->g_qb, nullptr, nullptr, 0, flags, beta, st, [&](cudaStream_t s) {
-    prof_open(h, ST_QB_QUANTILE, 2);
-    mark(h, ST_QB_QUANTILE, s);
-    qb_quantile_kernel<<<h->cfg.E, 256, 0, s>>>(h->hist, h->ntok, h->bias, h->cfg.E, h->cfg.k,
-                                                 (flags & LMOE_QB_LITERAL) ? 1 : 0, h->u, h->status);
-    CK(cudaGetLastError());
-    mark(h, ST_QB_APPLY, s);
-    qb_apply_kernel<<<1, 1024, 0, s>>>(h->bias, h->ntok, h->u, h->cfg.E, beta);
+    prof_open(h, ST_QB_UPDATE, 1);
+    mark(h, ST_QB_UPDATE, s);
+    qb_update_kernel<<<h->cfg.E, 256, 0, s>>>(h->hist, h->ntok, h->bias, h->cfg.E, h->cfg.k,
+                                               (flags & LMOE_QB_LITERAL) ? 1 : 0, beta, h->u, h->qb_done,
+                                               h->status);
     CK(cudaGetLastError());
     prof_close(h, s);
-    h->launches += 2;
+    h->launches += 1;
     return LMOE_OK;
   });
 }

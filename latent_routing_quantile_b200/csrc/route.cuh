@@ -48,23 +48,29 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 }
 
 // One warp per token, 4 tokens per warp, kTokBlock = 32 tokens per block.  Lane L holds the
-// scores of experts L, L+32, ...  k rounds of: local best (larger key, then lower index), warp
-// max of the keys (redux), warp min of the expert index among the lanes holding that key (redux),
-// broadcast of its unbiased score.  This is top-k of u = s + b in fp32 with ties to the lower
-// expert index.  Gates are the chosen s over their sum.  Each choice sets the token's bit in the
-// expert's shared mask; the token's rank inside the block for that expert is the number of set
-// bits below it, so the permutation is stable (token ascending) with no order-dependent atomics.
-// With bins != null it also stores each score's histogram bin, min(floor(s * 4096), 4095) as
-// uint16, expert-major (bins[e * ld_bins + t]) for the histogram kernel.
+// scores of experts L, L+32, ...; the scores of up to PF tokens are loaded before any of them is
+// ranked, so their memory latency overlaps.  k rounds of: local best (larger key, then lower
+// index), warp max of the keys (redux), warp min of the expert index among the lanes holding
+// that key (redux), broadcast of its unbiased score.  This is top-k of u = s + b in fp32 with
+// ties to the lower expert index.  Gates are the chosen s over their sum.  Each choice sets the
+// token's bit in the expert's shared mask; the token's rank inside the block for that expert is
+// the number of set bits below it, so the permutation is stable (token ascending) with no
+// order-dependent atomics.  With bins != null it also stores each score's histogram bin,
+// min(floor(s * 4096), 4095) as uint16, expert-major (bins[e * ld_bins + t]).
+__host__ __device__ constexpr int topk_prefetch(int nj) { return nj <= 8 ? 4 : (nj <= 16 ? 2 : 1); }
+
 template <int NJ>
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ s, const float* __restrict__ bias,
                                                    int ntok, int E, int k, int* __restrict__ idx,
                                                    float* __restrict__ gates, int* __restrict__ rank,
                                                    int* __restrict__ blkcnt, int* __restrict__ counts,
                                                    uint16_t* __restrict__ bins, int ld_bins, uint32_t* status) {
+  constexpr int TPW = kTokBlock / 8;  // tokens per warp
+  constexpr int PF = topk_prefetch(NJ);
   extern __shared__ uint32_t smem_topk[];
-  uint32_t* mask = smem_topk;                                          // [E]
-  uint16_t* sbins = reinterpret_cast<uint16_t*>(smem_topk + E);        // [E][32]
+  uint32_t* mask = smem_topk;                                    // [E]
+  uint16_t* sbins = reinterpret_cast<uint16_t*>(smem_topk + E);  // [32 tokens][E + 2] (padded rows)
+  const int bpitch = E + 2;
   const int blk = blockIdx.x, t0 = blk * kTokBlock;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < E; i += blockDim.x) mask[i] = 0;
@@ -76,68 +82,82 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ s, 
   }
   __syncthreads();
 
-  constexpr int TPW = kTokBlock / 8;  // tokens per warp
   int sel_q[TPW];
   bool nan = false;
 #pragma unroll
-  for (int q = 0; q < TPW; ++q) {
-    sel_q[q] = -1;
-    const int tl = warp * TPW + q, t = t0 + tl;
-    if (t >= ntok) break;
-    uint32_t key[NJ];
-    float sv[NJ];
+  for (int q0 = 0; q0 < TPW; q0 += PF) {
+    float vq[PF][NJ];
 #pragma unroll
-    for (int j = 0; j < NJ; ++j) {
-      const int e = j * 32 + lane;
-      if (e < E) {
-        const float v = s[(size_t)t * E + e];
-        nan |= (v != v);
-        sv[j] = (v == v) ? v : 0.f;
-        key[j] = order_key(v + bj[j]);
-        if (bins) sbins[e * kTokBlock + tl] = (uint16_t)(v >= 0.f ? min((int)(v * (float)LMOE_NBINS), LMOE_NBINS - 1) : 0);
-      } else {
-        sv[j] = 0.f;
-        key[j] = 0u;
-      }
-    }
-    int my_sel = -1;
-    float my_s = 0.f;
-    for (int i = 0; i < k; ++i) {
-      uint32_t bk = 0u;
-      uint32_t be = 0xffffffffu;
-      float bs = 0.f;
+    for (int p = 0; p < PF; ++p) {
+      const int t = t0 + warp * TPW + q0 + p;
 #pragma unroll
       for (int j = 0; j < NJ; ++j) {
-        if (key[j] > bk) {
-          bk = key[j];
-          be = (uint32_t)(j * 32 + lane);
-          bs = sv[j];
+        const int e = j * 32 + lane;
+        vq[p][j] = (t < ntok && e < E) ? s[(size_t)t * E + e] : 0.f;
+      }
+    }
+#pragma unroll
+    for (int p = 0; p < PF; ++p) {
+      const int tl = warp * TPW + q0 + p, t = t0 + tl;
+      sel_q[q0 + p] = -1;
+      if (t >= ntok) continue;  // warp-uniform
+      uint32_t key[NJ];
+      float sv[NJ];
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        const int e = j * 32 + lane;
+        const float v = vq[p][j];
+        if (e < E) {
+          nan |= (v != v);
+          sv[j] = (v == v) ? v : 0.f;
+          key[j] = order_key(v + bj[j]);
+          if (bins)
+            sbins[tl * bpitch + e] =
+                (uint16_t)(v >= 0.f ? min((int)(v * (float)LMOE_NBINS), LMOE_NBINS - 1) : 0);
+        } else {
+          sv[j] = 0.f;
+          key[j] = 0u;
         }
       }
-      const uint32_t wmax = __reduce_max_sync(kFull, bk);
-      const uint32_t emin = __reduce_min_sync(kFull, bk == wmax ? be : 0xffffffffu);
-      const float es = __shfl_sync(kFull, bs, (int)(emin & 31u));
+      int my_sel = -1;
+      float my_s = 0.f;
+      for (int i = 0; i < k; ++i) {
+        uint32_t bk = 0u;
+        uint32_t be = 0xffffffffu;
+        float bs = 0.f;
 #pragma unroll
-      for (int j = 0; j < NJ; ++j)
-        if ((uint32_t)(j * 32 + lane) == emin) key[j] = 0u;
-      if (lane == i) {
-        my_sel = (int)emin;
-        my_s = es;
-      }
-    }
-    float ssum = lane < k ? my_s : 0.f;
+        for (int j = 0; j < NJ; ++j) {
+          if (key[j] > bk) {
+            bk = key[j];
+            be = (uint32_t)(j * 32 + lane);
+            bs = sv[j];
+          }
+        }
+        const uint32_t wmax = __reduce_max_sync(kFull, bk);
+        const uint32_t emin = __reduce_min_sync(kFull, bk == wmax ? be : 0xffffffffu);
+        const float es = __shfl_sync(kFull, bs, (int)(emin & 31u));
 #pragma unroll
-    for (int off = 16; off; off >>= 1) ssum += __shfl_xor_sync(kFull, ssum, off);
-    if (lane < k) {
-      if (my_sel < 0 || my_sel >= E) {
-        set_status(status, LMOE_STATUS_BAD_INDEX);
-        my_sel = 0;
+        for (int j = 0; j < NJ; ++j)
+          if ((uint32_t)(j * 32 + lane) == emin) key[j] = 0u;
+        if (lane == i) {
+          my_sel = (int)emin;
+          my_s = es;
+        }
       }
-      idx[(size_t)t * k + lane] = my_sel;
-      gates[(size_t)t * k + lane] = my_s / ssum;
-      atomicOr(&mask[my_sel], 1u << tl);
+      float ssum = lane < k ? my_s : 0.f;
+#pragma unroll
+      for (int off = 16; off; off >>= 1) ssum += __shfl_xor_sync(kFull, ssum, off);
+      if (lane < k) {
+        if (my_sel < 0 || my_sel >= E) {
+          set_status(status, LMOE_STATUS_BAD_INDEX);
+          my_sel = 0;
+        }
+        idx[(size_t)t * k + lane] = my_sel;
+        gates[(size_t)t * k + lane] = my_s / ssum;
+        atomicOr(&mask[my_sel], 1u << tl);
+      }
+      sel_q[q0 + p] = my_sel;
     }
-    sel_q[q] = my_sel;
   }
   if (nan) set_status(status, LMOE_STATUS_NAN_SCORE);
   __syncthreads();
@@ -157,7 +177,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ s, 
     // expert-major store: one warp writes 32 tokens (64 bytes) of one expert per step
     const int nt = min(kTokBlock, ntok - t0);
     for (int e = warp; e < E; e += 8)
-      if (lane < nt) bins[(size_t)e * ld_bins + t0 + lane] = sbins[e * kTokBlock + lane];
+      if (lane < nt) bins[(size_t)e * ld_bins + t0 + lane] = sbins[lane * bpitch + e];
   }
 }
 
@@ -327,30 +347,37 @@ __global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ o, c
 }
 
 // --------------------------------------------------------------------------- QB update
-// Block per expert: m = ceil((E-k) N / E); the crossing bin j* is the first whose cumulative
-// count reaches m; q = (j* + (m - cum_{j*-1}) / cnt_{j*}) / 4096; u_e = q (+ b_e).  The row of
-// the histogram is cleared afterwards.
-__global__ void __launch_bounds__(256) qb_quantile_kernel(uint32_t* __restrict__ hist,
-                                                          const long long* __restrict__ ntok_acc,
-                                                          const float* __restrict__ bias, int E, int k,
-                                                          int literal, double* __restrict__ u_out,
-                                                          uint32_t* status) {
+// One kernel, block per expert.  Block e: m = ceil((E-k) N / E); the crossing bin j* is the first
+// whose cumulative count reaches m; q = (j* + (m - cum_{j*-1}) / cnt_{j*}) / 4096; u_e = q (+ b_e);
+// the expert's histogram row is cleared.  The last block to finish (a device-wide counter)
+// computes mean_e u and applies b_e <- b_e - beta (u_e - mean) to every expert, then clears N and
+// the counter.  Nothing happens when N == 0.
+__global__ void __launch_bounds__(256) qb_update_kernel(uint32_t* __restrict__ hist, long long* ntok_acc,
+                                                        float* __restrict__ bias, int E, int k, int literal,
+                                                        float beta, double* __restrict__ u_buf,
+                                                        unsigned int* done_counter, uint32_t* status) {
   __shared__ long long wsum[8];
+  __shared__ double wd[8];
+  __shared__ bool last;
   const int e = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const long long N = *ntok_acc;
   if (N <= 0) return;
   long long m = ((long long)(E - k) * N + E - 1) / E;
   m = m < 1 ? 1 : (m > N ? N : m);
-  uint32_t* row = hist + (size_t)e * LMOE_NBINS;
-  constexpr int PER = LMOE_NBINS / 256;
+  uint4* row4 = reinterpret_cast<uint4*>(hist + (size_t)e * LMOE_NBINS);
+  constexpr int PER = LMOE_NBINS / 256;  // 16 bins per thread, 4 x uint4
   uint32_t c[PER];
+#pragma unroll
+  for (int j = 0; j < PER / 4; ++j) {
+    const uint4 q = row4[tid * (PER / 4) + j];
+    c[4 * j] = q.x;
+    c[4 * j + 1] = q.y;
+    c[4 * j + 2] = q.z;
+    c[4 * j + 3] = q.w;
+  }
   long long local = 0;
 #pragma unroll
-  for (int j = 0; j < PER; ++j) {
-    c[j] = row[tid * PER + j];
-    local += c[j];
-  }
-  // inclusive scan of per-thread sums
+  for (int j = 0; j < PER; ++j) local += c[j];
   long long x = local;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
@@ -358,7 +385,7 @@ __global__ void __launch_bounds__(256) qb_quantile_kernel(uint32_t* __restrict__
     if (lane >= off) x += y;
   }
   if (lane == 31) wsum[warp] = x;
-  if (tid == 0) u_out[e] = literal ? 0.0 : (double)bias[e];
+  if (tid == 0) u_buf[e] = literal ? 0.0 : (double)bias[e];  // only if no crossing is found
   __syncthreads();
   long long before = x - local;
   for (int w = 0; w < warp; ++w) before += wsum[w];
@@ -369,7 +396,7 @@ __global__ void __launch_bounds__(256) qb_quantile_kernel(uint32_t* __restrict__
       if (cum + c[j] >= m) {
         const int jstar = tid * PER + j;
         const double q = ((double)jstar + (double)(m - cum) / (double)c[j]) / (double)LMOE_NBINS;
-        u_out[e] = literal ? q : q + (double)bias[e];
+        u_buf[e] = literal ? q : q + (double)bias[e];
         break;
       }
       cum += c[j];
@@ -377,33 +404,29 @@ __global__ void __launch_bounds__(256) qb_quantile_kernel(uint32_t* __restrict__
   }
   __syncthreads();
 #pragma unroll
-  for (int j = 0; j < PER; ++j) row[tid * PER + j] = 0u;
-}
-
-// b_e <- b_e - beta (u_e - mean_e u); then the token count is cleared.  One block.
-__global__ void __launch_bounds__(1024) qb_apply_kernel(float* __restrict__ bias, long long* ntok_acc,
-                                                        const double* __restrict__ u, int E, float beta) {
-  __shared__ double ws[32];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (*ntok_acc <= 0) return;
+  for (int j = 0; j < PER / 4; ++j) row4[tid * (PER / 4) + j] = make_uint4(0u, 0u, 0u, 0u);
+  // publish u_e, then count finished blocks
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) last = (atomicAdd(done_counter, 1u) == (unsigned)(E - 1));
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
   double v = 0.0;
-  for (int e = tid; e < E; e += blockDim.x) v += u[e];
+  for (int i = tid; i < E; i += blockDim.x) v += __ldcg(&u_buf[i]);
 #pragma unroll
   for (int off = 16; off; off >>= 1) v += __shfl_xor_sync(kFull, v, off);
-  if (lane == 0) ws[warp] = v;
+  if (lane == 0) wd[warp] = v;
   __syncthreads();
-  if (warp == 0) {
-    double w = ws[lane];
-#pragma unroll
-    for (int off = 16; off; off >>= 1) w += __shfl_xor_sync(kFull, w, off);
-    if (lane == 0) ws[0] = w;
+  double tot = 0.0;
+  for (int w = 0; w < 8; ++w) tot += wd[w];
+  const double mean = tot / E;
+  for (int i = tid; i < E; i += blockDim.x)
+    bias[i] = (float)((double)bias[i] - (double)beta * (__ldcg(&u_buf[i]) - mean));
+  if (tid == 0) {
+    *ntok_acc = 0;
+    *done_counter = 0u;
   }
-  __syncthreads();
-  const double mean = ws[0] / E;
-  for (int e = tid; e < E; e += blockDim.x)
-    bias[e] = (float)((double)bias[e] - (double)beta * (u[e] - mean));
-  __syncthreads();
-  if (tid == 0) *ntok_acc = 0;
 }
 
 // --------------------------------------------------------------------------- weight repacking
