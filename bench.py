@@ -64,6 +64,8 @@ def stage_work(shape, T):
         "rms": (0, T * w * d + 4 * T),
         "down_proj": (2 * T * d * l, T * w * d + l * d * w + 4 * T * l),
         "router": (2 * T * l * E, 4 * T * l + 4 * E * l + 4 * T * E),
+        "norm_down_router": (2 * T * d * l + 2 * T * l * E,
+                             T * (w * d + 2 * l + 4 * E + 4) + l * d * w + 4 * E * l),
         "topk": (0, 4 * T * E + 12 * TK),
         "plan": (0, 3 * 4 * nblk * E),
         "gather": (0, TK * (2 * w * l + 8)),

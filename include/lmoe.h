@@ -158,10 +158,11 @@ int lmoe_get_status(lmoe_handle *h, uint32_t *status);
 /* Measurement support.  With profiling enabled, every lmoe_forward, lmoe_route_scores and
  * lmoe_qb_update records a CUDA event on its stream before each of its stages and after the last
  * (at most 4096 calls between two reads; later calls go unrecorded).  lmoe_profile_read
- * synchronises the device, stores in ms[i] (n >= 13) the time of stage i summed over the recorded
+ * synchronises the device, stores in ms[i] (n >= 14) the time of stage i summed over the recorded
  * calls, the number of recorded forwards in *calls, and forgets the records.  Stage i is named by
- * lmoe_stage_name(i): rms, down_proj, router, topk, plan, gather, hist, shared_swiglu,
- * expert_swiglu, expert_down, combine, up_proj, qb_update. */
+ * lmoe_stage_name(i): rms, down_proj, router, norm_down_router (the three fused, when l and E are
+ * at most 256), topk, plan, gather, hist, shared_swiglu, expert_swiglu, expert_down, combine,
+ * up_proj, qb_update. */
 int lmoe_profile_enable(lmoe_handle *h, int32_t enable);
 int lmoe_profile_read(lmoe_handle *h, float *ms, int32_t n, int32_t *calls);
 const char *lmoe_stage_name(int32_t i);
@@ -180,7 +181,7 @@ int lmoe_launch_count(lmoe_handle *h, int64_t *n);
  * offsets [E+1] int32, perm [T*k] int32 (permuted row -> token), inv [T*k] int32, all device
  * buffers the caller owns.  1 <= k <= min(E, 32), E <= 1024.
  * Scratch: a static device array of LMOE_NOALLOC_SCRATCH_BYTES in the library image, which needs
- *   4*T*k + 8*ceil(T/32)*E + 8*(ceil(T*k/128) + E) bytes (each part rounded up to 256) + 256;
+ *   4*T*k + 8*ceil(T/32)*E + 8*(ceil(T*k/128) + E) + 132*E bytes (each part rounded up to 256) + 256;
  *   larger sizes return LMOE_EUNSUPPORTED (about T = 65536 at E = 256, k = 6).
  * The first call on each device takes the array's device address (cudaGetSymbolAddress); make
  * that first call before any stream capture.  All calls share the one array, which keeps the
@@ -191,11 +192,18 @@ int lmoe_route_noalloc(const float *scores_dev, const float *bias_dev, int32_t T
                        int32_t *idx, float *gates, int32_t *counts, int32_t *offsets, int32_t *perm,
                        int32_t *inv, void *stream);
 
+/* Failure-detection check of the bounded waits: one thread waits on an mbarrier that nothing ever
+ * completes, with the same wait loop every pipeline kernel uses but a limit of limit_us
+ * microseconds (1 .. 2e6); it gives up, sets LMOE_STATUS_WATCHDOG in *status_dev (device word,
+ * caller-owned) and returns, leaving the context usable.  No kernel of this library traps. */
+int lmoe_watchdog_selftest(uint32_t *status_dev, int32_t limit_us, void *stream);
+
 /* Static text for a return code. */
 const char *lmoe_strerror(int code);
 
 /* Check of the tensor-core GEMM engine on its own: C[M,N] (fp32) = A[M,K] B[N,K]^T with
- * A, B bf16 device buffers, K and N multiples of 64, row pitches equal to K.  For tests. */
+ * A, B bf16 device buffers, K and N multiples of 64, row pitches equal to K.  M >= 256 with N a
+ * multiple of 128 runs the two-CTA (cta_group::2, 256-row tile) variant.  For tests. */
 int lmoe_gemm_bf16(const void *a_dev, const void *b_dev, float *c_dev, int32_t M, int32_t N,
                    int32_t K, void *stream);
 

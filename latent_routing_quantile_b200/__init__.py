@@ -26,9 +26,9 @@ EXPORTED = (
     "lmoe_qb_update", "lmoe_route_scores", "lmoe_get_routing", "lmoe_get_bias", "lmoe_set_bias",
     "lmoe_get_hist", "lmoe_set_hist", "lmoe_get_status", "lmoe_strerror", "lmoe_gemm_bf16",
     "lmoe_profile_enable", "lmoe_profile_read", "lmoe_stage_name", "lmoe_launch_count",
-    "lmoe_route_noalloc",
+    "lmoe_route_noalloc", "lmoe_watchdog_selftest",
 )
-NUM_STAGES = 13
+NUM_STAGES = 14
 
 
 class LmoeError(RuntimeError):
@@ -76,6 +76,7 @@ def lib() -> ctypes.CDLL:
             "lmoe_profile_read": [vp, POINTER(c_float), i32, POINTER(i32)],
             "lmoe_launch_count": [vp, POINTER(ctypes.c_int64)],
             "lmoe_route_noalloc": [vp, vp, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp],
+            "lmoe_watchdog_selftest": [vp, i32, vp],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -243,6 +244,14 @@ class Layer:
             self.close()
         except Exception:
             pass
+
+
+def watchdog_selftest(limit_us: int = 20000, stream=None) -> int:
+    """Runs the bounded-wait check (a wait on a barrier nothing completes) and returns the status word."""
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    _check(lib().lmoe_watchdog_selftest(_ptr(st), int(limit_us), _stream(stream)), "lmoe_watchdog_selftest")
+    torch.cuda.synchronize()
+    return int(st.item()) & 0xffffffff
 
 
 def stage_name(i: int) -> str:

@@ -14,6 +14,7 @@
 #include "route.cuh"
 #include "simt_gemm.cuh"
 #include "tc_gemm.cuh"
+#include "k1_router.cuh"
 
 using namespace lmoe;
 
@@ -36,19 +37,29 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 matrix [rows, cols] with row pitch `pitch` elements; box = 64 columns x box_rows rows,
-// 128-byte swizzle (the layout the MMA descriptors expect).
-bool make_map(CUtensorMap* m, const void* base, long long rows, long long cols, long long pitch, int box_rows) {
+// Tensor map of a row-major matrix with a 128-byte swizzle (the layout the MMA descriptors and the
+// staged epilogue expect).
+bool make_map_t(CUtensorMap* m, const void* base, long long rows, long long cols, long long pitch, int box_rows,
+                bool f32) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
-  if (((uintptr_t)base & 15) || ((pitch * 2) & 15) || rows <= 0 || cols <= 0) return false;
+  const long long es_bytes = f32 ? 4 : 2;
+  if (((uintptr_t)base & 15) || ((pitch * es_bytes) & 15) || rows <= 0 || cols <= 0) return false;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)(pitch * 2)};
-  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(pitch * es_bytes)};
+  cuuint32_t box[2] = {f32 ? 32u : 64u, (cuuint32_t)box_rows};
   cuuint32_t es[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return enc(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
+             dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+// bf16 matrix [rows, cols], row pitch `pitch` elements; box = 64 columns (128 bytes) x box_rows.
+bool make_map(CUtensorMap* m, const void* base, long long rows, long long cols, long long pitch, int box_rows) {
+  return make_map_t(m, base, rows, cols, pitch, box_rows, false);
+}
+// fp32 matrix; box = 32 columns (128 bytes) x box_rows.
+bool make_map_f32(CUtensorMap* m, const void* base, long long rows, long long cols, long long pitch, int box_rows) {
+  return make_map_t(m, base, rows, cols, pitch, box_rows, true);
 }
 
 int pick_bn(int n) { return n % 256 == 0 ? 256 : (n % 128 == 0 ? 128 : 64); }
@@ -79,11 +90,36 @@ cudaError_t ensure_smem_attr(K kern, int bytes, unsigned& done) {
 
 template <int BN, int EPI>
 cudaError_t launch_tc_t(const TcParams& p, int grid, cudaStream_t st) {
-  auto kern = tc_gemm_kernel<BN, EPI>;
+  auto kern = tc_gemm_kernel<BN, EPI, 0>;
   static unsigned done = 0;
   cudaError_t e = ensure_smem_attr(kern, TcCfg<BN>::kSmemBytes, done);
   if (e != cudaSuccess) return e;
   kern<<<grid, kTcThreads, TcCfg<BN>::kSmemBytes, st>>>(p);
+  return cudaGetLastError();
+}
+
+// Two-CTA (cta_group::2) variant: clusters of 2 along x, grid even.
+template <int BN, int EPI>
+cudaError_t launch_tc_pair_t(const TcParams& p, int grid, cudaStream_t st) {
+  auto kern = tc_gemm_kernel<BN, EPI, 1>;
+  static unsigned done = 0;
+  cudaError_t e = ensure_smem_attr(kern, TcCfg<BN, 1>::kSmemBytes, done);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)(grid & ~1), 1, 1);
+  cfg.blockDim = dim3(kTcThreads, 1, 1);
+  cfg.dynamicSmemBytes = TcCfg<BN, 1>::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -108,11 +144,31 @@ cudaError_t launch_tc(const TcParams& p, int epi, int bn, int grid, cudaStream_t
   }
 }
 
+// Pair launches exist for tile widths 128 and 256 and the bf16 / SwiGLU / fp32 epilogues.
+cudaError_t launch_tc_pair(const TcParams& p, int epi, int bn, int grid, cudaStream_t st) {
+  if (epi == EPI_SWIGLU) return bn == 256 ? launch_tc_pair_t<256, EPI_SWIGLU>(p, grid, st)
+                                          : launch_tc_pair_t<128, EPI_SWIGLU>(p, grid, st);
+  if (epi == EPI_BF16) return bn == 256 ? launch_tc_pair_t<256, EPI_BF16>(p, grid, st)
+                                        : launch_tc_pair_t<128, EPI_BF16>(p, grid, st);
+  if (epi == EPI_F32) return bn == 256 ? launch_tc_pair_t<256, EPI_F32>(p, grid, st)
+                                       : launch_tc_pair_t<128, EPI_F32>(p, grid, st);
+  return cudaErrorInvalidValue;
+}
+
+// Pair tile width for M rows and N columns: the widest of 256/128 dividing N whose 256-row tiles
+// still give every pair of SMs one; 0 when N has no such width.
+int pick_pair_bn(long long M, int N, int sms) {
+  const long long mt = (M + 255) / 256;
+  for (int bn = 256; bn >= 128; bn >>= 1)
+    if (N % bn == 0 && mt * (N / bn) >= sms / 2) return bn;
+  return N % 128 == 0 ? 128 : 0;
+}
+
 struct TopkArgs {
   const float* s;
   const float* b;
   int T, E, k;
-  int *idx, *rank, *blkcnt, *counts;
+  int *idx, *rank, *blkcnt, *counts32;
   float* gates;
   uint16_t* bins;
   int ld_bins;
@@ -128,7 +184,7 @@ cudaError_t launch_topk_t(const TopkArgs& a, cudaStream_t st) {
     cudaError_t e = ensure_smem_attr(topk_kernel<NJ>, 64 * 1024 + 4 * 1024 + 1024, done);
     if (e != cudaSuccess) return e;
   }
-  topk_kernel<NJ><<<nblk, 256, smem, st>>>(a.s, a.b, a.T, a.E, a.k, a.idx, a.gates, a.rank, a.blkcnt, a.counts,
+  topk_kernel<NJ><<<nblk, 256, smem, st>>>(a.s, a.b, a.T, a.E, a.k, a.idx, a.gates, a.rank, a.blkcnt, a.counts32,
                                            a.bins, a.ld_bins, a.status);
   return cudaGetLastError();
 }
@@ -154,12 +210,12 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Stages timed by the optional per-stage profiler (lmoe_profile_enable).
 enum Stage : int {
-  ST_RMS = 0, ST_DOWN, ST_ROUTER, ST_TOPK, ST_PLAN, ST_GATHER, ST_HIST, ST_SHARED, ST_EXPERT1, ST_EXPERT2,
-  ST_COMBINE, ST_UP, ST_QB_UPDATE, ST_COUNT
+  ST_RMS = 0, ST_DOWN, ST_ROUTER, ST_K1, ST_TOPK, ST_PLAN, ST_GATHER, ST_HIST, ST_SHARED, ST_EXPERT1,
+  ST_EXPERT2, ST_COMBINE, ST_UP, ST_QB_UPDATE, ST_COUNT
 };
 const char* const kStageNames[ST_COUNT] = {
-    "rms", "down_proj", "router", "topk", "plan", "gather", "hist", "shared_swiglu", "expert_swiglu",
-    "expert_down", "combine", "up_proj", "qb_update"};
+    "rms", "down_proj", "router", "norm_down_router", "topk", "plan", "gather", "hist", "shared_swiglu",
+    "expert_swiglu", "expert_down", "combine", "up_proj", "qb_update"};
 constexpr int kProfRecords = 4096;
 
 // One cached CUDA graph of a call with fixed arguments (see lmoe_forward).
@@ -221,7 +277,10 @@ struct lmoe_handle {
   float* s = nullptr;
   uint16_t* bins = nullptr;  // [E, ld_bins] histogram bin of every score, expert-major
   int *idx = nullptr, *rank = nullptr, *blkcnt = nullptr, *blkbase = nullptr, *counts = nullptr;
+  int* counts32 = nullptr;  // [32][E] partial counts of the top-k blocks
   int *offsets = nullptr, *num_mtiles = nullptr, *perm = nullptr, *inv = nullptr;
+  int *pad_delta = nullptr, *prow = nullptr;  // padded expert layout of the grouped GEMMs
+  long long rows_pad = 0;                     // rows of that layout (upper bound)
   float* gates = nullptr;
   int2* mtiles = nullptr;
   void *a_perm = nullptr, *act = nullptr, *o = nullptr, *z = nullptr, *a_s = nullptr;
@@ -236,8 +295,10 @@ struct lmoe_handle {
   int last_T = 0;
   // tensor maps (bf16)
   // weight maps of the non-grouped GEMMs exist for each tile width 64/128/256 that divides N
-  CUtensorMap tm_hx, tm_aperm, tm_w13, tm_act, tm_w2, tm_z, tm_as;
+  CUtensorMap tm_hx, tm_aperm, tm_w13, tm_act, tm_w2, tm_z, tm_as, tm_o, tm_s;
   CUtensorMap tm_wr[3], tm_wdown[3], tm_ws13[3], tm_wy[3];
+  bool fused_k1 = false;       // l <= 256 and E <= 256: RMSNorm + W_down + router in one kernel
+  CUtensorMap tm_k1_wd, tm_k1_wr;
   int bn_e1 = 256, bn_e2 = 256;
   // launch counter and optional per-stage profiler
   long long launches = 0;
@@ -289,14 +350,18 @@ void plan_layout(lmoe_handle* h, Arena& a) {
   a.add((void**)&h->blkcnt, (size_t)h->nblk_max * E * 4);
   a.add((void**)&h->blkbase, (size_t)h->nblk_max * E * 4);
   a.add((void**)&h->counts, E * 4);
+  a.add((void**)&h->counts32, (size_t)kCountCopies * E * 4);
   a.add((void**)&h->offsets, (E + 1) * 4);
   a.add((void**)&h->num_mtiles, 4);
   a.add((void**)&h->mtiles, (size_t)h->max_mtiles * 8);
   a.add((void**)&h->perm, TK * 4);
   a.add((void**)&h->inv, TK * 4);
-  a.add(&h->a_perm, TK * l * es);
-  a.add(&h->act, TK * hh * es);
-  a.add(&h->o, TK * l * es);
+  a.add((void**)&h->prow, TK * 4);
+  a.add((void**)&h->pad_delta, E * 4);
+  const size_t RP = (size_t)h->rows_pad;
+  a.add(&h->a_perm, RP * l * es);
+  a.add(&h->act, RP * hh * es);
+  a.add(&h->o, RP * l * es);
   a.add(&h->z, Tm * l * es);
   if (hs) a.add(&h->a_s, Tm * hs * es);
   a.add(&h->x_stage, Tm * d * es);
@@ -355,13 +420,22 @@ int build_maps(lmoe_handle* h) {
   ok &= make_weight_maps(h->tm_wr, h->w_r, E, 3 * l);
   ok &= make_weight_maps(h->tm_wdown, h->w_down, l, h->unit_gain ? d : 2 * d);
   if (hs) ok &= make_weight_maps(h->tm_ws13, h->ws13, 2 * hs, d);
-  ok &= make_map(&h->tm_aperm, h->a_perm, TK, l, l, 128);
+  const long long RP = h->rows_pad;
+  (void)TK;
+  ok &= make_map(&h->tm_aperm, h->a_perm, RP, l, l, 128);
   ok &= make_map(&h->tm_w13, h->w13, E * 2 * hh, l, l, h->bn_e1);
-  ok &= make_map(&h->tm_act, h->act, TK, hh, hh, 128);
+  ok &= make_map(&h->tm_act, h->act, RP, hh, hh, 128);
+  ok &= make_map(&h->tm_o, h->o, RP, l, l, 128);
+  ok &= make_map_f32(&h->tm_s, h->s, Tm, E, E, 128);
   ok &= make_map(&h->tm_w2, h->w2, E * l, hh, hh, h->bn_e2);
   ok &= make_map(&h->tm_z, h->z, Tm, l, l, 128);
   if (hs) ok &= make_map(&h->tm_as, h->a_s, Tm, hs, hs, 128);
   ok &= make_weight_maps(h->tm_wy, h->wy, d, l + hs);
+  h->fused_k1 = c.l <= 256 && c.E <= 256;
+  if (h->fused_k1) {
+    ok &= make_map(&h->tm_k1_wd, h->w_down, l, h->unit_gain ? d : 2 * d, h->unit_gain ? d : 2 * d, (int)l);
+    ok &= make_map(&h->tm_k1_wr, h->w_r, E, 3 * l, 3 * l, (int)E);
+  }
   return ok ? LMOE_OK : LMOE_ECUDA;
 }
 
@@ -399,24 +473,24 @@ int route_from_scores(lmoe_handle* h, int T, uint32_t flags, cudaStream_t st) {
   const lmoe_config& c = h->cfg;
   const int nblk = (T + kTokBlock - 1) / kTokBlock;
   mark(h, ST_TOPK, st);
-  CK(cudaMemsetAsync(h->counts, 0, c.E * sizeof(int), st));
-  TopkArgs ta{h->s, h->bias, T, c.E, c.k, h->idx, h->rank, h->blkcnt, h->counts, h->gates,
+  CK(cudaMemsetAsync(h->counts32, 0, (size_t)kCountCopies * c.E * sizeof(int), st));
+  TopkArgs ta{h->s, h->bias, T, c.E, c.k, h->idx, h->rank, h->blkcnt, h->counts32, h->gates,
               (flags & LMOE_RECORD_STATS) ? h->bins : nullptr, h->ld_bins, h->status};
   CK(launch_topk(ta, st));
   mark(h, ST_PLAN, st);
-  plan_kernel<<<(c.E + 31) / 32, 1024, 0, st>>>(h->counts, h->blkcnt, nblk, c.E, h->offsets, h->blkbase,
-                                                  h->mtiles, h->num_mtiles);
+  plan_kernel<<<(c.E + 31) / 32, 1024, 0, st>>>(h->counts32, h->counts, h->blkcnt, nblk, c.E, h->offsets,
+                                                  h->pad_delta, h->blkbase, h->mtiles, h->num_mtiles);
   CK(cudaGetLastError());
   const int pairs = T * c.k;
   mark(h, ST_GATHER, st);
   if (h->bf) {
-    gather_kernel<bf16><<<(pairs + 7) / 8, 256, 0, st>>>((const bf16*)h->hx, 3 * c.l, c.l, h->idx, h->rank,
-                                                         h->blkbase, T, c.E, c.k, h->perm, h->inv,
-                                                         (bf16*)h->a_perm, h->status);
+    gather_kernel<bf16><<<(pairs + 8 * kGatherPairs - 1) / (8 * kGatherPairs), 256, 0, st>>>((const bf16*)h->hx, 3 * c.l, c.l, h->idx, h->rank,
+                                                         h->blkbase, h->pad_delta, T, c.E, c.k, h->perm, h->inv,
+                                                         h->prow, (bf16*)h->a_perm, h->status);
   } else {
-    gather_kernel<float><<<(pairs + 7) / 8, 256, 0, st>>>((const float*)h->hx, c.l, c.l, h->idx, h->rank,
-                                                          h->blkbase, T, c.E, c.k, h->perm, h->inv,
-                                                          (float*)h->a_perm, h->status);
+    gather_kernel<float><<<(pairs + 8 * kGatherPairs - 1) / (8 * kGatherPairs), 256, 0, st>>>((const float*)h->hx, c.l, c.l, h->idx, h->rank,
+                                                          h->blkbase, h->pad_delta, T, c.E, c.k, h->perm, h->inv,
+                                                          h->prow, (float*)h->a_perm, h->status);
   }
   CK(cudaGetLastError());
   mark(h, ST_HIST, st);
@@ -436,49 +510,78 @@ int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, 
   CUtensorMap tm_x;
   if (!make_map(&tm_x, x, T, c.d, c.d, 128)) return LMOE_EINVAL;
   mark(h, ST_RMS, st);
-  rms_kernel<bf16><<<(T + 7) / 8, 256, 0, st>>>((const bf16*)x, T, c.d, c.rms_eps, h->r);
-  CK(cudaGetLastError());
-  // h = r * (x Wdown^T), stored as hi | mid | lo bf16 parts
-  mark(h, ST_DOWN, st);
-  {
-    TcParams p = tc_base(h);
-    p.tmA[0] = tm_x;
-    p.tmA[1] = tm_x;
-    const int bn = pick_bn_for(T, c.l, h->sms, 64);
-    p.tmB = h->tm_wdown[bn_index(bn)];
-    p.nseg = h->unit_gain ? 1 : 2;
-    p.seg[0] = {0, 0, 0, c.d / 64};
-    p.seg[1] = {0, 0, c.d, c.d / 64};
-    p.M = T;
-    p.n_tiles = c.l / bn;
-    p.out = h->hx;
-    p.ldo = 3 * c.l;
-    p.split = c.l;
-    p.row_scale = h->r;
-    CK(launch_tc(p, EPI_DOWN3, bn, std::min(mt * p.n_tiles, h->sms), st));
-  }
-  // s = sigmoid(h Wr^T + c) from six bf16 x bf16 products of the hi/mid/lo parts
-  mark(h, ST_ROUTER, st);
-  {
-    TcParams p = tc_base(h);
-    p.tmA[0] = h->tm_hx;
-    p.tmA[1] = h->tm_hx;
-    const int bn = pick_bn_for(T, c.E, h->sms, 64);
-    p.tmB = h->tm_wr[bn_index(bn)];
-    const int L = c.l, nk = c.l / 64;
-    p.nseg = 6;
-    p.seg[0] = {0, L, L, nk};      // mid * mid
-    p.seg[1] = {0, 2 * L, 0, nk};  // lo * hi
-    p.seg[2] = {0, 0, 2 * L, nk};  // hi * lo
-    p.seg[3] = {0, L, 0, nk};      // mid * hi
-    p.seg[4] = {0, 0, L, nk};      // hi * mid
-    p.seg[5] = {0, 0, 0, nk};      // hi * hi
-    p.M = T;
-    p.n_tiles = c.E / bn;
-    p.out = h->s;
-    p.ldo = c.E;
-    p.col_bias = h->c;
-    CK(launch_tc(p, EPI_ROUTER, bn, std::min(mt * p.n_tiles, h->sms), st));
+  if (h->fused_k1) {
+    mark(h, ST_DOWN, st);
+    mark(h, ST_ROUTER, st);
+    mark(h, ST_K1, st);
+    K1Params kp;
+    memset(&kp, 0, sizeof(kp));
+    kp.tm_s = h->tm_s;
+    kp.tm_x = tm_x;
+    kp.tm_wd = h->tm_k1_wd;
+    kp.tm_hx = h->tm_hx;
+    kp.tm_wr = h->tm_k1_wr;
+    kp.T = T;
+    kp.d = c.d;
+    kp.l = c.l;
+    kp.E = c.E;
+    kp.wd_segments = h->unit_gain ? 1 : 2;
+    kp.eps = c.rms_eps;
+    kp.r = h->r;
+    kp.c = h->c;
+    kp.status = h->status;
+    static unsigned done = 0;
+    CK(ensure_smem_attr(k1_kernel, kK1SmemBytes, done));
+    k1_kernel<<<std::min(mt, h->sms), kTcThreads, kK1SmemBytes, st>>>(kp);
+    CK(cudaGetLastError());
+    h->launches += 1;
+  } else {
+    rms_kernel<bf16><<<(T + 7) / 8, 256, 0, st>>>((const bf16*)x, T, c.d, c.rms_eps, h->r);
+    CK(cudaGetLastError());
+    // h = r * (x Wdown^T), stored as hi | mid | lo bf16 parts
+    mark(h, ST_DOWN, st);
+    {
+      TcParams p = tc_base(h);
+      p.tmA[0] = tm_x;
+      p.tmA[1] = tm_x;
+      const int bn = pick_bn_for(T, c.l, h->sms, 64);
+      p.tmB = h->tm_wdown[bn_index(bn)];
+      p.nseg = h->unit_gain ? 1 : 2;
+      p.seg[0] = {0, 0, 0, c.d / 64};
+      p.seg[1] = {0, 0, c.d, c.d / 64};
+      p.M = T;
+      p.M_rows = T;
+      p.n_tiles = c.l / bn;
+      p.tmOut = h->tm_hx;
+      p.split = c.l;
+      p.row_scale = h->r;
+      CK(launch_tc(p, EPI_DOWN3, bn, std::min(mt * p.n_tiles, h->sms), st));
+    }
+    // s = sigmoid(h Wr^T + c) from six bf16 x bf16 products of the hi/mid/lo parts
+    mark(h, ST_ROUTER, st);
+    {
+      TcParams p = tc_base(h);
+      p.tmA[0] = h->tm_hx;
+      p.tmA[1] = h->tm_hx;
+      const int bn = pick_bn_for(T, c.E, h->sms, 64);
+      p.tmB = h->tm_wr[bn_index(bn)];
+      const int L = c.l, nk = c.l / 64;
+      p.nseg = 6;
+      p.seg[0] = {0, L, L, nk};      // mid * mid
+      p.seg[1] = {0, 2 * L, 0, nk};  // lo * hi
+      p.seg[2] = {0, 0, 2 * L, nk};  // hi * lo
+      p.seg[3] = {0, L, 0, nk};      // mid * hi
+      p.seg[4] = {0, 0, L, nk};      // hi * mid
+      p.seg[5] = {0, 0, 0, nk};      // hi * hi
+      p.M = T;
+      p.M_rows = T;
+      p.n_tiles = c.E / bn;
+      p.tmOut = h->tm_s;
+      p.col_bias = h->c;
+      CK(launch_tc(p, EPI_ROUTER, bn, std::min(mt * p.n_tiles, h->sms), st));
+    }
+    mark(h, ST_K1, st);
+    h->launches += 3;
   }
   int rc = route_from_scores(h, T, flags, st);
   if (rc) return rc;
@@ -488,16 +591,24 @@ int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, 
     TcParams p = tc_base(h);
     p.tmA[0] = tm_x;
     p.tmA[1] = tm_x;
-    const int bn = pick_bn_for(T, 2 * c.hs, h->sms, 128);
-    p.tmB = h->tm_ws13[bn_index(bn)];
     p.nseg = 1;
     p.seg[0] = {0, 0, 0, c.d / 64};
     p.M = T;
-    p.n_tiles = 2 * c.hs / bn;
-    p.out = h->a_s;
-    p.ldo = c.hs;
+    p.M_rows = T;
+    p.tmOut = h->tm_as;
     p.row_scale = h->r;
-    CK(launch_tc(p, EPI_SWIGLU, bn, std::min(mt * p.n_tiles, h->sms), st));
+    const int pbn = T >= 256 * 8 ? pick_pair_bn(T, 2 * c.hs, h->sms) : 0;
+    if (pbn) {  // two-CTA tiles: each CTA loads BN/2 rows of the weights
+      p.tmB = h->tm_ws13[bn_index(pbn / 2)];
+      p.n_tiles = 2 * c.hs / pbn;
+      const int tiles = (T + 255) / 256 * p.n_tiles;
+      CK(launch_tc_pair(p, EPI_SWIGLU, pbn, 2 * std::min(tiles, h->sms / 2), st));
+    } else {
+      const int bn = pick_bn_for(T, 2 * c.hs, h->sms, 128);
+      p.tmB = h->tm_ws13[bn_index(bn)];
+      p.n_tiles = 2 * c.hs / bn;
+      CK(launch_tc(p, EPI_SWIGLU, bn, std::min(mt * p.n_tiles, h->sms), st));
+    }
   }
   // routed experts, grouped over the permuted rows
   mark(h, ST_EXPERT1, st);
@@ -512,10 +623,8 @@ int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, 
     p.n_tiles = 2 * c.h / h->bn_e1;
     p.mtile_table = h->mtiles;
     p.num_mtiles = h->num_mtiles;
-    p.seg_off = h->offsets;
     p.b_rows_per_group = 2 * c.h;
-    p.out = h->act;
-    p.ldo = c.h;
+    p.tmOut = h->tm_act;
     CK(launch_tc(p, EPI_SWIGLU, h->bn_e1, h->sms, st));
   }
   mark(h, ST_EXPERT2, st);
@@ -530,14 +639,12 @@ int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, 
     p.n_tiles = c.l / h->bn_e2;
     p.mtile_table = h->mtiles;
     p.num_mtiles = h->num_mtiles;
-    p.seg_off = h->offsets;
     p.b_rows_per_group = c.l;
-    p.out = h->o;
-    p.ldo = c.l;
+    p.tmOut = h->tm_o;
     CK(launch_tc(p, EPI_BF16, h->bn_e2, h->sms, st));
   }
   mark(h, ST_COMBINE, st);
-  combine_kernel<bf16><<<(T + 7) / 8, 256, 0, st>>>((const bf16*)h->o, h->gates, h->inv, T, c.k, c.l,
+  combine_kernel<bf16><<<(T + 7) / 8, 256, 0, st>>>((const bf16*)h->o, h->gates, h->prow, T, c.k, c.l,
                                                     (bf16*)h->z);
   CK(cudaGetLastError());
   // y = [z | a_s] [W_up | Ws2]^T
@@ -546,18 +653,26 @@ int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, 
     TcParams p = tc_base(h);
     p.tmA[0] = h->tm_z;
     p.tmA[1] = c.hs ? h->tm_as : h->tm_z;
-    const int bn = pick_bn_for(T, c.d, h->sms, 64);
-    p.tmB = h->tm_wy[bn_index(bn)];
     p.nseg = c.hs ? 2 : 1;
     p.seg[0] = {0, 0, 0, c.l / 64};
     p.seg[1] = {1, 0, c.l, c.hs / 64};
     p.M = T;
-    p.n_tiles = c.d / bn;
-    p.out = y;
-    p.ldo = c.d;
-    CK(launch_tc(p, EPI_BF16, bn, std::min(mt * p.n_tiles, h->sms), st));
+    p.M_rows = T;
+    if (!make_map(&p.tmOut, y, T, c.d, c.d, 128)) return LMOE_EINVAL;
+    const int pbn = T >= 256 * 8 ? pick_pair_bn(T, c.d, h->sms) : 0;
+    if (pbn) {
+      p.tmB = h->tm_wy[bn_index(pbn / 2)];
+      p.n_tiles = c.d / pbn;
+      const int tiles = (T + 255) / 256 * p.n_tiles;
+      CK(launch_tc_pair(p, EPI_BF16, pbn, 2 * std::min(tiles, h->sms / 2), st));
+    } else {
+      const int bn = pick_bn_for(T, c.d, h->sms, 64);
+      p.tmB = h->tm_wy[bn_index(bn)];
+      p.n_tiles = c.d / bn;
+      CK(launch_tc(p, EPI_BF16, bn, std::min(mt * p.n_tiles, h->sms), st));
+    }
   }
-  h->launches += 4 + (c.hs ? 2 : 1) + 2;
+  h->launches += (c.hs ? 1 : 0) + 4;
   return LMOE_OK;
 }
 
@@ -589,6 +704,7 @@ int forward_f32(lmoe_handle* h, const void* xv, void* yv, int T, uint32_t flags,
     p.out = h->s; p.ldo = c.E; p.col_bias = h->c;
     CK(launch_simt<SE_ROUTER>(p, mt, st));
   }
+  mark(h, ST_K1, st);
   int rc = route_from_scores(h, T, flags, st);
   if (rc) return rc;
   mark(h, ST_SHARED, st);
@@ -604,27 +720,27 @@ int forward_f32(lmoe_handle* h, const void* xv, void* yv, int T, uint32_t flags,
   mark(h, ST_EXPERT1, st);
   {  // act = silu(A W1_e^T) * (A W3_e^T)
     SimtParams p = b;
-    p.A0 = (const float*)h->a_perm; p.lda0 = c.l; p.K0 = c.l; p.a_rows = T * c.k;
+    p.A0 = (const float*)h->a_perm; p.lda0 = c.l; p.K0 = c.l; p.a_rows = (int)h->rows_pad;
     p.B0 = (const float*)h->w13; p.B1 = (const float*)h->w3f; p.ldb = c.l;
     p.b_group_stride = (long long)c.h * c.l;
     p.N = c.h; p.grouped = 1;
-    p.mtile_table = h->mtiles; p.num_mtiles = h->num_mtiles; p.seg_off = h->offsets;
+    p.mtile_table = h->mtiles; p.num_mtiles = h->num_mtiles;
     p.out = (float*)h->act; p.ldo = c.h;
     CK(launch_simt<SE_SWIGLU>(p, gm, st));
   }
   mark(h, ST_EXPERT2, st);
   {  // o = act W2_e^T
     SimtParams p = b;
-    p.A0 = (const float*)h->act; p.lda0 = c.h; p.K0 = c.h; p.a_rows = T * c.k;
+    p.A0 = (const float*)h->act; p.lda0 = c.h; p.K0 = c.h; p.a_rows = (int)h->rows_pad;
     p.B0 = (const float*)h->w2; p.ldb = c.h;
     p.b_group_stride = (long long)c.l * c.h;
     p.N = c.l; p.grouped = 1;
-    p.mtile_table = h->mtiles; p.num_mtiles = h->num_mtiles; p.seg_off = h->offsets;
+    p.mtile_table = h->mtiles; p.num_mtiles = h->num_mtiles;
     p.out = (float*)h->o; p.ldo = c.l;
     CK(launch_simt<SE_STORE>(p, gm, st));
   }
   mark(h, ST_COMBINE, st);
-  combine_kernel<float><<<(T + 7) / 8, 256, 0, st>>>((const float*)h->o, h->gates, h->inv, T, c.k, c.l,
+  combine_kernel<float><<<(T + 7) / 8, 256, 0, st>>>((const float*)h->o, h->gates, h->prow, T, c.k, c.l,
                                                      (float*)h->z);
   CK(cudaGetLastError());
   mark(h, ST_UP, st);
@@ -779,6 +895,7 @@ static void size_handle(lmoe_handle* h, const lmoe_config* cfg) {
   h->nblk_max = (cfg->max_tokens + kTokBlock - 1) / kTokBlock;
   h->max_mtiles = (int)(((long long)cfg->max_tokens * cfg->k + kTileRows - 1) / kTileRows) + cfg->E;
   h->ld_bins = (cfg->max_tokens + 31) / 32 * 32;
+  h->rows_pad = (long long)cfg->max_tokens * cfg->k + (long long)kTileRows * cfg->E;
 }
 
 int lmoe_workspace_bytes(const lmoe_config* cfg, size_t* bytes) {
@@ -1002,18 +1119,24 @@ int lmoe_gemm_bf16(const void* a, const void* b, float* c, int32_t M, int32_t N,
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int bn = pick_bn(N);
+  const bool pair = M >= 256 && bn >= 128;  // the two-CTA variant, so tests exercise it
   TcParams p;
   memset(&p, 0, sizeof(p));
-  if (!make_map(&p.tmA[0], a, M, K, K, 128) || !make_map(&p.tmB, b, N, K, K, bn)) return LMOE_EINVAL;
+  if (!make_map(&p.tmA[0], a, M, K, K, 128) || !make_map(&p.tmB, b, N, K, K, pair ? bn / 2 : bn)) return LMOE_EINVAL;
   p.tmA[1] = p.tmA[0];
   p.nseg = 1;
   p.seg[0] = {0, 0, 0, K / 64};
   p.M = M;
+  p.M_rows = M;
   p.n_tiles = N / bn;
-  p.out = c;
-  p.ldo = N;
-  const int tiles = ((M + 127) / 128) * p.n_tiles;
-  CK(launch_tc(p, EPI_F32, bn, tiles < sms ? tiles : sms, (cudaStream_t)stream));
+  if (!make_map_f32(&p.tmOut, c, M, N, N, 128)) return LMOE_EINVAL;
+  if (pair) {
+    const int tiles = ((M + 255) / 256) * p.n_tiles;
+    CK(launch_tc_pair(p, EPI_F32, bn, 2 * (tiles < sms / 2 ? tiles : sms / 2), (cudaStream_t)stream));
+  } else {
+    const int tiles = ((M + 127) / 128) * p.n_tiles;
+    CK(launch_tc(p, EPI_F32, bn, tiles < sms ? tiles : sms, (cudaStream_t)stream));
+  }
   return LMOE_OK;
 }
 
@@ -1024,7 +1147,8 @@ int lmoe_gemm_bf16(const void* a, const void* b, float* c, int32_t M, int32_t N,
 static __device__ __align__(256) unsigned char g_noalloc_scratch[LMOE_NOALLOC_SCRATCH_BYTES];
 
 static size_t noalloc_bytes(long long T, long long E, long long k, size_t* off_rank, size_t* off_cnt,
-                            size_t* off_base, size_t* off_tiles, size_t* off_ntiles) {
+                            size_t* off_base, size_t* off_tiles, size_t* off_delta, size_t* off_c32,
+                            size_t* off_ntiles) {
   const long long nblk = (T + kTokBlock - 1) / kTokBlock;
   const long long mtiles = (T * k + kTileRows - 1) / kTileRows + E;
   size_t o = 0;
@@ -1036,6 +1160,10 @@ static size_t noalloc_bytes(long long T, long long E, long long k, size_t* off_r
   o += align_up((size_t)(nblk * E) * 4, 256);
   *off_tiles = o;
   o += align_up((size_t)mtiles * 8, 256);
+  *off_delta = o;
+  o += align_up((size_t)E * 4, 256);
+  *off_c32 = o;
+  o += align_up((size_t)kCountCopies * E * 4, 256);
   *off_ntiles = o;
   o += 256;
   return o;
@@ -1046,8 +1174,9 @@ int lmoe_route_noalloc(const float* scores, const float* bias, int32_t T, int32_
                        void* stream) {
   if (!scores || !bias || !idx || !gates || !counts || !offsets || !perm || !inv) return LMOE_EINVAL;
   if (T < 0 || E <= 0 || E > 1024 || k <= 0 || k > E || k > 32) return LMOE_EINVAL;
-  size_t o_rank, o_cnt, o_base, o_tiles, o_ntiles;
-  if (noalloc_bytes(T, E, k, &o_rank, &o_cnt, &o_base, &o_tiles, &o_ntiles) > LMOE_NOALLOC_SCRATCH_BYTES)
+  size_t o_rank, o_cnt, o_base, o_tiles, o_delta, o_c32, o_ntiles;
+  if (noalloc_bytes(T, E, k, &o_rank, &o_cnt, &o_base, &o_tiles, &o_delta, &o_c32, &o_ntiles) >
+      LMOE_NOALLOC_SCRATCH_BYTES)
     return LMOE_EUNSUPPORTED;
   // set-up, once per device: the device address of the scratch array
   static std::mutex mu;
@@ -1069,8 +1198,8 @@ int lmoe_route_noalloc(const float* scores, const float* bias, int32_t T, int32_
     base = base_of[dev];
   }
   cudaStream_t st = (cudaStream_t)stream;
-  CK(cudaMemsetAsync(counts, 0, (size_t)E * sizeof(int32_t), st));  // summed with atomics
   if (T == 0) {
+    CK(cudaMemsetAsync(counts, 0, (size_t)E * sizeof(int32_t), st));
     CK(cudaMemsetAsync(offsets, 0, (size_t)(E + 1) * sizeof(int32_t), st));
     return LMOE_OK;
   }
@@ -1078,18 +1207,47 @@ int lmoe_route_noalloc(const float* scores, const float* bias, int32_t T, int32_
   int* blkcnt = reinterpret_cast<int*>(base + o_cnt);
   int* blkbase = reinterpret_cast<int*>(base + o_base);
   int2* tiles = reinterpret_cast<int2*>(base + o_tiles);
+  int* delta = reinterpret_cast<int*>(base + o_delta);
+  int* counts32 = reinterpret_cast<int*>(base + o_c32);
   int* ntiles = reinterpret_cast<int*>(base + o_ntiles);
   uint32_t* status = reinterpret_cast<uint32_t*>(base + o_ntiles + 128);
-  // every scratch word is written before it is read, except the status word
+  // every scratch word is written before it is read, except the status word and the count copies,
+  // which the top-k blocks add into
   CK(cudaMemsetAsync(status, 0, sizeof(uint32_t), st));
-  TopkArgs ta{scores, bias, T, E, k, idx, rank, blkcnt, counts, gates, nullptr, 0, status};
+  CK(cudaMemsetAsync(counts32, 0, (size_t)kCountCopies * E * sizeof(int), st));
+  TopkArgs ta{scores, bias, T, E, k, idx, rank, blkcnt, counts32, gates, nullptr, 0, status};
   CK(launch_topk(ta, st));
   const int nblk = (T + kTokBlock - 1) / kTokBlock;
-  plan_kernel<<<(E + 31) / 32, 1024, 0, st>>>(counts, blkcnt, nblk, E, offsets, blkbase, tiles, ntiles);
+  plan_kernel<<<(E + 31) / 32, 1024, 0, st>>>(counts32, counts, blkcnt, nblk, E, offsets, delta, blkbase, tiles,
+                                               ntiles);
   CK(cudaGetLastError());
   const int pairs = T * k;
-  gather_kernel<float><<<(pairs + 7) / 8, 256, 0, st>>>(nullptr, 0, 0, idx, rank, blkbase, T, E, k, perm, inv,
-                                                        nullptr, status);
+  gather_kernel<float><<<(pairs + 8 * kGatherPairs - 1) / (8 * kGatherPairs), 256, 0, st>>>(
+      nullptr, 0, 0, idx, rank, blkbase, nullptr, T, E, k, perm, inv, nullptr, nullptr, status);
+  CK(cudaGetLastError());
+  return LMOE_OK;
+}
+
+// ---------------------------------------------------------------- failure-detection check
+// One thread waits, with the pipelines' bounded wait, on an mbarrier that nothing ever completes.
+__global__ void watchdog_selftest_kernel(uint32_t* status, long long limit_cycles) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (!mbar_wait(&bar, 0, &abort_flag, status, limit_cycles)) set_status(status, LMOE_STATUS_WATCHDOG);
+  }
+}
+
+int lmoe_watchdog_selftest(uint32_t* status_dev, int32_t limit_us, void* stream) {
+  if (!status_dev || limit_us <= 0 || limit_us > 2000000) return LMOE_EINVAL;
+  // ~2000 SM cycles per microsecond at B200 clocks; the exact bound only has to be finite
+  watchdog_selftest_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(status_dev, (long long)limit_us * 2000);
   CK(cudaGetLastError());
   return LMOE_OK;
 }

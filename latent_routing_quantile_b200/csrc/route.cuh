@@ -10,6 +10,7 @@
 namespace lmoe {
 
 constexpr int kTokBlock = 32;      // tokens per routing block: one rank-mask word per expert
+constexpr int kCountCopies = 32;   // per-expert counts are summed into this many copies (block % 32)
 constexpr int kTileRows = 128;     // rows per grouped-GEMM M-tile
 constexpr unsigned kFull = 0xffffffffu;
 
@@ -63,7 +64,7 @@ template <int NJ>
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ s, const float* __restrict__ bias,
                                                    int ntok, int E, int k, int* __restrict__ idx,
                                                    float* __restrict__ gates, int* __restrict__ rank,
-                                                   int* __restrict__ blkcnt, int* __restrict__ counts,
+                                                   int* __restrict__ blkcnt, int* __restrict__ counts32,
                                                    uint16_t* __restrict__ bins, int ld_bins, uint32_t* status) {
   constexpr int TPW = kTokBlock / 8;  // tokens per warp
   constexpr int PF = topk_prefetch(NJ);
@@ -168,10 +169,11 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ s, 
     if (t >= ntok) break;
     if (lane < k) rank[(size_t)t * k + lane] = __popc(mask[sel_q[q]] & ((1u << tl) - 1u));
   }
+  int* ccopy = counts32 + (size_t)(blk & (kCountCopies - 1)) * E;
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     const int c = __popc(mask[e]);
     blkcnt[(size_t)blk * E + e] = c;
-    if (c) atomicAdd(&counts[e], c);
+    if (c) atomicAdd(&ccopy[e], c);
   }
   if (bins) {
     // expert-major store: one warp writes 32 tokens (64 bytes) of one expert per step
@@ -209,28 +211,42 @@ __device__ __forceinline__ int block_exclusive_scan_1024(int v, int* sh /*[32]*/
   return incl - v;
 }
 
-// Grid: ceil(E/32) blocks of 1024 threads.  Every block recomputes the expert offsets (the
-// exclusive scan of counts); block 0 stores them and the grouped-GEMM tile table; each block
-// then fills blkbase[b][e] = off[e] + sum_{b' < b} blkcnt[b'][e] for its 32 experts.
-__global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ counts,
+// Grid: ceil(E/32) blocks of 1024 threads.  Every block sums the 32 count copies and recomputes
+// the expert offsets (their exclusive scan); block 0 stores counts, offsets, the grouped-GEMM
+// tile table and pad_delta;
+// each block then fills blkbase[b][e] = off[e] + sum_{b' < b} blkcnt[b'][e] for its 32 experts.
+// The grouped GEMMs use a padded row layout: expert e's rows start at pad_off[e], the exclusive
+// scan of counts rounded up to kTileRows, so no 128-row tile holds rows of two experts; a
+// permuted row pos of expert e sits at row pos + pad_delta[e] of that layout.
+__global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ counts32, int* __restrict__ counts,
                                                     const int* __restrict__ blkcnt, int nblk, int E,
-                                                    int* __restrict__ offsets, int* __restrict__ blkbase,
-                                                    int2* __restrict__ mtiles, int* __restrict__ num_mtiles) {
+                                                    int* __restrict__ offsets, int* __restrict__ pad_delta,
+                                                    int* __restrict__ blkbase, int2* __restrict__ mtiles,
+                                                    int* __restrict__ num_mtiles) {
   __shared__ int sh[32];
   __shared__ int s_off[1024];
   __shared__ int part[32][33];
   const int tid = threadIdx.x;
-  const int c = tid < E ? counts[tid] : 0;
+  int c = 0;
+  if (tid < E) {
+#pragma unroll 8
+    for (int j = 0; j < kCountCopies; ++j) c += counts32[(size_t)j * E + tid];
+  }
   int total;
   const int off = block_exclusive_scan_1024(c, sh, &total);
   s_off[tid] = off;
   if (blockIdx.x == 0) {
-    if (tid < E) offsets[tid] = off;
+    if (tid < E) {
+      offsets[tid] = off;
+      counts[tid] = c;
+    }
     if (tid == 0) offsets[E] = total;
     const int mt = (c + kTileRows - 1) / kTileRows;
     int mt_total;
     const int mt_start = block_exclusive_scan_1024(mt, sh, &mt_total);
-    for (int j = 0; j < mt; ++j) mtiles[mt_start + j] = make_int2(tid, off + j * kTileRows);
+    const int poff = mt_start * kTileRows;  // padded offset of this expert
+    if (tid < E) pad_delta[tid] = poff - off;
+    for (int j = 0; j < mt; ++j) mtiles[mt_start + j] = make_int2(tid, poff + j * kTileRows);
     if (tid == 0) *num_mtiles = mt_total;
   }
   __syncthreads();
@@ -256,33 +272,59 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ coun
 
 // --------------------------------------------------------------------------- gather
 // One warp per (token, slot): its permuted row pos = blkbase[block][e] + rank; records
-// perm[pos] = token and inv[(t, i)] = pos, and copies the token's latent row into A_perm[pos].
+// perm[pos] = token and inv[(t, i)] = pos, and copies the token's latent row into the padded
+// expert layout at row prow[(t, i)] = pos + pad_delta[e] (prow and dst may be null: then only the
+// permutation is written).
+constexpr int kGatherPairs = 4;  // (token, slot) pairs per warp, their row copies issued together
+
 template <typename T>
 __global__ void __launch_bounds__(256) gather_kernel(const T* __restrict__ src, int ld_src, int l,
                                                      const int* __restrict__ idx, const int* __restrict__ rank,
-                                                     const int* __restrict__ blkbase, int ntok, int E, int k,
+                                                     const int* __restrict__ blkbase,
+                                                     const int* __restrict__ pad_delta, int ntok, int E, int k,
                                                      int* __restrict__ perm, int* __restrict__ inv,
-                                                     T* __restrict__ dst, uint32_t* status) {
-  const int pair = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-  if (pair >= ntok * k) return;
-  const int t = pair / k, e = idx[pair];
-  if (e < 0 || e >= E) {
-    if (lane == 0) set_status(status, LMOE_STATUS_BAD_INDEX);
-    return;
+                                                     int* __restrict__ prow, T* __restrict__ dst,
+                                                     uint32_t* status) {
+  const int lane = threadIdx.x & 31;
+  const int pair0 = (blockIdx.x * 8 + (threadIdx.x >> 5)) * kGatherPairs;
+  const int npairs = ntok * k;
+  // lanes 0..3 resolve one pair each
+  int t = -1, prow_v = 0;
+  if (lane < kGatherPairs && pair0 + lane < npairs) {
+    const int pair = pair0 + lane;
+    const int tt = pair / k, e = idx[pair];
+    if (e < 0 || e >= E) {
+      set_status(status, LMOE_STATUS_BAD_INDEX);
+    } else {
+      const int pos = blkbase[(size_t)(tt / kTokBlock) * E + e] + rank[pair];
+      if (pos < 0 || pos >= npairs) {
+        set_status(status, LMOE_STATUS_BAD_INDEX);
+      } else {
+        t = tt;
+        prow_v = pad_delta ? pos + pad_delta[e] : pos;
+        inv[pair] = pos;
+        perm[pos] = tt;
+        if (prow) prow[pair] = prow_v;
+      }
+    }
   }
-  const int pos = blkbase[(size_t)(t / kTokBlock) * E + e] + rank[pair];
-  if (pos < 0 || pos >= ntok * k) {
-    if (lane == 0) set_status(status, LMOE_STATUS_BAD_INDEX);
-    return;
-  }
-  if (lane == 0) {
-    inv[pair] = pos;
-    perm[pos] = t;
-  }
+  if (!dst) return;
   constexpr int VEC = 16 / sizeof(T);
-  const uint4* s4 = reinterpret_cast<const uint4*>(src + (size_t)t * ld_src);
-  uint4* d4 = reinterpret_cast<uint4*>(dst + (size_t)pos * l);
-  for (int v = lane; v < l / VEC; v += 32) d4[v] = s4[v];
+  int ts[kGatherPairs], rows[kGatherPairs];
+#pragma unroll
+  for (int j = 0; j < kGatherPairs; ++j) {
+    ts[j] = __shfl_sync(kFull, t, j);
+    rows[j] = __shfl_sync(kFull, prow_v, j);
+  }
+  for (int v = lane; v < l / VEC; v += 32) {
+    uint4 q[kGatherPairs];
+#pragma unroll
+    for (int j = 0; j < kGatherPairs; ++j)
+      if (ts[j] >= 0) q[j] = reinterpret_cast<const uint4*>(src + (size_t)ts[j] * ld_src)[v];
+#pragma unroll
+    for (int j = 0; j < kGatherPairs; ++j)
+      if (ts[j] >= 0) reinterpret_cast<uint4*>(dst + (size_t)rows[j] * l)[v] = q[j];
+  }
 }
 
 // --------------------------------------------------------------------------- QB histogram
@@ -318,25 +360,39 @@ __global__ void __launch_bounds__(512) hist_kernel(const uint16_t* __restrict__ 
 }
 
 // --------------------------------------------------------------------------- combine
-// z_t = sum_i g_ti o[inv[t, i]] in rank order, fp32 accumulation; one warp per token.
+// z_t = sum_i g_ti o[prow[t, i]] in rank order (prow: the pair's row in the padded expert layout),
+// fp32 accumulation; one warp per token.
 template <typename T>
 __global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ o, const float* __restrict__ gates,
-                                                      const int* __restrict__ inv, int ntok, int k, int l,
+                                                      const int* __restrict__ prow, int ntok, int k, int l,
                                                       T* __restrict__ z) {
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (t >= ntok) return;
   constexpr int VEC = 16 / sizeof(T);
+  // lane i < k holds slot i's gate and row
+  const float g_l = lane < k ? gates[(size_t)t * k + lane] : 0.f;
+  const int r_l = lane < k ? prow[(size_t)t * k + lane] : 0;
   for (int v = lane; v < l / VEC; v += 32) {
     float acc[VEC];
 #pragma unroll
     for (int j = 0; j < VEC; ++j) acc[j] = 0.f;
-    for (int i = 0; i < k; ++i) {
-      const float g = gates[(size_t)t * k + i];
-      const int row = inv[(size_t)t * k + i];
-      uint4 q = reinterpret_cast<const uint4*>(o + (size_t)row * l)[v];
-      const T* e = reinterpret_cast<const T*>(&q);
+    for (int i0 = 0; i0 < k; i0 += 8) {
+      uint4 q[8];
+      float g[8];
 #pragma unroll
-      for (int j = 0; j < VEC; ++j) acc[j] = fmaf(g, to_f<T>(e[j]), acc[j]);
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u;
+        const int row = __shfl_sync(kFull, r_l, i & 31);
+        g[u] = __shfl_sync(kFull, g_l, i & 31);
+        if (i < k) q[u] = reinterpret_cast<const uint4*>(o + (size_t)row * l)[v];
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (i0 + u >= k) break;
+        const T* e = reinterpret_cast<const T*>(&q[u]);
+#pragma unroll
+        for (int j = 0; j < VEC; ++j) acc[j] = fmaf(g[u], to_f<T>(e[j]), acc[j]);
+      }
     }
     uint4 out;
     T* oe = reinterpret_cast<T*>(&out);

@@ -1,8 +1,9 @@
 // fp32 FFMA GEMM for the fp32 layer configuration: C = A B^T with both operands K-contiguous.
 // Tensor-core tf32 keeps 10 mantissa bits, which cannot meet fp32 accuracy, so the fp32 layer
 // runs its products here.  Tile 128 x 32 x 32, 256 threads, 4 x 4 outputs per thread.
-// Same A/B conventions and grouped-tile table as the tensor-core engine; an optional second B
-// operand (dual mode) gives the gate and linear halves of a SwiGLU in one pass.
+// Same A/B conventions and grouped-tile table (padded expert layout) as the tensor-core engine;
+// an optional second B operand (dual mode) gives the gate and linear halves of a SwiGLU in one
+// pass.
 #pragma once
 
 #include "common.cuh"
@@ -29,7 +30,6 @@ struct SimtParams {
   int grouped;
   const int2* mtile_table;
   const int* num_mtiles;
-  const int* seg_off;
   float* out;
   int ldo;
   const float* row_scale;
@@ -51,7 +51,7 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const SimtParams p) {
     int2 er = p.mtile_table[blockIdx.y];
     e = er.x;
     row0 = er.y;
-    row_end = p.seg_off[e + 1];
+    row_end = row0 + BM;  // padded expert layout: the whole tile belongs to expert e
   } else {
     row0 = blockIdx.y * BM;
     row_end = p.M;

@@ -5,13 +5,17 @@
 // tcgen05.mma (one thread) into one of two TMEM accumulators, warps 2-9 drain the other
 // accumulator (tcgen05.ld) through the epilogue while the next tile is multiplied.  Two
 // epilogue warps share each TMEM lane quarter and split its columns, so the element-wise
-// epilogue math keeps pace with the tensor core.  Tiles are
+// epilogue math keeps pace with the tensor core.  Results leave through shared memory: each
+// step the epilogue warps fill one 16 KB box (128 rows x 128 bytes, 128-byte swizzle) of a
+// two-box staging ring and warp 2 issues a TMA tensor store of it, so global writes are whole
+// lines instead of one 16-byte piece per row per thread.  Tiles are
 // 128 x BN, K steps of 64 (one 128-byte swizzle atom).  The grid is at most one CTA per SM and
 // walks the tile list with a stride of gridDim.x.
 //
 // Grouped mode (routed experts): M-tiles come from a device table of (expert, first row) built
-// after the routing counts, B rows are offset by expert * b_rows_per_group, and rows past the
-// expert's segment end are computed but never stored.
+// after the routing counts, and B rows are offset by expert * b_rows_per_group.  Every expert's
+// rows start on a multiple of 128, so a tile never holds rows of two experts; the padding rows
+// are computed and stored but never read.
 //
 // K is described by up to 6 segments, each naming which A tensor map and which A and B columns
 // its k-blocks read; this expresses concatenated-K products ([z | a_s] [W_up | Ws2]^T) and the
@@ -41,6 +45,7 @@ struct KSeg {
 struct TcParams {
   CUtensorMap tmA[2];
   CUtensorMap tmB;
+  CUtensorMap tmOut;          // output: box 64 x 128 (bf16) or 32 x 128 (fp32), 128-byte swizzle
   KSeg seg[6];
   int nseg;
   int grouped;
@@ -48,59 +53,61 @@ struct TcParams {
   int n_tiles;                // N / BN
   const int2* mtile_table;    // grouped: (expert, first row)
   const int* num_mtiles;      // grouped: number of table entries (device)
-  const int* seg_off;         // grouped: expert row offsets [E+1]
   int b_rows_per_group;       // grouped: B rows per expert
-  void* out;
-  int ldo;                    // output row pitch in elements
-  int split;                  // EPI_DOWN3: width of each of the three parts
+  int M_rows;                 // rows whose row_scale may be read (non-grouped: M)
+  int split;                  // EPI_DOWN3: column offset between the three parts
   const float* row_scale;
   const float* col_bias;
   uint32_t* status;
 };
 
-template <int BN>
+// PAIR = 1: a cluster of two CTAs computes one 256 x BN tile with tcgen05.mma.cta_group::2; each
+// CTA holds 128 rows of A and BN/2 rows of B per stage.
+template <int BN, int PAIR = 0>
 struct TcCfg {
   static constexpr int kABytes = 128 * 128;              // 128 rows x 64 bf16
-  static constexpr int kBBytes = BN * 128;
+  static constexpr int kBBytes = (PAIR ? BN / 2 : BN) * 128;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kStages = (192 * 1024) / kStageBytes;
   static constexpr int kTmemCols = 2 * BN;
-  static constexpr int kBarOffset = kStages * kStageBytes;
+  static constexpr int kOutOffset = kStages * kStageBytes;    // two 16 KB output boxes
+  static constexpr int kBarOffset = kOutOffset + 2 * 16384;
   static constexpr int kSmemBytes = kBarOffset + 256 + 1024;  // barriers + alignment slack
 };
 
 struct TileInfo {
-  int row0, row_end, b_row0, n0;
+  int row0, b_row0, n0;
 };
 
-__device__ __forceinline__ TileInfo tc_tile(const TcParams& p, int tile, int BN) {
+__device__ __forceinline__ TileInfo tc_tile(const TcParams& p, int tile, int BN, int pair, uint32_t rank) {
   TileInfo ti;
   int mt = tile / p.n_tiles, nt = tile - mt * p.n_tiles;
   ti.n0 = nt * BN;
-  if (p.grouped) {
+  if (pair) {  // 256-row tiles; this CTA owns rows 128*rank.. and B rows BN/2*rank..
+    ti.row0 = mt * 256 + (int)rank * 128;
+    ti.b_row0 = ti.n0 + (int)rank * (BN / 2);
+  } else if (p.grouped) {
     int2 e_r = p.mtile_table[mt];
     ti.row0 = e_r.y;
-    ti.row_end = p.seg_off[e_r.x + 1];
     ti.b_row0 = e_r.x * p.b_rows_per_group + ti.n0;
   } else {
     ti.row0 = mt * 128;
-    ti.row_end = p.M;
     ti.b_row0 = ti.n0;
   }
   return ti;
 }
 
-__device__ __forceinline__ int tc_num_tiles(const TcParams& p) {
-  int mt = p.grouped ? *p.num_mtiles : (p.M + 127) / 128;
+__device__ __forceinline__ int tc_num_tiles(const TcParams& p, int pair) {
+  int mt = p.grouped ? *p.num_mtiles : (pair ? (p.M + 255) / 256 : (p.M + 127) / 128);
   return mt * p.n_tiles;
 }
 
 constexpr int kEpiWarps = 8;
 constexpr int kTcThreads = 64 + 32 * kEpiWarps;
 
-template <int BN, int EPI>
+template <int BN, int EPI, int PAIR>
 __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_constant__ TcParams p) {
-  using C = TcCfg<BN>;
+  using C = TcCfg<BN, PAIR>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
@@ -109,11 +116,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
   uint64_t* empty = full + S;
   uint64_t* tfull = empty + S;
   uint64_t* tempty = tfull + 2;
-  uint64_t* drain = tempty + 2;
+  uint64_t* bfull = tempty + 2;   // output box written by all epilogue warps
+  uint64_t* bfree = bfull + 2;    // output box read by its TMA store
+  uint64_t* drain = bfree + 2;
+  uint8_t* obox = smem + C::kOutOffset;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;  // 0 = the pair's MMA issuer
+  const bool leader = rank == 0;
+  // pairs walk the tile list together: pair index and count
+  const int first = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int stride = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(&full[i], 1);
@@ -121,7 +136,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], kEpiWarps);
+      mbar_init(&tempty[i], PAIR ? 2 * kEpiWarps : kEpiWarps);
+      mbar_init(&bfull[i], kEpiWarps);
+      mbar_init(&bfree[i], 1);
     }
     mbar_init(drain, 1);
     *abort = 0;
@@ -129,16 +146,23 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     tma_prefetch_desc(&p.tmA[0]);
     tma_prefetch_desc(&p.tmA[1]);
     tma_prefetch_desc(&p.tmB);
+    tma_prefetch_desc(&p.tmOut);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::kTmemCols);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, C::kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, C::kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync_all();  // the peer's barriers exist before any remote signal
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int num_tiles = tc_num_tiles(p);
+  const int num_tiles = tc_num_tiles(p, PAIR);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -147,8 +171,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       uint32_t phase = 0;
       uint32_t armed = 0, armed_parity = 0;  // per-stage bits, for the abort drain
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-        TileInfo ti = tc_tile(p, tile, BN);
+      for (int tile = first; ok && tile < num_tiles; tile += stride) {
+        TileInfo ti = tc_tile(p, tile, BN, PAIR, rank);
         for (int s = 0; ok && s < p.nseg; ++s) {
           const KSeg sg = p.seg[s];
           for (int kb = 0; kb < sg.nkb; ++kb) {
@@ -158,9 +182,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             }
             uint8_t* a_dst = smem + stage * C::kStageBytes;
             uint8_t* b_dst = a_dst + C::kABytes;
-            mbar_expect_tx(&full[stage], C::kStageBytes);
-            tma_load_2d(a_dst, &p.tmA[sg.a_map], &full[stage], sg.a_col + kb * 64, ti.row0);
-            tma_load_2d(b_dst, &p.tmB, &full[stage], sg.b_col + kb * 64, ti.b_row0);
+            if constexpr (PAIR) {
+              // both CTAs' bytes complete the leader's full barrier; the leader expects all of them
+              const uint32_t bar0 = mapa_shared(smem_u32(&full[stage]), 0);
+              if (leader) mbar_expect_tx(&full[stage], 2 * C::kStageBytes);
+              tma_load_2d_pair(a_dst, &p.tmA[sg.a_map], bar0, sg.a_col + kb * 64, ti.row0);
+              tma_load_2d_pair(b_dst, &p.tmB, bar0, sg.b_col + kb * 64, ti.b_row0);
+            } else {
+              mbar_expect_tx(&full[stage], C::kStageBytes);
+              tma_load_2d(a_dst, &p.tmA[sg.a_map], &full[stage], sg.a_col + kb * 64, ti.row0);
+              tma_load_2d(b_dst, &p.tmB, &full[stage], sg.b_col + kb * 64, ti.b_row0);
+            }
             armed |= 1u << stage;
             armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
             if (++stage == S) {
@@ -170,21 +202,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
           }
         }
       }
-      if (!ok) {
-        // let every load this thread issued land before the CTA's shared memory is released
+      if (!ok && leader) {
+        // let every load issued land before shared memory is released (for a pair, the leader's
+        // barriers count both CTAs' loads, and the final cluster barrier holds the peer)
         for (int i = 0; i < S; ++i)
           if ((armed >> i) & 1u) mbar_drain(&full[i], (armed_parity >> i) & 1u);
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- MMA issuer
-      constexpr uint32_t idesc = idesc_bf16_f32(BN);
+    if (lane == 0 && leader) {
+      // ---------------- MMA issuer (the even CTA of a pair issues for both)
+      constexpr uint32_t idesc = idesc_bf16_f32(BN, PAIR ? 256 : 128);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++it) {
+      for (int tile = first; ok && tile < num_tiles; tile += stride, ++it) {
         const int acc = it & 1;
         const uint32_t acc_phase = (it >> 1) & 1;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort, p.status)) {
@@ -206,21 +239,36 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             const uint32_t b_addr = a_addr + C::kABytes;
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              tc_mma_bf16(d_tmem, smem_desc_sw128(a_addr + k * 32), smem_desc_sw128(b_addr + k * 32),
-                          idesc, (kbi | k) != 0);
+              if constexpr (PAIR)
+                tc_mma_bf16_pair(d_tmem, smem_desc_sw128(a_addr + k * 32), smem_desc_sw128(b_addr + k * 32), idesc,
+                                 (kbi | k) != 0);
+              else
+                tc_mma_bf16(d_tmem, smem_desc_sw128(a_addr + k * 32), smem_desc_sw128(b_addr + k * 32), idesc,
+                            (kbi | k) != 0);
             }
-            tc_commit(&empty[stage]);
+            if constexpr (PAIR)
+              tc_commit_pair(&empty[stage]);
+            else
+              tc_commit(&empty[stage]);
             if (++stage == S) {
               stage = 0;
               phase ^= 1u;
             }
           }
         }
-        if (ok) tc_commit(&tfull[acc]);
+        if (ok) {
+          if constexpr (PAIR)
+            tc_commit_pair(&tfull[acc]);
+          else
+            tc_commit(&tfull[acc]);
+        }
       }
       if (!ok) {
         // wait (bounded) for the MMAs already issued before TMEM is released
-        tc_commit(drain);
+        if constexpr (PAIR)
+          tc_commit_pair(drain);
+        else
+          tc_commit(drain);
         mbar_drain(drain, 0);
       }
     }
@@ -228,121 +276,169 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     // ---------------- epilogue warps 2..9: TMEM lane quarter (warp % 4), column half (warp-2)/4
     const int wq = warp & 3;
     const int half_id = (warp - 2) >> 2;
+    const int rl = wq * 32 + lane;          // row of the tile this thread owns
+    const bool storer = (warp == 2);        // warp 2 issues the TMA stores
     int it = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+    uint32_t step = 0;                      // output boxes so far (alternating staging buffers)
+    bool ok = true;
+    // Writes this thread's 64 bytes into the current box, then (storer) stores the box.
+    auto emit = [&](const uint32_t (&w)[16], int x, int y) -> bool {
+      const int buf = step & 1;
+      const uint32_t par = (step >> 1) & 1u;
+      bool good = mbar_wait(&bfree[buf], par ^ 1u, abort, p.status);
+      __syncwarp();
+      if (__any_sync(0xffffffffu, !good)) return false;
+      uint8_t* box = obox + buf * 16384;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<uint4*>(box + sw128_offset(rl, half_id * 4 + q)) =
+            make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bfull[buf]);
+      if (storer) {
+        good = mbar_wait(&bfull[buf], par, abort, p.status);
+        __syncwarp();
+        if (__any_sync(0xffffffffu, !good)) return false;
+        if (lane == 0) {
+          tma_store_2d(&p.tmOut, box, x, y);
+          bulk_commit();
+          if (step > 0) {
+            bulk_wait_read<1>();  // the previous box has been read: its buffer is free
+            mbar_arrive(&bfree[(step - 1) & 1]);
+          }
+        }
+        __syncwarp();
+      }
+      ++step;
+      return true;
+    };
+    for (int tile = first; ok && tile < num_tiles; tile += stride, ++it) {
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
-      bool ok = mbar_wait(&tfull[acc], acc_phase, abort, p.status);
+      float c_lane[BN / 32];  // router column offsets of this tile, one per lane and step
+      if constexpr (EPI == EPI_ROUTER) {
+        const int n0 = (tile % p.n_tiles) * BN;
+#pragma unroll
+        for (int j = 0; j < BN / 32; ++j) c_lane[j] = p.col_bias[n0 + j * 32 + lane];
+      } else {
+#pragma unroll
+        for (int j = 0; j < BN / 32; ++j) c_lane[j] = 0.f;
+      }
+      ok = mbar_wait(&tfull[acc], acc_phase, abort, p.status);
       __syncwarp();
-      if (__any_sync(0xffffffffu, !ok)) break;
+      if (__any_sync(0xffffffffu, !ok)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
-      TileInfo ti = tc_tile(p, tile, BN);
-      const int row = ti.row0 + wq * 32 + lane;
-      const bool valid = row < ti.row_end;
+      TileInfo ti = tc_tile(p, tile, BN, PAIR, rank);
+      const int row = ti.row0 + rl;
       const uint32_t tbase = tmem_base + ((uint32_t)(wq * 32) << 16) + acc * BN;
-      const float rs = (p.row_scale != nullptr && valid) ? p.row_scale[row] : 1.0f;
+      const float rs = (p.row_scale != nullptr && row < p.M_rows) ? p.row_scale[row] : 1.0f;
+      uint32_t w[16];
 
       if constexpr (EPI == EPI_SWIGLU) {
-        // item i = (group g = i / 2, part = i % 2): gate columns g*128 + part*32 .. +31, linear
-        // columns 64 further; items alternate between the two warps of a lane quarter
+        // step j: output columns n0/2 + j*64 .. +63; this warp's 32 of them come from gate
+        // columns j*128 + half*32 and linear columns 64 further
 #pragma unroll 1
-        for (int item = half_id; item < BN / 64; item += 2) {
-          const int g = item >> 1, part = item & 1;
+        for (int j = 0; ok && j < BN / 128; ++j) {
           uint32_t gv[32], uv[32];
-          tmem_ld32(tbase + g * 128 + part * 32, gv);
-          tmem_ld32(tbase + g * 128 + 64 + part * 32, uv);
+          tmem_ld32(tbase + j * 128 + half_id * 32, gv);
+          tmem_ld32(tbase + j * 128 + 64 + half_id * 32, uv);
           tc_wait_ld();
-          if (valid) {
-            bf16* o = reinterpret_cast<bf16*>(p.out) + (size_t)row * p.ldo + (ti.n0 >> 1) + g * 64 + part * 32;
-            uint32_t pk[16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float g0 = __uint_as_float(gv[2 * j]) * rs, g1 = __uint_as_float(gv[2 * j + 1]) * rs;
-              const float u0 = __uint_as_float(uv[2 * j]) * rs, u1 = __uint_as_float(uv[2 * j + 1]) * rs;
-              pk[j] = pack_bf16x2(silu_fast(g0) * u0, silu_fast(g1) * u1);
+          for (int q = 0; q < 16; ++q) {
+            const float g0 = __uint_as_float(gv[2 * q]) * rs, g1 = __uint_as_float(gv[2 * q + 1]) * rs;
+            const float u0 = __uint_as_float(uv[2 * q]) * rs, u1 = __uint_as_float(uv[2 * q + 1]) * rs;
+            w[q] = pack_bf16x2(silu_fast(g0) * u0, silu_fast(g1) * u1);
+          }
+          ok = emit(w, (ti.n0 >> 1) + j * 64, ti.row0);
+        }
+      } else if constexpr (EPI == EPI_BF16) {
+#pragma unroll 1
+        for (int j = 0; ok && j < BN / 64; ++j) {
+          uint32_t v[32];
+          tmem_ld32(tbase + j * 64 + half_id * 32, v);
+          tc_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 16; ++q) w[q] = pack_bf16x2(__uint_as_float(v[2 * q]), __uint_as_float(v[2 * q + 1]));
+          ok = emit(w, ti.n0 + j * 64, ti.row0);
+        }
+      } else if constexpr (EPI == EPI_DOWN3) {
+        // v = r * acc, stored as hi + mid + lo bf16 parts (exact to fp32's 24 bits), one box each
+#pragma unroll 1
+        for (int j = 0; ok && j < BN / 64; ++j) {
+          uint32_t v[32];
+          tmem_ld32(tbase + j * 64 + half_id * 32, v);
+          tc_wait_ld();
+          float a[32];
+#pragma unroll
+          for (int q = 0; q < 32; ++q) a[q] = __uint_as_float(v[q]) * rs;
+#pragma unroll 1
+          for (int part = 0; ok && part < 3; ++part) {
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+              const bf16 h0 = __float2bfloat16_rn(a[2 * q]), h1 = __float2bfloat16_rn(a[2 * q + 1]);
+              __nv_bfloat162 ph = __halves2bfloat162(h0, h1);
+              w[q] = *reinterpret_cast<uint32_t*>(&ph);
+              a[2 * q] -= __bfloat162float(h0);   // remainder for the next part
+              a[2 * q + 1] -= __bfloat162float(h1);
             }
-            uint4* o4 = reinterpret_cast<uint4*>(o);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) o4[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+            ok = emit(w, part * p.split + ti.n0 + j * 64, ti.row0);
           }
         }
       } else {
+        // EPI_F32 / EPI_ROUTER: step j = 32 fp32 columns, 16 per warp.  The router's column offsets
+        // of this tile sit one per lane (lane m: offset n0 + j*32 + m), loaded before the waits.
+        bool nan = false;
 #pragma unroll 1
-        for (int c = half_id; c < BN / 32; c += 2) {
-          uint32_t v[32];
-          tmem_ld32(tbase + c * 32, v);
+        for (int j = 0; ok && j < BN / 32; ++j) {
+          uint32_t v[16];
+          tmem_ld16(tbase + j * 32 + half_id * 16, v);
+          float cj = c_lane[0];
+#pragma unroll
+          for (int jj = 1; jj < BN / 32; ++jj)
+            if (jj == j) cj = c_lane[jj];
           tc_wait_ld();
-          if (!valid) continue;
-          const int col = ti.n0 + c * 32;
-          if constexpr (EPI == EPI_F32) {
-            float4* o4 = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + (size_t)row * p.ldo + col);
+          if constexpr (EPI == EPI_ROUTER) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              o4[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                                  __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
-          } else if constexpr (EPI == EPI_BF16) {
-            uint4* o4 = reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(p.out) + (size_t)row * p.ldo + col);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              o4[j] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * j]), __uint_as_float(v[8 * j + 1])),
-                                 pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
-                                 pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
-                                 pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7])));
-          } else if constexpr (EPI == EPI_DOWN3) {
-            // v = r * acc, stored as hi + mid + lo bf16 parts (exact to fp32's 24 bits)
-            bf16* base = reinterpret_cast<bf16*>(p.out) + (size_t)row * p.ldo + col;
-            uint32_t hi[16], mid[16], lo[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float a0 = __uint_as_float(v[2 * j]) * rs, a1 = __uint_as_float(v[2 * j + 1]) * rs;
-              const bf16 h0 = __float2bfloat16_rn(a0), h1 = __float2bfloat16_rn(a1);
-              const float r0 = a0 - __bfloat162float(h0), r1 = a1 - __bfloat162float(h1);
-              const bf16 m0 = __float2bfloat16_rn(r0), m1 = __float2bfloat16_rn(r1);
-              const float q0 = r0 - __bfloat162float(m0), q1 = r1 - __bfloat162float(m1);
-              __nv_bfloat162 ph = __halves2bfloat162(h0, h1), pm = __halves2bfloat162(m0, m1);
-              hi[j] = *reinterpret_cast<uint32_t*>(&ph);
-              mid[j] = *reinterpret_cast<uint32_t*>(&pm);
-              lo[j] = pack_bf16x2(q0, q1);
+            for (int q = 0; q < 16; ++q) {
+              const float o = sigmoidf_acc(__uint_as_float(v[q]) + __shfl_sync(0xffffffffu, cj, half_id * 16 + q));
+              nan |= (o != o);
+              w[q] = __float_as_uint(o);
             }
-            uint4* oh = reinterpret_cast<uint4*>(base);
-            uint4* om = reinterpret_cast<uint4*>(base + p.split);
-            uint4* ol = reinterpret_cast<uint4*>(base + 2 * p.split);
+          } else {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              oh[j] = make_uint4(hi[4 * j], hi[4 * j + 1], hi[4 * j + 2], hi[4 * j + 3]);
-              om[j] = make_uint4(mid[4 * j], mid[4 * j + 1], mid[4 * j + 2], mid[4 * j + 3]);
-              ol[j] = make_uint4(lo[4 * j], lo[4 * j + 1], lo[4 * j + 2], lo[4 * j + 3]);
-            }
-          } else if constexpr (EPI == EPI_ROUTER) {
-            float4* o4 = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + (size_t)row * p.ldo + col);
-            const float4* cb4 = reinterpret_cast<const float4*>(p.col_bias + col);
-            bool nan = false;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const float4 cb = cb4[j];
-              float4 o;
-              o.x = sigmoidf_acc(__uint_as_float(v[4 * j]) + cb.x);
-              o.y = sigmoidf_acc(__uint_as_float(v[4 * j + 1]) + cb.y);
-              o.z = sigmoidf_acc(__uint_as_float(v[4 * j + 2]) + cb.z);
-              o.w = sigmoidf_acc(__uint_as_float(v[4 * j + 3]) + cb.w);
-              nan |= (o.x != o.x) | (o.y != o.y) | (o.z != o.z) | (o.w != o.w);
-              o4[j] = o;
-            }
-            if (nan) set_status(p.status, LMOE_STATUS_NAN_SCORE);
+            for (int q = 0; q < 16; ++q) w[q] = v[q];
           }
+          ok = emit(w, ti.n0 + j * 32, ti.row0);
         }
+        if (nan && row < p.M_rows) set_status(p.status, LMOE_STATUS_NAN_SCORE);
       }
+      if (!ok) break;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (lane == 0) {
+        if constexpr (PAIR)
+          mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));  // the leader's barrier
+        else
+          mbar_arrive(&tempty[acc]);
+      }
     }
+    if (storer && lane == 0) bulk_wait_all();  // every store has left shared memory and landed
   }
 
   __syncthreads();
+  if constexpr (PAIR) cluster_sync_all();  // both CTAs are done with TMEM and each other's barriers
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::kTmemCols);
+    if constexpr (PAIR)
+      tmem_dealloc_pair(tmem_base, C::kTmemCols);
+    else
+      tmem_dealloc(tmem_base, C::kTmemCols);
   }
+  if constexpr (PAIR) cluster_sync_all();
 }
 
 }  // namespace lmoe

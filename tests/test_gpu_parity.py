@@ -134,6 +134,19 @@ def test_nan_score_is_flagged_and_never_chosen():
     layer.close()
 
 
+def test_bounded_wait_gives_up_and_the_context_stays_usable():
+    """A pipeline wait on a barrier that nothing completes must expire, report, and return."""
+    import time
+    t0 = time.time()
+    st = lq.watchdog_selftest(limit_us=20000)
+    assert st & lq.STATUS_WATCHDOG
+    assert time.time() - t0 < 30
+    y = lq.gemm_bf16(torch.ones(128, 64, dtype=torch.bfloat16, device="cuda"),
+                     torch.ones(64, 64, dtype=torch.bfloat16, device="cuda"))
+    torch.cuda.synchronize()
+    assert torch.all(y == 64)
+
+
 # --------------------------------------------------------------------------- QB update stage
 @pytest.mark.parametrize("literal", [False, True])
 def test_qb_update_stage(literal):
@@ -199,9 +212,10 @@ def test_tiny_fp32_layer_and_qb_update():
     layer.close()
 
 
-@pytest.mark.parametrize("gain", ["ones", "random"])
-def test_small_bf16_layer_ragged(gain):
-    shape = datagen.LayerShape("small", 1000, 256, 128, 64, 4, 128, 256, "bf16", seed=21, offset_var=0.5)
+@pytest.mark.parametrize("gain,E", [("ones", 64), ("random", 64), ("ones", 320), ("random", 320)])
+def test_small_bf16_layer_ragged(gain, E):
+    # E <= 256 runs the fused RMSNorm + W_down + router kernel, E = 320 the three separate ones
+    shape = datagen.LayerShape("small", 1000, 256, 128, E, 4, 128, 256, "bf16", seed=21, offset_var=0.5)
     w = datagen.layer_weights(shape, gain=gain)
     x = datagen.tokens(shape)
     layer, y, ro, stats = run_layer_check(shape, w, x)
