@@ -58,10 +58,12 @@ extern "C" {
 #define LMOE_BF16 1
 
 /* lmoe_forward flags */
-#define LMOE_RECORD_STATS 1u    /* add this forward's scores to the QB histogram (training);
-                                   without it the forward leaves the QB state untouched */
+#define LMOE_RECORD_STATS 1u    /* add this forward's scores to the QB histogram and its expert
+                                   loads to the load counters (training); without it the forward
+                                   leaves the balancing state untouched */
 /* lmoe_qb_update flags */
 #define LMOE_QB_LITERAL 1u      /* u_e = q_e (quantile of the unbiased column) */
+#define LMOE_BIAS_SIGN 2u       /* aux-loss-free sign rule instead of QB (see lmoe_qb_update) */
 
 /* device status bits (lmoe_get_status) */
 #define LMOE_STATUS_NAN_SCORE 1u   /* a router score was NaN; it was never selected */
@@ -126,10 +128,15 @@ int lmoe_forward(lmoe_handle *h, const void *x_dev, void *y_dev, int32_t T, uint
 int lmoe_forward_host(lmoe_handle *h, const void *x_host, void *y_host, int32_t T,
                       uint32_t flags, void *stream);
 
-/* Quantile Balancing step from everything recorded since the last update (N = the sum of T of
- * those forwards): m = ceil((E-k) N / E) (exact integer), q_e = histogram estimate of the m-th
- * smallest score of expert e, b updated as above with step `beta`; then the histogram and N are
- * cleared.  With N == 0 the bias is left unchanged.  Delayed: it changes only later forwards. */
+/* Bias update from everything recorded since the last update (N = the sum of T of those
+ * forwards).  Default, Quantile Balancing: m = ceil((E-k) N / E) (exact integer), q_e = histogram
+ * estimate of the m-th smallest score of expert e, b updated as above with step `beta`.
+ * With LMOE_BIAS_SIGN, the aux-loss-free sign rule of "Pretraining a Mini Kimi K3" (g.15386.cn),
+ * capsule 16: b_e <- b_e + beta * sign(mean_e' load_e' - load_e), load_e = (token, slot) pairs
+ * routed to expert e by the recorded forwards (that page's step is beta = 1e-2); the sign is
+ * decided in exact integers and the fp32 add is rounded once.  LMOE_QB_LITERAL together with
+ * LMOE_BIAS_SIGN is LMOE_EINVAL.  Either rule then clears the histogram, N and the loads.
+ * With N == 0 the bias is left unchanged.  Delayed: it changes only later forwards. */
 int lmoe_qb_update(lmoe_handle *h, float beta, uint32_t flags, void *stream);
 
 /* Routing stage on caller-given scores: runs biased top-k, gates, counts, offsets, the stable
@@ -151,6 +158,11 @@ int lmoe_get_bias(lmoe_handle *h, float *b_dev, void *stream);
 int lmoe_set_bias(lmoe_handle *h, const float *b_dev, void *stream);
 int lmoe_get_hist(lmoe_handle *h, uint32_t *hist_dev, int64_t *ntok_dev, void *stream);
 int lmoe_set_hist(lmoe_handle *h, const uint32_t *hist_dev, const int64_t *ntok_dev, void *stream);
+/* Expert loads recorded since the last update: load [E] int64, device.  Data-parallel ranks sum
+ * them (with the histogram and N) before a sign-rule update, as the same page's capsule 27
+ * ("Bug 2") requires: a rank that balanced its own slice would route a token by where it ran. */
+int lmoe_get_load(lmoe_handle *h, int64_t *load_dev, void *stream);
+int lmoe_set_load(lmoe_handle *h, const int64_t *load_dev, void *stream);
 
 /* Synchronises the device, then returns the status word in *status and clears it. */
 int lmoe_get_status(lmoe_handle *h, uint32_t *status);

@@ -18,13 +18,14 @@ LIB_PATH = os.path.join(_HERE, "liblmoe.so")
 F32, BF16 = 0, 1
 RECORD_STATS = 1
 QB_LITERAL = 1
+BIAS_SIGN = 2
 STATUS_NAN_SCORE, STATUS_WATCHDOG, STATUS_BAD_INDEX = 1, 2, 4
 NBINS = 4096
 
 EXPORTED = (
     "lmoe_create", "lmoe_destroy", "lmoe_workspace_bytes", "lmoe_forward", "lmoe_forward_host",
     "lmoe_qb_update", "lmoe_route_scores", "lmoe_get_routing", "lmoe_get_bias", "lmoe_set_bias",
-    "lmoe_get_hist", "lmoe_set_hist", "lmoe_get_status", "lmoe_strerror", "lmoe_gemm_bf16",
+    "lmoe_get_hist", "lmoe_set_hist", "lmoe_get_load", "lmoe_set_load", "lmoe_get_status", "lmoe_strerror", "lmoe_gemm_bf16",
     "lmoe_profile_enable", "lmoe_profile_read", "lmoe_stage_name", "lmoe_launch_count",
     "lmoe_route_noalloc", "lmoe_watchdog_selftest",
 )
@@ -70,6 +71,8 @@ def lib() -> ctypes.CDLL:
             "lmoe_set_bias": [vp, vp, vp],
             "lmoe_get_hist": [vp, vp, vp, vp],
             "lmoe_set_hist": [vp, vp, vp, vp],
+            "lmoe_get_load": [vp, vp, vp],
+            "lmoe_set_load": [vp, vp, vp],
             "lmoe_get_status": [vp, POINTER(u32)],
             "lmoe_gemm_bf16": [vp, vp, vp, i32, i32, i32, vp],
             "lmoe_profile_enable": [vp, i32],
@@ -174,9 +177,11 @@ class Layer:
                                        _stream(stream)), "lmoe_route_scores")
         self.last_T = T
 
-    def qb_update(self, beta, literal=False, stream=None):
-        _check(lib().lmoe_qb_update(self.handle, float(beta), QB_LITERAL if literal else 0, _stream(stream)),
-               "lmoe_qb_update")
+    def qb_update(self, beta, literal=False, sign_rule=False, stream=None):
+        """Bias update from the recorded statistics: Quantile Balancing, or with sign_rule=True the
+        aux-loss-free rule b_e += beta * sign(mean load - load_e)."""
+        flags = (QB_LITERAL if literal else 0) | (BIAS_SIGN if sign_rule else 0)
+        _check(lib().lmoe_qb_update(self.handle, float(beta), flags, _stream(stream)), "lmoe_qb_update")
 
     # ---------------------------------------------------------------- introspection
     def routing(self, stream=None):
@@ -213,6 +218,15 @@ class Layer:
         _dev(hist, torch.int32, (self.cfg.E, NBINS), "hist")
         _dev(ntok, torch.int64, (1,), "ntok")
         _check(lib().lmoe_set_hist(self.handle, _ptr(hist), _ptr(ntok), _stream(stream)), "lmoe_set_hist")
+
+    def load(self, stream=None):
+        load = torch.empty(self.cfg.E, dtype=torch.int64, device="cuda")
+        _check(lib().lmoe_get_load(self.handle, _ptr(load), _stream(stream)), "lmoe_get_load")
+        return load
+
+    def set_load(self, load, stream=None):
+        _dev(load, torch.int64, (self.cfg.E,), "load")
+        _check(lib().lmoe_set_load(self.handle, _ptr(load), _stream(stream)), "lmoe_set_load")
 
     def profile(self, enable: bool = True):
         _check(lib().lmoe_profile_enable(self.handle, 1 if enable else 0), "lmoe_profile_enable")
@@ -276,14 +290,17 @@ def gemm_bf16(a, b, stream=None):
     return c
 
 
-def sum_qb_statistics(hist, ntok, group=None):
-    """The data-parallel exchange step of QB: sums the integer histograms [E, 4096] and token
-    counts of all ranks in place (torch.distributed all-reduce), so every rank then applies the
-    same bias update as one device that saw every token."""
+def sum_qb_statistics(hist, ntok, load=None, group=None):
+    """The data-parallel exchange step of the bias update: sums the integer histograms [E, 4096],
+    token counts and (for the sign rule) expert loads [E] of all ranks in place (torch.distributed
+    all-reduce), so every rank then applies the same bias update as one device that saw every
+    token."""
     import torch.distributed as dist
     dist.all_reduce(hist, group=group)
     dist.all_reduce(ntok, group=group)
-    return hist, ntok
+    if load is not None:
+        dist.all_reduce(load, group=group)
+    return hist, ntok, load
 
 
 def route_noalloc(scores, bias, k, out=None, stream=None):

@@ -22,6 +22,17 @@ __device__ __forceinline__ void set_status(uint32_t* status, uint32_t bit) {
   if (status) atomicOr(status, bit);
 }
 
+// Programmatic dependent launch.  The layer's kernels are launched with programmatic stream
+// serialisation, so a kernel's blocks may be scheduled while its predecessor drains.  Each such
+// kernel calls pdl_wait() before its first access to global memory that another kernel writes or
+// reads: it returns once the preceding kernel has completed and its writes are visible.  Every
+// kernel of the chain waits, so completion of the predecessor implies completion of all earlier
+// kernels too.  pdl_trigger() allows the next kernel's blocks to be scheduled early; they then
+// hold only their own prologue until their own wait.  Without the launch attribute both are
+// no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -53,13 +64,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// The same test with acquire semantics at cluster scope, for a barrier that the other CTA of a
+// cluster arrives on (mbar_arrive_cluster releases at cluster scope).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase of `parity` to complete.  Returns false when *abort is raised by another
 // role or when the wait exceeded kWaitLimitCycles (then it raises *abort and the status bit).
+// cluster = true acquires at cluster scope (a barrier the peer CTA of a cluster arrives on).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          uint32_t* status, long long limit_cycles = kWaitLimitCycles) {
+                                          uint32_t* status, long long limit_cycles = kWaitLimitCycles,
+                                          bool cluster = false) {
   long long t0 = 0;
   for (uint32_t i = 0;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (cluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
     if ((i & 1023u) == 1023u) {
       if (*abort) return false;
       const long long now = clock64();
@@ -112,6 +139,10 @@ __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wa
 // Orders this thread's generic-proxy shared-memory writes before later async-proxy reads (TMA).
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// Orders this thread's view of global memory (generic proxy) before its later TMA accesses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 // Byte offset of 16-byte chunk `chunk` (0..7) of row `row` in a 128-byte-swizzled box.
 __device__ __forceinline__ uint32_t sw128_offset(int row, int chunk) {

@@ -1,7 +1,11 @@
 // Fused RMSNorm + latent down-projection + sigmoid router for sm_100a (l <= 256, E <= 256).
 //
-// One CTA per 128-token tile (persistent over tiles), 10 warps: warp 0 issues TMA loads into a
-// 4-stage shared-memory ring, warp 1 issues tcgen05.mma, warps 2-9 are the epilogue.
+// One CTA, or a cluster of ns = 2 CTAs, per 128-token tile (persistent over tiles), 10 warps: warp
+// 0 issues TMA loads into a 4-stage shared-memory ring, warp 1 issues tcgen05.mma, warps 2-9 are
+// the epilogue.  With ns = 2 (few tiles: twice the SMs at work) CTA rank r of the cluster
+// computes columns [r l/2, (r+1) l/2) of h and experts [r E/2, (r+1) E/2) of s: each loads half
+// of W_down and of the router weights, and both read all of h back in phase C, so phase C waits
+// until both CTAs' h stores have completed (each storer arrives on both CTAs' barrier).
 //   Phase A  h_acc[128, l] = x_tile W_down'^T in TMEM columns [0, l).  While each x stage sits in
 //            shared memory the epilogue warps add up the squares of their rows (a sum does not
 //            care about the 128-byte swizzle order), so r_t = 1/sqrt(mean x^2 + eps) costs no
@@ -24,10 +28,11 @@ namespace lmoe {
 struct K1Params {
   CUtensorMap tm_s;   // s [Tm, E] fp32, box 32 x 128 (output)
   CUtensorMap tm_x;   // x [T, d], box 64 x 128
-  CUtensorMap tm_wd;  // W_down' [l, d] or [l, 2d] (hi | lo when the gain is not one), box 64 x l
+  CUtensorMap tm_wd;  // W_down' [l, d] or [l, 2d] (hi | lo when the gain is not one), box 64 x l/ns
   CUtensorMap tm_hx;  // h parts [Tm, 3l], box 64 x 128 (output, then A of phase C)
-  CUtensorMap tm_wr;  // router parts [E, 3l], box 64 x E
+  CUtensorMap tm_wr;  // router parts [E, 3l], box 64 x E/ns
   int T, d, l, E;
+  int ns;             // CTAs per tile: 1, or 2 (launched as clusters of 2; l % 128 == 0, E % 64 == 0)
   int wd_segments;    // 1, or 2 when W_down' is split into hi | lo
   float eps;
   float* r;           // out: [T]
@@ -64,9 +69,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant
   uint8_t* obox = smem + kK1OutOffset;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ns = p.ns;
+  const uint32_t rank = ns == 2 ? cluster_ctarank() : 0u;
+  const int lh = p.l / ns, eh = p.E / ns;  // this CTA's columns of h and of s
+  const int first = (int)blockIdx.x / ns, stride = (int)gridDim.x / ns;
+  const uint32_t tmem_cols = ns == 2 ? 256u : 512u;
   const int nkd = p.d / 64, nkl = p.l / 64;
   const int nkbA = nkd * p.wd_segments, nkbC = 6 * nkl;
-  const uint32_t bytesA = 16384u + (uint32_t)p.l * 128u, bytesC = 16384u + (uint32_t)p.E * 128u;
+  const uint32_t bytesA = 16384u + (uint32_t)lh * 128u, bytesC = 16384u + (uint32_t)eh * 128u;
   // the six significant products of (hi, mid, lo) parts, smallest first, as (A part, B part):
   // (mid, mid), (lo, hi), (hi, lo), (mid, hi), (hi, mid), (hi, hi); three bits per product
   constexpr uint32_t kProdA = 1u | (2u << 3) | (0u << 6) | (1u << 9) | (0u << 12) | (0u << 15);
@@ -80,7 +90,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant
     }
     mbar_init(tfullA, 1);
     mbar_init(tempA, kEpiWarps);
-    mbar_init(hxr, 1);  // the storer, once the h parts have landed
+    mbar_init(hxr, ns);  // the storer of every CTA of the tile, once its h parts have landed
     mbar_init(tfullC, 1);
     mbar_init(tempC, kEpiWarps);
     mbar_init(rmsx, kEpiWarps);
@@ -98,13 +108,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant
     tma_prefetch_desc(&p.tm_s);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 512);
+    tmem_alloc(tmem_slot, tmem_cols);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
+  if (ns == 2) cluster_sync_all();  // the peer's barriers exist before any remote arrival
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // x may come from an earlier kernel; hx and s are read by earlier ones
+  pdl_trigger();
   const int num_tiles = (p.T + 127) / 128;
 
   if (warp == 0) {
@@ -117,12 +130,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant
       uint32_t rms_cnt = 0;                  // per-stage use counts (bit = parity) of the rmsd barrier
       bool ok = true;
       int it = 0;
-      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++it) {
+      for (int tile = first; ok && tile < num_tiles; tile += stride, ++it) {
         const int row0 = tile * 128;
         for (int kb = 0; ok && kb < nkbA + nkbC; ++kb) {
-          if (kb == nkbA && !mbar_wait(hxr, it & 1, abort, p.status)) {  // h parts stored
-            ok = false;
-            break;
+          if (kb == nkbA) {  // every CTA's h parts are stored
+            if (!mbar_wait(hxr, it & 1, abort, p.status, kWaitLimitCycles, ns == 2)) {
+              ok = false;
+              break;
+            }
+            fence_proxy_async_global();
           }
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort, p.status)) {
             ok = false;
@@ -141,7 +157,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant
             const int seg = kb / nkd, kk = kb - seg * nkd;
             mbar_expect_tx(&full[stage], bytesA);
             tma_load_2d(a_dst, &p.tm_x, &full[stage], kk * 64, row0);
-            tma_load_2d(b_dst, &p.tm_wd, &full[stage], seg * p.d + kk * 64, 0);
+            tma_load_2d(b_dst, &p.tm_wd, &full[stage], seg * p.d + kk * 64, (int)rank * lh);
             if (seg == 0) {
               rms_pend |= 1u << stage;
               rms_par = (rms_par & ~(1u << stage)) | (((rms_cnt >> stage) & 1u) << stage);
@@ -152,7 +168,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant
             mbar_expect_tx(&full[stage], bytesC);
             const int pa = (int)((kProdA >> (3 * pr)) & 7u), pb = (int)((kProdB >> (3 * pr)) & 7u);
             tma_load_2d(a_dst, &p.tm_hx, &full[stage], pa * p.l + kk * 64, row0);
-            tma_load_2d(b_dst, &p.tm_wr, &full[stage], pb * p.l + kk * 64, 0);
+            tma_load_2d(b_dst, &p.tm_wr, &full[stage], pb * p.l + kk * 64, (int)rank * eh);
           }
           armed |= 1u << stage;
           armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
@@ -169,12 +185,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer
-      const uint32_t idescA = idesc_bf16_f32(p.l), idescC = idesc_bf16_f32(p.E);
+      const uint32_t idescA = idesc_bf16_f32(lh), idescC = idesc_bf16_f32(eh);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       int it = 0;
-      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++it) {
+      for (int tile = first; ok && tile < num_tiles; tile += stride, ++it) {
         for (int ph = 0; ok && ph < 2; ++ph) {
           const int nkb = ph == 0 ? nkbA : nkbC;
           if (!mbar_wait(ph == 0 ? tempA : tempC, (it & 1) ^ 1u, abort, p.status)) {
@@ -182,7 +198,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant
             break;
           }
           tc_fence_after();
-          const uint32_t d_tmem = tmem_base + (ph == 0 ? 0u : (uint32_t)p.l);
+          const uint32_t d_tmem = tmem_base + (ph == 0 ? 0u : (uint32_t)lh);
           const uint32_t idesc = ph == 0 ? idescA : idescC;
           for (int kb = 0; kb < nkb; ++kb) {
             if (!mbar_wait(&full[stage], phase, abort, p.status)) {
@@ -256,8 +272,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant
     // once, long before phase D uses them
     float c_lane[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) c_lane[j] = (j * 32 + lane < p.E) ? p.c[j * 32 + lane] : 0.f;
-    for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++it) {
+    for (int j = 0; j < 8; ++j) c_lane[j] = (j * 32 + lane < eh) ? p.c[(int)rank * eh + j * 32 + lane] : 0.f;
+    for (int tile = first; ok && tile < num_tiles; tile += stride, ++it) {
       const int row0 = tile * 128, row = row0 + rl;
       const bool valid = row < p.T;
       // phase A: squares of this row's half of every x stage (first W_down segment only)
@@ -300,7 +316,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant
       if (__any_sync(0xffffffffu, !ok)) break;
       const float rr =
           (float)(1.0 / sqrt(((double)rms_part[rl] + (double)rms_part[128 + rl]) / p.d + (double)p.eps));
-      if (half_id == 0 && valid) p.r[row] = rr;
+      if (half_id == 0 && valid && rank == 0) p.r[row] = rr;
       // phase B: h = r * acc as hi | mid | lo bf16 parts, one staged box per part and 64 columns
       ok = mbar_wait(tfullA, it & 1, abort, p.status);
       __syncwarp();
@@ -309,7 +325,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant
       const uint32_t tbase = tmem_base + ((uint32_t)(wq * 32) << 16);
       uint32_t w[16];
 #pragma unroll 1
-      for (int j = 0; ok && j < p.l / 64; ++j) {
+      for (int j = 0; ok && j < lh / 64; ++j) {
         uint32_t v[32];
         tmem_ld32(tbase + j * 64 + half_id * 32, v);
         tc_wait_ld();
@@ -326,7 +342,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant
             a[2 * q] -= __bfloat162float(h0);
             a[2 * q + 1] -= __bfloat162float(h1);
           }
-          ok = emit(w, &p.tm_hx, part * p.l + j * 64, row0);
+          ok = emit(w, &p.tm_hx, part * p.l + (int)rank * lh + j * 64, row0);
         }
       }
       if (!ok) break;
@@ -336,7 +352,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant
       if (storer) {
         if (lane == 0) {
           bulk_wait_all();  // the h parts are in global memory before phase C loads them
-          mbar_arrive(hxr);
+          mbar_arrive(hxr);  // own barrier first: the peer's next arrival comes after it
+          if (ns == 2) mbar_arrive_cluster(mapa_shared(smem_u32(hxr), rank ^ 1u));
         }
         __syncwarp();
       }
@@ -347,9 +364,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant
       tc_fence_after();
       bool nan = false;
 #pragma unroll 1
-      for (int j = 0; ok && j < p.E / 32; ++j) {
+      for (int j = 0; ok && j < eh / 32; ++j) {
         uint32_t v[16];
-        tmem_ld16(tbase + p.l + j * 32 + half_id * 16, v);
+        tmem_ld16(tbase + lh + j * 32 + half_id * 16, v);
         float cj = c_lane[0];  // select by unrolled compares: no dynamic register indexing
 #pragma unroll
         for (int jj = 1; jj < 8; ++jj)
@@ -363,7 +380,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant
           nan |= (o != o);
           w[q] = __float_as_uint(o);
         }
-        ok = emit(w, &p.tm_s, j * 32, row0);
+        ok = emit(w, &p.tm_s, (int)rank * eh + j * 32, row0);
       }
       if (!ok) break;
       if (nan && valid) set_status(p.status, LMOE_STATUS_NAN_SCORE);
@@ -375,9 +392,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant
   }
 
   __syncthreads();
+  if (ns == 2) cluster_sync_all();  // no remote arrival is still on its way to this CTA
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 512);
+    tmem_dealloc(tmem_base, tmem_cols);
   }
 }
 

@@ -88,14 +88,44 @@ cudaError_t ensure_smem_attr(K kern, int bytes, unsigned& done) {
   return e;
 }
 
+// Launches `kern` with programmatic stream serialisation, so its blocks may be scheduled while
+// the previous kernel of the stream drains (every kernel of the layer calls pdl_wait() before
+// touching data another kernel writes), and for cluster_x > 1 in clusters of cluster_x CTAs.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, int cluster_x,
+                     Args... args) {
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  memset(attr, 0, sizeof(attr));
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 template <int BN, int EPI>
 cudaError_t launch_tc_t(const TcParams& p, int grid, cudaStream_t st) {
   auto kern = tc_gemm_kernel<BN, EPI, 0>;
   static unsigned done = 0;
   cudaError_t e = ensure_smem_attr(kern, TcCfg<BN>::kSmemBytes, done);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kTcThreads, TcCfg<BN>::kSmemBytes, st>>>(p);
-  return cudaGetLastError();
+  return launch_k(kern, dim3(grid), dim3(kTcThreads), TcCfg<BN>::kSmemBytes, st, 1, p);
 }
 
 // Two-CTA (cta_group::2) variant: clusters of 2 along x, grid even.
@@ -105,22 +135,7 @@ cudaError_t launch_tc_pair_t(const TcParams& p, int grid, cudaStream_t st) {
   static unsigned done = 0;
   cudaError_t e = ensure_smem_attr(kern, TcCfg<BN, 1>::kSmemBytes, done);
   if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg;
-  memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = dim3((unsigned)(grid & ~1), 1, 1);
-  cfg.blockDim = dim3(kTcThreads, 1, 1);
-  cfg.dynamicSmemBytes = TcCfg<BN, 1>::kSmemBytes;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, p);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+  return launch_k(kern, dim3((unsigned)(grid & ~1)), dim3(kTcThreads), TcCfg<BN, 1>::kSmemBytes, st, 2, p);
 }
 
 template <int EPI>
@@ -184,9 +199,9 @@ cudaError_t launch_topk_t(const TopkArgs& a, cudaStream_t st) {
     cudaError_t e = ensure_smem_attr(topk_kernel<NJ>, 64 * 1024 + 4 * 1024 + 1024, done);
     if (e != cudaSuccess) return e;
   }
-  topk_kernel<NJ><<<nblk, 256, smem, st>>>(a.s, a.b, a.T, a.E, a.k, a.idx, a.gates, a.rank, a.blkcnt, a.counts32,
-                                           a.bins, a.ld_bins, a.status);
-  return cudaGetLastError();
+  return launch_k(topk_kernel<NJ>, dim3(nblk), dim3(32 * topk_warps(NJ)), smem, st, 1, a.s, a.b, a.T, a.E, a.k,
+                  a.idx, a.gates,
+                  a.rank, a.blkcnt, a.counts32, a.bins, a.ld_bins, a.status);
 }
 
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st) {
@@ -201,9 +216,17 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st) {
 
 template <int EPI>
 cudaError_t launch_simt(const SimtParams& p, int mtiles, cudaStream_t st) {
-  dim3 grid(p.N / 32, mtiles);
-  simt_gemm_kernel<EPI><<<grid, 256, 0, st>>>(p);
-  return cudaGetLastError();
+  return launch_k(simt_gemm_kernel<EPI>, dim3(p.N / 32, mtiles), dim3(256), 0, st, 1, p);
+}
+
+template <typename T>
+cudaError_t launch_combine(const T* o, const float* gates, const int* prow, int T_, int k, int l, T* z,
+                           cudaStream_t st) {
+  const dim3 grid((T_ + 7) / 8), block(256);
+  if (k <= 2) return launch_k(combine_kernel<T, 2>, grid, block, 0, st, 1, o, gates, prow, T_, k, l, z);
+  if (k <= 4) return launch_k(combine_kernel<T, 4>, grid, block, 0, st, 1, o, gates, prow, T_, k, l, z);
+  if (k <= 6) return launch_k(combine_kernel<T, 6>, grid, block, 0, st, 1, o, gates, prow, T_, k, l, z);
+  return launch_k(combine_kernel<T, 8>, grid, block, 0, st, 1, o, gates, prow, T_, k, l, z);
 }
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -278,6 +301,7 @@ struct lmoe_handle {
   uint16_t* bins = nullptr;  // [E, ld_bins] histogram bin of every score, expert-major
   int *idx = nullptr, *rank = nullptr, *blkcnt = nullptr, *blkbase = nullptr, *counts = nullptr;
   int* counts32 = nullptr;  // [32][E] partial counts of the top-k blocks
+  bool counts32_dirty = true;
   int *offsets = nullptr, *num_mtiles = nullptr, *perm = nullptr, *inv = nullptr;
   int *pad_delta = nullptr, *prow = nullptr;  // padded expert layout of the grouped GEMMs
   long long rows_pad = 0;                     // rows of that layout (upper bound)
@@ -289,6 +313,7 @@ struct lmoe_handle {
   float* bias = nullptr;
   uint32_t* hist = nullptr;
   long long* ntok = nullptr;
+  long long* load = nullptr;  // [E] (token, slot) pairs routed to each expert since the last update
   uint32_t* status = nullptr;
   double* u = nullptr;
   unsigned int* qb_done = nullptr;  // block counter of the QB update kernel (zero between calls)
@@ -298,7 +323,9 @@ struct lmoe_handle {
   CUtensorMap tm_hx, tm_aperm, tm_w13, tm_act, tm_w2, tm_z, tm_as, tm_o, tm_s;
   CUtensorMap tm_wr[3], tm_wdown[3], tm_ws13[3], tm_wy[3];
   bool fused_k1 = false;       // l <= 256 and E <= 256: RMSNorm + W_down + router in one kernel
-  CUtensorMap tm_k1_wd, tm_k1_wr;
+  CUtensorMap tm_k1_wd, tm_k1_wr;        // boxes of the whole of l and E rows (one CTA per tile)
+  CUtensorMap tm_k1_wd2, tm_k1_wr2;      // boxes of l/2 and E/2 rows (a cluster of two per tile)
+  bool k1_split = false;                 // the two-CTA form exists (l % 128 == 0, E % 64 == 0)
   int bn_e1 = 256, bn_e2 = 256;
   // launch counter and optional per-stage profiler
   long long launches = 0;
@@ -370,6 +397,7 @@ void plan_layout(lmoe_handle* h, Arena& a) {
   a.add((void**)&h->bias, E * 4);
   a.add((void**)&h->hist, E * LMOE_NBINS * 4);
   a.add((void**)&h->ntok, 8);
+  a.add((void**)&h->load, E * 8);
   a.add((void**)&h->status, 4);
   a.add((void**)&h->u, E * 8);
   a.add((void**)&h->qb_done, 4);
@@ -435,6 +463,11 @@ int build_maps(lmoe_handle* h) {
   if (h->fused_k1) {
     ok &= make_map(&h->tm_k1_wd, h->w_down, l, h->unit_gain ? d : 2 * d, h->unit_gain ? d : 2 * d, (int)l);
     ok &= make_map(&h->tm_k1_wr, h->w_r, E, 3 * l, 3 * l, (int)E);
+    h->k1_split = c.l % 128 == 0 && c.E % 64 == 0;
+    if (h->k1_split) {
+      ok &= make_map(&h->tm_k1_wd2, h->w_down, l, h->unit_gain ? d : 2 * d, h->unit_gain ? d : 2 * d, (int)l / 2);
+      ok &= make_map(&h->tm_k1_wr2, h->w_r, E, 3 * l, 3 * l, (int)E / 2);
+    }
   }
   return ok ? LMOE_OK : LMOE_ECUDA;
 }
@@ -473,31 +506,37 @@ int route_from_scores(lmoe_handle* h, int T, uint32_t flags, cudaStream_t st) {
   const lmoe_config& c = h->cfg;
   const int nblk = (T + kTokBlock - 1) / kTokBlock;
   mark(h, ST_TOPK, st);
-  CK(cudaMemsetAsync(h->counts32, 0, (size_t)kCountCopies * c.E * sizeof(int), st));
+  // the count copies are zero between routings (the gather kernel clears them after the plan
+  // kernel has read them) unless an earlier routing stopped half-way
+  if (h->counts32_dirty) CK(cudaMemsetAsync(h->counts32, 0, (size_t)kCountCopies * c.E * sizeof(int), st));
+  h->counts32_dirty = true;
   TopkArgs ta{h->s, h->bias, T, c.E, c.k, h->idx, h->rank, h->blkcnt, h->counts32, h->gates,
               (flags & LMOE_RECORD_STATS) ? h->bins : nullptr, h->ld_bins, h->status};
   CK(launch_topk(ta, st));
   mark(h, ST_PLAN, st);
-  plan_kernel<<<(c.E + 31) / 32, 1024, 0, st>>>(h->counts32, h->counts, h->blkcnt, nblk, c.E, h->offsets,
-                                                  h->pad_delta, h->blkbase, h->mtiles, h->num_mtiles);
-  CK(cudaGetLastError());
+  CK(launch_k(plan_kernel, dim3((c.E + 31) / 32), dim3(1024), 0, st, 1, (const int*)h->counts32, h->counts,
+              (const int*)h->blkcnt, nblk, c.E, h->offsets, h->pad_delta, h->blkbase, h->mtiles, h->num_mtiles,
+              (flags & LMOE_RECORD_STATS) ? h->load : (long long*)nullptr));
   const int pairs = T * c.k;
+  const dim3 ggrid((pairs + 8 * kGatherPairs - 1) / (8 * kGatherPairs));
+  int4* clear = reinterpret_cast<int4*>(h->counts32);
+  const int nclear = kCountCopies * c.E / 4;
   mark(h, ST_GATHER, st);
   if (h->bf) {
-    gather_kernel<bf16><<<(pairs + 8 * kGatherPairs - 1) / (8 * kGatherPairs), 256, 0, st>>>((const bf16*)h->hx, 3 * c.l, c.l, h->idx, h->rank,
-                                                         h->blkbase, h->pad_delta, T, c.E, c.k, h->perm, h->inv,
-                                                         h->prow, (bf16*)h->a_perm, h->status);
+    CK(launch_k(gather_kernel<bf16>, ggrid, dim3(256), 0, st, 1, (const bf16*)h->hx, 3 * c.l, c.l,
+                (const int*)h->idx, (const int*)h->rank, (const int*)h->blkbase, (const int*)h->pad_delta, T, c.E,
+                c.k, h->perm, h->inv, h->prow, (bf16*)h->a_perm, clear, nclear, h->status));
   } else {
-    gather_kernel<float><<<(pairs + 8 * kGatherPairs - 1) / (8 * kGatherPairs), 256, 0, st>>>((const float*)h->hx, c.l, c.l, h->idx, h->rank,
-                                                          h->blkbase, h->pad_delta, T, c.E, c.k, h->perm, h->inv,
-                                                          h->prow, (float*)h->a_perm, h->status);
+    CK(launch_k(gather_kernel<float>, ggrid, dim3(256), 0, st, 1, (const float*)h->hx, c.l, c.l,
+                (const int*)h->idx, (const int*)h->rank, (const int*)h->blkbase, (const int*)h->pad_delta, T, c.E,
+                c.k, h->perm, h->inv, h->prow, (float*)h->a_perm, clear, nclear, h->status));
   }
-  CK(cudaGetLastError());
+  h->counts32_dirty = false;
   mark(h, ST_HIST, st);
   h->launches += 3;
   if (flags & LMOE_RECORD_STATS) {
-    hist_kernel<<<c.E, 512, 0, st>>>(h->bins, h->ld_bins, T, h->hist, h->ntok);
-    CK(cudaGetLastError());
+    CK(launch_k(hist_kernel, dim3(c.E), dim3(kHistThreads), 0, st, 1, (const uint16_t*)h->bins, h->ld_bins, T,
+                h->hist, h->ntok));
     h->launches += 1;
   }
   h->last_T = T;
@@ -514,13 +553,16 @@ int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, 
     mark(h, ST_DOWN, st);
     mark(h, ST_ROUTER, st);
     mark(h, ST_K1, st);
+    // a cluster of two CTAs per tile while the tiles fill at most half of the SMs
+    const int ns = (h->k1_split && 2 * mt <= h->sms) ? 2 : 1;
     K1Params kp;
     memset(&kp, 0, sizeof(kp));
     kp.tm_s = h->tm_s;
     kp.tm_x = tm_x;
-    kp.tm_wd = h->tm_k1_wd;
+    kp.tm_wd = ns == 2 ? h->tm_k1_wd2 : h->tm_k1_wd;
     kp.tm_hx = h->tm_hx;
-    kp.tm_wr = h->tm_k1_wr;
+    kp.tm_wr = ns == 2 ? h->tm_k1_wr2 : h->tm_k1_wr;
+    kp.ns = ns;
     kp.T = T;
     kp.d = c.d;
     kp.l = c.l;
@@ -532,12 +574,10 @@ int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, 
     kp.status = h->status;
     static unsigned done = 0;
     CK(ensure_smem_attr(k1_kernel, kK1SmemBytes, done));
-    k1_kernel<<<std::min(mt, h->sms), kTcThreads, kK1SmemBytes, st>>>(kp);
-    CK(cudaGetLastError());
+    CK(launch_k(k1_kernel, dim3(ns * std::min(mt, h->sms / ns)), dim3(kTcThreads), kK1SmemBytes, st, ns, kp));
     h->launches += 1;
   } else {
-    rms_kernel<bf16><<<(T + 7) / 8, 256, 0, st>>>((const bf16*)x, T, c.d, c.rms_eps, h->r);
-    CK(cudaGetLastError());
+    CK(launch_k(rms_kernel<bf16>, dim3((T + 7) / 8), dim3(256), 0, st, 1, (const bf16*)x, T, c.d, c.rms_eps, h->r));
     // h = r * (x Wdown^T), stored as hi | mid | lo bf16 parts
     mark(h, ST_DOWN, st);
     {
@@ -644,9 +684,7 @@ int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, 
     CK(launch_tc(p, EPI_BF16, h->bn_e2, h->sms, st));
   }
   mark(h, ST_COMBINE, st);
-  combine_kernel<bf16><<<(T + 7) / 8, 256, 0, st>>>((const bf16*)h->o, h->gates, h->prow, T, c.k, c.l,
-                                                    (bf16*)h->z);
-  CK(cudaGetLastError());
+  CK(launch_combine((const bf16*)h->o, h->gates, h->prow, T, c.k, c.l, (bf16*)h->z, st));
   // y = [z | a_s] [W_up | Ws2]^T
   mark(h, ST_UP, st);
   {
@@ -681,8 +719,7 @@ int forward_f32(lmoe_handle* h, const void* xv, void* yv, int T, uint32_t flags,
   const float* x = (const float*)xv;
   const int mt = (T + 127) / 128;
   mark(h, ST_RMS, st);
-  rms_kernel<float><<<(T + 7) / 8, 256, 0, st>>>(x, T, c.d, c.rms_eps, h->r);
-  CK(cudaGetLastError());
+  CK(launch_k(rms_kernel<float>, dim3((T + 7) / 8), dim3(256), 0, st, 1, x, T, c.d, c.rms_eps, h->r));
   SimtParams b;
   memset(&b, 0, sizeof(b));
   b.status = h->status;
@@ -740,9 +777,7 @@ int forward_f32(lmoe_handle* h, const void* xv, void* yv, int T, uint32_t flags,
     CK(launch_simt<SE_STORE>(p, gm, st));
   }
   mark(h, ST_COMBINE, st);
-  combine_kernel<float><<<(T + 7) / 8, 256, 0, st>>>((const float*)h->o, h->gates, h->prow, T, c.k, c.l,
-                                                     (float*)h->z);
-  CK(cudaGetLastError());
+  CK(launch_combine((const float*)h->o, h->gates, h->prow, T, c.k, c.l, (float*)h->z, st));
   mark(h, ST_UP, st);
   {  // y = [z | a_s] [W_up | Ws2]^T
     SimtParams p = b;
@@ -944,6 +979,7 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, void* stream, lmo
   if (!rc && cudaMemsetAsync(h->bias, 0, cfg->E * 4, st) != cudaSuccess) rc = LMOE_ECUDA;
   if (!rc && cudaMemsetAsync(h->hist, 0, (size_t)cfg->E * LMOE_NBINS * 4, st) != cudaSuccess) rc = LMOE_ECUDA;
   if (!rc && cudaMemsetAsync(h->ntok, 0, 8, st) != cudaSuccess) rc = LMOE_ECUDA;
+  if (!rc && cudaMemsetAsync(h->load, 0, (size_t)cfg->E * 8, st) != cudaSuccess) rc = LMOE_ECUDA;
   if (!rc && cudaMemsetAsync(h->status, 0, 4, st) != cudaSuccess) rc = LMOE_ECUDA;
   if (!rc && cudaMemsetAsync(h->qb_done, 0, 4, st) != cudaSuccess) rc = LMOE_ECUDA;
   if (!rc && h->bf) rc = build_maps(h);
@@ -1012,14 +1048,14 @@ int lmoe_route_scores(lmoe_handle* h, const float* scores, int32_t T, uint32_t f
 
 int lmoe_qb_update(lmoe_handle* h, float beta, uint32_t flags, void* stream) {
   if (!h || !(beta == beta)) return LMOE_EINVAL;
+  if ((flags & LMOE_QB_LITERAL) && (flags & LMOE_BIAS_SIGN)) return LMOE_EINVAL;
   cudaStream_t st = (cudaStream_t)stream;
   return run_cached(h, h->g_qb, nullptr, nullptr, 0, flags, beta, st, [&](cudaStream_t s) {
     prof_open(h, ST_QB_UPDATE, 1);
     mark(h, ST_QB_UPDATE, s);
-    qb_update_kernel<<<h->cfg.E, 256, 0, s>>>(h->hist, h->ntok, h->bias, h->cfg.E, h->cfg.k,
-                                               (flags & LMOE_QB_LITERAL) ? 1 : 0, beta, h->u, h->qb_done,
-                                               h->status);
-    CK(cudaGetLastError());
+    CK(launch_k(qb_update_kernel, dim3(h->cfg.E), dim3(256), 0, s, 1, h->hist, h->ntok, h->load, h->bias,
+                h->cfg.E, h->cfg.k, (flags & LMOE_QB_LITERAL) ? 1 : 0, (flags & LMOE_BIAS_SIGN) ? 1 : 0, beta,
+                h->u, h->qb_done, h->status));
     prof_close(h, s);
     h->launches += 1;
     return LMOE_OK;
@@ -1069,6 +1105,18 @@ int lmoe_set_hist(lmoe_handle* h, const uint32_t* hist, const int64_t* ntok, voi
   cudaStream_t st = (cudaStream_t)stream;
   CK(cudaMemcpyAsync(h->hist, hist, (size_t)h->cfg.E * LMOE_NBINS * 4, cudaMemcpyDeviceToDevice, st));
   CK(cudaMemcpyAsync(h->ntok, ntok, 8, cudaMemcpyDeviceToDevice, st));
+  return LMOE_OK;
+}
+
+int lmoe_get_load(lmoe_handle* h, int64_t* load, void* stream) {
+  if (!h || !load) return LMOE_EINVAL;
+  CK(cudaMemcpyAsync(load, h->load, (size_t)h->cfg.E * 8, cudaMemcpyDeviceToDevice, (cudaStream_t)stream));
+  return LMOE_OK;
+}
+
+int lmoe_set_load(lmoe_handle* h, const int64_t* load, void* stream) {
+  if (!h || !load) return LMOE_EINVAL;
+  CK(cudaMemcpyAsync(h->load, load, (size_t)h->cfg.E * 8, cudaMemcpyDeviceToDevice, (cudaStream_t)stream));
   return LMOE_OK;
 }
 
@@ -1219,11 +1267,11 @@ int lmoe_route_noalloc(const float* scores, const float* bias, int32_t T, int32_
   CK(launch_topk(ta, st));
   const int nblk = (T + kTokBlock - 1) / kTokBlock;
   plan_kernel<<<(E + 31) / 32, 1024, 0, st>>>(counts32, counts, blkcnt, nblk, E, offsets, delta, blkbase, tiles,
-                                               ntiles);
+                                               ntiles, nullptr);
   CK(cudaGetLastError());
   const int pairs = T * k;
   gather_kernel<float><<<(pairs + 8 * kGatherPairs - 1) / (8 * kGatherPairs), 256, 0, st>>>(
-      nullptr, 0, 0, idx, rank, blkbase, nullptr, T, E, k, perm, inv, nullptr, nullptr, status);
+      nullptr, 0, 0, idx, rank, blkbase, nullptr, T, E, k, perm, inv, nullptr, nullptr, nullptr, 0, status);
   CK(cudaGetLastError());
   return LMOE_OK;
 }

@@ -19,6 +19,8 @@ constexpr unsigned kFull = 0xffffffffu;
 template <typename T>
 __global__ void __launch_bounds__(256) rms_kernel(const T* __restrict__ x, int ntok, int d, float eps,
                                                   float* __restrict__ r) {
+  pdl_wait();
+  pdl_trigger();
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (row >= ntok) return;
   constexpr int VEC = 16 / sizeof(T);
@@ -48,25 +50,31 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-// One warp per token, 4 tokens per warp, kTokBlock = 32 tokens per block.  Lane L holds the
-// scores of experts L, L+32, ...; the scores of up to PF tokens are loaded before any of them is
-// ranked, so their memory latency overlaps.  k rounds of: local best (larger key, then lower
-// index), warp max of the keys (redux), warp min of the expert index among the lanes holding
-// that key (redux), broadcast of its unbiased score.  This is top-k of u = s + b in fp32 with
-// ties to the lower expert index.  Gates are the chosen s over their sum.  Each choice sets the
-// token's bit in the expert's shared mask; the token's rank inside the block for that expert is
-// the number of set bits below it, so the permutation is stable (token ascending) with no
-// order-dependent atomics.  With bins != null it also stores each score's histogram bin,
-// min(floor(s * 4096), 4095) as uint16, expert-major (bins[e * ld_bins + t]).
-__host__ __device__ constexpr int topk_prefetch(int nj) { return nj <= 8 ? 4 : (nj <= 16 ? 2 : 1); }
+// One warp per token; a block of W warps ranks kTokBlock = 32 tokens (32 / W per warp; W = 16
+// for E <= 256, whose registers allow two such blocks per SM, else 8).  Lane L holds the scores
+// of experts L, L+32, ...; the scores of up to PF tokens are loaded before any of them is ranked,
+// so their memory latency overlaps.  k rounds of: local best (larger key, then lower index),
+// warp max of the keys (redux), warp min of the expert index among the lanes holding that key
+// (redux); lane i keeps the i-th choice.  This is top-k of u = s + b in fp32 with ties to the
+// lower expert index.  Gates are the chosen s (reloaded by the lanes that keep a choice) over
+// their sum.  Each choice sets the token's bit in the expert's shared mask; the token's rank
+// inside the block for that expert is the number of set bits below it, so the permutation is
+// stable (token ascending) with no order-dependent atomics.  With bins != null it also stores
+// each score's histogram bin, min(floor(s * 4096), 4095) as uint16, expert-major
+// (bins[e * ld_bins + t]).
+__host__ __device__ constexpr int topk_warps(int nj) { return nj <= 8 ? 16 : 8; }
+__host__ __device__ constexpr int topk_prefetch(int nj) {
+  return nj <= 8 ? kTokBlock / topk_warps(nj) : (nj <= 16 ? 2 : 1);
+}
 
 template <int NJ>
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ s, const float* __restrict__ bias,
-                                                   int ntok, int E, int k, int* __restrict__ idx,
-                                                   float* __restrict__ gates, int* __restrict__ rank,
-                                                   int* __restrict__ blkcnt, int* __restrict__ counts32,
-                                                   uint16_t* __restrict__ bins, int ld_bins, uint32_t* status) {
-  constexpr int TPW = kTokBlock / 8;  // tokens per warp
+__global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 : 1)
+    topk_kernel(const float* __restrict__ s, const float* __restrict__ bias, int ntok, int E, int k,
+                int* __restrict__ idx, float* __restrict__ gates, int* __restrict__ rank,
+                int* __restrict__ blkcnt, int* __restrict__ counts32, uint16_t* __restrict__ bins, int ld_bins,
+                uint32_t* status) {
+  constexpr int W = topk_warps(NJ);
+  constexpr int TPW = kTokBlock / W;  // tokens per warp
   constexpr int PF = topk_prefetch(NJ);
   extern __shared__ uint32_t smem_topk[];
   uint32_t* mask = smem_topk;                                    // [E]
@@ -75,6 +83,8 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ s, 
   const int blk = blockIdx.x, t0 = blk * kTokBlock;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < E; i += blockDim.x) mask[i] = 0;
+  pdl_wait();
+  pdl_trigger();
   float bj[NJ];
 #pragma unroll
   for (int j = 0; j < NJ; ++j) {
@@ -103,56 +113,51 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ s, 
       sel_q[q0 + p] = -1;
       if (t >= ntok) continue;  // warp-uniform
       uint32_t key[NJ];
-      float sv[NJ];
 #pragma unroll
       for (int j = 0; j < NJ; ++j) {
         const int e = j * 32 + lane;
         const float v = vq[p][j];
         if (e < E) {
           nan |= (v != v);
-          sv[j] = (v == v) ? v : 0.f;
           key[j] = order_key(v + bj[j]);
           if (bins)
             sbins[tl * bpitch + e] =
                 (uint16_t)(v >= 0.f ? min((int)(v * (float)LMOE_NBINS), LMOE_NBINS - 1) : 0);
         } else {
-          sv[j] = 0.f;
           key[j] = 0u;
         }
       }
       int my_sel = -1;
-      float my_s = 0.f;
       for (int i = 0; i < k; ++i) {
         uint32_t bk = 0u;
-        uint32_t be = 0xffffffffu;
-        float bs = 0.f;
+        int bjx = 0;
 #pragma unroll
         for (int j = 0; j < NJ; ++j) {
           if (key[j] > bk) {
             bk = key[j];
-            be = (uint32_t)(j * 32 + lane);
-            bs = sv[j];
+            bjx = j;
           }
         }
         const uint32_t wmax = __reduce_max_sync(kFull, bk);
-        const uint32_t emin = __reduce_min_sync(kFull, bk == wmax ? be : 0xffffffffu);
-        const float es = __shfl_sync(kFull, bs, (int)(emin & 31u));
+        const uint32_t emin = __reduce_min_sync(kFull, bk == wmax ? (uint32_t)(bjx * 32 + lane) : 0xffffffffu);
 #pragma unroll
         for (int j = 0; j < NJ; ++j)
           if ((uint32_t)(j * 32 + lane) == emin) key[j] = 0u;
-        if (lane == i) {
-          my_sel = (int)emin;
-          my_s = es;
-        }
+        if (lane == i) my_sel = (int)emin;
       }
-      float ssum = lane < k ? my_s : 0.f;
-#pragma unroll
-      for (int off = 16; off; off >>= 1) ssum += __shfl_xor_sync(kFull, ssum, off);
+      float my_s = 0.f;
       if (lane < k) {
         if (my_sel < 0 || my_sel >= E) {
           set_status(status, LMOE_STATUS_BAD_INDEX);
           my_sel = 0;
         }
+        my_s = s[(size_t)t * E + my_sel];
+        if (my_s != my_s) my_s = 0.f;
+      }
+      float ssum = my_s;
+#pragma unroll
+      for (int off = 16; off; off >>= 1) ssum += __shfl_xor_sync(kFull, ssum, off);
+      if (lane < k) {
         idx[(size_t)t * k + lane] = my_sel;
         gates[(size_t)t * k + lane] = my_s / ssum;
         atomicOr(&mask[my_sel], 1u << tl);
@@ -178,7 +183,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ s, 
   if (bins) {
     // expert-major store: one warp writes 32 tokens (64 bytes) of one expert per step
     const int nt = min(kTokBlock, ntok - t0);
-    for (int e = warp; e < E; e += 8)
+    for (int e = warp; e < E; e += W)
       if (lane < nt) bins[(size_t)e * ld_bins + t0 + lane] = sbins[lane * bpitch + e];
   }
 }
@@ -222,11 +227,13 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ coun
                                                     const int* __restrict__ blkcnt, int nblk, int E,
                                                     int* __restrict__ offsets, int* __restrict__ pad_delta,
                                                     int* __restrict__ blkbase, int2* __restrict__ mtiles,
-                                                    int* __restrict__ num_mtiles) {
+                                                    int* __restrict__ num_mtiles, long long* __restrict__ load) {
   __shared__ int sh[32];
   __shared__ int s_off[1024];
   __shared__ int part[32][33];
   const int tid = threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
   int c = 0;
   if (tid < E) {
 #pragma unroll 8
@@ -239,6 +246,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ coun
     if (tid < E) {
       offsets[tid] = off;
       counts[tid] = c;
+      if (load) load[tid] += c;
     }
     if (tid == 0) offsets[E] = total;
     const int mt = (c + kTileRows - 1) / kTileRows;
@@ -284,7 +292,13 @@ __global__ void __launch_bounds__(256) gather_kernel(const T* __restrict__ src, 
                                                      const int* __restrict__ pad_delta, int ntok, int E, int k,
                                                      int* __restrict__ perm, int* __restrict__ inv,
                                                      int* __restrict__ prow, T* __restrict__ dst,
-                                                     uint32_t* status) {
+                                                     int4* __restrict__ clear, int nclear, uint32_t* status) {
+  pdl_wait();
+  pdl_trigger();
+  // the top-k count copies were last read by the plan kernel: the last block clears them for
+  // the next routing (nclear 16-byte words)
+  if (clear && blockIdx.x == gridDim.x - 1)
+    for (int i = threadIdx.x; i < nclear; i += blockDim.x) clear[i] = make_int4(0, 0, 0, 0);
   const int lane = threadIdx.x & 31;
   const int pair0 = (blockIdx.x * 8 + (threadIdx.x >> 5)) * kGatherPairs;
   const int npairs = ntok * k;
@@ -330,12 +344,20 @@ __global__ void __launch_bounds__(256) gather_kernel(const T* __restrict__ src, 
 // --------------------------------------------------------------------------- QB histogram
 // Block per expert: counts that expert's uint16 bins (written expert-major by the top-k kernel)
 // in a shared 4096-bin histogram, then adds it into the expert's global row, which no other
-// block touches.  Block 0 adds T to the recorded token count.
-__global__ void __launch_bounds__(512) hist_kernel(const uint16_t* __restrict__ bins, int ld_bins, int ntok,
-                                                   uint32_t* __restrict__ hist, long long* ntok_acc) {
-  __shared__ uint32_t sh[LMOE_NBINS];
+// block touches.  Thread i owns bins [8i, 8i + 8) of the row; it loads them before counting so
+// their latency overlaps the counting.  Block 0 adds T to the recorded token count.
+constexpr int kHistThreads = LMOE_NBINS / 8;
+
+__global__ void __launch_bounds__(kHistThreads) hist_kernel(const uint16_t* __restrict__ bins, int ld_bins,
+                                                            int ntok, uint32_t* __restrict__ hist,
+                                                            long long* ntok_acc) {
+  __shared__ __align__(16) uint32_t sh[LMOE_NBINS];
   const int e = blockIdx.x;
   for (int i = threadIdx.x; i < LMOE_NBINS; i += blockDim.x) sh[i] = 0;
+  pdl_wait();
+  pdl_trigger();
+  uint4* hrow4 = reinterpret_cast<uint4*>(hist + (size_t)e * LMOE_NBINS) + 2 * threadIdx.x;
+  uint4 g0 = hrow4[0], g1 = hrow4[1];
   __syncthreads();
   const uint16_t* row = bins + (size_t)e * ld_bins;
   const int nvec = ntok / 8;  // ld_bins is a multiple of 32, so rows are 16-byte aligned
@@ -351,21 +373,26 @@ __global__ void __launch_bounds__(512) hist_kernel(const uint16_t* __restrict__ 
   }
   for (int t = nvec * 8 + threadIdx.x; t < ntok; t += blockDim.x) atomicAdd(&sh[row[t]], 1u);
   __syncthreads();
-  uint32_t* hrow = hist + (size_t)e * LMOE_NBINS;
-  for (int i = threadIdx.x; i < LMOE_NBINS; i += blockDim.x) {
-    const uint32_t v = sh[i];
-    if (v) hrow[i] += v;
-  }
+  const uint4 a0 = reinterpret_cast<const uint4*>(sh)[2 * threadIdx.x];
+  const uint4 a1 = reinterpret_cast<const uint4*>(sh)[2 * threadIdx.x + 1];
+  g0.x += a0.x; g0.y += a0.y; g0.z += a0.z; g0.w += a0.w;
+  g1.x += a1.x; g1.y += a1.y; g1.z += a1.z; g1.w += a1.w;
+  hrow4[0] = g0;
+  hrow4[1] = g1;
   if (e == 0 && threadIdx.x == 0) *ntok_acc += ntok;
 }
 
 // --------------------------------------------------------------------------- combine
 // z_t = sum_i g_ti o[prow[t, i]] in rank order (prow: the pair's row in the padded expert layout),
-// fp32 accumulation; one warp per token.
-template <typename T>
-__global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ o, const float* __restrict__ gates,
-                                                      const int* __restrict__ prow, int ntok, int k, int l,
-                                                      T* __restrict__ z) {
+// fp32 accumulation; one warp per token.  The row loads of G slots are issued together before
+// their FMAs (G >= k where possible: the launch picks the smallest of 2, 4, 6, 8 that covers k),
+// and G sizes the registers, so small k keeps more warps resident.
+template <typename T, int G>
+__global__ void __launch_bounds__(256, (G <= 6 && sizeof(T) == 2) ? 4 : 3) combine_kernel(const T* __restrict__ o, const float* __restrict__ gates,
+                                                         const int* __restrict__ prow, int ntok, int k, int l,
+                                                         T* __restrict__ z) {
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (t >= ntok) return;
   constexpr int VEC = 16 / sizeof(T);
@@ -376,18 +403,18 @@ __global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ o, c
     float acc[VEC];
 #pragma unroll
     for (int j = 0; j < VEC; ++j) acc[j] = 0.f;
-    for (int i0 = 0; i0 < k; i0 += 8) {
-      uint4 q[8];
-      float g[8];
+    for (int i0 = 0; i0 < k; i0 += G) {
+      uint4 q[G];
+      float g[G];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < G; ++u) {
         const int i = i0 + u;
         const int row = __shfl_sync(kFull, r_l, i & 31);
         g[u] = __shfl_sync(kFull, g_l, i & 31);
         if (i < k) q[u] = reinterpret_cast<const uint4*>(o + (size_t)row * l)[v];
       }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < G; ++u) {
         if (i0 + u >= k) break;
         const T* e = reinterpret_cast<const T*>(&q[u]);
 #pragma unroll
@@ -403,82 +430,112 @@ __global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ o, c
 }
 
 // --------------------------------------------------------------------------- QB update
-// One kernel, block per expert.  Block e: m = ceil((E-k) N / E); the crossing bin j* is the first
-// whose cumulative count reaches m; q = (j* + (m - cum_{j*-1}) / cnt_{j*}) / 4096; u_e = q (+ b_e);
-// the expert's histogram row is cleared.  The last block to finish (a device-wide counter)
-// computes mean_e u and applies b_e <- b_e - beta (u_e - mean) to every expert, then clears N and
-// the counter.  Nothing happens when N == 0.
+// One kernel, block per expert, for both bias rules; nothing happens when N == 0.
+//  QB (sign_rule == 0): block e finds m = ceil((E-k) N / E), the crossing bin j* (the first whose
+//   cumulative count reaches m) and q = (j* + (m - cum_{j*-1}) / cnt_{j*}) / 4096, then u_e = q
+//   (+ b_e unless literal).  The last block to finish (a device-wide counter) computes mean_e u and
+//   applies b_e <- b_e - beta (u_e - mean) to every expert.
+//  Sign rule (sign_rule == 1): the last block applies b_e <- b_e + beta sign(mean load - load_e),
+//   the sign taken in integers as sign(sum_e' load_e' - E load_e).
+// Either way every block clears its histogram row, and the last block clears N, the loads and
+// the counter: an update consumes all statistics recorded since the previous one.
 __global__ void __launch_bounds__(256) qb_update_kernel(uint32_t* __restrict__ hist, long long* ntok_acc,
-                                                        float* __restrict__ bias, int E, int k, int literal,
-                                                        float beta, double* __restrict__ u_buf,
-                                                        unsigned int* done_counter, uint32_t* status) {
+                                                        long long* __restrict__ load, float* __restrict__ bias,
+                                                        int E, int k, int literal, int sign_rule, float beta,
+                                                        double* __restrict__ u_buf, unsigned int* done_counter,
+                                                        uint32_t* status) {
   __shared__ long long wsum[8];
   __shared__ double wd[8];
+  __shared__ double u_sh;
   __shared__ bool last;
   const int e = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_wait();
+  pdl_trigger();
   const long long N = *ntok_acc;
   if (N <= 0) return;
-  long long m = ((long long)(E - k) * N + E - 1) / E;
-  m = m < 1 ? 1 : (m > N ? N : m);
   uint4* row4 = reinterpret_cast<uint4*>(hist + (size_t)e * LMOE_NBINS);
   constexpr int PER = LMOE_NBINS / 256;  // 16 bins per thread, 4 x uint4
-  uint32_t c[PER];
+  if (!sign_rule) {
+    long long m = ((long long)(E - k) * N + E - 1) / E;
+    m = m < 1 ? 1 : (m > N ? N : m);
+    uint32_t c[PER];
 #pragma unroll
-  for (int j = 0; j < PER / 4; ++j) {
-    const uint4 q = row4[tid * (PER / 4) + j];
-    c[4 * j] = q.x;
-    c[4 * j + 1] = q.y;
-    c[4 * j + 2] = q.z;
-    c[4 * j + 3] = q.w;
-  }
-  long long local = 0;
-#pragma unroll
-  for (int j = 0; j < PER; ++j) local += c[j];
-  long long x = local;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const long long y = __shfl_up_sync(kFull, x, off);
-    if (lane >= off) x += y;
-  }
-  if (lane == 31) wsum[warp] = x;
-  if (tid == 0) u_buf[e] = literal ? 0.0 : (double)bias[e];  // only if no crossing is found
-  __syncthreads();
-  long long before = x - local;
-  for (int w = 0; w < warp; ++w) before += wsum[w];
-  if (before < m && m <= before + local) {
-    long long cum = before;
-#pragma unroll
-    for (int j = 0; j < PER; ++j) {
-      if (cum + c[j] >= m) {
-        const int jstar = tid * PER + j;
-        const double q = ((double)jstar + (double)(m - cum) / (double)c[j]) / (double)LMOE_NBINS;
-        u_buf[e] = literal ? q : q + (double)bias[e];
-        break;
-      }
-      cum += c[j];
+    for (int j = 0; j < PER / 4; ++j) {
+      const uint4 q = row4[tid * (PER / 4) + j];
+      c[4 * j] = q.x;
+      c[4 * j + 1] = q.y;
+      c[4 * j + 2] = q.z;
+      c[4 * j + 3] = q.w;
     }
+    long long local = 0;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) local += c[j];
+    long long x = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const long long y = __shfl_up_sync(kFull, x, off);
+      if (lane >= off) x += y;
+    }
+    if (lane == 31) wsum[warp] = x;
+    if (tid == 0) u_sh = literal ? 0.0 : (double)bias[e];  // only if no crossing is found
+    __syncthreads();
+    long long before = x - local;
+    for (int w = 0; w < warp; ++w) before += wsum[w];
+    if (before < m && m <= before + local) {
+      long long cum = before;
+#pragma unroll
+      for (int j = 0; j < PER; ++j) {
+        if (cum + c[j] >= m) {
+          const int jstar = tid * PER + j;
+          const double q = ((double)jstar + (double)(m - cum) / (double)c[j]) / (double)LMOE_NBINS;
+          u_sh = literal ? q : q + (double)bias[e];
+          break;
+        }
+        cum += c[j];
+      }
+    }
+    __syncthreads();
   }
-  __syncthreads();
 #pragma unroll
   for (int j = 0; j < PER / 4; ++j) row4[tid * (PER / 4) + j] = make_uint4(0u, 0u, 0u, 0u);
-  // publish u_e, then count finished blocks
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) last = (atomicAdd(done_counter, 1u) == (unsigned)(E - 1));
+  // thread 0 publishes u_e, then counts finished blocks (the cleared rows are read only by later
+  // kernels, so they need no fence)
+  if (tid == 0) {
+    if (!sign_rule) u_buf[e] = u_sh;
+    __threadfence();
+    last = (atomicAdd(done_counter, 1u) == (unsigned)(E - 1));
+  }
   __syncthreads();
   if (!last) return;
   __threadfence();
-  double v = 0.0;
-  for (int i = tid; i < E; i += blockDim.x) v += __ldcg(&u_buf[i]);
+  if (sign_rule) {
+    long long v = 0;
+    for (int i = tid; i < E; i += blockDim.x) v += __ldcg(&load[i]);
 #pragma unroll
-  for (int off = 16; off; off >>= 1) v += __shfl_xor_sync(kFull, v, off);
-  if (lane == 0) wd[warp] = v;
-  __syncthreads();
-  double tot = 0.0;
-  for (int w = 0; w < 8; ++w) tot += wd[w];
-  const double mean = tot / E;
-  for (int i = tid; i < E; i += blockDim.x)
-    bias[i] = (float)((double)bias[i] - (double)beta * (__ldcg(&u_buf[i]) - mean));
+    for (int off = 16; off; off >>= 1) v += __shfl_xor_sync(kFull, v, off);
+    if (lane == 0) wsum[warp] = v;
+    __syncthreads();
+    long long tot = 0;
+    for (int w = 0; w < 8; ++w) tot += wsum[w];
+    for (int i = tid; i < E; i += blockDim.x) {
+      const long long diff = tot - (long long)E * __ldcg(&load[i]);
+      const float dir = diff > 0 ? 1.f : (diff < 0 ? -1.f : 0.f);
+      bias[i] = __fadd_rn(bias[i], beta * dir);
+    }
+  } else {
+    double v = 0.0;
+    for (int i = tid; i < E; i += blockDim.x) v += __ldcg(&u_buf[i]);
+#pragma unroll
+    for (int off = 16; off; off >>= 1) v += __shfl_xor_sync(kFull, v, off);
+    if (lane == 0) wd[warp] = v;
+    __syncthreads();
+    double tot = 0.0;
+    for (int w = 0; w < 8; ++w) tot += wd[w];
+    const double mean = tot / E;
+    for (int i = tid; i < E; i += blockDim.x)
+      bias[i] = (float)((double)bias[i] - (double)beta * (__ldcg(&u_buf[i]) - mean));
+  }
+  for (int i = tid; i < E; i += blockDim.x) load[i] = 0;
   if (tid == 0) {
     *ntok_acc = 0;
     *done_counter = 0u;

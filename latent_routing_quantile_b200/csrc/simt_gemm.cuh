@@ -45,6 +45,8 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const SimtParams p) {
   __shared__ float Bs[BK][BN + 4];
   __shared__ float Bs1[kDual ? BK : 1][BN + 4];
 
+  pdl_wait();
+  pdl_trigger();
   int row0, row_end, e = 0;
   if (p.grouped) {
     if ((int)blockIdx.y >= *p.num_mtiles) return;

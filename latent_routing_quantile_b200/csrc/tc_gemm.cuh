@@ -162,6 +162,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
   if constexpr (PAIR) cluster_sync_all();  // the peer's barriers exist before any remote signal
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // operands, tile table and row scales come from earlier kernels
+  pdl_trigger();
   const int num_tiles = tc_num_tiles(p, PAIR);
 
   if (warp == 0) {

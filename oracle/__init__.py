@@ -22,7 +22,7 @@ Sources, cited by page title and section:
   [course] "Attention→K3 三十天课 · Day 28" (ai.air7.fun): design survival
           table (Stable LatentMoE 896 choose 16, QB, RMSNorm).
   [ebook] "免费电子书:Pretraining a Mini Kimi K3" (g.15386.cn): capsule 16
-          (aux-loss-free bias rule), capsule 20 and 25 (batched experts,
+          (aux-loss-free sign rule for the bias, gamma 1e-2), capsule 20 and 25 (batched experts,
           dispatch buffer without silent fallback), capsule 27 Bug 2
           (all-reduce of load statistics before the bias update).
   [blog]  "Kimi K3登顶开源第一，靠的是把浪费逼到墙角" (cge.wang): latent
@@ -307,6 +307,23 @@ def qb_update(b, hist: np.ndarray, N: int, k: int, beta: float, literal: bool = 
     q = np.array([histogram_quantile(hist[e], m, nbins) for e in range(E)])
     u = q if literal else q + b
     return b - beta * (u - u.mean())
+
+
+def sign_rule_update(b, load: np.ndarray, gamma: float) -> np.ndarray:
+    """The aux-loss-free bias rule: b_e <- b_e + gamma * sign(mean load - load_e).
+
+    [ebook] capsule 16 gives the rule with gamma = 1e-2 as the fix for expert
+    collapse; load_e is the number of (token, slot) pairs routed to expert e
+    since the previous update (expert_counts summed over those forwards), and
+    with data-parallel ranks it is the sum over all ranks (capsule 27, Bug 2).
+    The sign is taken exactly: mean load - load_e has the sign of
+    sum(load) - E * load_e, an integer.
+    """
+    b = f64(b)
+    load = np.asarray(load, dtype=np.int64)
+    E = load.shape[0]
+    direction = np.sign(load.sum() - E * load).astype(np.float64)
+    return b + float(gamma) * direction
 
 
 def load_ratio(counts: np.ndarray) -> float:

@@ -311,6 +311,94 @@ def test_qb_skewed_router_run():
     layer.close()
 
 
+def test_sign_rule_update_stage_exact():
+    """The sign-rule bias update on given loads is bit-exact against the oracle's rule, clears the
+    histogram, N and the loads, leaves the bias alone when nothing was recorded, and refuses the
+    literal-QB flag beside it."""
+    shape = datagen.LayerShape("sign_stage", 64, 64, 64, 256, 6, 64, 0, "bf16", seed=5)
+    E = shape.E
+    layer = make_layer(shape, datagen.layer_weights(shape))
+    rng = np.random.default_rng(5)
+    gamma = np.float32(1e-2)
+    for trial in range(4):
+        load = rng.integers(0, 50, E).astype(np.int64)
+        if trial == 1:
+            load[:] = 7  # every expert on the mean
+        if trial == 2:
+            load[: E // 2], load[E // 2:] = 3, 9
+        if trial == 3:
+            load[:] = 0
+            load[:14] = 1000  # a collapsed router: most experts never chosen
+        b = (rng.standard_normal(E) * 0.1).astype(np.float32)
+        layer.set_bias(torch.from_numpy(b).cuda())
+        layer.set_load(torch.from_numpy(load).cuda())
+        layer.set_hist(torch.ones((E, lq.NBINS), dtype=torch.int32, device="cuda"),
+                       torch.tensor([4096], dtype=torch.int64, device="cuda"))
+        layer.qb_update(float(gamma), sign_rule=True)
+        got = layer.bias().cpu().numpy()
+        want = oracle.sign_rule_update(b, load, gamma).astype(np.float32)
+        assert np.array_equal(got, want), trial
+        hist, n = layer.hist()
+        assert int(n.item()) == 0 and int(hist.abs().sum().item()) == 0
+        assert int(layer.load().abs().sum().item()) == 0
+    before = layer.bias().clone()
+    layer.qb_update(float(gamma), sign_rule=True)  # nothing recorded since the last update
+    assert torch.equal(layer.bias(), before)
+    with pytest.raises(lq.LmoeError, match="invalid"):
+        layer.qb_update(0.01, literal=True, sign_rule=True)
+    layer.close()
+
+
+def test_sign_rule_on_skewed_router_and_qb_beside_it():
+    """50 forward + update steps on the skewed router with the sign rule (gamma 1e-2, the
+    e-book's capsule 16 value), bias teacher-forced from the oracle as in the QB run: the loads a
+    forward records are its routing counts; the GPU's update equals the oracle's rule on those
+    loads bit for bit; the counts match the oracle's routing at the same bias up to near-ties.
+    Then the same 50 steps once more, free-running on the GPU alone with QB (beta 0.05), so the
+    two balancers' max/min load trajectories sit side by side in the output."""
+    shape = datagen.WORKLOADS["qb_skewed"]
+    a = json.load(open(os.path.join(GOLDEN, "qb_skew_offset.json")))["a"]
+    c = np.zeros(shape.E, dtype=np.float32)
+    c[0] = a
+    w = datagen.layer_weights(shape, router_offsets=c)
+    gamma = np.float32(1e-2)
+    layer = make_layer(shape, w)
+    b = np.zeros(shape.E, dtype=np.float32)
+    sign_ratios, nmism, load_diff = [], 0, 0
+    for step in range(shape.steps):
+        layer.set_bias(torch.from_numpy(b).cuda())
+        x = datagen.tokens(shape, seed=shape.seed + step)
+        layer.forward(x.cuda(), record_stats=True)
+        r = layer.routing()
+        load = layer.load().cpu().numpy()
+        counts = r["counts"].cpu().numpy()
+        assert np.array_equal(load, counts)
+        layer.qb_update(float(gamma), sign_rule=True)
+        b_gpu = layer.bias().cpu().numpy()
+        assert np.array_equal(b_gpu, oracle.sign_rule_update(b, load, gamma).astype(np.float32)), step
+        ro = oracle.layer_routing(x, w, b.astype(np.float64), shape.k, shape.rms_eps)
+        set_diff, order_diff = routing_mismatches(r["idx"].cpu().numpy(), ro)
+        nmism += int((set_diff | order_diff).sum())
+        load_diff += int(np.abs(counts - oracle.expert_counts(ro["idx"], shape.E)).sum())
+        sign_ratios.append(oracle.load_ratio(counts))
+        b = oracle.sign_rule_update(b, oracle.expert_counts(ro["idx"], shape.E), gamma).astype(np.float32)
+    layer.close()
+    layer = make_layer(shape, w)
+    qb_ratios = []
+    for step in range(shape.steps):
+        layer.forward(datagen.tokens(shape, seed=shape.seed + step).cuda(), record_stats=True)
+        qb_ratios.append(oracle.load_ratio(layer.routing()["counts"].cpu().numpy()))
+        layer.qb_update(shape.beta)
+    layer.close()
+    print("balancers_skewed", json.dumps(dict(sign_rule=[round(v, 3) for v in sign_ratios],
+                                              qb=[round(v, 3) for v in qb_ratios], mismatched_tokens=nmism,
+                                              load_diff=load_diff)))
+    assert nmism <= 1e-4 * shape.T * shape.steps
+    assert load_diff <= 2 * nmism
+    assert sign_ratios[0] >= 3.5 and max(sign_ratios[-10:]) < sign_ratios[0] / 2.5
+    assert qb_ratios[0] >= 3.5 and qb_ratios[-1] < 2.0
+
+
 @pytest.mark.slow
 def test_wide_stress_sampled():
     shape = datagen.WORKLOADS["wide_stress"]

@@ -61,8 +61,18 @@ MUTANTS = {
                     lambda hist_e, m, nbins=4096: _HQ(hist_e, m + 1, nbins),
                     [lambda: [pins.test_histogram_quantile_within_one_bin_of_exact(c)
                               for c in ("uniform", "sigmoid", "duplicates", "one_bin", "edges")]]),
+    # sign rule: direction flipped (hot experts pushed further up)
+    "sign_rule_flipped": ("sign_rule_update",
+                          lambda b, load, gamma: 2 * oracle.f64(b) - _SR(b, load, gamma),
+                          [pins.test_sign_rule_worked_example, pins.test_sign_rule_revives_a_collapsed_router]),
+    # sign rule: compared with the largest load instead of the mean (no bias ever falls)
+    "sign_rule_vs_max": ("sign_rule_update",
+                         lambda b, load, gamma: oracle.f64(b) + gamma * np.sign(np.max(load) - np.asarray(load)),
+                         [pins.test_sign_rule_worked_example,
+                          lambda: pins.test_sign_rule_sign_against_exact_rational_mean(0)]),
 }
 
+_SR = oracle.sign_rule_update
 _QB = oracle.qb_update
 _HQ = oracle.histogram_quantile
 

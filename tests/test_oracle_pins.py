@@ -343,6 +343,52 @@ def test_qb_single_step_at_beta_one():
     assert after < before / 3
 
 
+def test_sign_rule_worked_example():
+    """Hand-computed: loads (3, 1, 2, 2) have mean 2, so expert 0 (hot) steps down by gamma,
+    expert 1 (cold) up, experts 2 and 3 (at the mean) stay ([ebook] capsule 16)."""
+    b = np.array([0.5, -0.25, 0.0, 0.125])
+    got = oracle.sign_rule_update(b, np.array([3, 1, 2, 2]), 0.01)
+    np.testing.assert_array_equal(got, [0.49, -0.24, 0.0, 0.125])
+    # equal loads: nothing moves
+    np.testing.assert_array_equal(oracle.sign_rule_update(b, np.array([5, 5, 5, 5]), 0.01), b)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_sign_rule_sign_against_exact_rational_mean(seed):
+    """Brute force with exact rationals: the step is +gamma below the mean load, -gamma above it,
+    0 at it, for small integer loads that often sit exactly on the mean."""
+    from fractions import Fraction
+    rng = np.random.default_rng(seed)
+    E = int(rng.integers(2, 9))
+    load = rng.integers(0, 4, E)
+    b = rng.standard_normal(E)
+    got = oracle.sign_rule_update(b, load, 0.25)
+    mean = Fraction(int(load.sum()), E)
+    for e in range(E):
+        want = b[e] + (0.25 if load[e] < mean else (-0.25 if load[e] > mean else 0.0))
+        assert got[e] == want
+
+
+def test_sign_rule_revives_a_collapsed_router():
+    """[ebook] capsule 16: most experts dead (never selected) and the sign rule as the fix.  On
+    fixed scores where 4 of 32 experts take every token, repeated steps of gamma = 1e-2 bring
+    every expert back; each step moves each bias by exactly 0 or gamma."""
+    rng = np.random.default_rng(11)
+    N, E, k = 2048, 32, 2
+    off = np.zeros(E)
+    off[:4] = 3.0
+    s = oracle.sigmoid(rng.standard_normal((N, E)) * 0.5 + off)
+    b = np.zeros(E)
+    dead0 = int((oracle.expert_counts(oracle.biased_topk(s, b, k), E) == 0).sum())
+    assert dead0 >= 24
+    for _ in range(200):
+        load = oracle.expert_counts(oracle.biased_topk(s, b, k), E)
+        b1 = oracle.sign_rule_update(b, load, 1e-2)
+        assert set(np.round(np.abs(b1 - b), 12)) <= {0.0, 0.01}
+        b = b1
+    assert int((oracle.expert_counts(oracle.biased_topk(s, b, k), E) == 0).sum()) == 0
+
+
 @pytest.mark.slow
 def test_qb_skewed_router_converges_like_the_demo():
     """50 steps, beta 0.05, fresh tokens each step: max/min load starts at >= 3.5 and ends near
