@@ -291,10 +291,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&p);
 }
-// Router sigmoid: CUDA's __expf (error 2 + 1.16|z| ulp) and a correctly rounded reciprocal.  The
-// error of s = 1/(1 + e^-z) is s(1-s) times the relative error of e^-z, at most ~6e-8 (at z = 0,
-// where s(1-s) = 1/4); far from zero s(1-s) shrinks faster than the exp error grows.
-__device__ __forceinline__ float sigmoidf_acc(float z) { return __frcp_rn(1.0f + __expf(-z)); }
+// Router sigmoid: CUDA's __expf (error 2 + 1.16|z| ulp) and its fast reciprocal (__fdividef,
+// about 2 ulp).  The error of s = 1/(1 + e^-z) is s(1-s) times the relative error of e^-z plus
+// that of the reciprocal: a few 1e-7 at most, an order below the 1e-5 near-tie margin of the
+// routing checks.  A correctly rounded reciprocal (__frcp_rn) costs several times more per score
+// than the rest of the epilogue.  z below about -88 gives e^-z = inf and s = 0; NaN stays NaN.
+__device__ __forceinline__ float sigmoidf_acc(float z) { return __fdividef(1.0f, 1.0f + __expf(-z)); }
 __device__ __forceinline__ float siluf(float v) { return v / (1.0f + expf(-v)); }
 // SiLU for bf16 outputs: hardware exp2 and fast division, relative error ~1e-6, far below the
 // 2^-9 rounding of the bf16 result.  Large negative v gives exp overflow -> v / inf = -0.

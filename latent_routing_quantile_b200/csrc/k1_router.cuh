@@ -15,7 +15,13 @@
 //            the shared expert.  The parts leave by TMA stores (staged 16 KB boxes, as in the GEMM
 //            engine), stay in L2 and are loaded back by TMA once the stores have completed.
 //   Phase C  z[128, E] = six bf16 x bf16 products of the h parts with the hi/mid/lo parts of the
-//            fp32 router weights, in TMEM columns [l, l + E).
+//            fp32 router weights.  When E/ns <= l/ns (the usual case) phase C walks K chunk by
+//            chunk: the three h parts and the three weight parts of a 64-column chunk are loaded
+//            once (three ring stages) and feed all six products; hi x hi accumulates in TMEM
+//            columns [l/ns, l/ns + E/ns) and the five smaller products in columns [0, E/ns) (h's
+//            accumulator, free once phase B has read it), so the small terms are summed among
+//            themselves before phase D adds the two.  Otherwise it walks product by product
+//            (smallest first) into one accumulator, reloading parts.
 //   Phase D  epilogue: s = sigmoid(z + c), fp32.
 // Every wait is bounded as in the GEMM engine; a wait that expires sets LMOE_STATUS_WATCHDOG and
 // the CTA winds down.
@@ -40,14 +46,19 @@ struct K1Params {
   uint32_t* status;
 };
 
-constexpr int kK1Stages = 4;
-constexpr int kK1StageBytes = 16384 + 256 * 128;
-constexpr int kK1OutOffset = kK1Stages * kK1StageBytes;  // two 16 KB output boxes
+// A stage holds a 16 KB x (or h part) box and the B rows of one k-block (at most 256 x 128 bytes);
+// the ring gets as many stages as fit in 192 KB: 4 when B has 256 rows, 6 with 128 rows.
+constexpr int kK1RingBytes = 192 * 1024;
+constexpr int kK1MaxStages = 8;
+constexpr int kK1OutOffset = kK1RingBytes;  // two 16 KB output boxes
 constexpr int kK1BarOffset = kK1OutOffset + 2 * 16384;
-constexpr int kK1SmemBytes = kK1BarOffset + 1280 + 1024;  // barriers, RMS partials, alignment slack
+constexpr int kK1SmemBytes = kK1BarOffset + 384 + 1024 + 1024;  // barriers, RMS partials, alignment slack
 
 __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant__ K1Params p) {
-  constexpr int S = kK1Stages;
+  const int brows = (p.l > p.E ? p.l : p.E) / p.ns;  // B rows per stage
+  const int stage_bytes = 16384 + brows * 128;
+  int S = kK1RingBytes / stage_bytes;
+  S = S > kK1MaxStages ? kK1MaxStages : S;  // 3 x S + 11 barriers and two words fit in 384 bytes
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* smem = smem_raw + pad;
@@ -65,7 +76,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant
   uint64_t* drain = bfree + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* rms_part = reinterpret_cast<float*>(smem + kK1BarOffset + 256);  // [2][128]
+  float* rms_part = reinterpret_cast<float*>(smem + kK1BarOffset + 384);  // [2][128]
   uint8_t* obox = smem + kK1OutOffset;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -75,7 +86,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant
   const int first = (int)blockIdx.x / ns, stride = (int)gridDim.x / ns;
   const uint32_t tmem_cols = ns == 2 ? 256u : 512u;
   const int nkd = p.d / 64, nkl = p.l / 64;
-  const int nkbA = nkd * p.wd_segments, nkbC = 6 * nkl;
+  const bool dual = eh <= lh;  // phase C chunk-major with a second accumulator (see above)
+  const int nkbA = nkd * p.wd_segments, nkbC = (dual ? 3 : 6) * nkl;
   const uint32_t bytesA = 16384u + (uint32_t)lh * 128u, bytesC = 16384u + (uint32_t)eh * 128u;
   // the six significant products of (hi, mid, lo) parts, smallest first, as (A part, B part):
   // (mid, mid), (lo, hi), (hi, lo), (mid, hi), (hi, mid), (hi, hi); three bits per product
@@ -151,7 +163,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant
             }
             rms_pend &= ~(1u << stage);
           }
-          uint8_t* a_dst = smem + stage * kK1StageBytes;
+          uint8_t* a_dst = smem + stage * stage_bytes;
           uint8_t* b_dst = a_dst + 16384;
           if (kb < nkbA) {
             const int seg = kb / nkd, kk = kb - seg * nkd;
@@ -164,9 +176,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant
               rms_cnt ^= 1u << stage;
             }
           } else {
-            const int pr = (kb - nkbA) / nkl, kk = (kb - nkbA) - pr * nkl;
+            int kk, pa, pb;
+            if (dual) {  // chunk kk, part pa = pb of h and of the router weights
+              kk = (kb - nkbA) / 3;
+              pa = pb = (kb - nkbA) - 3 * kk;
+            } else {     // product pr, chunk kk
+              const int pr = (kb - nkbA) / nkl;
+              kk = (kb - nkbA) - pr * nkl;
+              pa = (int)((kProdA >> (3 * pr)) & 7u);
+              pb = (int)((kProdB >> (3 * pr)) & 7u);
+            }
             mbar_expect_tx(&full[stage], bytesC);
-            const int pa = (int)((kProdA >> (3 * pr)) & 7u), pb = (int)((kProdB >> (3 * pr)) & 7u);
             tma_load_2d(a_dst, &p.tm_hx, &full[stage], pa * p.l + kk * 64, row0);
             tma_load_2d(b_dst, &p.tm_wr, &full[stage], pb * p.l + kk * 64, (int)rank * eh);
           }
@@ -197,7 +217,52 @@ __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant
             ok = false;
             break;
           }
+          // dual phase C writes columns [0, E/ns): the epilogue must have read h out of them, and
+          // the next phase A must wait until phase D has read the small products
+          if (dual && !mbar_wait(ph == 0 ? tempC : tempA, ph == 0 ? (it & 1) ^ 1u : (it & 1), abort, p.status)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
+          if (ph == 1 && dual) {
+            const uint32_t d_big = tmem_base + (uint32_t)lh, d_small = tmem_base;
+            for (int kk = 0; ok && kk < nkl; ++kk) {
+              uint32_t a_addr[3], b_addr[3];
+              int st3[3];
+#pragma unroll
+              for (int q = 0; q < 3; ++q) {
+                if (!mbar_wait(&full[stage], phase, abort, p.status)) {
+                  ok = false;
+                  break;
+                }
+                a_addr[q] = smem_u32(smem + stage * stage_bytes);
+                b_addr[q] = a_addr[q] + 16384;
+                st3[q] = stage;
+                if (++stage == S) {
+                  stage = 0;
+                  phase ^= 1u;
+                }
+              }
+              if (!ok) break;
+              tc_fence_after();
+#pragma unroll
+              for (int pr = 0; pr < 5; ++pr) {  // (mid,mid) (lo,hi) (hi,lo) (mid,hi) (hi,mid)
+                const int pa = (int)((kProdA >> (3 * pr)) & 7u), pb = (int)((kProdB >> (3 * pr)) & 7u);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                  tc_mma_bf16(d_small, smem_desc_sw128(a_addr[pa] + k * 32), smem_desc_sw128(b_addr[pb] + k * 32),
+                              idescC, (kk | pr | k) != 0);
+              }
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                tc_mma_bf16(d_big, smem_desc_sw128(a_addr[0] + k * 32), smem_desc_sw128(b_addr[0] + k * 32), idescC,
+                            (kk | k) != 0);
+#pragma unroll
+              for (int q = 0; q < 3; ++q) tc_commit(&empty[st3[q]]);
+            }
+            if (ok) tc_commit(tfullC);
+            continue;
+          }
           const uint32_t d_tmem = tmem_base + (ph == 0 ? 0u : (uint32_t)lh);
           const uint32_t idesc = ph == 0 ? idescA : idescC;
           for (int kb = 0; kb < nkb; ++kb) {
@@ -206,7 +271,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant
               break;
             }
             tc_fence_after();
-            const uint32_t a_addr = smem_u32(smem + stage * kK1StageBytes);
+            const uint32_t a_addr = smem_u32(smem + stage * stage_bytes);
             const uint32_t b_addr = a_addr + 16384;
 #pragma unroll
             for (int k = 0; k < 4; ++k)
@@ -286,7 +351,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant
             ok = false;
             break;
           }
-          const uint8_t* a_row = smem + stage * kK1StageBytes + rl * 128;
+          const uint8_t* a_row = smem + stage * stage_bytes + rl * 128;
           float f = 0.f;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
@@ -365,13 +430,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant
       bool nan = false;
 #pragma unroll 1
       for (int j = 0; ok && j < eh / 32; ++j) {
-        uint32_t v[16];
+        uint32_t v[16], vs[16];
         tmem_ld16(tbase + lh + j * 32 + half_id * 16, v);
+        if (dual) tmem_ld16(tbase + j * 32 + half_id * 16, vs);
         float cj = c_lane[0];  // select by unrolled compares: no dynamic register indexing
 #pragma unroll
         for (int jj = 1; jj < 8; ++jj)
           if (jj == j) cj = c_lane[jj];
         tc_wait_ld();
+        if (dual) {
+#pragma unroll
+          for (int q = 0; q < 16; ++q) v[q] = __float_as_uint(__uint_as_float(v[q]) + __uint_as_float(vs[q]));
+        }
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
           // lane m of the warp holds offset j*32 + m (loaded at the start of the kernel)
