@@ -58,7 +58,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant
   const int brows = (p.l > p.E ? p.l : p.E) / p.ns;  // B rows per stage
   const int stage_bytes = 16384 + brows * 128;
   int S = kK1RingBytes / stage_bytes;
-  S = S > kK1MaxStages ? kK1MaxStages : S;  // 3 x S + 11 barriers and two words fit in 384 bytes
+  S = S > kK1MaxStages ? kK1MaxStages : S;  // 3 x S + 13 barriers and two words fit in 384 bytes
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* smem = smem_raw + pad;
@@ -74,7 +74,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant
   uint64_t* bfull = rmsx + 1;  // output box written by all epilogue warps
   uint64_t* bfree = bfull + 2; // output box read by its TMA store
   uint64_t* drain = bfree + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* hxs = drain + 1;   // every epilogue warp has staged its h parts in the ring
+  uint64_t* sds = hxs + 1;     // every epilogue warp has staged its scores in the ring (last tile)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sds + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* rms_part = reinterpret_cast<float*>(smem + kK1BarOffset + 384);  // [2][128]
   uint8_t* obox = smem + kK1OutOffset;
@@ -111,6 +113,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant
       mbar_init(&bfree[i], 1);
     }
     mbar_init(drain, 1);
+    mbar_init(hxs, kEpiWarps);
+    mbar_init(sds, kEpiWarps);
     *abort = 0;
     fence_mbar_init();
     tma_prefetch_desc(&p.tm_x);
@@ -382,23 +386,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant
       const float rr =
           (float)(1.0 / sqrt(((double)rms_part[rl] + (double)rms_part[128 + rl]) / p.d + (double)p.eps));
       if (half_id == 0 && valid && rank == 0) p.r[row] = rr;
-      // phase B: h = r * acc as hi | mid | lo bf16 parts, one staged box per part and 64 columns
+      // phase B: h = r * acc as hi | mid | lo bf16 parts.  The ring is idle until every part is
+      // stored (phase A's loads are consumed, and the producer waits for hxr before phase C), so
+      // box (chunk j, part) is staged at ring offset (3 j + part) * 16 KB and the storer issues
+      // all the TMA stores at once.
       ok = mbar_wait(tfullA, it & 1, abort, p.status);
       __syncwarp();
       if (__any_sync(0xffffffffu, !ok)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(wq * 32) << 16);
-      uint32_t w[16];
 #pragma unroll 1
-      for (int j = 0; ok && j < lh / 64; ++j) {
+      for (int j = 0; j < lh / 64; ++j) {
         uint32_t v[32];
         tmem_ld32(tbase + j * 64 + half_id * 32, v);
         tc_wait_ld();
         float a[32];
 #pragma unroll
         for (int q = 0; q < 32; ++q) a[q] = __uint_as_float(v[q]) * rr;
-#pragma unroll 1
-        for (int part = 0; ok && part < 3; ++part) {
+#pragma unroll
+        for (int part = 0; part < 3; ++part) {
+          uint32_t w[16];
 #pragma unroll
           for (int q = 0; q < 16; ++q) {
             const bf16 h0 = __float2bfloat16_rn(a[2 * q]), h1 = __float2bfloat16_rn(a[2 * q + 1]);
@@ -407,27 +414,45 @@ __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant
             a[2 * q] -= __bfloat162float(h0);
             a[2 * q + 1] -= __bfloat162float(h1);
           }
-          ok = emit(w, &p.tm_hx, part * p.l + (int)rank * lh + j * 64, row0);
+          uint8_t* box = smem + (3 * j + part) * 16384;
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4*>(box + sw128_offset(rl, half_id * 4 + q)) =
+                make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
         }
       }
-      if (!ok) break;
+      fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(tempA);
+      if (lane == 0) {
+        mbar_arrive(tempA);
+        mbar_arrive(hxs);
+      }
       if (storer) {
+        ok = mbar_wait(hxs, it & 1, abort, p.status);
+        __syncwarp();
+        if (__any_sync(0xffffffffu, !ok)) break;
         if (lane == 0) {
-          bulk_wait_all();  // the h parts are in global memory before phase C loads them
+          for (int j = 0; j < lh / 64; ++j)
+            for (int part = 0; part < 3; ++part)
+              tma_store_2d(&p.tm_hx, smem + (3 * j + part) * 16384, part * p.l + (int)rank * lh + j * 64, row0);
+          bulk_commit();
+          bulk_wait_all();  // the h parts are in global memory (and the ring is free) before phase C
           mbar_arrive(hxr);  // own barrier first: the peer's next arrival comes after it
           if (ns == 2) mbar_arrive_cluster(mapa_shared(smem_u32(hxr), rank ^ 1u));
         }
         __syncwarp();
       }
-      // phase D: s = sigmoid(z + c), fp32, 32 columns per box (16 per warp)
+      // phase D: s = sigmoid(z + c), fp32, 32 columns per box (16 per warp).  On this CTA's last
+      // tile the ring is idle once phase C's products are done (no loads follow), so every box is
+      // staged there (box j at j * 16 KB) and stored at once; otherwise the two-box ring of emit.
       ok = mbar_wait(tfullC, it & 1, abort, p.status);
       __syncwarp();
       if (__any_sync(0xffffffffu, !ok)) break;
       tc_fence_after();
+      const bool last_tile = tile + stride >= num_tiles;
       bool nan = false;
+      uint32_t w[16];
 #pragma unroll 1
       for (int j = 0; ok && j < eh / 32; ++j) {
         uint32_t v[16], vs[16];
@@ -450,9 +475,32 @@ __global__ void __launch_bounds__(kTcThreads, 1) k1_kernel(const __grid_constant
           nan |= (o != o);
           w[q] = __float_as_uint(o);
         }
-        ok = emit(w, &p.tm_s, (int)rank * eh + j * 32, row0);
+        if (last_tile) {
+          uint8_t* box = smem + j * 16384;
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4*>(box + sw128_offset(rl, half_id * 4 + q)) =
+                make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+        } else {
+          ok = emit(w, &p.tm_s, (int)rank * eh + j * 32, row0);
+        }
       }
       if (!ok) break;
+      if (last_tile) {
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sds);
+        if (storer) {
+          ok = mbar_wait(sds, 0, abort, p.status);
+          __syncwarp();
+          if (__any_sync(0xffffffffu, !ok)) break;
+          if (lane == 0) {
+            for (int j = 0; j < eh / 32; ++j) tma_store_2d(&p.tm_s, smem + j * 16384, (int)rank * eh + j * 32, row0);
+            bulk_commit();
+          }
+          __syncwarp();
+        }
+      }
       if (nan && valid) set_status(p.status, LMOE_STATUS_NAN_SCORE);
       tc_fence_before();
       __syncwarp();

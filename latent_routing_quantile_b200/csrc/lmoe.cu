@@ -321,6 +321,9 @@ struct lmoe_handle {
   // tensor maps (bf16)
   // weight maps of the non-grouped GEMMs exist for each tile width 64/128/256 that divides N
   CUtensorMap tm_hx, tm_aperm, tm_w13, tm_act, tm_w2, tm_z, tm_as, tm_o, tm_s;
+  // A_perm, act and o with boxes of 32, 64 and 96 rows: the grouped GEMMs move only the valid
+  // rows of an expert's last tile
+  CUtensorMap tm_aperm_part[3], tm_act_part[3], tm_o_part[3];
   CUtensorMap tm_wr[3], tm_wdown[3], tm_ws13[3], tm_wy[3];
   bool fused_k1 = false;       // l <= 256 and E <= 256: RMSNorm + W_down + router in one kernel
   CUtensorMap tm_k1_wd, tm_k1_wr;        // boxes of the whole of l and E rows (one CTA per tile)
@@ -454,6 +457,11 @@ int build_maps(lmoe_handle* h) {
   ok &= make_map(&h->tm_w13, h->w13, E * 2 * hh, l, l, h->bn_e1);
   ok &= make_map(&h->tm_act, h->act, RP, hh, hh, 128);
   ok &= make_map(&h->tm_o, h->o, RP, l, l, 128);
+  for (int i = 0; i < 3; ++i) {
+    ok &= make_map(&h->tm_aperm_part[i], h->a_perm, RP, l, l, 32 * (i + 1));
+    ok &= make_map(&h->tm_act_part[i], h->act, RP, hh, hh, 32 * (i + 1));
+    ok &= make_map(&h->tm_o_part[i], h->o, RP, l, l, 32 * (i + 1));
+  }
   ok &= make_map_f32(&h->tm_s, h->s, Tm, E, E, 128);
   ok &= make_map(&h->tm_w2, h->w2, E * l, hh, hh, h->bn_e2);
   ok &= make_map(&h->tm_z, h->z, Tm, l, l, 128);
@@ -665,6 +673,13 @@ int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, 
     p.num_mtiles = h->num_mtiles;
     p.b_rows_per_group = 2 * c.h;
     p.tmOut = h->tm_act;
+    p.trim = 1;
+    for (int i = 0; i < 3; ++i) {
+      p.tmA_part[i] = h->tm_aperm_part[i];
+      p.tmOut_part[i] = h->tm_act_part[i];
+    }
+    p.hint_b = 1;    // each expert's weights serve its few tiles, then not again this step
+    p.hint_out = 1;  // act is read by the next GEMM
     CK(launch_tc(p, EPI_SWIGLU, h->bn_e1, h->sms, st));
   }
   mark(h, ST_EXPERT2, st);
@@ -681,6 +696,14 @@ int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, 
     p.num_mtiles = h->num_mtiles;
     p.b_rows_per_group = c.l;
     p.tmOut = h->tm_o;
+    p.trim = 1;
+    for (int i = 0; i < 3; ++i) {
+      p.tmA_part[i] = h->tm_act_part[i];
+      p.tmOut_part[i] = h->tm_o_part[i];
+    }
+    p.hint_a = 1;    // last read of act
+    p.hint_b = 1;
+    p.hint_out = 1;  // o is read by the combine kernel
     CK(launch_tc(p, EPI_BF16, h->bn_e2, h->sms, st));
   }
   mark(h, ST_COMBINE, st);

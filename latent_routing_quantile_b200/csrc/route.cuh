@@ -254,7 +254,9 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ coun
     const int mt_start = block_exclusive_scan_1024(mt, sh, &mt_total);
     const int poff = mt_start * kTileRows;  // padded offset of this expert
     if (tid < E) pad_delta[tid] = poff - off;
-    for (int j = 0; j < mt; ++j) mtiles[mt_start + j] = make_int2(tid, poff + j * kTileRows);
+    // entry: x = expert | (valid rows of the tile << 16), y = first row in the padded layout
+    for (int j = 0; j < mt; ++j)
+      mtiles[mt_start + j] = make_int2(tid | (min(kTileRows, c - j * kTileRows) << 16), poff + j * kTileRows);
     if (tid == 0) *num_mtiles = mt_total;
   }
   __syncthreads();

@@ -51,7 +51,7 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const SimtParams p) {
   if (p.grouped) {
     if ((int)blockIdx.y >= *p.num_mtiles) return;
     int2 er = p.mtile_table[blockIdx.y];
-    e = er.x;
+    e = er.x & 0xFFFF;  // the high half holds the tile's valid rows
     row0 = er.y;
     row_end = row0 + BM;  // padded expert layout: the whole tile belongs to expert e
   } else {

@@ -12,10 +12,13 @@
 // 128 x BN, K steps of 64 (one 128-byte swizzle atom).  The grid is at most one CTA per SM and
 // walks the tile list with a stride of gridDim.x.
 //
-// Grouped mode (routed experts): M-tiles come from a device table of (expert, first row) built
-// after the routing counts, and B rows are offset by expert * b_rows_per_group.  Every expert's
-// rows start on a multiple of 128, so a tile never holds rows of two experts; the padding rows
-// are computed and stored but never read.
+// Grouped mode (routed experts): M-tiles come from a device table of (expert, valid rows, first
+// row) built after the routing counts, and B rows are offset by expert * b_rows_per_group.
+// Every expert's rows start on a multiple of 128, so a tile never holds rows of two experts.
+// With `trim`, a tile with R < 128 valid rows loads and stores only ceil(R/32)*32 rows (tensor
+// maps with 32/64/96-row boxes): the padding rows cost no memory traffic.  The MMA still runs
+// 128 rows; rows past the load hold stale shared memory, and only their own output rows, which
+// are never stored, depend on them.
 //
 // K is described by up to 6 segments, each naming which A tensor map and which A and B columns
 // its k-blocks read; this expresses concatenated-K products ([z | a_s] [W_up | Ws2]^T) and the
@@ -46,6 +49,8 @@ struct TcParams {
   CUtensorMap tmA[2];
   CUtensorMap tmB;
   CUtensorMap tmOut;          // output: box 64 x 128 (bf16) or 32 x 128 (fp32), 128-byte swizzle
+  CUtensorMap tmA_part[3];    // trim: tmA[0] with boxes of 32, 64, 96 rows
+  CUtensorMap tmOut_part[3];  // trim: tmOut with boxes of 32, 64, 96 rows
   KSeg seg[6];
   int nseg;
   int grouped;
@@ -58,6 +63,9 @@ struct TcParams {
   int split;                  // EPI_DOWN3: column offset between the three parts
   const float* row_scale;
   const float* col_bias;
+  int trim;                   // grouped: move only the valid rows of a tile, rounded up to 32
+  int hint_a, hint_b;         // 1: load A / B with L2 evict_first (read once, not again soon)
+  int hint_out;               // 1: store the output with L2 evict_last (the next kernel reads it)
   uint32_t* status;
 };
 
@@ -77,19 +85,22 @@ struct TcCfg {
 
 struct TileInfo {
   int row0, b_row0, n0;
+  int q;  // 32-row quarters of the tile that are loaded and stored (4 = all)
 };
 
 __device__ __forceinline__ TileInfo tc_tile(const TcParams& p, int tile, int BN, int pair, uint32_t rank) {
   TileInfo ti;
   int mt = tile / p.n_tiles, nt = tile - mt * p.n_tiles;
   ti.n0 = nt * BN;
+  ti.q = 4;
   if (pair) {  // 256-row tiles; this CTA owns rows 128*rank.. and B rows BN/2*rank..
     ti.row0 = mt * 256 + (int)rank * 128;
     ti.b_row0 = ti.n0 + (int)rank * (BN / 2);
   } else if (p.grouped) {
     int2 e_r = p.mtile_table[mt];
     ti.row0 = e_r.y;
-    ti.b_row0 = e_r.x * p.b_rows_per_group + ti.n0;
+    ti.b_row0 = (e_r.x & 0xFFFF) * p.b_rows_per_group + ti.n0;
+    if (p.trim) ti.q = ((e_r.x >> 16) + 31) >> 5;
   } else {
     ti.row0 = mt * 128;
     ti.b_row0 = ti.n0;
@@ -147,6 +158,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     tma_prefetch_desc(&p.tmA[1]);
     tma_prefetch_desc(&p.tmB);
     tma_prefetch_desc(&p.tmOut);
+    if (p.trim)
+      for (int i = 0; i < 3; ++i) {
+        tma_prefetch_desc(&p.tmA_part[i]);
+        tma_prefetch_desc(&p.tmOut_part[i]);
+      }
   }
   if (warp == 1) {
     if constexpr (PAIR) {
@@ -172,6 +188,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed = 0, armed_parity = 0;  // per-stage bits, for the abort drain
+      const uint64_t pol_first = l2_evict_first();
       bool ok = true;
       for (int tile = first; ok && tile < num_tiles; tile += stride) {
         TileInfo ti = tc_tile(p, tile, BN, PAIR, rank);
@@ -191,9 +208,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
               tma_load_2d_pair(a_dst, &p.tmA[sg.a_map], bar0, sg.a_col + kb * 64, ti.row0);
               tma_load_2d_pair(b_dst, &p.tmB, bar0, sg.b_col + kb * 64, ti.b_row0);
             } else {
-              mbar_expect_tx(&full[stage], C::kStageBytes);
-              tma_load_2d(a_dst, &p.tmA[sg.a_map], &full[stage], sg.a_col + kb * 64, ti.row0);
-              tma_load_2d(b_dst, &p.tmB, &full[stage], sg.b_col + kb * 64, ti.b_row0);
+              const CUtensorMap* amap = ti.q < 4 ? &p.tmA_part[ti.q - 1] : &p.tmA[sg.a_map];
+              mbar_expect_tx(&full[stage], (uint32_t)(ti.q * 32 * 128 + C::kBBytes));
+              if (p.hint_a)
+                tma_load_2d_hint(a_dst, amap, &full[stage], sg.a_col + kb * 64, ti.row0, pol_first);
+              else
+                tma_load_2d(a_dst, amap, &full[stage], sg.a_col + kb * 64, ti.row0);
+              if (p.hint_b)
+                tma_load_2d_hint(b_dst, &p.tmB, &full[stage], sg.b_col + kb * 64, ti.b_row0, pol_first);
+              else
+                tma_load_2d(b_dst, &p.tmB, &full[stage], sg.b_col + kb * 64, ti.b_row0);
             }
             armed |= 1u << stage;
             armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
@@ -284,6 +308,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     uint32_t step = 0;                      // output boxes so far (alternating staging buffers)
     bool ok = true;
     // Writes this thread's 64 bytes into the current box, then (storer) stores the box.
+    const CUtensorMap* omap = &p.tmOut;  // this tile's output map (trim: only its valid rows)
     auto emit = [&](const uint32_t (&w)[16], int x, int y) -> bool {
       const int buf = step & 1;
       const uint32_t par = (step >> 1) & 1u;
@@ -303,7 +328,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         __syncwarp();
         if (__any_sync(0xffffffffu, !good)) return false;
         if (lane == 0) {
-          tma_store_2d(&p.tmOut, box, x, y);
+          if (p.hint_out)
+            tma_store_2d_hint(omap, box, x, y, l2_evict_last());
+          else
+            tma_store_2d(omap, box, x, y);
           bulk_commit();
           if (step > 0) {
             bulk_wait_read<1>();  // the previous box has been read: its buffer is free
@@ -335,6 +363,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       }
       tc_fence_after();
       TileInfo ti = tc_tile(p, tile, BN, PAIR, rank);
+      omap = ti.q < 4 ? &p.tmOut_part[ti.q - 1] : &p.tmOut;
       const int row = ti.row0 + rl;
       const uint32_t tbase = tmem_base + ((uint32_t)(wq * 32) << 16) + acc * BN;
       const float rs = (p.row_scale != nullptr && row < p.M_rows) ? p.row_scale[row] : 1.0f;
