@@ -153,7 +153,10 @@ int lmoe_get_routing(lmoe_handle *h, int32_t *idx, float *gates, float *scores, 
                      int32_t *offsets, int32_t *perm, int32_t *inv, void *stream);
 
 /* QB state: bias b [E] fp32 (device), histogram [E, 4096] uint32 and token count N (int64),
- * all device pointers. */
+ * all device pointers.  The scores of the last recorded forward are kept as per-score bins and
+ * counted by the next lmoe_qb_update directly; lmoe_get_hist (and a second recorded forward)
+ * first adds them to the histogram, so what it returns always covers every recorded forward.
+ * lmoe_set_hist replaces all statistics recorded so far. */
 int lmoe_get_bias(lmoe_handle *h, float *b_dev, void *stream);
 int lmoe_set_bias(lmoe_handle *h, const float *b_dev, void *stream);
 int lmoe_get_hist(lmoe_handle *h, uint32_t *hist_dev, int64_t *ntok_dev, void *stream);

@@ -249,12 +249,13 @@ struct GraphCache {
   int T = -1;
   uint32_t flags = 0;
   float beta = 0.f;
+  uint64_t state = 0;  // the statistics state the call started from (it decides the kernels)
   int seen = 0;
   long long kernels = 0;
-  bool same(const void* x_, void* y_, int T_, uint32_t f_, float b_) const {
-    return x == x_ && y == y_ && T == T_ && flags == f_ && beta == b_;
+  bool same(const void* x_, void* y_, int T_, uint32_t f_, float b_, uint64_t s_) const {
+    return x == x_ && y == y_ && T == T_ && flags == f_ && beta == b_ && state == s_;
   }
-  void reset(const void* x_, void* y_, int T_, uint32_t f_, float b_) {
+  void reset(const void* x_, void* y_, int T_, uint32_t f_, float b_, uint64_t s_) {
     if (exec) cudaGraphExecDestroy(exec);
     exec = nullptr;
     x = x_;
@@ -262,9 +263,21 @@ struct GraphCache {
     T = T_;
     flags = f_;
     beta = b_;
+    state = s_;
     seen = 0;
     kernels = 0;
   }
+};
+
+// Where the statistics of recorded forwards stand.  A recorded forward's score bins stay in one
+// of two bin buffers, uncounted ("pending"), until the next lmoe_qb_update counts them into its
+// histogram quantiles directly, or another recorded forward or lmoe_get_hist adds them to the
+// accumulated histogram (hist_live: the accumulated rows may be non-zero).
+struct StatsState {
+  int pend_T = 0;      // tokens of the pending bins (0: none)
+  int pend_buf = 0;    // bin buffer holding them
+  bool hist_live = false;
+  uint64_t key() const { return ((uint64_t)(uint32_t)pend_T << 2) | ((uint64_t)pend_buf << 1) | (hist_live ? 1u : 0u); }
 };
 
 struct ProfRecord {
@@ -298,7 +311,8 @@ struct lmoe_handle {
   float* r = nullptr;
   void* hx = nullptr;       // bf16 [Tm, 3l] (hi|mid|lo of h); f32 [Tm, l]
   float* s = nullptr;
-  uint16_t* bins = nullptr;  // [E, ld_bins] histogram bin of every score, expert-major
+  uint16_t* bins = nullptr;  // 2 x [E, ld_bins] histogram bin of every score, expert-major
+  StatsState ss;
   int *idx = nullptr, *rank = nullptr, *blkcnt = nullptr, *blkbase = nullptr, *counts = nullptr;
   int* counts32 = nullptr;  // [32][E] partial counts of the top-k blocks
   bool counts32_dirty = true;
@@ -373,7 +387,7 @@ void plan_layout(lmoe_handle* h, Arena& a) {
   a.add((void**)&h->r, Tm * 4);
   a.add(&h->hx, h->bf ? Tm * 3 * l * 2 : Tm * l * 4);
   a.add((void**)&h->s, Tm * E * 4);
-  a.add((void**)&h->bins, (size_t)h->ld_bins * E * 2);
+  a.add((void**)&h->bins, 2 * (size_t)h->ld_bins * E * 2);
   a.add((void**)&h->idx, TK * 4);
   a.add((void**)&h->gates, TK * 4);
   a.add((void**)&h->rank, TK * 4);
@@ -510,7 +524,29 @@ TcParams tc_base(lmoe_handle* h) {
 }
 
 // ---- stages shared by lmoe_forward and lmoe_route_scores
-int route_from_scores(lmoe_handle* h, int T, uint32_t flags, cudaStream_t st) {
+uint16_t* bin_buffer(lmoe_handle* h, int i) { return h->bins + (size_t)i * h->ld_bins * h->cfg.E; }
+
+// State after a routing of T tokens with `flags` that started from `pre`.
+StatsState after_routing(const StatsState& pre, int T, uint32_t flags) {
+  StatsState post = pre;
+  if (flags & LMOE_RECORD_STATS) {
+    if (pre.pend_T) post.hist_live = true;
+    post.pend_buf = pre.pend_T ? pre.pend_buf ^ 1 : pre.pend_buf;
+    post.pend_T = T;
+  }
+  return post;
+}
+
+// Adds pending bins (pend_T tokens, buffer buf) to the accumulated histogram and N.
+int flush_bins(lmoe_handle* h, int pend_T, int buf, cudaStream_t st) {
+  CK(launch_k(hist_kernel, dim3(h->cfg.E), dim3(kHistThreads), 0, st, 1, (const uint16_t*)bin_buffer(h, buf),
+              h->ld_bins, pend_T, h->hist, h->ntok));
+  h->launches += 1;
+  return LMOE_OK;
+}
+
+int route_from_scores(lmoe_handle* h, int T, uint32_t flags, const StatsState& pre, cudaStream_t st) {
+  const StatsState post = after_routing(pre, T, flags);
   const lmoe_config& c = h->cfg;
   const int nblk = (T + kTokBlock - 1) / kTokBlock;
   mark(h, ST_TOPK, st);
@@ -519,7 +555,7 @@ int route_from_scores(lmoe_handle* h, int T, uint32_t flags, cudaStream_t st) {
   if (h->counts32_dirty) CK(cudaMemsetAsync(h->counts32, 0, (size_t)kCountCopies * c.E * sizeof(int), st));
   h->counts32_dirty = true;
   TopkArgs ta{h->s, h->bias, T, c.E, c.k, h->idx, h->rank, h->blkcnt, h->counts32, h->gates,
-              (flags & LMOE_RECORD_STATS) ? h->bins : nullptr, h->ld_bins, h->status};
+              (flags & LMOE_RECORD_STATS) ? bin_buffer(h, post.pend_buf) : nullptr, h->ld_bins, h->status};
   CK(launch_topk(ta, st));
   mark(h, ST_PLAN, st);
   CK(launch_k(plan_kernel, dim3((c.E + 31) / 32), dim3(1024), 0, st, 1, (const int*)h->counts32, h->counts,
@@ -542,16 +578,18 @@ int route_from_scores(lmoe_handle* h, int T, uint32_t flags, cudaStream_t st) {
   h->counts32_dirty = false;
   mark(h, ST_HIST, st);
   h->launches += 3;
-  if (flags & LMOE_RECORD_STATS) {
-    CK(launch_k(hist_kernel, dim3(c.E), dim3(kHistThreads), 0, st, 1, (const uint16_t*)h->bins, h->ld_bins, T,
-                h->hist, h->ntok));
-    h->launches += 1;
+  // the bins of an earlier recorded forward that no update has counted yet join the histogram
+  // before their buffer is reused (this forward's own bins stay pending for lmoe_qb_update)
+  if ((flags & LMOE_RECORD_STATS) && pre.pend_T) {
+    int rc = flush_bins(h, pre.pend_T, pre.pend_buf, st);
+    if (rc) return rc;
   }
   h->last_T = T;
   return LMOE_OK;
 }
 
-int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, cudaStream_t st) {
+int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, const StatsState& pre,
+                 cudaStream_t st) {
   const lmoe_config& c = h->cfg;
   const int mt = (T + 127) / 128;
   CUtensorMap tm_x;
@@ -631,7 +669,7 @@ int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, 
     mark(h, ST_K1, st);
     h->launches += 3;
   }
-  int rc = route_from_scores(h, T, flags, st);
+  int rc = route_from_scores(h, T, flags, pre, st);
   if (rc) return rc;
   // shared expert, first half: a_s = silu(r x Ws1^T) * (r x Ws3^T)
   mark(h, ST_SHARED, st);
@@ -737,7 +775,8 @@ int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, 
   return LMOE_OK;
 }
 
-int forward_f32(lmoe_handle* h, const void* xv, void* yv, int T, uint32_t flags, cudaStream_t st) {
+int forward_f32(lmoe_handle* h, const void* xv, void* yv, int T, uint32_t flags, const StatsState& pre,
+                cudaStream_t st) {
   const lmoe_config& c = h->cfg;
   const float* x = (const float*)xv;
   const int mt = (T + 127) / 128;
@@ -765,7 +804,7 @@ int forward_f32(lmoe_handle* h, const void* xv, void* yv, int T, uint32_t flags,
     CK(launch_simt<SE_ROUTER>(p, mt, st));
   }
   mark(h, ST_K1, st);
-  int rc = route_from_scores(h, T, flags, st);
+  int rc = route_from_scores(h, T, flags, pre, st);
   if (rc) return rc;
   mark(h, ST_SHARED, st);
   if (c.hs) {  // a_s = silu(r x Ws1'^T) * (r x Ws3'^T)
@@ -892,12 +931,12 @@ bool gain_is_unit(const lmoe_config& c, const void* g) {
 // stream.  Eager whenever profiling is on or the caller's stream is itself being captured.
 template <typename F>
 int run_cached(lmoe_handle* h, GraphCache& g, const void* x, void* y, int T, uint32_t flags, float beta,
-               cudaStream_t st, F body) {
+               uint64_t state, cudaStream_t st, F body) {
   cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
   if (h->profiling || cudaStreamIsCapturing(st, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) {
     return body(st);
   }
-  if (!g.same(x, y, T, flags, beta)) g.reset(x, y, T, flags, beta);
+  if (!g.same(x, y, T, flags, beta, state)) g.reset(x, y, T, flags, beta, state);
   if (g.exec) {
     CK(cudaGraphLaunch(g.exec, st));
     h->launches += g.kernels;
@@ -1022,8 +1061,8 @@ int lmoe_destroy(lmoe_handle* h) {
   cudaDeviceSynchronize();
   for (auto& r : h->prof)
     for (auto& e : r.ev) cudaEventDestroy(e);
-  h->g_fwd.reset(nullptr, nullptr, -1, 0, 0.f);
-  h->g_qb.reset(nullptr, nullptr, -1, 0, 0.f);
+  h->g_fwd.reset(nullptr, nullptr, -1, 0, 0.f, 0);
+  h->g_qb.reset(nullptr, nullptr, -1, 0, 0.f, 0);
   if (h->cap) cudaStreamDestroy(h->cap);
   cudaFree(h->arena);
   delete h;
@@ -1038,12 +1077,15 @@ int lmoe_forward(lmoe_handle* h, const void* x, void* y, int32_t T, uint32_t fla
   if ((const char*)x < (const char*)y + bytes && (const char*)y < (const char*)x + bytes) return LMOE_EINVAL;
   cudaStream_t st = (cudaStream_t)stream;
   h->last_T = T;
-  return run_cached(h, h->g_fwd, x, y, T, flags, 0.f, st, [&](cudaStream_t s) {
+  const StatsState pre = h->ss;
+  int rc = run_cached(h, h->g_fwd, x, y, T, flags, 0.f, pre.key(), st, [&](cudaStream_t s) {
     prof_open(h, ST_RMS, ST_UP - ST_RMS + 1);
-    int rc = h->bf ? forward_bf16(h, x, y, T, flags, s) : forward_f32(h, x, y, T, flags, s);
+    int r = h->bf ? forward_bf16(h, x, y, T, flags, pre, s) : forward_f32(h, x, y, T, flags, pre, s);
     prof_close(h, s);
-    return rc;
+    return r;
   });
+  if (rc == LMOE_OK) h->ss = after_routing(pre, T, flags);
+  return rc;
 }
 
 int lmoe_forward_host(lmoe_handle* h, const void* x_host, void* y_host, int32_t T, uint32_t flags, void* stream) {
@@ -1064,8 +1106,10 @@ int lmoe_route_scores(lmoe_handle* h, const float* scores, int32_t T, uint32_t f
   cudaStream_t st = (cudaStream_t)stream;
   CK(cudaMemcpyAsync(h->s, scores, (size_t)T * h->cfg.E * 4, cudaMemcpyDeviceToDevice, st));
   prof_open(h, ST_TOPK, ST_HIST - ST_TOPK + 1);
-  int rc = route_from_scores(h, T, flags, st);
+  const StatsState pre = h->ss;
+  int rc = route_from_scores(h, T, flags, pre, st);
   prof_close(h, st);
+  if (rc == LMOE_OK) h->ss = after_routing(pre, T, flags);
   return rc;
 }
 
@@ -1073,16 +1117,23 @@ int lmoe_qb_update(lmoe_handle* h, float beta, uint32_t flags, void* stream) {
   if (!h || !(beta == beta)) return LMOE_EINVAL;
   if ((flags & LMOE_QB_LITERAL) && (flags & LMOE_BIAS_SIGN)) return LMOE_EINVAL;
   cudaStream_t st = (cudaStream_t)stream;
-  return run_cached(h, h->g_qb, nullptr, nullptr, 0, flags, beta, st, [&](cudaStream_t s) {
+  const StatsState pre = h->ss;
+  int rc = run_cached(h, h->g_qb, nullptr, nullptr, 0, flags, beta, pre.key(), st, [&](cudaStream_t s) {
     prof_open(h, ST_QB_UPDATE, 1);
     mark(h, ST_QB_UPDATE, s);
-    CK(launch_k(qb_update_kernel, dim3(h->cfg.E), dim3(256), 0, s, 1, h->hist, h->ntok, h->load, h->bias,
+    CK(launch_k(qb_update_kernel, dim3(h->cfg.E), dim3(kQbThreads), 0, s, 1, h->hist, h->ntok, h->load, h->bias,
                 h->cfg.E, h->cfg.k, (flags & LMOE_QB_LITERAL) ? 1 : 0, (flags & LMOE_BIAS_SIGN) ? 1 : 0, beta,
-                h->u, h->qb_done, h->status));
+                h->u, h->qb_done, (const uint16_t*)bin_buffer(h, pre.pend_buf), h->ld_bins, pre.pend_T,
+                pre.hist_live ? 1 : 0, h->status));
     prof_close(h, s);
     h->launches += 1;
     return LMOE_OK;
   });
+  if (rc == LMOE_OK) {
+    h->ss.pend_T = 0;
+    h->ss.hist_live = false;
+  }
+  return rc;
 }
 
 int lmoe_get_routing(lmoe_handle* h, int32_t* idx, float* gates, float* scores, int32_t* counts, int32_t* offsets,
@@ -1118,6 +1169,12 @@ int lmoe_set_bias(lmoe_handle* h, const float* b, void* stream) {
 int lmoe_get_hist(lmoe_handle* h, uint32_t* hist, int64_t* ntok, void* stream) {
   if (!h) return LMOE_EINVAL;
   cudaStream_t st = (cudaStream_t)stream;
+  if (h->ss.pend_T) {  // count the pending bins into the accumulated histogram first
+    int rc = flush_bins(h, h->ss.pend_T, h->ss.pend_buf, st);
+    if (rc) return rc;
+    h->ss.pend_T = 0;
+    h->ss.hist_live = true;
+  }
   if (hist) CK(cudaMemcpyAsync(hist, h->hist, (size_t)h->cfg.E * LMOE_NBINS * 4, cudaMemcpyDeviceToDevice, st));
   if (ntok) CK(cudaMemcpyAsync(ntok, h->ntok, 8, cudaMemcpyDeviceToDevice, st));
   return LMOE_OK;
@@ -1128,6 +1185,8 @@ int lmoe_set_hist(lmoe_handle* h, const uint32_t* hist, const int64_t* ntok, voi
   cudaStream_t st = (cudaStream_t)stream;
   CK(cudaMemcpyAsync(h->hist, hist, (size_t)h->cfg.E * LMOE_NBINS * 4, cudaMemcpyDeviceToDevice, st));
   CK(cudaMemcpyAsync(h->ntok, ntok, 8, cudaMemcpyDeviceToDevice, st));
+  h->ss.pend_T = 0;  // the given statistics replace everything recorded so far
+  h->ss.hist_live = true;
   return LMOE_OK;
 }
 

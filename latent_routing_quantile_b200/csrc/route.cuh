@@ -236,8 +236,11 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ coun
   pdl_trigger();
   int c = 0;
   if (tid < E) {
-#pragma unroll 8
-    for (int j = 0; j < kCountCopies; ++j) c += counts32[(size_t)j * E + tid];
+    int cc[kCountCopies];  // all copies in flight at once
+#pragma unroll
+    for (int j = 0; j < kCountCopies; ++j) cc[j] = counts32[(size_t)j * E + tid];
+#pragma unroll
+    for (int j = 0; j < kCountCopies; ++j) c += cc[j];
   }
   int total;
   const int off = block_exclusive_scan_1024(c, sh, &total);
@@ -264,18 +267,38 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ coun
   const int e = blockIdx.x * 32 + tx;
   const int chunk = (nblk + 31) / 32;
   const int b0 = ty * chunk, b1 = min(nblk, b0 + chunk);
+  // the chunk's counts are loaded in batches of 8 independent loads (one latency per batch);
+  // chunks of up to 8 blocks keep them in registers for the second pass
+  constexpr int kBatch = 8;
+  int keep[kBatch];
   int sum = 0;
   if (e < E)
-    for (int b = b0; b < b1; ++b) sum += blkcnt[(size_t)b * E + e];
+    for (int b = b0; b < b1; b += kBatch) {
+      int v[kBatch];
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) v[i] = (b + i < b1) ? blkcnt[(size_t)(b + i) * E + e] : 0;
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        sum += v[i];
+        keep[i] = v[i];
+      }
+    }
   part[ty][tx] = sum;
   __syncthreads();
   if (e < E) {
     int run = s_off[e];
     for (int q = 0; q < ty; ++q) run += part[q][tx];
-    for (int b = b0; b < b1; ++b) {
-      const int v = blkcnt[(size_t)b * E + e];
-      blkbase[(size_t)b * E + e] = run;
-      run += v;
+    for (int b = b0; b < b1; b += kBatch) {
+      int v[kBatch];
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i)
+        v[i] = chunk <= kBatch ? keep[i] : ((b + i < b1) ? blkcnt[(size_t)(b + i) * E + e] : 0);
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i)
+        if (b + i < b1) {
+          blkbase[(size_t)(b + i) * E + e] = run;
+          run += v[i];
+        }
     }
   }
 }
@@ -432,20 +455,29 @@ __global__ void __launch_bounds__(256, (G <= 6 && sizeof(T) == 2) ? 4 : 3) combi
 }
 
 // --------------------------------------------------------------------------- QB update
-// One kernel, block per expert, for both bias rules; nothing happens when N == 0.
-//  QB (sign_rule == 0): block e finds m = ceil((E-k) N / E), the crossing bin j* (the first whose
-//   cumulative count reaches m) and q = (j* + (m - cum_{j*-1}) / cnt_{j*}) / 4096, then u_e = q
-//   (+ b_e unless literal).  The last block to finish (a device-wide counter) computes mean_e u and
-//   applies b_e <- b_e - beta (u_e - mean) to every expert.
+// One kernel, block per expert, for both bias rules.  The statistics are the accumulated
+// histogram rows (when hist_live; otherwise they are known to be zero and are not touched) plus,
+// when pend_T > 0, the bins of the last recorded forward that no kernel has counted yet (bins
+// [E, ld_bins], pend_T tokens): N = *ntok_acc + pend_T; with N == 0 the bias is left unchanged.
+//  QB (sign_rule == 0): block e counts its expert's row into a shared 4096-bin histogram, finds
+//   m = ceil((E-k) N / E), the crossing bin j* (the first whose cumulative count reaches m) and
+//   q = (j* + (m - cum_{j*-1}) / cnt_{j*}) / 4096, then u_e = q (+ b_e unless literal).  The last
+//   block to finish (a device-wide counter) computes mean_e u and applies
+//   b_e <- b_e - beta (u_e - mean) to every expert.
 //  Sign rule (sign_rule == 1): the last block applies b_e <- b_e + beta sign(mean load - load_e),
 //   the sign taken in integers as sign(sum_e' load_e' - E load_e).
-// Either way every block clears its histogram row, and the last block clears N, the loads and
-// the counter: an update consumes all statistics recorded since the previous one.
-__global__ void __launch_bounds__(256) qb_update_kernel(uint32_t* __restrict__ hist, long long* ntok_acc,
-                                                        long long* __restrict__ load, float* __restrict__ bias,
-                                                        int E, int k, int literal, int sign_rule, float beta,
-                                                        double* __restrict__ u_buf, unsigned int* done_counter,
-                                                        uint32_t* status) {
+// Either way the accumulated rows are cleared, and the last block clears N, the loads and the
+// counter: an update consumes all statistics recorded since the previous one.
+constexpr int kQbThreads = 256;
+
+__global__ void __launch_bounds__(kQbThreads) qb_update_kernel(uint32_t* __restrict__ hist, long long* ntok_acc,
+                                                               long long* __restrict__ load,
+                                                               float* __restrict__ bias, int E, int k, int literal,
+                                                               int sign_rule, float beta, double* __restrict__ u_buf,
+                                                               unsigned int* done_counter,
+                                                               const uint16_t* __restrict__ bins, int ld_bins,
+                                                               int pend_T, int hist_live, uint32_t* status) {
+  __shared__ __align__(16) uint32_t sh[LMOE_NBINS];
   __shared__ long long wsum[8];
   __shared__ double wd[8];
   __shared__ double u_sh;
@@ -453,22 +485,41 @@ __global__ void __launch_bounds__(256) qb_update_kernel(uint32_t* __restrict__ h
   const int e = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   pdl_wait();
   pdl_trigger();
-  const long long N = *ntok_acc;
-  if (N <= 0) return;
+  const long long N = *ntok_acc + (long long)pend_T;
   uint4* row4 = reinterpret_cast<uint4*>(hist + (size_t)e * LMOE_NBINS);
-  constexpr int PER = LMOE_NBINS / 256;  // 16 bins per thread, 4 x uint4
+  constexpr int PER = LMOE_NBINS / kQbThreads;  // 16 bins per thread, 4 x uint4
+  if (N <= 0) {  // nothing recorded: the bias stays; rows set without tokens are dropped
+    if (hist_live)
+      for (int j = 0; j < PER / 4; ++j) row4[tid * (PER / 4) + j] = make_uint4(0u, 0u, 0u, 0u);
+    return;
+  }
   if (!sign_rule) {
+    // shared histogram = accumulated row + the pending bins of this expert
+    uint4* sh4 = reinterpret_cast<uint4*>(sh);
+#pragma unroll
+    for (int j = 0; j < PER / 4; ++j)
+      sh4[tid * (PER / 4) + j] = hist_live ? row4[tid * (PER / 4) + j] : make_uint4(0u, 0u, 0u, 0u);
+    __syncthreads();
+    if (pend_T > 0) {
+      const uint16_t* brow = bins + (size_t)e * ld_bins;
+      const int nvec = pend_T / 8;  // ld_bins is a multiple of 32, so rows are 16-byte aligned
+      for (int v = tid; v < nvec; v += kQbThreads) {
+        const uint4 q = reinterpret_cast<const uint4*>(brow)[v];
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          atomicAdd(&sh[w[j] & 0xFFFFu], 1u);
+          atomicAdd(&sh[w[j] >> 16], 1u);
+        }
+      }
+      for (int t = nvec * 8 + tid; t < pend_T; t += kQbThreads) atomicAdd(&sh[brow[t]], 1u);
+      __syncthreads();
+    }
     long long m = ((long long)(E - k) * N + E - 1) / E;
     m = m < 1 ? 1 : (m > N ? N : m);
     uint32_t c[PER];
 #pragma unroll
-    for (int j = 0; j < PER / 4; ++j) {
-      const uint4 q = row4[tid * (PER / 4) + j];
-      c[4 * j] = q.x;
-      c[4 * j + 1] = q.y;
-      c[4 * j + 2] = q.z;
-      c[4 * j + 3] = q.w;
-    }
+    for (int j = 0; j < PER; ++j) c[j] = sh[tid * PER + j];
     long long local = 0;
 #pragma unroll
     for (int j = 0; j < PER; ++j) local += c[j];
@@ -498,8 +549,10 @@ __global__ void __launch_bounds__(256) qb_update_kernel(uint32_t* __restrict__ h
     }
     __syncthreads();
   }
+  if (hist_live) {
 #pragma unroll
-  for (int j = 0; j < PER / 4; ++j) row4[tid * (PER / 4) + j] = make_uint4(0u, 0u, 0u, 0u);
+    for (int j = 0; j < PER / 4; ++j) row4[tid * (PER / 4) + j] = make_uint4(0u, 0u, 0u, 0u);
+  }
   // thread 0 publishes u_e, then counts finished blocks (the cleared rows are read only by later
   // kernels, so they need no fence)
   if (tid == 0) {

@@ -311,6 +311,46 @@ def test_qb_skewed_router_run():
     layer.close()
 
 
+def test_recorded_statistics_accumulate_across_forwards():
+    """Two recorded forwards, then one update.  The last forward's bins are counted by the update
+    itself, the first one's are added to the histogram when the second arrives; reading the
+    histogram in between (which adds pending bins first) must not change the update, which must
+    match the oracle's update from the histogram of all 2T scores (bin edges aside)."""
+    shape = datagen.LayerShape("acc", 500, 256, 128, 64, 4, 128, 256, "bf16", seed=23, offset_var=0.5, beta=0.05)
+    w = datagen.layer_weights(shape)
+    xs = [datagen.tokens(shape, seed=23 + i) for i in range(2)]
+    biases, hists = [], []
+    for read_between in (False, True):
+        layer = make_layer(shape, w)
+        for x in xs:
+            layer.forward(x.cuda(), record_stats=True)
+            if read_between:
+                hists.append(layer.hist())
+        if not read_between:
+            hists.append(layer.hist())  # adds the pending bins, then the update sees them as history
+            layer.set_hist(*hists[-1])
+        layer.qb_update(shape.beta)
+        biases.append(layer.bias().cpu().numpy())
+        layer.close()
+    # the same statistics through three paths give the same bias, bit for bit
+    layer = make_layer(shape, w)
+    for x in xs:
+        layer.forward(x.cuda(), record_stats=True)
+    layer.qb_update(shape.beta)
+    biases.append(layer.bias().cpu().numpy())
+    layer.close()
+    assert np.array_equal(biases[0], biases[1]) and np.array_equal(biases[0], biases[2])
+    hist, n = hists[0]
+    assert int(n.item()) == 2 * shape.T
+    assert torch.equal(hist, hists[-1][0])  # read after both forwards, both ways
+    s_all = np.concatenate([oracle.layer_routing(x, w, np.zeros(shape.E), shape.k, shape.rms_eps)["s"] for x in xs])
+    ho = oracle.score_histogram(s_all)
+    edge = np.abs(s_all * 4096 - np.round(s_all * 4096)) < 1e-6 * 4096
+    assert np.all(np.abs(hist.cpu().numpy() - ho).sum(1) <= 2 * edge.sum(0))
+    b_ref = oracle.qb_update(np.zeros(shape.E), ho, 2 * shape.T, shape.k, shape.beta)
+    np.testing.assert_allclose(biases[2], b_ref, rtol=0, atol=shape.beta * 2 / 4096 + 1e-6)
+
+
 def test_sign_rule_update_stage_exact():
     """The sign-rule bias update on given loads is bit-exact against the oracle's rule, clears the
     histogram, N and the loads, leaves the bias alone when nothing was recorded, and refuses the
