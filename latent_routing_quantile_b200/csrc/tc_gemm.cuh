@@ -190,8 +190,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       uint32_t armed = 0, armed_parity = 0;  // per-stage bits, for the abort drain
       const uint64_t pol_first = l2_evict_first();
       bool ok = true;
+      // the tile after this one is looked up one tile ahead: in grouped mode that is a global load
+      // whose latency would otherwise stall the issue of every tile's first loads
+      TileInfo ti_next = tc_tile(p, first < num_tiles ? first : 0, BN, PAIR, rank);
       for (int tile = first; ok && tile < num_tiles; tile += stride) {
-        TileInfo ti = tc_tile(p, tile, BN, PAIR, rank);
+        const TileInfo ti = ti_next;
+        if (tile + stride < num_tiles) ti_next = tc_tile(p, tile + stride, BN, PAIR, rank);
         for (int s = 0; ok && s < p.nseg; ++s) {
           const KSeg sg = p.seg[s];
           for (int kb = 0; kb < sg.nkb; ++kb) {
@@ -355,6 +359,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
 #pragma unroll
         for (int j = 0; j < BN / 32; ++j) c_lane[j] = 0.f;
       }
+      // tile table entry and row scale are loaded before the wait, so their latency overlaps it
+      const TileInfo ti = tc_tile(p, tile, BN, PAIR, rank);
+      const int row = ti.row0 + rl;
+      const float rs = (p.row_scale != nullptr && row < p.M_rows) ? p.row_scale[row] : 1.0f;
       ok = mbar_wait(&tfull[acc], acc_phase, abort, p.status);
       __syncwarp();
       if (__any_sync(0xffffffffu, !ok)) {
@@ -362,11 +370,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         break;
       }
       tc_fence_after();
-      TileInfo ti = tc_tile(p, tile, BN, PAIR, rank);
       omap = ti.q < 4 ? &p.tmOut_part[ti.q - 1] : &p.tmOut;
-      const int row = ti.row0 + rl;
       const uint32_t tbase = tmem_base + ((uint32_t)(wq * 32) << 16) + acc * BN;
-      const float rs = (p.row_scale != nullptr && row < p.M_rows) ? p.row_scale[row] : 1.0f;
       uint32_t w[16];
 
       if constexpr (EPI == EPI_SWIGLU) {

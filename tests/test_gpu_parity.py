@@ -48,9 +48,19 @@ def routing_mismatches(gpu_idx, ora, slack=0.0):
     return set_diff, order_diff
 
 
-def check_routing(gpu_idx, ora):
-    """Every mismatch is a near-tie, and mismatched tokens are under 1e-4 of all tokens."""
-    set_diff, order_diff = routing_mismatches(gpu_idx, ora)
+def score_tolerance(shape):
+    """Bound on |s_gpu - s_oracle|.  The scores carry the fp32 accumulation error of the longer of
+    the two dot products behind them (the down projection over d, the six split-precision router
+    products over l), which grows like the square root of its length; 2e-6 is the bound at
+    d = 1024 (the configuration it was measured and asserted on), never tightened below it."""
+    return 2e-6 * max(1.0, np.sqrt(max(shape.d, 6 * shape.l) / 1024))
+
+
+def check_routing(gpu_idx, ora, s_tol=2e-6):
+    """Every mismatch is a near-tie, and mismatched tokens are under 1e-4 of all tokens.  Two
+    scores that each move by up to s_tol can swap when they are within 2 s_tol, so the near-tie
+    margin grows with it beyond NEAR_TIE."""
+    set_diff, order_diff = routing_mismatches(gpu_idx, ora, slack=max(0.0, 2 * s_tol - NEAR_TIE))
     mism = set_diff | order_diff
     frac = float(mism.mean())
     assert mism.sum() <= int(1e-4 * len(mism)), f"mismatch fraction {frac}"
@@ -186,8 +196,9 @@ def run_layer_check(shape, w, x, b=None, sample=None, record=True):
     ro = oracle.layer_routing(x, w, b64, k, shape.rms_eps)
     s_gpu = r["scores"].cpu().numpy()
     s_err = float(np.max(np.abs(s_gpu - ro["s"])))
-    assert s_err < 2e-6, f"router scores off by {s_err}"
-    frac = check_routing(r["idx"].cpu().numpy(), ro)
+    s_tol = score_tolerance(shape)
+    assert s_err < s_tol, f"router scores off by {s_err} (bound {s_tol})"
+    frac = check_routing(r["idx"].cpu().numpy(), ro, s_tol)
     check_permutation(r, T, k, E)
     rows = np.arange(T) if sample is None else sample
     xs = x[torch.from_numpy(rows)]
