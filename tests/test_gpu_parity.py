@@ -7,6 +7,7 @@ differ, and such tokens must stay under 1e-4 of all tokens.  Stage tests feed th
 same fp32 scores the oracle sees, so there every decision is taken in the same precision.
 Layer outputs: max|y - y_ref| / max|y_ref| <= 2e-2 for bf16, 1e-4 for fp32.
 """
+import dataclasses
 import json
 import os
 
@@ -237,6 +238,18 @@ def test_small_bf16_layer_ragged(gain, E):
     diff = np.abs(hist.cpu().numpy() - ho).sum(1)
     assert np.all(diff <= 2 * edge.sum(0))
     assert int(ntok.item()) == shape.T
+    layer.close()
+
+
+def test_sweep_65536_tokens_sampled():
+    """The token sweep's 65536-token point (the sweep workload's seeded inputs, as bench.py --workload
+    sweep --tokens 65536 uses them; mini_replica widths): routing parity on every token,
+    outputs on every 64th (1024 tokens), as the sweep's parity check asks for T >= 16384."""
+    shape = dataclasses.replace(datagen.WORKLOADS["sweep"], T=65536)
+    w = datagen.layer_weights(shape)
+    x = datagen.tokens(shape)
+    layer, y, ro, stats = run_layer_check(shape, w, x, sample=np.arange(0, shape.T, 64))
+    print("sweep_65536", json.dumps(stats))
     layer.close()
 
 
