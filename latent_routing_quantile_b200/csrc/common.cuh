@@ -155,6 +155,8 @@ __device__ __forceinline__ void tma_store_2d_hint(const CUtensorMap* m, const vo
                "r"(smem_u32(src)), "r"(x), "r"(y), "l"(pol)
                : "memory");
 }
+// Prefetch of the 128-byte line at p into L2.
+__device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Waits until at most N committed bulk groups still read their shared-memory source.
 template <int N>

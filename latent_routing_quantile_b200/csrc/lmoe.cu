@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdio>
+#include <cmath>
 #include <cstring>
 #include <mutex>
 #include <new>
@@ -187,6 +188,7 @@ struct TopkArgs {
   float* gates;
   uint16_t* bins;
   int ld_bins;
+  TopkRefine rf;
   uint32_t* status;
 };
 
@@ -201,7 +203,7 @@ cudaError_t launch_topk_t(const TopkArgs& a, cudaStream_t st) {
   }
   return launch_k(topk_kernel<NJ>, dim3(nblk), dim3(32 * topk_warps(NJ)), smem, st, 1, a.s, a.b, a.T, a.E, a.k,
                   a.idx, a.gates,
-                  a.rank, a.blkcnt, a.counts32, a.bins, a.ld_bins, a.status);
+                  a.rank, a.blkcnt, a.counts32, a.bins, a.ld_bins, a.rf, a.status);
 }
 
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st) {
@@ -301,6 +303,8 @@ struct lmoe_handle {
   void* w_down = nullptr;   // bf16 [l, d] or [l, 2d] (hi|lo); f32 [l, d]
   void* w_r = nullptr;      // bf16 [E, 3l] (hi|mid|lo); f32 [E, l]
   float* c = nullptr;       // [E]
+  double* wc = nullptr;     // W_comb [E, d] fp64 (exact decision of ambiguous top-k)
+  float tau = 0.f;          // near-tie width below which a token's top-k is decided in fp64
   void* ws13 = nullptr;     // bf16 [2hs, d] interleaved; f32: ws1 [hs, d]
   void* ws3f = nullptr;     // f32 only: ws3 [hs, d]
   void* w13 = nullptr;      // bf16 [E, 2h, l] interleaved; f32: w1 [E, h, l]
@@ -375,6 +379,7 @@ void plan_layout(lmoe_handle* h, Arena& a) {
   a.add(&h->w_down, (h->bf && !h->unit_gain ? 2 : 1) * l * d * es);
   a.add(&h->w_r, h->bf ? E * 3 * l * 2 : E * l * 4);
   a.add((void**)&h->c, E * 4);
+  a.add((void**)&h->wc, E * d * 8);
   if (hs) {
     a.add(&h->ws13, 2 * hs * d * es);
     if (!h->bf) a.add(&h->ws3f, hs * d * es);
@@ -545,7 +550,8 @@ int flush_bins(lmoe_handle* h, int pend_T, int buf, cudaStream_t st) {
   return LMOE_OK;
 }
 
-int route_from_scores(lmoe_handle* h, int T, uint32_t flags, const StatsState& pre, cudaStream_t st) {
+int route_from_scores(lmoe_handle* h, int T, uint32_t flags, const StatsState& pre, const void* x,
+                      cudaStream_t st) {
   const StatsState post = after_routing(pre, T, flags);
   const lmoe_config& c = h->cfg;
   const int nblk = (T + kTokBlock - 1) / kTokBlock;
@@ -555,7 +561,8 @@ int route_from_scores(lmoe_handle* h, int T, uint32_t flags, const StatsState& p
   if (h->counts32_dirty) CK(cudaMemsetAsync(h->counts32, 0, (size_t)kCountCopies * c.E * sizeof(int), st));
   h->counts32_dirty = true;
   TopkArgs ta{h->s, h->bias, T, c.E, c.k, h->idx, h->rank, h->blkcnt, h->counts32, h->gates,
-              (flags & LMOE_RECORD_STATS) ? bin_buffer(h, post.pend_buf) : nullptr, h->ld_bins, h->status};
+              (flags & LMOE_RECORD_STATS) ? bin_buffer(h, post.pend_buf) : nullptr, h->ld_bins,
+              TopkRefine{x, h->bf ? 1 : 0, c.d, h->wc, h->c, c.rms_eps, h->tau}, h->status};
   CK(launch_topk(ta, st));
   mark(h, ST_PLAN, st);
   CK(launch_k(plan_kernel, dim3((c.E + 31) / 32), dim3(1024), 0, st, 1, (const int*)h->counts32, h->counts,
@@ -669,7 +676,7 @@ int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, 
     mark(h, ST_K1, st);
     h->launches += 3;
   }
-  int rc = route_from_scores(h, T, flags, pre, st);
+  int rc = route_from_scores(h, T, flags, pre, x, st);
   if (rc) return rc;
   // shared expert, first half: a_s = silu(r x Ws1^T) * (r x Ws3^T)
   mark(h, ST_SHARED, st);
@@ -804,7 +811,7 @@ int forward_f32(lmoe_handle* h, const void* xv, void* yv, int T, uint32_t flags,
     CK(launch_simt<SE_ROUTER>(p, mt, st));
   }
   mark(h, ST_K1, st);
-  int rc = route_from_scores(h, T, flags, pre, st);
+  int rc = route_from_scores(h, T, flags, pre, xv, st);
   if (rc) return rc;
   mark(h, ST_SHARED, st);
   if (c.hs) {  // a_s = silu(r x Ws1'^T) * (r x Ws3'^T)
@@ -897,6 +904,16 @@ int repack(lmoe_handle* h, const lmoe_weights* w, cudaStream_t st) {
     if (hs)
       fold_gain_kernel<float><<<grid_1d(d * hs, TPB), TPB, 0, st>>>((const float*)w->ws2, nullptr, d, hs,
                                                                     (float*)h->wy, l + hs, l);
+  }
+  {  // W_comb = W_r (W_down g) in fp64, for the exact decision of ambiguous top-k choices
+    const dim3 grid((unsigned)((d + 255) / 256), (unsigned)E);
+    if (h->bf)
+      combine_router_kernel<bf16><<<grid, 256, 0, st>>>(w->w_router, (const bf16*)w->w_down,
+                                                        h->unit_gain ? nullptr : (const bf16*)w->rms_gain, (int)l,
+                                                        (int)d, h->wc);
+    else
+      combine_router_kernel<float><<<grid, 256, 0, st>>>(w->w_router, (const float*)w->w_down,
+                                                         (const float*)w->rms_gain, (int)l, (int)d, h->wc);
   }
   CK(cudaGetLastError());
   if (w->router_bias)
@@ -1027,6 +1044,10 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, void* stream, lmo
   h->device = dev;
   h->sms = sms;
   h->unit_gain = gain_is_unit(*cfg, w->rms_gain);
+  // near-tie width for the exact decision: 2.5 times the bound on the scores' fp32 error (2e-6 at
+  // d = 1024, growing like the square root of the longer accumulation: d, or the router's six
+  // products over l), so two scores that each err by up to the bound cannot swap unnoticed
+  h->tau = 5e-6f * (float)std::max(1.0, std::sqrt(std::max((double)cfg->d, 6.0 * cfg->l) / 1024.0));
   Arena a;
   plan_layout(h, a);
   if (cudaMalloc(&h->arena, a.off) != cudaSuccess) {
@@ -1107,7 +1128,7 @@ int lmoe_route_scores(lmoe_handle* h, const float* scores, int32_t T, uint32_t f
   CK(cudaMemcpyAsync(h->s, scores, (size_t)T * h->cfg.E * 4, cudaMemcpyDeviceToDevice, st));
   prof_open(h, ST_TOPK, ST_HIST - ST_TOPK + 1);
   const StatsState pre = h->ss;
-  int rc = route_from_scores(h, T, flags, pre, st);
+  int rc = route_from_scores(h, T, flags, pre, nullptr, st);
   prof_close(h, st);
   if (rc == LMOE_OK) h->ss = after_routing(pre, T, flags);
   return rc;
@@ -1345,7 +1366,7 @@ int lmoe_route_noalloc(const float* scores, const float* bias, int32_t T, int32_
   // which the top-k blocks add into
   CK(cudaMemsetAsync(status, 0, sizeof(uint32_t), st));
   CK(cudaMemsetAsync(counts32, 0, (size_t)kCountCopies * E * sizeof(int), st));
-  TopkArgs ta{scores, bias, T, E, k, idx, rank, blkcnt, counts32, gates, nullptr, 0, status};
+  TopkArgs ta{scores, bias, T, E, k, idx, rank, blkcnt, counts32, gates, nullptr, 0, TopkRefine{}, status};
   CK(launch_topk(ta, st));
   const int nblk = (T + kTokBlock - 1) / kTokBlock;
   plan_kernel<<<(E + 31) / 32, 1024, 0, st>>>(counts32, counts, blkcnt, nblk, E, offsets, delta, blkbase, tiles,

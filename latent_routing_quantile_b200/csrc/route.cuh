@@ -49,6 +49,36 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   const uint32_t b = __float_as_uint(f);
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
+// Inverse of order_key for keys of numbers (>= 2).
+__device__ __forceinline__ float key_value(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
+
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int off = 16; off; off >>= 1) v += __shfl_xor_sync(kFull, v, off);
+  return v;
+}
+
+// Inputs of the exact decision of ambiguous tokens (x == nullptr: decide every token in fp32).
+struct TopkRefine {
+  const void* x;      // layer input [T, d], bf16 (x_bf16) or fp32
+  int x_bf16, d;
+  const double* wc;   // W_comb [E, d] fp64
+  const float* cz;    // router column offsets [E]
+  float eps, tau;
+};
+constexpr int kRefineExtra = 8;  // candidates beyond the k-th that an exact decision considers
+
+// The exact decision of a token whose fp32 top-k is ambiguous (two of its top k+1 biased scores
+// within tau of each other, so the scores' fp32 rounding could order them either way).  Its
+// candidates are every expert whose fp32 biased score lies within tau of the k-th (at most
+// kRefineExtra beyond the k-th).  Each candidate's biased score is recomputed in fp64 as the layer
+// defines it, u = sigmoid(r * (x . W_comb[e]) + c_e) + b_e with r = 1/sqrt(mean x^2 + eps) and
+// W_comb the router and down-projection weights multiplied out in fp64 (the same logit as
+// h W_r^T + c up to fp64 rounding), and the candidates are ranked by (u descending, expert
+// ascending).  The whole block computes each such token's dot products together (one memory
+// round trip instead of one per 32 elements), after its warps have ranked every other token.
 
 // One warp per token; a block of W warps ranks kTokBlock = 32 tokens (32 / W per warp; W = 16
 // for E <= 256, whose registers allow two such blocks per SM, else 8).  Lane L holds the scores
@@ -72,7 +102,7 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 
     topk_kernel(const float* __restrict__ s, const float* __restrict__ bias, int ntok, int E, int k,
                 int* __restrict__ idx, float* __restrict__ gates, int* __restrict__ rank,
                 int* __restrict__ blkcnt, int* __restrict__ counts32, uint16_t* __restrict__ bins, int ld_bins,
-                uint32_t* status) {
+                const TopkRefine rf, uint32_t* status) {
   constexpr int W = topk_warps(NJ);
   constexpr int TPW = kTokBlock / W;  // tokens per warp
   constexpr int PF = topk_prefetch(NJ);
@@ -82,7 +112,14 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 
   const int bpitch = E + 2;
   const int blk = blockIdx.x, t0 = blk * kTokBlock;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // tokens of the block that wait for the exact decision: candidates, (token | count << 8)
+  __shared__ int def_e[kTokBlock][32];
+  __shared__ int def_info[kTokBlock];
+  __shared__ int def_n;
+  __shared__ double red[W][9];
+  __shared__ double def_z[48];  // [0, 32): candidate dot products; [32, 41): first group's sums; 40: x^2
   for (int i = threadIdx.x; i < E; i += blockDim.x) mask[i] = 0;
+  if (threadIdx.x == 0) def_n = 0;
   pdl_wait();
   pdl_trigger();
   float bj[NJ];
@@ -93,8 +130,29 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 
   }
   __syncthreads();
 
-  int sel_q[TPW];
+  int sel_q[TPW], slot_q[TPW];
+  uint32_t deferred = 0;  // tokens of this warp whose choice waits for the exact decision
   bool nan = false;
+  // stores token t's choice (lane i < k holds the i-th expert): index, gate, rank-mask bit
+  auto commit = [&](int t, int tl, int& my_sel) {
+    float my_s = 0.f;
+    if (lane < k) {
+      if (my_sel < 0 || my_sel >= E) {
+        set_status(status, LMOE_STATUS_BAD_INDEX);
+        my_sel = 0;
+      }
+      my_s = s[(size_t)t * E + my_sel];
+      if (my_s != my_s) my_s = 0.f;
+    }
+    float ssum = my_s;
+#pragma unroll
+    for (int off = 16; off; off >>= 1) ssum += __shfl_xor_sync(kFull, ssum, off);
+    if (lane < k) {
+      idx[(size_t)t * k + lane] = my_sel;
+      gates[(size_t)t * k + lane] = my_s / ssum;
+      atomicOr(&mask[my_sel], 1u << tl);
+    }
+  };
 #pragma unroll
   for (int q0 = 0; q0 < TPW; q0 += PF) {
     float vq[PF][NJ];
@@ -128,7 +186,13 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 
         }
       }
       int my_sel = -1;
-      for (int i = 0; i < k; ++i) {
+      // k rounds of selection; with the exact decision enabled, further rounds collect the
+      // experts within tau of the k-th (at most kRefineExtra), and near-ties mark the token
+      const int kmax = rf.x ? min(min(k + kRefineExtra, 32), E) : k;
+      float u_prev = 0.f, u_k1 = 0.f;
+      bool amb = false;
+      int nc = 0;
+      for (int i = 0; i < kmax; ++i) {
         uint32_t bk = 0u;
         int bjx = 0;
 #pragma unroll
@@ -139,32 +203,128 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 
           }
         }
         const uint32_t wmax = __reduce_max_sync(kFull, bk);
+        if (i >= k) {  // an extra candidate: only within tau of the k-th, and only a number
+          if (wmax < 2u || !(key_value(wmax) >= u_k1 - rf.tau)) break;
+        }
         const uint32_t emin = __reduce_min_sync(kFull, bk == wmax ? (uint32_t)(bjx * 32 + lane) : 0xffffffffu);
 #pragma unroll
         for (int j = 0; j < NJ; ++j)
           if ((uint32_t)(j * 32 + lane) == emin) key[j] = 0u;
         if (lane == i) my_sel = (int)emin;
-      }
-      float my_s = 0.f;
-      if (lane < k) {
-        if (my_sel < 0 || my_sel >= E) {
-          set_status(status, LMOE_STATUS_BAD_INDEX);
-          my_sel = 0;
+        if (rf.x) {
+          const float ui = wmax >= 2u ? key_value(wmax) : 0.f;
+          if (i > 0 && wmax >= 2u && u_prev - ui < rf.tau) amb = true;
+          if (i == k - 1) u_k1 = ui;
+          u_prev = ui;
         }
-        my_s = s[(size_t)t * E + my_sel];
-        if (my_s != my_s) my_s = 0.f;
+        nc = i + 1;
       }
-      float ssum = my_s;
-#pragma unroll
-      for (int off = 16; off; off >>= 1) ssum += __shfl_xor_sync(kFull, ssum, off);
-      if (lane < k) {
-        idx[(size_t)t * k + lane] = my_sel;
-        gates[(size_t)t * k + lane] = my_s / ssum;
-        atomicOr(&mask[my_sel], 1u << tl);
+      if (amb) {  // warp-uniform: decided by the whole block after the token loop
+        int slot = 0;
+        if (lane == 0) slot = atomicAdd(&def_n, 1);
+        slot = __shfl_sync(kFull, slot, 0);
+        def_e[slot][lane] = lane < nc ? my_sel : -1;
+        if (lane == 0) def_info[slot] = tl | (nc << 8);
+        // warm L2 with the candidates' fp64 weight rows and the token's input row while the warp
+        // ranks its other tokens
+        for (int c = 0; c < nc; ++c) {
+          const char* row = reinterpret_cast<const char*>(rf.wc + (size_t)__shfl_sync(kFull, my_sel, c) * rf.d);
+          for (int b = lane * 128; b < rf.d * 8; b += 32 * 128) prefetch_l2(row + b);
+        }
+        const char* xr = reinterpret_cast<const char*>(rf.x) + (size_t)t * rf.d * (rf.x_bf16 ? 2 : 4);
+        for (int b = lane * 128; b < rf.d * (rf.x_bf16 ? 2 : 4); b += 32 * 128) prefetch_l2(xr + b);
+        deferred |= 1u << (q0 + p);
+        slot_q[q0 + p] = slot;
+        continue;
       }
+      if (lane >= k) my_sel = -1;
+      commit(t, tl, my_sel);
       sel_q[q0 + p] = my_sel;
     }
   }
+  __syncthreads();  // every deferred token is listed
+  const int ndef = def_n;
+  for (int di = 0; di < ndef; ++di) {  // block-uniform
+    const int tl = def_info[di] & 255, nc = def_info[di] >> 8, t = t0 + tl;
+    const size_t xoff = (size_t)t * rf.d;
+    auto xval = [&](int j) -> double {
+      return rf.x_bf16 ? (double)__bfloat162float(reinterpret_cast<const bf16*>(rf.x)[xoff + j])
+                       : (double)reinterpret_cast<const float*>(rf.x)[xoff + j];
+    };
+    // block sums: warp shuffles, then one partial per warp in red[][u]
+    auto block_sum = [&](double (&v)[9], int nv, double* out) {
+#pragma unroll
+      for (int u = 0; u < 9; ++u) {
+        if (u < nv) {
+          const double a = warp_sum_d(v[u]);
+          if (lane == 0) red[warp][u] = a;
+        }
+      }
+      __syncthreads();
+      if (threadIdx.x < nv) {
+        double a = 0.0;
+        for (int w = 0; w < W; ++w) a += red[w][threadIdx.x];
+        out[threadIdx.x] = a;
+      }
+      __syncthreads();
+    };
+    // group g sums x . W_comb[e] for candidates 8g..8g+7 (group 0 also sums x^2 for r)
+    double v[9];
+    for (int c0 = 0; c0 < nc; c0 += 8) {
+      const int ng = min(8, nc - c0);
+      const double* wrow[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        v[u] = 0.0;
+        wrow[u] = rf.wc + (size_t)def_e[di][min(c0 + u, nc - 1)] * rf.d;
+      }
+      v[8] = 0.0;
+      for (int j = threadIdx.x; j < rf.d; j += blockDim.x) {
+        const double xv = xval(j);
+        v[8] = fma(xv, xv, v[8]);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = fma(xv, wrow[u][j], v[u]);
+      }
+      if (c0 == 0) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (u == ng) v[u] = v[8];  // x^2 rides in slot ng of the first group's sums
+        block_sum(v, ng + 1, def_z + 32);
+        for (int u = 0; u < ng; ++u) {
+          if (threadIdx.x == 0) def_z[u] = def_z[32 + u];
+        }
+        if (threadIdx.x == 0) def_z[40] = def_z[32 + ng];
+        __syncthreads();
+      } else {
+        block_sum(v, ng, def_z + c0);
+      }
+    }
+    const double r = 1.0 / sqrt(def_z[40] / rf.d + (double)rf.eps);
+    if (warp == 0) {  // rank the candidates and store the choice like any other token's
+      const int e_lane = def_e[di][lane];
+      double my_u = 0.0;
+      if (lane < nc) my_u = 1.0 / (1.0 + exp(-(r * def_z[lane] + (double)rf.cz[e_lane]))) + (double)bias[e_lane];
+      int rk = 0;
+      for (int c = 0; c < nc; ++c) {
+        const double uc = __shfl_sync(kFull, my_u, c);
+        const int ec = __shfl_sync(kFull, e_lane, c);
+        if (uc > my_u || (uc == my_u && ec < e_lane)) ++rk;
+      }
+      int sel = -1;
+      for (int i = 0; i < k; ++i) {
+        const unsigned who = __ballot_sync(kFull, lane < nc && rk == i);
+        const int src = who ? __ffs(who) - 1 : 0;
+        const int ei = __shfl_sync(kFull, e_lane, src);
+        if (lane == i && who) sel = ei;
+      }
+      commit(t, tl, sel);
+      def_e[di][lane] = sel;  // the owning warp reads its choice back for the ranks
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int q = 0; q < TPW; ++q)
+    if ((deferred >> q) & 1u) sel_q[q] = def_e[slot_q[q]][lane];
   if (nan) set_status(status, LMOE_STATUS_NAN_SCORE);
   __syncthreads();
 
@@ -598,6 +758,21 @@ __global__ void __launch_bounds__(kQbThreads) qb_update_kernel(uint32_t* __restr
 }
 
 // --------------------------------------------------------------------------- weight repacking
+// W_comb[e, j] = g_j * sum_i W_r[e, i] W_down[i, j] in fp64 (g = null: gain one): the router logit
+// as a single map of x (z = r * x W_comb^T + c), for the exact decision of ambiguous tokens.
+// Grid (ceil(d / 256), E), one output per thread.
+template <typename T>
+__global__ void __launch_bounds__(256) combine_router_kernel(const float* __restrict__ w_r,
+                                                             const T* __restrict__ w_down, const T* __restrict__ g,
+                                                             int l, int d, double* __restrict__ wc) {
+  const int e = blockIdx.y, j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= d) return;
+  double acc = 0.0;
+  for (int i = 0; i < l; ++i)
+    acc = fma((double)w_r[(size_t)e * l + i], (double)to_f<T>(w_down[(size_t)i * d + j]), acc);
+  wc[(size_t)e * d + j] = g ? acc * (double)to_f<T>(g[j]) : acc;
+}
+
 // out[r, c] = g[c] * w[r, c] in the storage type (gain folded into an (out, in) matrix).
 template <typename T>
 __global__ void fold_gain_kernel(const T* __restrict__ w, const T* __restrict__ g, int rows, int cols,
