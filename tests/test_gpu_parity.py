@@ -200,6 +200,8 @@ def run_layer_check(shape, w, x, b=None, sample=None, record=True):
     s_tol = score_tolerance(shape)
     assert s_err < s_tol, f"router scores off by {s_err} (bound {s_tol})"
     frac = check_routing(r["idx"].cpu().numpy(), ro, s_tol)
+    # ambiguous tokens are decided in fp64, so every choice (set and rank order) is the oracle's
+    assert frac == 0.0, f"mismatch fraction {frac}"
     check_permutation(r, T, k, E)
     rows = np.arange(T) if sample is None else sample
     xs = x[torch.from_numpy(rows)]
@@ -328,7 +330,7 @@ def test_qb_skewed_router_run():
     frac = nmism / (shape.T * shape.steps)
     print("qb_skewed", json.dumps(dict(ratio_first=ratios[0], ratio_last=ratios[-1], ratios=ratios,
                                        max_q_err=max(qerr), max_update_diff=max(berr), mismatch_frac=frac)))
-    assert nmism <= 1e-4 * shape.T * shape.steps
+    assert nmism == 0  # ambiguous tokens are decided in fp64
     assert max(berr) <= shape.beta * 2 / 4096 + 1e-6
     assert ratios[0] >= 3.5 and ratios[-1] < 2.0
     assert max(qerr) <= 1 / 4096 + 1e-7
@@ -457,8 +459,7 @@ def test_sign_rule_on_skewed_router_and_qb_beside_it():
     print("balancers_skewed", json.dumps(dict(sign_rule=[round(v, 3) for v in sign_ratios],
                                               qb=[round(v, 3) for v in qb_ratios], mismatched_tokens=nmism,
                                               load_diff=load_diff)))
-    assert nmism <= 1e-4 * shape.T * shape.steps
-    assert load_diff <= 2 * nmism
+    assert nmism == 0 and load_diff == 0  # ambiguous tokens are decided in fp64
     assert sign_ratios[0] >= 3.5 and max(sign_ratios[-10:]) < sign_ratios[0] / 2.5
     assert qb_ratios[0] >= 3.5 and qb_ratios[-1] < 2.0
 
