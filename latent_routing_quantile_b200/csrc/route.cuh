@@ -186,13 +186,15 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 
         }
       }
       int my_sel = -1;
-      // k rounds of selection; with the exact decision enabled, further rounds collect the
-      // experts within tau of the k-th (at most kRefineExtra), and near-ties mark the token
+      // k rounds of selection.  With the exact decision enabled, near-ties among the chosen and
+      // with the best unchosen expert (a warp max of the remaining keys) mark the token, and
+      // only then do further rounds collect the experts within tau of the k-th (at most
+      // kRefineExtra)
       const int kmax = rf.x ? min(min(k + kRefineExtra, 32), E) : k;
       float u_prev = 0.f, u_k1 = 0.f;
       bool amb = false;
-      int nc = 0;
-      for (int i = 0; i < kmax; ++i) {
+      int nc = 0, lim = k;
+      for (int i = 0; i < lim; ++i) {
         uint32_t bk = 0u;
         int bjx = 0;
 #pragma unroll
@@ -214,7 +216,15 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 
         if (rf.x) {
           const float ui = wmax >= 2u ? key_value(wmax) : 0.f;
           if (i > 0 && wmax >= 2u && u_prev - ui < rf.tau) amb = true;
-          if (i == k - 1) u_k1 = ui;
+          if (i == k - 1) {
+            u_k1 = ui;
+            uint32_t nk = 0u;  // best remaining key
+#pragma unroll
+            for (int j = 0; j < NJ; ++j) nk = max(nk, key[j]);
+            nk = __reduce_max_sync(kFull, nk);
+            if (nk >= 2u && ui - key_value(nk) < rf.tau) amb = true;
+            if (amb) lim = kmax;
+          }
           u_prev = ui;
         }
         nc = i + 1;
