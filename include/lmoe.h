@@ -123,8 +123,12 @@ int lmoe_forward(lmoe_handle *h, const void *x_dev, void *y_dev, int32_t T, uint
                  void *stream);
 
 /* The same forward with host buffers: copies x_host to the device, runs lmoe_forward into a
- * handle-owned buffer and copies the result to y_host, all enqueued on `stream`.  y_host is
- * valid after the stream synchronises. */
+ * handle-owned buffer and copies the result to y_host.  The forward and the copy to y_host are
+ * enqueued on `stream`; the copy from x_host runs on a handle-owned copy stream into one of two
+ * staging buffers (ordered by events: it waits for the forward that last read that buffer, and
+ * the forward waits for it), so one call's input copy overlaps the previous call's forward.
+ * y_host is valid, and x_host may change, after `stream` synchronises.  Under stream capture of
+ * `stream` everything stays on `stream`. */
 int lmoe_forward_host(lmoe_handle *h, const void *x_host, void *y_host, int32_t T,
                       uint32_t flags, void *stream);
 

@@ -327,6 +327,13 @@ struct lmoe_handle {
   int2* mtiles = nullptr;
   void *a_perm = nullptr, *act = nullptr, *o = nullptr, *z = nullptr, *a_s = nullptr;
   void *x_stage = nullptr, *y_stage = nullptr;
+  // lmoe_forward_host: two input staging buffers, so the next call's host-to-device copy (on its
+  // own stream) overlaps this call's forward
+  void* x_stage2 = nullptr;
+  int host_slot = 0;
+  cudaStream_t cp_in = nullptr;
+  cudaEvent_t ev_in[2] = {nullptr, nullptr}, ev_fwd[2] = {nullptr, nullptr};
+  bool fwd_recorded[2] = {false, false};
   // state
   float* bias = nullptr;
   uint32_t* hist = nullptr;
@@ -356,7 +363,9 @@ struct lmoe_handle {
   ProfRecord* cur = nullptr;
   // graph replay of repeated calls
   cudaStream_t cap = nullptr;
-  GraphCache g_fwd, g_qb;
+  GraphCache g_fwd[2], g_qb;  // two forward graphs (the host path alternates input buffers)
+  long long g_tick = 0;
+  long long g_used[2] = {0, 0};
 };
 
 namespace {
@@ -414,6 +423,7 @@ void plan_layout(lmoe_handle* h, Arena& a) {
   a.add(&h->z, Tm * l * es);
   if (hs) a.add(&h->a_s, Tm * hs * es);
   a.add(&h->x_stage, Tm * d * es);
+  a.add(&h->x_stage2, Tm * d * es);
   a.add(&h->y_stage, Tm * d * es);
   // state
   a.add((void**)&h->bias, E * 4);
@@ -1067,6 +1077,11 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, void* stream, lmo
   if (!rc && cudaMemsetAsync(h->qb_done, 0, 4, st) != cudaSuccess) rc = LMOE_ECUDA;
   if (!rc && h->bf) rc = build_maps(h);
   if (!rc && cudaStreamCreateWithFlags(&h->cap, cudaStreamNonBlocking) != cudaSuccess) rc = LMOE_ECUDA;
+  if (!rc && cudaStreamCreateWithFlags(&h->cp_in, cudaStreamNonBlocking) != cudaSuccess) rc = LMOE_ECUDA;
+  for (int i = 0; !rc && i < 2; ++i)
+    if (cudaEventCreateWithFlags(&h->ev_in[i], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&h->ev_fwd[i], cudaEventDisableTiming) != cudaSuccess)
+      rc = LMOE_ECUDA;
   if (rc) {
     cudaStreamSynchronize(st);
     cudaFree(h->arena);
@@ -1082,9 +1097,14 @@ int lmoe_destroy(lmoe_handle* h) {
   cudaDeviceSynchronize();
   for (auto& r : h->prof)
     for (auto& e : r.ev) cudaEventDestroy(e);
-  h->g_fwd.reset(nullptr, nullptr, -1, 0, 0.f, 0);
+  for (auto& g : h->g_fwd) g.reset(nullptr, nullptr, -1, 0, 0.f, 0);
   h->g_qb.reset(nullptr, nullptr, -1, 0, 0.f, 0);
   if (h->cap) cudaStreamDestroy(h->cap);
+  if (h->cp_in) cudaStreamDestroy(h->cp_in);
+  for (int i = 0; i < 2; ++i) {
+    if (h->ev_in[i]) cudaEventDestroy(h->ev_in[i]);
+    if (h->ev_fwd[i]) cudaEventDestroy(h->ev_fwd[i]);
+  }
   cudaFree(h->arena);
   delete h;
   return LMOE_OK;
@@ -1099,7 +1119,12 @@ int lmoe_forward(lmoe_handle* h, const void* x, void* y, int32_t T, uint32_t fla
   cudaStream_t st = (cudaStream_t)stream;
   h->last_T = T;
   const StatsState pre = h->ss;
-  int rc = run_cached(h, h->g_fwd, x, y, T, flags, 0.f, pre.key(), st, [&](cudaStream_t s) {
+  // the cached graph of these arguments, else the least recently used one
+  int gi = h->g_fwd[0].same(x, y, T, flags, 0.f, pre.key()) ? 0
+           : h->g_fwd[1].same(x, y, T, flags, 0.f, pre.key()) ? 1
+           : (h->g_used[0] <= h->g_used[1] ? 0 : 1);
+  h->g_used[gi] = ++h->g_tick;
+  int rc = run_cached(h, h->g_fwd[gi], x, y, T, flags, 0.f, pre.key(), st, [&](cudaStream_t s) {
     prof_open(h, ST_RMS, ST_UP - ST_RMS + 1);
     int r = h->bf ? forward_bf16(h, x, y, T, flags, pre, s) : forward_f32(h, x, y, T, flags, pre, s);
     prof_close(h, s);
@@ -1114,9 +1139,28 @@ int lmoe_forward_host(lmoe_handle* h, const void* x_host, void* y_host, int32_t 
   if (T == 0) return LMOE_OK;
   cudaStream_t st = (cudaStream_t)stream;
   const size_t bytes = (size_t)T * h->cfg.d * h->es;
-  CK(cudaMemcpyAsync(h->x_stage, x_host, bytes, cudaMemcpyHostToDevice, st));
-  int rc = lmoe_forward(h, h->x_stage, h->y_stage, T, flags, stream);
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) {
+    // under the caller's stream capture everything stays on its stream
+    CK(cudaMemcpyAsync(h->x_stage, x_host, bytes, cudaMemcpyHostToDevice, st));
+    int rc = lmoe_forward(h, h->x_stage, h->y_stage, T, flags, stream);
+    if (rc) return rc;
+    CK(cudaMemcpyAsync(y_host, h->y_stage, bytes, cudaMemcpyDeviceToHost, st));
+    return LMOE_OK;
+  }
+  // the input copy runs on the handle's copy stream into the staging buffer this call owns, once
+  // the forward that last read that buffer has finished; the forward waits for the copy
+  const int sl = h->host_slot;
+  void* xs = sl ? h->x_stage2 : h->x_stage;
+  if (h->fwd_recorded[sl]) CK(cudaStreamWaitEvent(h->cp_in, h->ev_fwd[sl], 0));
+  CK(cudaMemcpyAsync(xs, x_host, bytes, cudaMemcpyHostToDevice, h->cp_in));
+  CK(cudaEventRecord(h->ev_in[sl], h->cp_in));
+  CK(cudaStreamWaitEvent(st, h->ev_in[sl], 0));
+  int rc = lmoe_forward(h, xs, h->y_stage, T, flags, stream);
   if (rc) return rc;
+  CK(cudaEventRecord(h->ev_fwd[sl], st));
+  h->fwd_recorded[sl] = true;
+  h->host_slot ^= 1;
   CK(cudaMemcpyAsync(y_host, h->y_stage, bytes, cudaMemcpyDeviceToHost, st));
   return LMOE_OK;
 }
