@@ -4,9 +4,10 @@
 A step is one pass of the whole hot path over one batch of synthetic tokens already resident
 in HBM: lmoe_forward with QB statistics recorded (RMSNorm, latent down-projection, sigmoid
 router, biased top-k and gates, histogram, dispatch plan and permutation, routed SwiGLU
-experts, shared SwiGLU expert, combine, up-projection), then lmoe_qb_update.  With N > 1 ranks
-every rank runs its own tokens (weak scaling) and the ranks sum their QB histograms with one
-NCCL all-reduce before the update, so every rank keeps the same bias.
+experts, shared SwiGLU expert, combine, up-projection) and the QB bias update.  On one rank the
+update runs inside the forward (LMOE_UPDATE_BIAS: a graph branch that starts once routing is
+done); with N > 1 ranks every rank runs its own tokens (weak scaling) and the ranks sum their QB
+histograms with one NCCL all-reduce before lmoe_qb_update, so every rank keeps the same bias.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mini_replica] [--tokens T]
     python bench.py --impl reference ...   # the CPU oracle on the host cores, same metric
@@ -149,13 +150,18 @@ def run_ours(args, rank, world, local_rank):
     x = x_cpu.cuda()
     y = torch.empty_like(x)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    # one rank: the update runs inside the forward, as a branch after routing
+    layer.set_update(BETA)
 
     def step():
+        if world == 1:
+            layer.forward(x, y, update_bias=True)
+            return
         layer.forward(x, y, record_stats=True)
-        if world > 1:  # the one exchange step: sum the QB statistics of all ranks
-            hist, n = layer.hist()
-            lq.sum_qb_statistics(hist, n)
-            layer.set_hist(hist, n)
+        # the one exchange step: sum the QB statistics of all ranks
+        hist, n = layer.hist()
+        lq.sum_qb_statistics(hist, n)
+        layer.set_hist(hist, n)
         layer.qb_update(BETA)
 
     def barrier():
@@ -204,11 +210,13 @@ def run_ours(args, rank, world, local_rank):
     yh = torch.empty_like(xh).pin_memory()
 
     def step_host():
+        if world == 1:
+            layer.forward_host(xh, yh, update_bias=True)
+            return
         layer.forward_host(xh, yh, record_stats=True)
-        if world > 1:
-            hist, n = layer.hist()
-            lq.sum_qb_statistics(hist, n)
-            layer.set_hist(hist, n)
+        hist, n = layer.hist()
+        lq.sum_qb_statistics(hist, n)
+        layer.set_hist(hist, n)
         layer.qb_update(BETA)
 
     for _ in range(3):
@@ -286,13 +294,15 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None, "dtype": shape.dtype, "data": "synthetic (seeded; x ~ N(0,1), weights ~ N(0,1/fan_in))",
         "config": {"workload": shape.name, "T": T, "d": shape.d, "l": shape.l, "E": shape.E, "k": shape.k,
                    "h": shape.h, "hs": shape.hs, "tokens_per_gpu": T, "global_tokens": T * world,
-                   "step": "forward with QB statistics + QB update", "beta": BETA,
+                   "step": "forward with QB statistics + QB update"
+                           + (" (update inside the forward, after routing)" if world == 1 else ""), "beta": BETA,
                    "l2": "flushed between steps (256 MiB write outside the timed events)",
                    "parallelism": f"dp{world}" + (" (histogram all-reduce)" if world > 1 else "")},
         "e2e": {"value": round(T * world / (e2e_ms / 1e3), 1), "unit": UNIT, "ms_per_step": round(e2e_ms, 5),
                 "h2d_bytes_per_step": T * shape.d * (2 if shape.dtype == "bf16" else 4),
                 "d2h_bytes_per_step": T * shape.d * (2 if shape.dtype == "bf16" else 4),
-                "api": "lmoe_forward_host + lmoe_qb_update, pinned host buffers"},
+                "api": ("lmoe_forward_host with LMOE_UPDATE_BIAS" if world == 1 else
+                        "lmoe_forward_host + histogram all-reduce + lmoe_qb_update") + ", pinned host buffers"},
         "gpu_launches": launches,
         "kernel_timing": "CUDA events before every stage on the launching stream, in a second pass of the "
                          "same K steps with eager launches (the timed region replays each call as a CUDA graph)",

@@ -61,6 +61,11 @@ extern "C" {
 #define LMOE_RECORD_STATS 1u    /* add this forward's scores to the QB histogram and its expert
                                    loads to the load counters (training); without it the forward
                                    leaves the balancing state untouched */
+#define LMOE_UPDATE_BIAS 4u     /* with LMOE_RECORD_STATS: the bias update of lmoe_qb_update, with
+                                   the step and flags set by lmoe_set_update, runs inside this
+                                   forward right after its routing (a parallel branch of the
+                                   forward's work) on everything recorded up to and including
+                                   this forward; it changes only later forwards */
 /* lmoe_qb_update flags */
 #define LMOE_QB_LITERAL 1u      /* u_e = q_e (quantile of the unbiased column) */
 #define LMOE_BIAS_SIGN 2u       /* aux-loss-free sign rule instead of QB (see lmoe_qb_update) */
@@ -142,6 +147,14 @@ int lmoe_forward_host(lmoe_handle *h, const void *x_host, void *y_host, int32_t 
  * LMOE_BIAS_SIGN is LMOE_EINVAL.  Either rule then clears the histogram, N and the loads.
  * With N == 0 the bias is left unchanged.  Delayed: it changes only later forwards. */
 int lmoe_qb_update(lmoe_handle *h, float beta, uint32_t flags, void *stream);
+
+/* Step and flags (LMOE_QB_LITERAL or LMOE_BIAS_SIGN, as for lmoe_qb_update) of the update that
+ * forwards with LMOE_UPDATE_BIAS run.  LMOE_EINVAL for a NaN step or both flags.  A forward with
+ * LMOE_UPDATE_BIAS before any lmoe_set_update, or without LMOE_RECORD_STATS, is LMOE_EINVAL.
+ * The result equals lmoe_forward with LMOE_RECORD_STATS followed by lmoe_qb_update on the same
+ * stream: the update reads only statistics that are final once routing is done, and nothing
+ * later in the forward reads the bias or the statistics. */
+int lmoe_set_update(lmoe_handle *h, float beta, uint32_t flags);
 
 /* Routing stage on caller-given scores: runs biased top-k, gates, counts, offsets, the stable
  * permutation and (with LMOE_RECORD_STATS) the histogram on scores_dev[T,E] fp32, exactly as

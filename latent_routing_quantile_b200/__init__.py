@@ -17,6 +17,7 @@ LIB_PATH = os.path.join(_HERE, "liblmoe.so")
 
 F32, BF16 = 0, 1
 RECORD_STATS = 1
+UPDATE_BIAS = 4
 QB_LITERAL = 1
 BIAS_SIGN = 2
 STATUS_NAN_SCORE, STATUS_WATCHDOG, STATUS_BAD_INDEX = 1, 2, 4
@@ -24,7 +25,7 @@ NBINS = 4096
 
 EXPORTED = (
     "lmoe_create", "lmoe_destroy", "lmoe_workspace_bytes", "lmoe_forward", "lmoe_forward_host",
-    "lmoe_qb_update", "lmoe_route_scores", "lmoe_get_routing", "lmoe_get_bias", "lmoe_set_bias",
+    "lmoe_qb_update", "lmoe_set_update", "lmoe_route_scores", "lmoe_get_routing", "lmoe_get_bias", "lmoe_set_bias",
     "lmoe_get_hist", "lmoe_set_hist", "lmoe_get_load", "lmoe_set_load", "lmoe_get_status", "lmoe_strerror", "lmoe_gemm_bf16",
     "lmoe_profile_enable", "lmoe_profile_read", "lmoe_stage_name", "lmoe_launch_count",
     "lmoe_route_noalloc", "lmoe_watchdog_selftest",
@@ -65,6 +66,7 @@ def lib() -> ctypes.CDLL:
             "lmoe_forward": [vp, vp, vp, i32, u32, vp],
             "lmoe_forward_host": [vp, vp, vp, i32, u32, vp],
             "lmoe_qb_update": [vp, c_float, u32, vp],
+            "lmoe_set_update": [vp, c_float, u32],
             "lmoe_route_scores": [vp, vp, i32, u32, vp],
             "lmoe_get_routing": [vp, vp, vp, vp, vp, vp, vp, vp, vp],
             "lmoe_get_bias": [vp, vp, vp],
@@ -148,24 +150,30 @@ class Layer:
         self.last_T = 0
 
     # ---------------------------------------------------------------- forward
-    def forward(self, x, y=None, record_stats=False, stream=None):
+    @staticmethod
+    def _fwd_flags(record_stats, update_bias):
+        # update_bias records this forward's statistics too (the update counts them)
+        return (RECORD_STATS if (record_stats or update_bias) else 0) | (UPDATE_BIAS if update_bias else 0)
+
+    def forward(self, x, y=None, record_stats=False, update_bias=False, stream=None):
+        """update_bias=True also runs the bias update set by set_update inside this forward."""
         T = x.shape[0]
         _dev(x, self.dtype, (T, self.cfg.d), "x")
         if y is None:
             y = torch.empty_like(x)
         _dev(y, self.dtype, (T, self.cfg.d), "y")
-        _check(lib().lmoe_forward(self.handle, _ptr(x), _ptr(y), T, RECORD_STATS if record_stats else 0,
+        _check(lib().lmoe_forward(self.handle, _ptr(x), _ptr(y), T, self._fwd_flags(record_stats, update_bias),
                                   _stream(stream)), "lmoe_forward")
         self.last_T = T
         return y
 
-    def forward_host(self, x_host, y_host, record_stats=False, stream=None):
+    def forward_host(self, x_host, y_host, record_stats=False, update_bias=False, stream=None):
         """Host tensors (pinned for asynchronous copies); y_host is valid after the stream syncs."""
         T = x_host.shape[0]
         if x_host.is_cuda or y_host.is_cuda or x_host.dtype != self.dtype or y_host.dtype != self.dtype:
             raise LmoeError("forward_host takes host tensors of the layer dtype")
         _check(lib().lmoe_forward_host(self.handle, c_void_p(x_host.data_ptr()), c_void_p(y_host.data_ptr()), T,
-                                       RECORD_STATS if record_stats else 0, _stream(stream)),
+                                       self._fwd_flags(record_stats, update_bias), _stream(stream)),
                "lmoe_forward_host")
         self.last_T = T
         return y_host
@@ -182,6 +190,11 @@ class Layer:
         aux-loss-free rule b_e += beta * sign(mean load - load_e)."""
         flags = (QB_LITERAL if literal else 0) | (BIAS_SIGN if sign_rule else 0)
         _check(lib().lmoe_qb_update(self.handle, float(beta), flags, _stream(stream)), "lmoe_qb_update")
+
+    def set_update(self, beta, literal=False, sign_rule=False):
+        """Step and rule of the update that forward(..., update_bias=True) runs after its routing."""
+        flags = (QB_LITERAL if literal else 0) | (BIAS_SIGN if sign_rule else 0)
+        _check(lib().lmoe_set_update(self.handle, float(beta), flags), "lmoe_set_update")
 
     # ---------------------------------------------------------------- introspection
     def routing(self, stream=None):

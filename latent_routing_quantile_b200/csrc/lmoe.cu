@@ -364,6 +364,12 @@ struct lmoe_handle {
   // graph replay of repeated calls
   cudaStream_t cap = nullptr;
   GraphCache g_fwd[2], g_qb;  // two forward graphs (the host path alternates input buffers)
+  // LMOE_UPDATE_BIAS: the update's step and flags, and the branch it runs on
+  bool upd_set = false;
+  float upd_beta = 0.f;
+  uint32_t upd_flags = 0;
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
   long long g_tick = 0;
   long long g_used[2] = {0, 0};
 };
@@ -560,6 +566,52 @@ int flush_bins(lmoe_handle* h, int pend_T, int buf, cudaStream_t st) {
   return LMOE_OK;
 }
 
+// The bias update (QB, or the sign rule) from the statistics state `at`.  `pdl` = false launches
+// it without programmatic serialisation: on a side branch its blocks would otherwise become
+// resident as soon as the kernel before the fork allowed dependents, and sit in their wait
+// holding SM slots that the persistent GEMMs of the main branch need.
+int launch_qb(lmoe_handle* h, float beta, uint32_t flags, const StatsState& at, cudaStream_t s, bool pdl = true) {
+  const int literal = (flags & LMOE_QB_LITERAL) ? 1 : 0, sign = (flags & LMOE_BIAS_SIGN) ? 1 : 0;
+  const uint16_t* bins = (const uint16_t*)bin_buffer(h, at.pend_buf);
+  if (pdl) {
+    CK(launch_k(qb_update_kernel, dim3(h->cfg.E), dim3(kQbThreads), 0, s, 1, h->hist, h->ntok, h->load, h->bias,
+                h->cfg.E, h->cfg.k, literal, sign, beta, h->u, h->qb_done, bins, h->ld_bins, at.pend_T,
+                at.hist_live ? 1 : 0, h->status));
+  } else {
+    qb_update_kernel<<<h->cfg.E, kQbThreads, 0, s>>>(h->hist, h->ntok, h->load, h->bias, h->cfg.E, h->cfg.k,
+                                                     literal, sign, beta, h->u, h->qb_done, bins, h->ld_bins,
+                                                     at.pend_T, at.hist_live ? 1 : 0, h->status);
+    CK(cudaGetLastError());
+  }
+  h->launches += 1;
+  return LMOE_OK;
+}
+
+// LMOE_UPDATE_BIAS without profiling: the update is a branch that forks off `st` once every
+// statistic it reads is final and joins `st` at the end of the forward (no later kernel of the
+// forward reads or writes the bias or the statistics).  QB reads the histogram, N and the bins
+// that top-k writes, so it forks right after top-k, beside the latency-bound plan kernel, unless
+// bins of an earlier forward still have to be flushed into the histogram; the plan kernel then
+// leaves the loads alone (the update zeroes them, as it would after adding them).  The sign rule
+// reads the loads that the plan kernel adds, so it forks after routing.
+bool fork_after_topk(lmoe_handle* h, uint32_t flags, const StatsState& pre) {
+  return !(h->upd_flags & LMOE_BIAS_SIGN) && !pre.pend_T && (flags & LMOE_UPDATE_BIAS) && !h->profiling;
+}
+int fork_update(lmoe_handle* h, int T, uint32_t flags, const StatsState& pre, cudaStream_t st) {
+  if (!(flags & LMOE_UPDATE_BIAS) || h->profiling) return LMOE_OK;
+  CK(cudaEventRecord(h->ev_fork, st));
+  CK(cudaStreamWaitEvent(h->side, h->ev_fork, 0));
+  int rc = launch_qb(h, h->upd_beta, h->upd_flags, after_routing(pre, T, flags), h->side, false);
+  if (rc) return rc;
+  CK(cudaEventRecord(h->ev_join, h->side));
+  return LMOE_OK;
+}
+int join_update(lmoe_handle* h, uint32_t flags, cudaStream_t st) {
+  if (!(flags & LMOE_UPDATE_BIAS) || h->profiling) return LMOE_OK;
+  CK(cudaStreamWaitEvent(st, h->ev_join, 0));
+  return LMOE_OK;
+}
+
 int route_from_scores(lmoe_handle* h, int T, uint32_t flags, const StatsState& pre, const void* x,
                       cudaStream_t st) {
   const StatsState post = after_routing(pre, T, flags);
@@ -574,10 +626,16 @@ int route_from_scores(lmoe_handle* h, int T, uint32_t flags, const StatsState& p
               (flags & LMOE_RECORD_STATS) ? bin_buffer(h, post.pend_buf) : nullptr, h->ld_bins,
               TopkRefine{x, h->bf ? 1 : 0, c.d, h->wc, h->c, c.rms_eps, h->tau}, h->status};
   CK(launch_topk(ta, st));
+  const bool early = fork_after_topk(h, flags, pre);
+  if (early) {
+    int rc = fork_update(h, T, flags, pre, st);
+    if (rc) return rc;
+  }
   mark(h, ST_PLAN, st);
   CK(launch_k(plan_kernel, dim3((c.E + 31) / 32), dim3(1024), 0, st, 1, (const int*)h->counts32, h->counts,
               (const int*)h->blkcnt, nblk, c.E, h->offsets, h->pad_delta, h->blkbase, h->mtiles, h->num_mtiles,
-              (flags & LMOE_RECORD_STATS) ? h->load : (long long*)nullptr));
+              // an update already forked clears the loads itself, which equals adding them first
+              ((flags & LMOE_RECORD_STATS) && !early) ? h->load : (long long*)nullptr));
   const int pairs = T * c.k;
   const dim3 ggrid((pairs + 8 * kGatherPairs - 1) / (8 * kGatherPairs));
   int4* clear = reinterpret_cast<int4*>(h->counts32);
@@ -602,7 +660,7 @@ int route_from_scores(lmoe_handle* h, int T, uint32_t flags, const StatsState& p
     if (rc) return rc;
   }
   h->last_T = T;
-  return LMOE_OK;
+  return early ? LMOE_OK : fork_update(h, T, flags, pre, st);
 }
 
 int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, const StatsState& pre,
@@ -789,7 +847,7 @@ int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, 
     }
   }
   h->launches += (c.hs ? 1 : 0) + 4;
-  return LMOE_OK;
+  return join_update(h, flags, st);
 }
 
 int forward_f32(lmoe_handle* h, const void* xv, void* yv, int T, uint32_t flags, const StatsState& pre,
@@ -868,7 +926,7 @@ int forward_f32(lmoe_handle* h, const void* xv, void* yv, int T, uint32_t flags,
     CK(launch_simt<SE_STORE>(p, mt, st));
   }
   h->launches += 4 + (c.hs ? 2 : 1) + 2;
-  return LMOE_OK;
+  return join_update(h, flags, st);
 }
 
 int repack(lmoe_handle* h, const lmoe_weights* w, cudaStream_t st) {
@@ -1078,6 +1136,10 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, void* stream, lmo
   if (!rc && h->bf) rc = build_maps(h);
   if (!rc && cudaStreamCreateWithFlags(&h->cap, cudaStreamNonBlocking) != cudaSuccess) rc = LMOE_ECUDA;
   if (!rc && cudaStreamCreateWithFlags(&h->cp_in, cudaStreamNonBlocking) != cudaSuccess) rc = LMOE_ECUDA;
+  if (!rc && cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking) != cudaSuccess) rc = LMOE_ECUDA;
+  if (!rc && (cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+              cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming) != cudaSuccess))
+    rc = LMOE_ECUDA;
   for (int i = 0; !rc && i < 2; ++i)
     if (cudaEventCreateWithFlags(&h->ev_in[i], cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&h->ev_fwd[i], cudaEventDisableTiming) != cudaSuccess)
@@ -1101,6 +1163,9 @@ int lmoe_destroy(lmoe_handle* h) {
   h->g_qb.reset(nullptr, nullptr, -1, 0, 0.f, 0);
   if (h->cap) cudaStreamDestroy(h->cap);
   if (h->cp_in) cudaStreamDestroy(h->cp_in);
+  if (h->side) cudaStreamDestroy(h->side);
+  if (h->ev_fork) cudaEventDestroy(h->ev_fork);
+  if (h->ev_join) cudaEventDestroy(h->ev_join);
   for (int i = 0; i < 2; ++i) {
     if (h->ev_in[i]) cudaEventDestroy(h->ev_in[i]);
     if (h->ev_fwd[i]) cudaEventDestroy(h->ev_fwd[i]);
@@ -1118,19 +1183,36 @@ int lmoe_forward(lmoe_handle* h, const void* x, void* y, int32_t T, uint32_t fla
   if ((const char*)x < (const char*)y + bytes && (const char*)y < (const char*)x + bytes) return LMOE_EINVAL;
   cudaStream_t st = (cudaStream_t)stream;
   h->last_T = T;
+  const bool upd = (flags & LMOE_UPDATE_BIAS) != 0;
+  if (upd && (!(flags & LMOE_RECORD_STATS) || !h->upd_set)) return LMOE_EINVAL;
   const StatsState pre = h->ss;
+  // graph key: the arguments, the update's step and flags, the statistics state
+  const uint32_t kflags = flags | (upd ? h->upd_flags << 16 : 0u);
+  const float kbeta = upd ? h->upd_beta : 0.f;
   // the cached graph of these arguments, else the least recently used one
-  int gi = h->g_fwd[0].same(x, y, T, flags, 0.f, pre.key()) ? 0
-           : h->g_fwd[1].same(x, y, T, flags, 0.f, pre.key()) ? 1
+  int gi = h->g_fwd[0].same(x, y, T, kflags, kbeta, pre.key()) ? 0
+           : h->g_fwd[1].same(x, y, T, kflags, kbeta, pre.key()) ? 1
            : (h->g_used[0] <= h->g_used[1] ? 0 : 1);
   h->g_used[gi] = ++h->g_tick;
-  int rc = run_cached(h, h->g_fwd[gi], x, y, T, flags, 0.f, pre.key(), st, [&](cudaStream_t s) {
+  int rc = run_cached(h, h->g_fwd[gi], x, y, T, kflags, kbeta, pre.key(), st, [&](cudaStream_t s) {
     prof_open(h, ST_RMS, ST_UP - ST_RMS + 1);
     int r = h->bf ? forward_bf16(h, x, y, T, flags, pre, s) : forward_f32(h, x, y, T, flags, pre, s);
     prof_close(h, s);
+    if (!r && upd && h->profiling) {  // profiled: the update after the forward, timed as its own stage
+      prof_open(h, ST_QB_UPDATE, 1);
+      mark(h, ST_QB_UPDATE, s);
+      r = launch_qb(h, h->upd_beta, h->upd_flags, after_routing(pre, T, flags), s);
+      prof_close(h, s);
+    }
     return r;
   });
-  if (rc == LMOE_OK) h->ss = after_routing(pre, T, flags);
+  if (rc == LMOE_OK) {
+    h->ss = after_routing(pre, T, flags);
+    if (upd) {  // the update consumed every statistic recorded so far
+      h->ss.pend_T = 0;
+      h->ss.hist_live = false;
+    }
+  }
   return rc;
 }
 
@@ -1172,6 +1254,7 @@ int lmoe_route_scores(lmoe_handle* h, const float* scores, int32_t T, uint32_t f
   CK(cudaMemcpyAsync(h->s, scores, (size_t)T * h->cfg.E * 4, cudaMemcpyDeviceToDevice, st));
   prof_open(h, ST_TOPK, ST_HIST - ST_TOPK + 1);
   const StatsState pre = h->ss;
+  flags &= LMOE_RECORD_STATS;  // the routing stage alone runs no update
   int rc = route_from_scores(h, T, flags, pre, nullptr, st);
   prof_close(h, st);
   if (rc == LMOE_OK) h->ss = after_routing(pre, T, flags);
@@ -1186,19 +1269,24 @@ int lmoe_qb_update(lmoe_handle* h, float beta, uint32_t flags, void* stream) {
   int rc = run_cached(h, h->g_qb, nullptr, nullptr, 0, flags, beta, pre.key(), st, [&](cudaStream_t s) {
     prof_open(h, ST_QB_UPDATE, 1);
     mark(h, ST_QB_UPDATE, s);
-    CK(launch_k(qb_update_kernel, dim3(h->cfg.E), dim3(kQbThreads), 0, s, 1, h->hist, h->ntok, h->load, h->bias,
-                h->cfg.E, h->cfg.k, (flags & LMOE_QB_LITERAL) ? 1 : 0, (flags & LMOE_BIAS_SIGN) ? 1 : 0, beta,
-                h->u, h->qb_done, (const uint16_t*)bin_buffer(h, pre.pend_buf), h->ld_bins, pre.pend_T,
-                pre.hist_live ? 1 : 0, h->status));
+    int r = launch_qb(h, beta, flags, pre, s);
     prof_close(h, s);
-    h->launches += 1;
-    return LMOE_OK;
+    return r;
   });
   if (rc == LMOE_OK) {
     h->ss.pend_T = 0;
     h->ss.hist_live = false;
   }
   return rc;
+}
+
+int lmoe_set_update(lmoe_handle* h, float beta, uint32_t flags) {
+  if (!h || !(beta == beta)) return LMOE_EINVAL;
+  if ((flags & LMOE_QB_LITERAL) && (flags & LMOE_BIAS_SIGN)) return LMOE_EINVAL;
+  h->upd_beta = beta;
+  h->upd_flags = flags & (LMOE_QB_LITERAL | LMOE_BIAS_SIGN);
+  h->upd_set = true;
+  return LMOE_OK;
 }
 
 int lmoe_get_routing(lmoe_handle* h, int32_t* idx, float* gates, float* scores, int32_t* counts, int32_t* offsets,

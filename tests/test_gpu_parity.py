@@ -473,3 +473,99 @@ def test_wide_stress_sampled():
     layer, y, ro, stats = run_layer_check(shape, w, x, sample=sample)
     print("wide_stress", json.dumps(stats))
     layer.close()
+
+
+@pytest.mark.parametrize("dtype,rule", [("bf16", "qb"), ("bf16", "sign"), ("f32", "qb")])
+def test_update_inside_forward_matches_separate_update(dtype, rule):
+    """A training loop whose forwards run the bias update themselves (LMOE_UPDATE_BIAS) gives,
+    step by step and bit for bit, the outputs and biases of the loop that records statistics and
+    calls the update after each forward; that holds with per-stage profiling on (the update then
+    runs after the forward), through the host-buffer entry point, and when a plain recorded
+    forward precedes the fused one (its statistics are counted by the fused update).  The QB
+    branch starts right after top-k unless earlier bins wait to be flushed; either way the
+    loads and N are zero after the step, as after a separate update."""
+    shape = datagen.LayerShape("fused_upd", 300, 128, 64, 64, 4, 64, 128, dtype, seed=31,
+                               offset_var=0.5, beta=0.05)
+    w = datagen.layer_weights(shape)
+    xs = [datagen.tokens(shape, seed=31 + i) for i in range(5)]
+    sign = rule == "sign"
+    beta = 1e-2 if sign else shape.beta
+
+    def loop(mode):
+        layer = make_layer(shape, w)
+        if mode != "separate":
+            layer.set_update(beta, sign_rule=sign)
+        if mode == "profiled":
+            layer.profile(True)
+        ys, bs, ls = [], [], []
+        for i, x in enumerate(xs):
+            if mode == "separate" or (mode == "preceded" and i % 2 == 0):
+                y = layer.forward(x.cuda(), record_stats=True)
+                if mode == "separate":
+                    layer.qb_update(beta, sign_rule=sign)
+            elif mode == "host":
+                xh = x.pin_memory()
+                y = torch.empty_like(xh).pin_memory()
+                layer.forward_host(xh, y, update_bias=True)
+            else:
+                y = layer.forward(x.cuda(), update_bias=True)
+            torch.cuda.synchronize()
+            ys.append(y.cpu().clone())
+            bs.append(layer.bias().cpu().clone())
+            # reading the histogram flushes pending bins: not after a plain recorded forward, so
+            # that the next fused forward still has to flush them itself
+            plain = mode == "preceded" and i % 2 == 0
+            ls.append((layer.load().cpu().clone(), None if plain else int(layer.hist()[1].item())))
+        layer.close()
+        return ys, bs, ls
+
+    ys0, bs0, ls0 = loop("separate")
+    assert all(int(ld.abs().sum()) == 0 and n == 0 for ld, n in ls0)
+    assert not torch.equal(bs0[-1], torch.zeros_like(bs0[-1]))  # the bias did move
+    for mode in ("fused", "profiled", "host"):
+        ys, bs, ls = loop(mode)
+        for i in range(len(xs)):
+            assert torch.equal(ys[i], ys0[i]), (mode, i)
+            assert torch.equal(bs[i], bs0[i]), (mode, i)
+            assert torch.equal(ls[i][0], ls0[i][0]) and ls[i][1] == 0, (mode, i)
+    # a plain recorded forward, then a fused one: one update over both, like record+record+update
+    layer = make_layer(shape, w)
+    for i in (0, 1):
+        layer.forward(xs[i].cuda(), record_stats=True)
+    layer.qb_update(beta, sign_rule=sign)
+    b_sep = layer.bias().cpu().clone()
+    layer.close()
+    ys, bs, ls = loop("preceded")
+    assert torch.equal(bs[1], b_sep)
+    assert int(ls[1][0].abs().sum()) == 0 and ls[1][1] == 0
+    assert int(ls[0][0].sum()) == shape.T * shape.k  # recorded, not yet consumed
+
+
+def test_update_inside_forward_argument_errors():
+    shape = datagen.LayerShape("fused_err", 64, 64, 64, 64, 4, 64, 0, "bf16", seed=3)
+    layer = make_layer(shape, datagen.layer_weights(shape))
+    x = datagen.tokens(shape, seed=3).cuda()
+    y = torch.empty_like(x)
+    L = lq.lib()
+    stream = torch.cuda.current_stream().cuda_stream
+    import ctypes
+    # no step set yet
+    rc = L.lmoe_forward(layer.handle, ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(y.data_ptr()), shape.T,
+                        lq.RECORD_STATS | lq.UPDATE_BIAS, ctypes.c_void_p(stream))
+    assert rc != 0
+    with pytest.raises(lq.LmoeError):
+        layer.set_update(0.1, literal=True, sign_rule=True)
+    with pytest.raises(lq.LmoeError):
+        layer.set_update(float("nan"))
+    layer.set_update(0.1)
+    # the update needs the statistics of this forward recorded
+    rc = L.lmoe_forward(layer.handle, ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(y.data_ptr()), shape.T,
+                        lq.UPDATE_BIAS, ctypes.c_void_p(stream))
+    assert rc != 0
+    b0 = layer.bias().cpu().clone()
+    layer.forward(x, y, update_bias=True)
+    torch.cuda.synchronize()
+    assert not torch.equal(layer.bias().cpu(), b0)
+    hist, n = layer.hist()
+    assert int(n.item()) == 0 and int(hist.sum().item()) == 0  # the update consumed the statistics
+    layer.close()
