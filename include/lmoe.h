@@ -66,6 +66,9 @@ extern "C" {
                                    forward right after its routing (a parallel branch of the
                                    forward's work) on everything recorded up to and including
                                    this forward; it changes only later forwards */
+#define LMOE_ASYNC_OUTPUT 8u     /* lmoe_forward_host only: the copy to y_host runs on a handle-owned
+                                   stream, so the next call's forward overlaps it; y_host is valid
+                                   only after lmoe_host_wait (see there) */
 /* lmoe_qb_update flags */
 #define LMOE_QB_LITERAL 1u      /* u_e = q_e (quantile of the unbiased column) */
 #define LMOE_BIAS_SIGN 2u       /* aux-loss-free sign rule instead of QB (see lmoe_qb_update) */
@@ -133,9 +136,21 @@ int lmoe_forward(lmoe_handle *h, const void *x_dev, void *y_dev, int32_t T, uint
  * staging buffers (ordered by events: it waits for the forward that last read that buffer, and
  * the forward waits for it), so one call's input copy overlaps the previous call's forward.
  * y_host is valid, and x_host may change, after `stream` synchronises.  Under stream capture of
- * `stream` everything stays on `stream`. */
+ * `stream` everything stays on `stream` (LMOE_EINVAL while an LMOE_ASYNC_OUTPUT copy is
+ * outstanding: call lmoe_host_wait and synchronise first).
+ * With LMOE_ASYNC_OUTPUT the forward writes one of two handle-owned output buffers and the copy
+ * to y_host runs on a second handle-owned copy stream once the forward is done; `stream` does not
+ * wait for it, so a serving loop overlaps the output copy of call i with the input copy and
+ * forward of call i+1 (a forward into a buffer waits for the copy that last read it).  y_host must
+ * then stay allocated and unread until lmoe_host_wait has been enqueued on a stream and that
+ * stream has synchronised; x_host may change after `stream` synchronises, as above. */
 int lmoe_forward_host(lmoe_handle *h, const void *x_host, void *y_host, int32_t T,
                       uint32_t flags, void *stream);
+
+/* Makes `stream` wait for every LMOE_ASYNC_OUTPUT output copy enqueued so far (they run in call
+ * order on one stream).  After `stream` synchronises, every such y_host holds its forward's
+ * output.  A no-op when there are none. */
+int lmoe_host_wait(lmoe_handle *h, void *stream);
 
 /* Bias update from everything recorded since the last update (N = the sum of T of those
  * forwards).  Default, Quantile Balancing: m = ceil((E-k) N / E) (exact integer), q_e = histogram

@@ -18,13 +18,14 @@ LIB_PATH = os.path.join(_HERE, "liblmoe.so")
 F32, BF16 = 0, 1
 RECORD_STATS = 1
 UPDATE_BIAS = 4
+ASYNC_OUTPUT = 8
 QB_LITERAL = 1
 BIAS_SIGN = 2
 STATUS_NAN_SCORE, STATUS_WATCHDOG, STATUS_BAD_INDEX = 1, 2, 4
 NBINS = 4096
 
 EXPORTED = (
-    "lmoe_create", "lmoe_destroy", "lmoe_workspace_bytes", "lmoe_forward", "lmoe_forward_host",
+    "lmoe_create", "lmoe_destroy", "lmoe_workspace_bytes", "lmoe_forward", "lmoe_forward_host", "lmoe_host_wait",
     "lmoe_qb_update", "lmoe_set_update", "lmoe_route_scores", "lmoe_get_routing", "lmoe_get_bias", "lmoe_set_bias",
     "lmoe_get_hist", "lmoe_set_hist", "lmoe_get_load", "lmoe_set_load", "lmoe_get_status", "lmoe_strerror", "lmoe_gemm_bf16",
     "lmoe_profile_enable", "lmoe_profile_read", "lmoe_stage_name", "lmoe_launch_count",
@@ -65,6 +66,7 @@ def lib() -> ctypes.CDLL:
             "lmoe_workspace_bytes": [POINTER(lmoe_config), POINTER(c_size_t)],
             "lmoe_forward": [vp, vp, vp, i32, u32, vp],
             "lmoe_forward_host": [vp, vp, vp, i32, u32, vp],
+            "lmoe_host_wait": [vp, vp],
             "lmoe_qb_update": [vp, c_float, u32, vp],
             "lmoe_set_update": [vp, c_float, u32],
             "lmoe_route_scores": [vp, vp, i32, u32, vp],
@@ -167,16 +169,23 @@ class Layer:
         self.last_T = T
         return y
 
-    def forward_host(self, x_host, y_host, record_stats=False, update_bias=False, stream=None):
-        """Host tensors (pinned for asynchronous copies); y_host is valid after the stream syncs."""
+    def forward_host(self, x_host, y_host, record_stats=False, update_bias=False, async_output=False,
+                     stream=None):
+        """Host tensors (pinned for asynchronous copies); y_host is valid after the stream syncs,
+        or with async_output=True after host_wait() and a sync of that stream."""
         T = x_host.shape[0]
         if x_host.is_cuda or y_host.is_cuda or x_host.dtype != self.dtype or y_host.dtype != self.dtype:
             raise LmoeError("forward_host takes host tensors of the layer dtype")
         _check(lib().lmoe_forward_host(self.handle, c_void_p(x_host.data_ptr()), c_void_p(y_host.data_ptr()), T,
-                                       self._fwd_flags(record_stats, update_bias), _stream(stream)),
+                                       self._fwd_flags(record_stats, update_bias) | (ASYNC_OUTPUT if async_output else 0),
+                                       _stream(stream)),
                "lmoe_forward_host")
         self.last_T = T
         return y_host
+
+    def host_wait(self, stream=None):
+        """Makes the stream wait for every async_output copy enqueued so far."""
+        _check(lib().lmoe_host_wait(self.handle, _stream(stream)), "lmoe_host_wait")
 
     def route_scores(self, scores, record_stats=False, stream=None):
         T = scores.shape[0]

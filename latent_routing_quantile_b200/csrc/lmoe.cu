@@ -330,10 +330,17 @@ struct lmoe_handle {
   // lmoe_forward_host: two input staging buffers, so the next call's host-to-device copy (on its
   // own stream) overlaps this call's forward
   void* x_stage2 = nullptr;
+  void* y_stage2 = nullptr;
   int host_slot = 0;
   cudaStream_t cp_in = nullptr;
   cudaEvent_t ev_in[2] = {nullptr, nullptr}, ev_fwd[2] = {nullptr, nullptr};
   bool fwd_recorded[2] = {false, false};
+  // LMOE_ASYNC_OUTPUT: output copies on their own stream; out_pending[i] = an output copy from
+  // staging slot i was enqueued there and no forward into that slot has waited for it yet
+  cudaStream_t cp_out = nullptr;
+  cudaEvent_t ev_out[2] = {nullptr, nullptr};
+  bool out_pending[2] = {false, false};
+  int last_out = -1;  // slot of the last output copy enqueued on cp_out
   // state
   float* bias = nullptr;
   uint32_t* hist = nullptr;
@@ -431,6 +438,7 @@ void plan_layout(lmoe_handle* h, Arena& a) {
   a.add(&h->x_stage, Tm * d * es);
   a.add(&h->x_stage2, Tm * d * es);
   a.add(&h->y_stage, Tm * d * es);
+  a.add(&h->y_stage2, Tm * d * es);
   // state
   a.add((void**)&h->bias, E * 4);
   a.add((void**)&h->hist, E * LMOE_NBINS * 4);
@@ -1136,13 +1144,15 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, void* stream, lmo
   if (!rc && h->bf) rc = build_maps(h);
   if (!rc && cudaStreamCreateWithFlags(&h->cap, cudaStreamNonBlocking) != cudaSuccess) rc = LMOE_ECUDA;
   if (!rc && cudaStreamCreateWithFlags(&h->cp_in, cudaStreamNonBlocking) != cudaSuccess) rc = LMOE_ECUDA;
+  if (!rc && cudaStreamCreateWithFlags(&h->cp_out, cudaStreamNonBlocking) != cudaSuccess) rc = LMOE_ECUDA;
   if (!rc && cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking) != cudaSuccess) rc = LMOE_ECUDA;
   if (!rc && (cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
               cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming) != cudaSuccess))
     rc = LMOE_ECUDA;
   for (int i = 0; !rc && i < 2; ++i)
     if (cudaEventCreateWithFlags(&h->ev_in[i], cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&h->ev_fwd[i], cudaEventDisableTiming) != cudaSuccess)
+        cudaEventCreateWithFlags(&h->ev_fwd[i], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&h->ev_out[i], cudaEventDisableTiming) != cudaSuccess)
       rc = LMOE_ECUDA;
   if (rc) {
     cudaStreamSynchronize(st);
@@ -1163,12 +1173,14 @@ int lmoe_destroy(lmoe_handle* h) {
   h->g_qb.reset(nullptr, nullptr, -1, 0, 0.f, 0);
   if (h->cap) cudaStreamDestroy(h->cap);
   if (h->cp_in) cudaStreamDestroy(h->cp_in);
+  if (h->cp_out) cudaStreamDestroy(h->cp_out);
   if (h->side) cudaStreamDestroy(h->side);
   if (h->ev_fork) cudaEventDestroy(h->ev_fork);
   if (h->ev_join) cudaEventDestroy(h->ev_join);
   for (int i = 0; i < 2; ++i) {
     if (h->ev_in[i]) cudaEventDestroy(h->ev_in[i]);
     if (h->ev_fwd[i]) cudaEventDestroy(h->ev_fwd[i]);
+    if (h->ev_out[i]) cudaEventDestroy(h->ev_out[i]);
   }
   cudaFree(h->arena);
   delete h;
@@ -1183,6 +1195,7 @@ int lmoe_forward(lmoe_handle* h, const void* x, void* y, int32_t T, uint32_t fla
   if ((const char*)x < (const char*)y + bytes && (const char*)y < (const char*)x + bytes) return LMOE_EINVAL;
   cudaStream_t st = (cudaStream_t)stream;
   h->last_T = T;
+  flags &= ~LMOE_ASYNC_OUTPUT;  // a host-buffer option only
   const bool upd = (flags & LMOE_UPDATE_BIAS) != 0;
   if (upd && (!(flags & LMOE_RECORD_STATS) || !h->upd_set)) return LMOE_EINVAL;
   const StatsState pre = h->ss;
@@ -1223,27 +1236,51 @@ int lmoe_forward_host(lmoe_handle* h, const void* x_host, void* y_host, int32_t 
   const size_t bytes = (size_t)T * h->cfg.d * h->es;
   cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
   if (cudaStreamIsCapturing(st, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) {
-    // under the caller's stream capture everything stays on its stream
+    // under the caller's stream capture everything stays on its stream (an output copy still in
+    // flight on the handle's own stream would race with this forward's output)
+    if (h->out_pending[0] || h->out_pending[1]) return LMOE_EINVAL;
     CK(cudaMemcpyAsync(h->x_stage, x_host, bytes, cudaMemcpyHostToDevice, st));
-    int rc = lmoe_forward(h, h->x_stage, h->y_stage, T, flags, stream);
+    int rc = lmoe_forward(h, h->x_stage, h->y_stage, T, flags & ~LMOE_ASYNC_OUTPUT, stream);
     if (rc) return rc;
     CK(cudaMemcpyAsync(y_host, h->y_stage, bytes, cudaMemcpyDeviceToHost, st));
     return LMOE_OK;
   }
   // the input copy runs on the handle's copy stream into the staging buffer this call owns, once
-  // the forward that last read that buffer has finished; the forward waits for the copy
+  // the forward that last read that buffer has finished; the forward waits for the copy (and for
+  // an output copy still reading this slot's output buffer)
   const int sl = h->host_slot;
   void* xs = sl ? h->x_stage2 : h->x_stage;
+  void* ys = sl ? h->y_stage2 : h->y_stage;
   if (h->fwd_recorded[sl]) CK(cudaStreamWaitEvent(h->cp_in, h->ev_fwd[sl], 0));
   CK(cudaMemcpyAsync(xs, x_host, bytes, cudaMemcpyHostToDevice, h->cp_in));
   CK(cudaEventRecord(h->ev_in[sl], h->cp_in));
   CK(cudaStreamWaitEvent(st, h->ev_in[sl], 0));
-  int rc = lmoe_forward(h, xs, h->y_stage, T, flags, stream);
+  if (h->out_pending[sl]) {
+    CK(cudaStreamWaitEvent(st, h->ev_out[sl], 0));
+    h->out_pending[sl] = false;
+  }
+  int rc = lmoe_forward(h, xs, ys, T, flags & ~LMOE_ASYNC_OUTPUT, stream);
   if (rc) return rc;
   CK(cudaEventRecord(h->ev_fwd[sl], st));
   h->fwd_recorded[sl] = true;
   h->host_slot ^= 1;
-  CK(cudaMemcpyAsync(y_host, h->y_stage, bytes, cudaMemcpyDeviceToHost, st));
+  if (flags & LMOE_ASYNC_OUTPUT) {
+    // the output copy leaves `stream`: the next call's forward overlaps it
+    CK(cudaStreamWaitEvent(h->cp_out, h->ev_fwd[sl], 0));
+    CK(cudaMemcpyAsync(y_host, ys, bytes, cudaMemcpyDeviceToHost, h->cp_out));
+    CK(cudaEventRecord(h->ev_out[sl], h->cp_out));
+    h->out_pending[sl] = true;
+    h->last_out = sl;
+  } else {
+    CK(cudaMemcpyAsync(y_host, ys, bytes, cudaMemcpyDeviceToHost, st));
+  }
+  return LMOE_OK;
+}
+
+int lmoe_host_wait(lmoe_handle* h, void* stream) {
+  if (!h) return LMOE_EINVAL;
+  // cp_out runs its copies in order, so the last one's event covers every earlier one
+  if (h->last_out >= 0) CK(cudaStreamWaitEvent((cudaStream_t)stream, h->ev_out[h->last_out], 0));
   return LMOE_OK;
 }
 

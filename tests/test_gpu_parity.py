@@ -569,3 +569,45 @@ def test_update_inside_forward_argument_errors():
     hist, n = layer.hist()
     assert int(n.item()) == 0 and int(hist.sum().item()) == 0  # the update consumed the statistics
     layer.close()
+
+
+def test_host_forward_async_output_matches_device_forward():
+    """With LMOE_ASYNC_OUTPUT the output copies leave the caller's stream; after lmoe_host_wait
+    every host output equals the device-buffer forward of the same input, bit for bit, also when
+    synchronous and asynchronous calls alternate and more calls than staging buffers are in
+    flight.  Under stream capture an outstanding asynchronous copy is refused."""
+    shape = datagen.LayerShape("async_out", 384, 256, 128, 64, 4, 128, 256, "bf16", seed=41, offset_var=0.5)
+    w = datagen.layer_weights(shape)
+    xs = [datagen.tokens(shape, seed=41 + i) for i in range(5)]
+    ref = make_layer(shape, w)
+    want = [ref.forward(x.cuda()).cpu() for x in xs]
+    torch.cuda.synchronize()
+    ref.close()
+    layer = make_layer(shape, w)
+    xh = [x.pin_memory() for x in xs]
+    yh = [torch.empty_like(x).pin_memory() for x in xs]
+    modes = [True, True, False, True, True]
+    for i in range(5):
+        layer.forward_host(xh[i], yh[i], async_output=modes[i])
+    layer.host_wait()
+    torch.cuda.synchronize()
+    for i in range(5):
+        assert torch.equal(yh[i], want[i]), i
+    # a second round reusing one host output buffer: the copies land in call order
+    y_one = torch.empty_like(xh[0]).pin_memory()
+    for i in range(3):
+        layer.forward_host(xh[i], y_one, async_output=True)
+    layer.host_wait()
+    torch.cuda.synchronize()
+    assert torch.equal(y_one, want[2])
+    # capture with an asynchronous copy outstanding is refused
+    layer.forward_host(xh[0], yh[0], async_output=True)
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with pytest.raises(lq.LmoeError), pytest.warns(UserWarning):  # the graph stays empty
+        with torch.cuda.graph(g, stream=s):
+            layer.forward_host(xh[1], yh[1], stream=s)
+    layer.host_wait()
+    torch.cuda.synchronize()
+    assert torch.equal(yh[0], want[0])
+    layer.close()
