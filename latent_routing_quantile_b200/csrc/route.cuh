@@ -72,13 +72,17 @@ constexpr int kRefineExtra = 8;  // candidates beyond the k-th that an exact dec
 
 // The exact decision of a token whose fp32 top-k is ambiguous (two of its top k+1 biased scores
 // within tau of each other, so the scores' fp32 rounding could order them either way).  Its
-// candidates are every expert whose fp32 biased score lies within tau of the k-th (at most
-// kRefineExtra beyond the k-th).  Each candidate's biased score is recomputed in fp64 as the layer
-// defines it, u = sigmoid(r * (x . W_comb[e]) + c_e) + b_e with r = 1/sqrt(mean x^2 + eps) and
-// W_comb the router and down-projection weights multiplied out in fp64 (the same logit as
-// h W_r^T + c up to fp64 rounding), and the candidates are ranked by (u descending, expert
-// ascending).  The whole block computes each such token's dot products together (one memory
-// round trip instead of one per 32 elements), after its warps have ranked every other token.
+// candidates are its top k and every expert whose fp32 biased score lies within tau of the k-th
+// (at most kRefineExtra beyond the k-th), in fp32 order.  Consecutive candidates closer than tau
+// are linked; a maximal run of linked candidates is a cluster.  The fp32 error of a score is below
+// tau / 2, so candidates of different clusters are in their exact order already, and only the
+// members of clusters of two or more are rescored: each one's biased score is recomputed in fp64
+// as the layer defines it, u = sigmoid(r * (x . W_comb[e]) + c_e) + b_e with r = 1/sqrt(mean x^2
+// + eps) and W_comb the router and down-projection weights multiplied out in fp64 (the same logit
+// as h W_r^T + c up to fp64 rounding), and each cluster's members are ranked among its positions by
+// (u descending, expert ascending).  The whole block computes each such token's dot products
+// together (one memory round trip instead of one per 32 elements), after its warps have ranked
+// every other token.
 
 // One warp per token; a block of W warps ranks kTokBlock = 32 tokens (32 / W per warp; W = 16
 // for E <= 256, whose registers allow two such blocks per SM, else 8).  Lane L holds the scores
@@ -114,7 +118,9 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // tokens of the block that wait for the exact decision: candidates, (token | count << 8)
   __shared__ int def_e[kTokBlock][32];
-  __shared__ int def_info[kTokBlock];
+  __shared__ unsigned char def_mi[kTokBlock][32];  // candidate positions of the cluster members
+  __shared__ unsigned def_lp[kTokBlock];           // bit c: candidate c is linked to candidate c-1
+  __shared__ int def_info[kTokBlock];              // token | candidates << 8 | members << 16
   __shared__ int def_n;
   __shared__ double red[W][9];
   __shared__ double def_z[48];  // [0, 32): candidate dot products; [32, 41): first group's sums; 40: x^2
@@ -191,8 +197,8 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 
       // only then do further rounds collect the experts within tau of the k-th (at most
       // kRefineExtra)
       const int kmax = rf.x ? min(min(k + kRefineExtra, 32), E) : k;
-      float u_prev = 0.f, u_k1 = 0.f;
-      bool amb = false;
+      float u_prev = 0.f, u_k1 = 0.f, my_u = 0.f;
+      bool amb = false, odd = false;  // odd: a candidate without a numeric score
       int nc = 0, lim = k;
       for (int i = 0; i < lim; ++i) {
         uint32_t bk = 0u;
@@ -215,6 +221,8 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 
         if (lane == i) my_sel = (int)emin;
         if (rf.x) {
           const float ui = wmax >= 2u ? key_value(wmax) : 0.f;
+          if (wmax < 2u) odd = true;
+          if (lane == i) my_u = ui;
           if (i > 0 && wmax >= 2u && u_prev - ui < rf.tau) amb = true;
           if (i == k - 1) {
             u_k1 = ui;
@@ -233,11 +241,21 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 
         int slot = 0;
         if (lane == 0) slot = atomicAdd(&def_n, 1);
         slot = __shfl_sync(kFull, slot, 0);
+        // clusters: candidate c is linked to c-1 when their fp32 scores are within tau (every
+        // candidate is, when one of them has no numeric score)
+        const float u_up = __shfl_up_sync(kFull, my_u, 1);
+        const unsigned lpm = __ballot_sync(kFull, lane > 0 && lane < nc && (odd || u_up - my_u < rf.tau));
+        const unsigned mm = lpm | (lpm >> 1);  // members: linked to the previous or the next
         def_e[slot][lane] = lane < nc ? my_sel : -1;
-        if (lane == 0) def_info[slot] = tl | (nc << 8);
-        // warm L2 with the candidates' fp64 weight rows and the token's input row while the warp
+        if ((mm >> lane) & 1u) def_mi[slot][__popc(mm & ((1u << lane) - 1u))] = (unsigned char)lane;
+        if (lane == 0) {
+          def_lp[slot] = lpm;
+          def_info[slot] = tl | (nc << 8) | (__popc(mm) << 16);
+        }
+        // warm L2 with the members' fp64 weight rows and the token's input row while the warp
         // ranks its other tokens
-        for (int c = 0; c < nc; ++c) {
+        for (unsigned m = mm; m; m &= m - 1u) {
+          const int c = __ffs(m) - 1;
           const char* row = reinterpret_cast<const char*>(rf.wc + (size_t)__shfl_sync(kFull, my_sel, c) * rf.d);
           for (int b = lane * 128; b < rf.d * 8; b += 32 * 128) prefetch_l2(row + b);
         }
@@ -255,7 +273,7 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 
   __syncthreads();  // every deferred token is listed
   const int ndef = def_n;
   for (int di = 0; di < ndef; ++di) {  // block-uniform
-    const int tl = def_info[di] & 255, nc = def_info[di] >> 8, t = t0 + tl;
+    const int tl = def_info[di] & 255, nc = (def_info[di] >> 8) & 255, nm = def_info[di] >> 16, t = t0 + tl;
     const size_t xoff = (size_t)t * rf.d;
     auto xval = [&](int j) -> double {
       return rf.x_bf16 ? (double)__bfloat162float(reinterpret_cast<const bf16*>(rf.x)[xoff + j])
@@ -278,15 +296,15 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 
       }
       __syncthreads();
     };
-    // group g sums x . W_comb[e] for candidates 8g..8g+7 (group 0 also sums x^2 for r)
+    // group g sums x . W_comb[e] for members 8g..8g+7 (group 0 also sums x^2 for r)
     double v[9];
-    for (int c0 = 0; c0 < nc; c0 += 8) {
-      const int ng = min(8, nc - c0);
+    for (int c0 = 0; c0 < nm; c0 += 8) {
+      const int ng = min(8, nm - c0);
       const double* wrow[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         v[u] = 0.0;
-        wrow[u] = rf.wc + (size_t)def_e[di][min(c0 + u, nc - 1)] * rf.d;
+        wrow[u] = rf.wc + (size_t)def_e[di][def_mi[di][min(c0 + u, nm - 1)]] * rf.d;
       }
       v[8] = 0.0;
       for (int j = threadIdx.x; j < rf.d; j += blockDim.x) {
@@ -312,13 +330,23 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 
     const double r = 1.0 / sqrt(def_z[40] / rf.d + (double)rf.eps);
     if (warp == 0) {  // rank the candidates and store the choice like any other token's
       const int e_lane = def_e[di][lane];
+      const unsigned lpm = def_lp[di], mm = lpm | (lpm >> 1);
+      const bool member = (mm >> lane) & 1u;
       double my_u = 0.0;
-      if (lane < nc) my_u = 1.0 / (1.0 + exp(-(r * def_z[lane] + (double)rf.cz[e_lane]))) + (double)bias[e_lane];
-      int rk = 0;
+      if (member) {
+        const double z = def_z[__popc(mm & ((1u << lane) - 1u))];
+        my_u = 1.0 / (1.0 + exp(-(r * z + (double)rf.cz[e_lane]))) + (double)bias[e_lane];
+      }
+      // a cluster starts at every candidate not linked to the previous one; a member's rank is
+      // its cluster's first position plus the members of its cluster that precede it exactly
+      const unsigned below = lane == 31 ? kFull : ((2u << lane) - 1u);
+      const int a = 31 - __clz(~lpm & below);
+      int rk = member ? a : lane;
       for (int c = 0; c < nc; ++c) {
         const double uc = __shfl_sync(kFull, my_u, c);
         const int ec = __shfl_sync(kFull, e_lane, c);
-        if (uc > my_u || (uc == my_u && ec < e_lane)) ++rk;
+        const int ac = __shfl_sync(kFull, a, c);
+        if (member && c != lane && ac == a && (uc > my_u || (uc == my_u && ec < e_lane))) ++rk;
       }
       int sel = -1;
       for (int i = 0; i < k; ++i) {
