@@ -142,7 +142,9 @@ cudaError_t launch_tc_pair_t(const TcParams& p, int grid, cudaStream_t st) {
 template <int EPI>
 cudaError_t launch_tc_e(const TcParams& p, int bn, int grid, cudaStream_t st) {
   switch (bn) {
-    case 256: return launch_tc_t<256, EPI>(p, grid, st);
+    case 256:
+      if constexpr (EPI == EPI_ROUTER) return cudaErrorInvalidValue;  // two accumulators: BN <= 128
+      else return launch_tc_t<256, EPI>(p, grid, st);
     case 128: return launch_tc_t<128, EPI>(p, grid, st);
     default:
       if constexpr (EPI == EPI_SWIGLU) return cudaErrorInvalidValue;
@@ -726,22 +728,20 @@ int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, 
       p.row_scale = h->r;
       CK(launch_tc(p, EPI_DOWN3, bn, std::min(mt * p.n_tiles, h->sms), st));
     }
-    // s = sigmoid(h Wr^T + c) from six bf16 x bf16 products of the hi/mid/lo parts
+    // s = sigmoid(h Wr^T + c) from six bf16 x bf16 products of the hi/mid/lo parts, walked chunk
+    // by chunk over the three parts (the engine's split-router mode; tiles at most 128 wide)
     mark(h, ST_ROUTER, st);
     {
       TcParams p = tc_base(h);
       p.tmA[0] = h->tm_hx;
       p.tmA[1] = h->tm_hx;
-      const int bn = pick_bn_for(T, c.E, h->sms, 64);
+      const int bn = std::min(pick_bn_for(T, c.E, h->sms, 64), 128);
       p.tmB = h->tm_wr[bn_index(bn)];
       const int L = c.l, nk = c.l / 64;
-      p.nseg = 6;
-      p.seg[0] = {0, L, L, nk};      // mid * mid
-      p.seg[1] = {0, 2 * L, 0, nk};  // lo * hi
-      p.seg[2] = {0, 0, 2 * L, nk};  // hi * lo
-      p.seg[3] = {0, L, 0, nk};      // mid * hi
-      p.seg[4] = {0, 0, L, nk};      // hi * mid
-      p.seg[5] = {0, 0, 0, nk};      // hi * hi
+      p.nseg = 3;
+      p.seg[0] = {0, 0, 0, nk};          // hi parts
+      p.seg[1] = {0, L, L, nk};          // mid parts
+      p.seg[2] = {0, 2 * L, 2 * L, nk};  // lo parts
       p.M = T;
       p.M_rows = T;
       p.n_tiles = c.E / bn;

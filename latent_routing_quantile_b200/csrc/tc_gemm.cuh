@@ -21,8 +21,15 @@
 // are never stored, depend on them.
 //
 // K is described by up to 6 segments, each naming which A tensor map and which A and B columns
-// its k-blocks read; this expresses concatenated-K products ([z | a_s] [W_up | Ws2]^T) and the
-// split-precision router (hi/mid/lo products) without copying operands.
+// its k-blocks read; this expresses concatenated-K products ([z | a_s] [W_up | Ws2]^T) without
+// copying operands.
+//
+// EPI_ROUTER (the split-precision router, not paired) reads three segments, the hi, mid and lo
+// parts of h and of the router weights, chunk by chunk: the three stages of a 64-column chunk
+// (part q of A and of B in stage q) feed all six significant products, five small ones
+// ((mid,mid) (lo,hi) (hi,lo) (mid,hi) (hi,mid)) into one accumulator and (hi,hi) into a second,
+// so each part is loaded once and the small terms are summed among themselves; the epilogue adds
+// the two.  Its accumulators take 2 BN TMEM columns each (BN <= 128).
 #pragma once
 
 #include "common.cuh"
@@ -120,6 +127,10 @@ template <int BN, int EPI, int PAIR>
 __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_constant__ TcParams p) {
   using C = TcCfg<BN, PAIR>;
   constexpr int S = C::kStages;
+  constexpr bool kSplit3 = EPI == EPI_ROUTER && !PAIR;  // chunk-major split-precision products
+  constexpr int kAccCols = kSplit3 ? 2 * BN : BN;       // TMEM columns of one accumulator buffer
+  constexpr uint32_t kTmemCols = 2 * kAccCols;
+  static_assert(kTmemCols <= 512 && (!kSplit3 || S >= 3), "router tiles are at most 128 wide");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* smem = smem_raw + pad;
@@ -166,10 +177,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
   }
   if (warp == 1) {
     if constexpr (PAIR) {
-      tmem_alloc_pair(tmem_slot, C::kTmemCols);
+      tmem_alloc_pair(tmem_slot, kTmemCols);
       tmem_relinquish_pair();
     } else {
-      tmem_alloc(tmem_slot, C::kTmemCols);
+      tmem_alloc(tmem_slot, kTmemCols);
       tmem_relinquish();
     }
   }
@@ -196,9 +207,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       for (int tile = first; ok && tile < num_tiles; tile += stride) {
         const TileInfo ti = ti_next;
         if (tile + stride < num_tiles) ti_next = tc_tile(p, tile + stride, BN, PAIR, rank);
-        for (int s = 0; ok && s < p.nseg; ++s) {
-          const KSeg sg = p.seg[s];
-          for (int kb = 0; kb < sg.nkb; ++kb) {
+        // k-blocks segment by segment, or (split router) chunk by chunk over the three segments
+        const int nouter = kSplit3 ? p.seg[0].nkb : p.nseg;
+        for (int o = 0; ok && o < nouter; ++o) {
+          const int ninner = kSplit3 ? 3 : p.seg[o].nkb;
+          for (int in = 0; in < ninner; ++in) {
+            const KSeg sg = p.seg[kSplit3 ? in : o];
+            const int kb = kSplit3 ? o : in;
             if (!mbar_wait(&empty[stage], phase ^ 1u, abort, p.status)) {
               ok = false;
               break;
@@ -255,7 +270,50 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * BN;
+        const uint32_t d_tmem = tmem_base + acc * kAccCols;
+        if constexpr (kSplit3) {
+          // per chunk: stage q holds part q (hi, mid, lo) of A and of B; small products into the
+          // accumulator's first BN columns, smallest first, (hi, hi) into the second BN
+          constexpr uint32_t kPa = 1u | (2u << 2) | (0u << 4) | (1u << 6) | (0u << 8);
+          constexpr uint32_t kPb = 1u | (0u << 2) | (2u << 4) | (0u << 6) | (1u << 8);
+          const int nch = p.seg[0].nkb;
+          for (int kk = 0; ok && kk < nch; ++kk) {
+            uint32_t a_addr[3], b_addr[3];
+            int st3[3];
+#pragma unroll
+            for (int q = 0; q < 3; ++q) {
+              if (!mbar_wait(&full[stage], phase, abort, p.status)) {
+                ok = false;
+                break;
+              }
+              a_addr[q] = smem_u32(smem + stage * C::kStageBytes);
+              b_addr[q] = a_addr[q] + C::kABytes;
+              st3[q] = stage;
+              if (++stage == S) {
+                stage = 0;
+                phase ^= 1u;
+              }
+            }
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int pr = 0; pr < 5; ++pr) {
+              const int pa = (int)((kPa >> (2 * pr)) & 3u), pb = (int)((kPb >> (2 * pr)) & 3u);
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                tc_mma_bf16(d_tmem, smem_desc_sw128(a_addr[pa] + k * 32), smem_desc_sw128(b_addr[pb] + k * 32), idesc,
+                            (kk | pr | k) != 0);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              tc_mma_bf16(d_tmem + BN, smem_desc_sw128(a_addr[0] + k * 32), smem_desc_sw128(b_addr[0] + k * 32), idesc,
+                          (kk | k) != 0);
+#pragma unroll
+            for (int q = 0; q < 3; ++q) tc_commit(&empty[st3[q]]);
+          }
+          if (ok) tc_commit(&tfull[acc]);
+          continue;
+        }
         int kbi = 0;
         for (int s = 0; ok && s < p.nseg; ++s) {
           const int nkb = p.seg[s].nkb;
@@ -371,7 +429,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       }
       tc_fence_after();
       omap = ti.q < 4 ? &p.tmOut_part[ti.q - 1] : &p.tmOut;
-      const uint32_t tbase = tmem_base + ((uint32_t)(wq * 32) << 16) + acc * BN;
+      const uint32_t tbase = tmem_base + ((uint32_t)(wq * 32) << 16) + acc * kAccCols;
       uint32_t w[16];
 
       if constexpr (EPI == EPI_SWIGLU) {
@@ -430,13 +488,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         bool nan = false;
 #pragma unroll 1
         for (int j = 0; ok && j < BN / 32; ++j) {
-          uint32_t v[16];
-          tmem_ld16(tbase + j * 32 + half_id * 16, v);
+          uint32_t v[16], vs[16];
+          if constexpr (kSplit3) {
+            tmem_ld16(tbase + BN + j * 32 + half_id * 16, v);  // (hi, hi)
+            tmem_ld16(tbase + j * 32 + half_id * 16, vs);      // the five small products
+          } else {
+            tmem_ld16(tbase + j * 32 + half_id * 16, v);
+          }
           float cj = c_lane[0];
 #pragma unroll
           for (int jj = 1; jj < BN / 32; ++jj)
             if (jj == j) cj = c_lane[jj];
           tc_wait_ld();
+          if constexpr (kSplit3) {
+#pragma unroll
+            for (int q = 0; q < 16; ++q) v[q] = __float_as_uint(__uint_as_float(v[q]) + __uint_as_float(vs[q]));
+          }
           if constexpr (EPI == EPI_ROUTER) {
 #pragma unroll
             for (int q = 0; q < 16; ++q) {
@@ -470,9 +537,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
   if (warp == 1) {
     tc_fence_after();
     if constexpr (PAIR)
-      tmem_dealloc_pair(tmem_base, C::kTmemCols);
+      tmem_dealloc_pair(tmem_base, kTmemCols);
     else
-      tmem_dealloc(tmem_base, C::kTmemCols);
+      tmem_dealloc(tmem_base, kTmemCols);
   }
   if constexpr (PAIR) cluster_sync_all();
 }
