@@ -44,10 +44,11 @@ __global__ void __launch_bounds__(256) rms_kernel(const T* __restrict__ x, int n
 // Order-preserving map of a float to uint32 (larger float -> larger key); 0 is kept free to mark
 // taken or absent experts and 1 for a NaN score, which ranks below every number.
 __device__ __forceinline__ uint32_t order_key(float f) {
-  if (f != f) return 1u;
-  if (f == 0.f) f = 0.f;  // -0 and +0 compare equal, so give them one key
-  const uint32_t b = __float_as_uint(f);
-  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+  // -0 + 0 = +0 under round-to-nearest (every other value is unchanged), so -0 and +0, which
+  // compare equal, get one key; negative numbers have all bits flipped, the others the sign bit
+  const uint32_t b = __float_as_uint(__fadd_rn(f, 0.0f));
+  const uint32_t key = b ^ ((uint32_t)((int32_t)b >> 31) | 0x80000000u);
+  return f != f ? 1u : key;
 }
 // Inverse of order_key for keys of numbers (>= 2).
 __device__ __forceinline__ float key_value(uint32_t key) {
@@ -184,9 +185,9 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 
         if (e < E) {
           nan |= (v != v);
           key[j] = order_key(v + bj[j]);
-          if (bins)
-            sbins[tl * bpitch + e] =
-                (uint16_t)(v >= 0.f ? min((int)(v * (float)LMOE_NBINS), LMOE_NBINS - 1) : 0);
+          // bin min(floor(s * 4096), 4095); the unsigned conversion takes negative scores and NaN
+          // to 0 and saturates large ones
+          if (bins) sbins[tl * bpitch + e] = (uint16_t)min(__float2uint_rz(v * (float)LMOE_NBINS), LMOE_NBINS - 1u);
         } else {
           key[j] = 0u;
         }
@@ -215,9 +216,10 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 
           if (wmax < 2u || !(key_value(wmax) >= u_k1 - rf.tau)) break;
         }
         const uint32_t emin = __reduce_min_sync(kFull, bk == wmax ? (uint32_t)(bjx * 32 + lane) : 0xffffffffu);
+        const uint32_t dj = emin - (uint32_t)lane;  // j * 32 in the lane that holds the choice
 #pragma unroll
         for (int j = 0; j < NJ; ++j)
-          if ((uint32_t)(j * 32 + lane) == emin) key[j] = 0u;
+          if (dj == (uint32_t)(j * 32)) key[j] = 0u;
         if (lane == i) my_sel = (int)emin;
         if (rf.x) {
           const float ui = wmax >= 2u ? key_value(wmax) : 0.f;
@@ -622,7 +624,12 @@ __global__ void __launch_bounds__(256, (G <= 6 && sizeof(T) == 2) ? 4 : 3) combi
   // lane i < k holds slot i's gate and row
   const float g_l = lane < k ? gates[(size_t)t * k + lane] : 0.f;
   const int r_l = lane < k ? prow[(size_t)t * k + lane] : 0;
-  for (int v = lane; v < l / VEC; v += 32) {
+  // every lane runs every trip (a row narrower than 32 vectors leaves some lanes idle), so the
+  // shuffles that hand out slot i's gate and row always see the lane that holds them
+  const int nvec = l / VEC;
+  for (int v0 = 0; v0 < nvec; v0 += 32) {
+    const int v = v0 + lane;
+    const bool act = v < nvec;
     float acc[VEC];
 #pragma unroll
     for (int j = 0; j < VEC; ++j) acc[j] = 0.f;
@@ -634,7 +641,7 @@ __global__ void __launch_bounds__(256, (G <= 6 && sizeof(T) == 2) ? 4 : 3) combi
         const int i = i0 + u;
         const int row = __shfl_sync(kFull, r_l, i & 31);
         g[u] = __shfl_sync(kFull, g_l, i & 31);
-        if (i < k) q[u] = reinterpret_cast<const uint4*>(o + (size_t)row * l)[v];
+        if (act && i < k) q[u] = reinterpret_cast<const uint4*>(o + (size_t)row * l)[v];
       }
 #pragma unroll
       for (int u = 0; u < G; ++u) {
@@ -644,6 +651,7 @@ __global__ void __launch_bounds__(256, (G <= 6 && sizeof(T) == 2) ? 4 : 3) combi
         for (int j = 0; j < VEC; ++j) acc[j] = fmaf(g[u], to_f<T>(e[j]), acc[j]);
       }
     }
+    if (!act) continue;
     uint4 out;
     T* oe = reinterpret_cast<T*>(&out);
 #pragma unroll

@@ -611,3 +611,26 @@ def test_host_forward_async_output_matches_device_forward():
     torch.cuda.synchronize()
     assert torch.equal(yh[0], want[0])
     layer.close()
+
+
+@pytest.mark.parametrize("name,T,d,l,E,k,h,hs,dtype", [
+    ("one_token", 1, 256, 128, 64, 4, 128, 256, "bf16"),        # a single token: one ragged tile
+    ("top1", 300, 256, 128, 64, 1, 128, 256, "bf16"),           # k = 1: every gate is exactly 1
+    ("no_shared", 333, 256, 128, 64, 6, 128, 0, "bf16"),        # hs = 0: no shared expert
+    ("all_experts", 200, 256, 64, 32, 32, 64, 0, "f32"),        # E = k: every expert, gates s / sum s
+])
+def test_degenerate_layers_match_oracle(name, T, d, l, E, k, h, hs, dtype):
+    """The method's degenerate cases through the whole CUDA forward against the oracle: one
+    token, top-1 routing, no shared expert, and every expert chosen."""
+    shape = datagen.LayerShape(name, T, d, l, E, k, h, hs, dtype, seed=51, offset_var=0.5)
+    w = datagen.layer_weights(shape)
+    x = datagen.tokens(shape)
+    layer, y, ro, stats = run_layer_check(shape, w, x)
+    r = layer.routing()
+    gates = r["gates"].cpu().numpy().astype(np.float64)
+    if k == 1:
+        assert np.all(gates == 1.0)
+    if E == k:
+        assert np.array_equal(np.sort(r["idx"].cpu().numpy(), 1), np.tile(np.arange(E), (T, 1)))
+    np.testing.assert_allclose(gates.sum(1), 1.0, rtol=0, atol=1e-5 * k)
+    layer.close()
