@@ -467,9 +467,9 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ coun
   const int e = blockIdx.x * 32 + tx;
   const int chunk = (nblk + 31) / 32;
   const int b0 = ty * chunk, b1 = min(nblk, b0 + chunk);
-  // the chunk's counts are loaded in batches of 8 independent loads (one latency per batch);
-  // chunks of up to 8 blocks keep them in registers for the second pass
-  constexpr int kBatch = 8;
+  // the chunk's counts are loaded in batches of 16 independent loads (one latency per batch);
+  // chunks of up to 16 blocks keep them in registers for the second pass
+  constexpr int kBatch = 16;
   int keep[kBatch];
   int sum = 0;
   if (e < E)
