@@ -46,11 +46,20 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def csrc_digest() -> str:
+# the sources that define and launch each kernel whose DRAM traffic profiles/traffic.json records:
+# a recorded figure counts only while these files are the ones it was measured on
+TRAFFIC_SOURCES = {
+    "shared_swiglu": ("common.cuh", "tc_gemm.cuh", "lmoe.cu"),
+    "norm_down_router": ("common.cuh", "k1_router.cuh", "lmoe.cu"),
+}
+
+
+def csrc_digest(files=None) -> str:
+    """sha256 (16 hex digits) of the named CUDA sources, or of all of them."""
     d = os.path.join(ROOT, "latent_routing_quantile_b200", "csrc")
     h = hashlib.sha256()
     for f in sorted(os.listdir(d)):
-        if f.endswith((".cu", ".cuh")):
+        if f.endswith((".cu", ".cuh")) and (files is None or f in files):
             h.update(open(os.path.join(d, f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -283,7 +292,8 @@ def run_ours(args, rank, world, local_rank):
     if os.path.exists(tpath):
         tj = json.load(open(tpath))
         ent = tj.get("kernels", {}).get(dom)
-        if ent and tj.get("csrc_digest") == csrc_digest() and tj.get("workload") == shape.name:
+        if (ent and dom in TRAFFIC_SOURCES and ent.get("src_digest") == csrc_digest(TRAFFIC_SOURCES[dom])
+                and tj.get("workload") == shape.name):
             traffic = ent["dram_bytes_per_launch"]
     if kd["bound"] == "tensor":
         roof = {"bound": "tensor", "achieved": kd["tflops"], "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}

@@ -46,9 +46,10 @@ __global__ void __launch_bounds__(256) rms_kernel(const T* __restrict__ x, int n
 __device__ __forceinline__ uint32_t order_key(float f) {
   // -0 + 0 = +0 under round-to-nearest (every other value is unchanged), so -0 and +0, which
   // compare equal, get one key; negative numbers have all bits flipped, the others the sign bit
-  const uint32_t b = __float_as_uint(__fadd_rn(f, 0.0f));
-  const uint32_t key = b ^ ((uint32_t)((int32_t)b >> 31) | 0x80000000u);
-  return f != f ? 1u : key;
+  if (f != f) return 1u;
+  if (f == 0.f) f = 0.f;
+  const uint32_t b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 // Inverse of order_key for keys of numbers (>= 2).
 __device__ __forceinline__ float key_value(uint32_t key) {
@@ -187,7 +188,9 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 
           key[j] = order_key(v + bj[j]);
           // bin min(floor(s * 4096), 4095); the unsigned conversion takes negative scores and NaN
           // to 0 and saturates large ones
-          if (bins) sbins[tl * bpitch + e] = (uint16_t)min(__float2uint_rz(v * (float)LMOE_NBINS), LMOE_NBINS - 1u);
+          if (bins)
+            sbins[tl * bpitch + e] =
+                (uint16_t)(v >= 0.f ? min((int)(v * (float)LMOE_NBINS), LMOE_NBINS - 1) : 0);
         } else {
           key[j] = 0u;
         }
@@ -216,10 +219,9 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 
           if (wmax < 2u || !(key_value(wmax) >= u_k1 - rf.tau)) break;
         }
         const uint32_t emin = __reduce_min_sync(kFull, bk == wmax ? (uint32_t)(bjx * 32 + lane) : 0xffffffffu);
-        const uint32_t dj = emin - (uint32_t)lane;  // j * 32 in the lane that holds the choice
 #pragma unroll
         for (int j = 0; j < NJ; ++j)
-          if (dj == (uint32_t)(j * 32)) key[j] = 0u;
+          if ((uint32_t)(j * 32 + lane) == emin) key[j] = 0u;
         if (lane == i) my_sel = (int)emin;
         if (rf.x) {
           const float ui = wmax >= 2u ? key_value(wmax) : 0.f;
@@ -469,7 +471,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ coun
   const int b0 = ty * chunk, b1 = min(nblk, b0 + chunk);
   // the chunk's counts are loaded in batches of 16 independent loads (one latency per batch);
   // chunks of up to 16 blocks keep them in registers for the second pass
-  constexpr int kBatch = 16;
+  constexpr int kBatch = 8;
   int keep[kBatch];
   int sum = 0;
   if (e < E)
