@@ -136,8 +136,10 @@ int lmoe_forward(lmoe_handle *h, const void *x_dev, void *y_dev, int32_t T, uint
  * staging buffers (ordered by events: it waits for the forward that last read that buffer, and
  * the forward waits for it), so one call's input copy overlaps the previous call's forward.
  * y_host is valid, and x_host may change, after `stream` synchronises.  Under stream capture of
- * `stream` everything stays on `stream` (LMOE_EINVAL while an LMOE_ASYNC_OUTPUT copy is
- * outstanding: call lmoe_host_wait and synchronise first).
+ * `stream` everything stays on `stream`; that form is LMOE_EINVAL while the handle still counts
+ * an LMOE_ASYNC_OUTPUT copy as outstanding, which lasts until a later uncaptured host-buffer
+ * forward into the same staging buffer (the two buffers alternate, so the second call after it)
+ * has been ordered after that copy.
  * With LMOE_ASYNC_OUTPUT the forward writes one of two handle-owned output buffers and the copy
  * to y_host runs on a second handle-owned copy stream once the forward is done; `stream` does not
  * wait for it, so a serving loop overlaps the output copy of call i with the input copy and
