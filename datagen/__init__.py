@@ -10,8 +10,8 @@ weights or one 1024-row chunk of tokens can be regenerated on its own: the
 oracle recomputes a token subset of the 16384-token, 896-expert workload
 without holding every expert in fp64.
 
-Distributions follow the workload table of the pages' layer (SURVEY: the
-five workloads): tokens x ~ N(0, 1); every weight ~ N(0, 1/fan_in) where
+Distributions follow the layer's five synthetic workloads (the pages give
+only 896-choose-16 and top-6 routing): tokens x ~ N(0, 1); every weight ~ N(0, 1/fan_in) where
 fan_in is the input width of that projection; RMSNorm gain 1; router column
 offsets c_e ~ N(0, 0.5) (variance 0.5) where the workload says so.
 """
