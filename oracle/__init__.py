@@ -33,7 +33,7 @@ contract this library implements fixes them: RMSNorm with eps 1e-6, a sigmoid
 router in fp32, SwiGLU as a marked stand-in for SiTU-GLU, a 4096-bin
 histogram over [0, 1] for the QB quantile.
 
-Readings where the pages are silent (each also listed in the design notes):
+Readings where the pages are silent:
   * QB quantile is the type-1 (inverse empirical CDF) quantile at rank
     m = ceil((E - k) * N / E), computed in exact integer arithmetic.
   * Bin rule min(floor(s * 4096), 4095) on the fp32 score (the layer keeps s in

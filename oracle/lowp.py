@@ -8,7 +8,7 @@ The pages say only that the K3 model runs its experts with 4-bit weights and 8-b
 ("Kimi K3登顶开源第一，靠的是把浪费逼到墙角", the QAT paragraph) and that the replica's FP8 attempt
 lost on H200 (the wink.run summary of "Pretraining a Mini Kimi K3": 0.19x).  They fix no format,
 block size or scale rule.  Readings taken (the plainest that block-scaled tensor-core operands
-support; each is listed in the design notes):
+support):
   * Elements are E4M3: 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits, no infinities,
     largest finite magnitude 448 (exponent field 15, mantissa 110), subnormals down to 2^-9.
     A value is rounded to the nearest element, ties to the even mantissa, and magnitudes beyond
