@@ -68,3 +68,19 @@ def test_product_path_never_imports_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 src = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in src and "from oracle" not in src, f
+
+
+def test_binding_constants_match_the_header():
+    """Every flag, mode and status bit the binding passes or reads has the header's value."""
+    text = open(os.path.join(ROOT, "include", "lmoe.h")).read()
+    defs = {m.group(1): int(m.group(2), 0)
+            for m in re.finditer(r"#define\s+LMOE_([A-Z0-9_]+)\s+\(?(-?(?:0x)?[0-9a-fA-F]+)u?\)?", text)}
+    pairs = {"F32": lq.F32, "BF16": lq.BF16, "RECORD_STATS": lq.RECORD_STATS, "UPDATE_BIAS": lq.UPDATE_BIAS,
+             "ASYNC_OUTPUT": lq.ASYNC_OUTPUT, "QB_LITERAL": lq.QB_LITERAL, "BIAS_SIGN": lq.BIAS_SIGN,
+             "STATUS_NAN_SCORE": lq.STATUS_NAN_SCORE, "STATUS_WATCHDOG": lq.STATUS_WATCHDOG,
+             "STATUS_BAD_INDEX": lq.STATUS_BAD_INDEX, "NBINS": lq.NBINS}
+    for name, value in pairs.items():
+        assert defs.get(name) == value, (name, defs.get(name), value)
+    # the forward flags are distinct bits, and the update's rule flags stay out of their way
+    fwd = [defs["RECORD_STATS"], defs["UPDATE_BIAS"], defs["ASYNC_OUTPUT"]]
+    assert len(set(fwd)) == 3 and all(f & (f - 1) == 0 for f in fwd)
