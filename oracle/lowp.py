@@ -103,5 +103,27 @@ def e4m3_half_step(v) -> np.ndarray:
     return step / 2
 
 
+
+
+def routed_outputs_mxfp8(h, idx, w1, w3, w2, block: int = MX_BLOCK) -> np.ndarray:
+    """o[t, i] = SwiGLU_{idx[t,i]}(h[t]) with every GEMM operand in MXFP8, for each chosen pair.
+
+    The same expert FFN as the forward oracle's routed_outputs (SwiGLU, the stand-in for SiTU-GLU),
+    with 8-bit operands: the expert's rows of h and its W1, W3 are quantised along l (their K),
+    act = silu(p1) * p3 and W2 along h; each product is the float64 product of the dequantised
+    operands, and silu and the elementwise product are float64 as well."""
+    h = np.asarray(h, dtype=np.float64)
+    T, k = idx.shape
+    o = np.zeros((T, k, np.shape(w2)[1]), dtype=np.float64)
+    for e in np.unique(idx):
+        t, i = np.nonzero(idx == e)
+        a = h[t]
+        p1 = mxfp8_matmul(a, np.asarray(w1[e], dtype=np.float64), block)
+        p3 = mxfp8_matmul(a, np.asarray(w3[e], dtype=np.float64), block)
+        act = p1 / (1.0 + np.exp(-p1)) * p3
+        o[t, i] = mxfp8_matmul(act, np.asarray(w2[e], dtype=np.float64), block)
+    return o
+
+
 __all__ = ["E4M3_MAX", "MX_BLOCK", "e4m3_decode", "round_e4m3", "mx_scale_exponent", "mxfp8_quantize",
-           "mxfp8_dequantize", "mxfp8_matmul", "e4m3_half_step"]
+           "mxfp8_dequantize", "mxfp8_matmul", "e4m3_half_step", "routed_outputs_mxfp8"]

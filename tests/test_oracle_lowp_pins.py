@@ -130,3 +130,46 @@ def test_a_lowp_pin_catches_the_mutant(name, monkeypatch):
     target, mutant, pin_list = LOWP_MUTANTS[name]
     monkeypatch.setattr(lp, target, mutant)
     assert any(_fails(p) for p in pin_list), f"no pin caught mutant {name}"
+
+
+def _expert_problem(seed=75):
+    rng = np.random.default_rng(seed)
+    T, l, h, E, k = 40, 64, 96, 5, 2
+    hid = rng.standard_normal((T, l))
+    w1, w3 = rng.standard_normal((E, h, l)) / 8, rng.standard_normal((E, h, l)) / 8
+    w2 = rng.standard_normal((E, l, h)) / 10
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)])
+    return hid, idx, w1, w3, w2
+
+
+def test_mxfp8_experts_are_exact_under_power_of_two_scaling_of_w2():
+    """A power-of-two factor on W2 moves every block scale by the same power and no element:
+    the 8-bit expert output scales by exactly that factor."""
+    hid, idx, w1, w3, w2 = _expert_problem()
+    o = lp.routed_outputs_mxfp8(hid, idx, w1, w3, w2)
+    for j in (-5, 3):
+        assert np.array_equal(lp.routed_outputs_mxfp8(hid, idx, w1, w3, np.ldexp(w2, j)), np.ldexp(o, j))
+
+
+def test_mxfp8_experts_ignore_the_order_of_k_blocks():
+    """Quantisation acts on 32-element blocks along K only: permuting whole blocks of l in h, W1
+    and W3 together (and of h in W1, W3 rows and W2 columns together) changes no output beyond
+    the float64 summation order."""
+    hid, idx, w1, w3, w2 = _expert_problem()
+    o = lp.routed_outputs_mxfp8(hid, idx, w1, w3, w2)
+    pl = np.concatenate([np.arange(32, 64), np.arange(0, 32)])            # swap the two blocks of l
+    ph = np.concatenate([np.arange(64, 96), np.arange(0, 32), np.arange(32, 64)])  # rotate h's blocks
+    o2 = lp.routed_outputs_mxfp8(hid[:, pl], idx, w1[:, ph][:, :, pl], w3[:, ph][:, :, pl], w2[:, :, ph])
+    np.testing.assert_allclose(o2, o, rtol=1e-12, atol=1e-12)
+
+
+def test_mxfp8_experts_stay_near_the_full_precision_experts():
+    """A check of the wiring against the forward oracle's float64 experts: each 8-bit operand is
+    within 1/8 of its value (the element pins above), so the outputs stay within 10% of the output
+    scale, while a lost block scale or a misplaced operand moves them by orders of magnitude."""
+    import oracle
+    hid, idx, w1, w3, w2 = _expert_problem()
+    o8 = lp.routed_outputs_mxfp8(hid, idx, w1, w3, w2)
+    o = oracle.routed_outputs(hid, idx, w1, w3, w2)
+    rel = np.max(np.abs(o8 - o)) / np.max(np.abs(o))
+    assert 0 < rel < 0.1, rel
