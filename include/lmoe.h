@@ -114,8 +114,8 @@ typedef struct {
 
 /* Validates cfg, repacks the weights (gain folded into W_down and the shared expert, gate and
  * linear projections interleaved, [W_up | Ws2] concatenated along K), allocates the workspace
- * for max_tokens and sets b = 0 and an empty histogram.  On error *out is NULL and nothing is
- * leaked. */
+ * for max_tokens and sets b = 0 and an empty histogram.  On error *out is NULL and the device
+ * memory it allocated is released. */
 int lmoe_create(const lmoe_config *cfg, const lmoe_weights *w, void *stream, lmoe_handle **out);
 
 /* Releases every device allocation of the handle (synchronises the device first). */
