@@ -412,3 +412,28 @@ def test_qb_skewed_router_converges_like_the_demo():
     assert ratios[0] >= 3.5
     assert min(ratios[-5:]) <= pages["max_min_load_ratio_after_qb"] * 1.1
     assert max(ratios[-5:]) < ratios[0] / 2.5
+
+
+def test_topk_margins_by_repeated_maximum():
+    """The near-tie margins the parity checks lean on: u_(k) - u_(k+1) and the smallest gap among
+    the top k+1, found here by taking the maximum k+1 times (no sort)."""
+    rng = np.random.default_rng(91)
+    for trial in range(40):
+        E = int(rng.integers(2, 12))
+        k = int(rng.integers(1, E + 1))
+        s = rng.uniform(0, 1, (5, E))
+        if trial % 4 == 0:
+            s = np.round(s * 8) / 8  # exact ties
+        b = rng.normal(0, 0.1, E)
+        gap, ogap = oracle.topk_gap(s, b, k), oracle.topk_order_gap(s, b, k)
+        for t in range(5):
+            u = list(s[t] + b)
+            tops = []
+            for _ in range(min(k + 1, E)):
+                m = max(u)
+                tops.append(m)
+                u.remove(m)
+            want_gap = tops[k - 1] - tops[k] if k < E else np.inf
+            diffs = [tops[i] - tops[i + 1] for i in range(len(tops) - 1)]
+            want_ogap = min(diffs) if diffs else np.inf
+            assert gap[t] == want_gap and ogap[t] == want_ogap
