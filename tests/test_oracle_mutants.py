@@ -70,9 +70,26 @@ MUTANTS = {
                          lambda b, load, gamma: oracle.f64(b) + gamma * np.sign(np.max(load) - np.asarray(load)),
                          [pins.test_sign_rule_worked_example,
                           lambda: pins.test_sign_rule_sign_against_exact_rational_mean(0)]),
+    # routing oracle: RMSNorm gain dropped
+    "routing_no_gain": ("layer_routing",
+                        lambda x, w, b, k, eps=1e-6: _LR(x, {**w, "rms_gain": np.ones(len(w["rms_gain"]))}, b, k, eps),
+                        [pins.test_layer_routing_worked_example_closed_forms,
+                         pins.test_layer_routing_equals_the_forward_routing]),
+    # routing oracle: router column offsets dropped
+    "routing_no_offsets": ("layer_routing",
+                           lambda x, w, b, k, eps=1e-6:
+                           _LR(x, {**w, "router_bias": np.zeros(len(w["router_bias"]))}, b, k, eps),
+                           [pins.test_layer_routing_worked_example_closed_forms,
+                            pins.test_layer_routing_equals_the_forward_routing]),
+    # routing oracle: the bias ignored in the choice
+    "routing_no_bias": ("layer_routing",
+                        lambda x, w, b, k, eps=1e-6: _LR(x, w, np.zeros_like(oracle.f64(b)), k, eps),
+                        [pins.test_layer_routing_worked_example_closed_forms,
+                         pins.test_layer_routing_equals_the_forward_routing]),
 }
 
 _SR = oracle.sign_rule_update
+_LR = oracle.layer_routing
 _QB = oracle.qb_update
 _HQ = oracle.histogram_quantile
 

@@ -81,6 +81,31 @@ def test_worked_example_closed_forms():
     np.testing.assert_allclose(out["y"], y_exp, rtol=1e-13)
 
 
+def test_layer_routing_worked_example_closed_forms():
+    """The routing half on its own (the routing oracle of every GPU layer test) takes the worked
+    example's closed forms: the gain 2 on column 1 sets h0[1] = 1/2 and the router column offsets
+    set s, so dropping either changes h, s and the choice."""
+    x, w, b = worked_example()
+    r = oracle.layer_routing(x, w, b, k=2, eps=0.0)
+    np.testing.assert_allclose(r["h"], [[1, 0.5], [1, -0.5]], rtol=1e-15)
+    np.testing.assert_allclose(r["s"], [[0.75, 0.75, 0.5, 0.8], [0.75, 0.25, 0.5, 0.8]], rtol=1e-14)
+    assert r["idx"].tolist() == [[0, 1], [0, 3]]
+    np.testing.assert_allclose(r["gates"], [[0.5, 0.5], [15 / 31, 16 / 31]], rtol=1e-14)
+    np.testing.assert_allclose(r["gap"], [0.2, 0.05], rtol=1e-12)
+    np.testing.assert_allclose(r["order_gap"], [0.0, 0.05], atol=1e-15)
+
+
+def test_layer_routing_equals_the_forward_routing():
+    """On a layer with a random gain, router offsets and a non-zero bias, the routing oracle's
+    h, s, choice, gates and margins are those of the whole forward, bit for bit."""
+    shape, w, x = small_layer()
+    b = datagen.normal_bias(shape.E, seed=13, std=0.1).astype(np.float64)
+    full = oracle.layer_forward(x, w, b, shape.k, shape.rms_eps)
+    r = oracle.layer_routing(x, w, b, shape.k, shape.rms_eps)
+    for name in ("h", "s", "idx", "gates", "gap", "order_gap"):
+        assert np.array_equal(r[name], full[name]), name
+
+
 # ---------------------------------------------------------------------------
 # Library routines.
 # ---------------------------------------------------------------------------
