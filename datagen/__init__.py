@@ -19,6 +19,8 @@ from __future__ import annotations
 
 import dataclasses
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass
 
 import numpy as np
@@ -102,9 +104,20 @@ def _matrix(seed, name, rows, cols, fan_in, dtype, sub=0):
 
 
 def _experts(seed, name, E, rows, cols, fan_in, dtype):
+    """Expert e's matrix comes from its own stream (sub-index e), so the experts are drawn on
+    several host threads (numpy and torch release the GIL) with the same values as one by one."""
     out = torch.empty((E, rows, cols), dtype=dtype)
-    for e in range(E):
+
+    def fill(e):
         out[e] = _matrix(seed, name, rows, cols, fan_in, dtype, sub=e)
+
+    workers = min(16, os.cpu_count() or 1, E)
+    if workers <= 1 or E * rows * cols < (1 << 22):
+        for e in range(E):
+            fill(e)
+    else:
+        with ThreadPoolExecutor(workers) as ex:
+            list(ex.map(fill, range(E)))
     return out
 
 

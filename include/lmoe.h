@@ -219,19 +219,24 @@ const char *lmoe_stage_name(int32_t i);
 /* Number of kernels the handle has launched since it was created. */
 int lmoe_launch_count(lmoe_handle *h, int64_t *n);
 
-/* Routing stage for callers that cannot allocate device memory: code running while a stream is
- * being captured into a CUDA graph (cudaMalloc is not allowed there and synchronises the device
- * otherwise), plug-ins whose host owns every byte of device memory, or real-time loops that must
- * not enter the allocator.  It needs no handle and calls no cudaMalloc, cudaFree or allocating
- * library routine.  The pages have no counterpart of this entry point.
+/* Routing stage for callers that cannot allocate device memory: plug-ins whose host application
+ * owns every byte of device memory and hands out only fixed buffers, code that runs inside another
+ * memory manager (a caching allocator or a memory pool, which must not call back into itself), and
+ * real-time loops that must not enter the driver's allocator, which can synchronise the device.
+ * It needs no handle and calls no cudaMalloc, cudaFree or allocating library routine.  The pages
+ * have no counterpart of this entry point.
  *
  * Computes, on scores_dev [T,E] fp32 and bias_dev [E] fp32 (device, caller-owned), the same
  * routing as lmoe_route_scores: idx [T,k] int32 (rank order), gates [T,k] fp32, counts [E] int32,
  * offsets [E+1] int32, perm [T*k] int32 (permuted row -> token), inv [T*k] int32, all device
- * buffers the caller owns.  1 <= k <= min(E, 32), E <= 1024.
+ * buffers the caller owns.  status_dev is a caller-owned device word: the call clears it, then
+ * its kernels OR in LMOE_STATUS_NAN_SCORE (a NaN score, never selected) and LMOE_STATUS_BAD_INDEX
+ * (an expert index or permuted row out of range); read it after the stream synchronises.
+ * 1 <= k <= E (else LMOE_EINVAL); E <= 1024 and k <= 32 (else LMOE_EUNSUPPORTED, as lmoe_create).
  * Scratch: a static device array of LMOE_NOALLOC_SCRATCH_BYTES in the library image, which needs
  *   4*T*k + 8*ceil(T/32)*E + 8*(ceil(T*k/128) + E) + 132*E bytes (each part rounded up to 256) + 256;
- *   larger sizes return LMOE_EUNSUPPORTED (about T = 65536 at E = 256, k = 6).
+ *   larger sizes return LMOE_EUNSUPPORTED.  The largest T is 94,496 at E = 256, k = 6 and 28,576 at
+ *   E = 896, k = 16.
  * The first call on each device takes the array's device address (cudaGetSymbolAddress); make
  * that first call before any stream capture.  All calls share the one array, which keeps the
  * last call's contents: calls whose work overlaps on the GPU (other streams, other threads)
@@ -239,7 +244,7 @@ int lmoe_launch_count(lmoe_handle *h, int64_t *n);
 #define LMOE_NOALLOC_SCRATCH_BYTES (8u << 20)
 int lmoe_route_noalloc(const float *scores_dev, const float *bias_dev, int32_t T, int32_t E, int32_t k,
                        int32_t *idx, float *gates, int32_t *counts, int32_t *offsets, int32_t *perm,
-                       int32_t *inv, void *stream);
+                       int32_t *inv, uint32_t *status_dev, void *stream);
 
 /* Failure-detection check of the bounded waits: one thread waits on an mbarrier that nothing ever
  * completes, with the same wait loop every pipeline kernel uses but a limit of limit_us

@@ -82,7 +82,7 @@ def lib() -> ctypes.CDLL:
             "lmoe_profile_enable": [vp, i32],
             "lmoe_profile_read": [vp, POINTER(c_float), i32, POINTER(i32)],
             "lmoe_launch_count": [vp, POINTER(ctypes.c_int64)],
-            "lmoe_route_noalloc": [vp, vp, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp],
+            "lmoe_route_noalloc": [vp, vp, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp],
             "lmoe_watchdog_selftest": [vp, i32, vp],
         }
         for name, args in sig.items():
@@ -325,23 +325,42 @@ def sum_qb_statistics(hist, ntok, load=None, group=None):
     return hist, ntok, load
 
 
+def dp_qb_update(layer, beta, literal=False, sign_rule=False, group=None, stream=None):
+    """The data-parallel bias update, on every rank of `group`: read this rank's statistics
+    recorded since the last update (histogram, token count and, for the sign rule, expert loads),
+    sum them over the ranks with sum_qb_statistics, set the sums back, and run the update.  Every
+    rank then applies the update one device would apply after seeing every rank's tokens, and all
+    ranks keep the same bias ("Pretraining a Mini Kimi K3", capsule 27, Bug 2: the all-reduce
+    comes before the update)."""
+    hist, n = layer.hist(stream)
+    load = layer.load(stream) if sign_rule else None
+    sum_qb_statistics(hist, n, load, group)
+    layer.set_hist(hist, n, stream)
+    if load is not None:
+        layer.set_load(load, stream)
+    layer.qb_update(beta, literal=literal, sign_rule=sign_rule, stream=stream)
+
+
 def route_noalloc(scores, bias, k, out=None, stream=None):
     """Routing of fp32 scores [T, E] with bias [E] through lmoe_route_noalloc, which allocates no
     device memory (its scratch is a static array in the library).  `out` may pass preallocated
-    buffers (idx, gates, counts, offsets, perm, inv); missing ones are allocated here by torch."""
+    buffers (idx, gates, counts, offsets, perm, inv, status); missing ones are allocated here by
+    torch.  out["status"] (one int32 word) holds the call's fault bits once the stream syncs."""
     T, E = scores.shape
     _dev(scores, torch.float32, (T, E), "scores")
     _dev(bias, torch.float32, (E,), "bias")
     dev = scores.device
     shapes = dict(idx=((T, k), torch.int32), gates=((T, k), torch.float32), counts=((E,), torch.int32),
-                  offsets=((E + 1,), torch.int32), perm=((T * k,), torch.int32), inv=((T * k,), torch.int32))
+                  offsets=((E + 1,), torch.int32), perm=((T * k,), torch.int32), inv=((T * k,), torch.int32),
+                  status=((1,), torch.int32))
     out = dict(out or {})
     for n, (shp, dt) in shapes.items():
         if n not in out:
             out[n] = torch.empty(shp, dtype=dt, device=dev)
         _dev(out[n], dt, shp, n)
     _check(lib().lmoe_route_noalloc(_ptr(scores), _ptr(bias), T, E, k,
-                                    *(_ptr(out[n]) for n in ("idx", "gates", "counts", "offsets", "perm", "inv")),
+                                    *(_ptr(out[n]) for n in ("idx", "gates", "counts", "offsets", "perm", "inv",
+                                                             "status")),
                                     _stream(stream)), "lmoe_route_noalloc")
     return out
 

@@ -1491,9 +1491,10 @@ static size_t noalloc_bytes(long long T, long long E, long long k, size_t* off_r
 
 int lmoe_route_noalloc(const float* scores, const float* bias, int32_t T, int32_t E, int32_t k, int32_t* idx,
                        float* gates, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
-                       void* stream) {
-  if (!scores || !bias || !idx || !gates || !counts || !offsets || !perm || !inv) return LMOE_EINVAL;
-  if (T < 0 || E <= 0 || E > 1024 || k <= 0 || k > E || k > 32) return LMOE_EINVAL;
+                       uint32_t* status, void* stream) {
+  if (!scores || !bias || !idx || !gates || !counts || !offsets || !perm || !inv || !status) return LMOE_EINVAL;
+  if (T < 0 || E <= 0 || k <= 0 || k > E) return LMOE_EINVAL;
+  if (E > 1024 || k > 32) return LMOE_EUNSUPPORTED;  // the same limits as lmoe_create
   size_t o_rank, o_cnt, o_base, o_tiles, o_delta, o_c32, o_ntiles;
   if (noalloc_bytes(T, E, k, &o_rank, &o_cnt, &o_base, &o_tiles, &o_delta, &o_c32, &o_ntiles) >
       LMOE_NOALLOC_SCRATCH_BYTES)
@@ -1518,6 +1519,7 @@ int lmoe_route_noalloc(const float* scores, const float* bias, int32_t T, int32_
     base = base_of[dev];
   }
   cudaStream_t st = (cudaStream_t)stream;
+  CK(cudaMemsetAsync(status, 0, sizeof(uint32_t), st));  // this call's faults only
   if (T == 0) {
     CK(cudaMemsetAsync(counts, 0, (size_t)E * sizeof(int32_t), st));
     CK(cudaMemsetAsync(offsets, 0, (size_t)(E + 1) * sizeof(int32_t), st));
@@ -1530,10 +1532,8 @@ int lmoe_route_noalloc(const float* scores, const float* bias, int32_t T, int32_
   int* delta = reinterpret_cast<int*>(base + o_delta);
   int* counts32 = reinterpret_cast<int*>(base + o_c32);
   int* ntiles = reinterpret_cast<int*>(base + o_ntiles);
-  uint32_t* status = reinterpret_cast<uint32_t*>(base + o_ntiles + 128);
-  // every scratch word is written before it is read, except the status word and the count copies,
-  // which the top-k blocks add into
-  CK(cudaMemsetAsync(status, 0, sizeof(uint32_t), st));
+  // every scratch word is written before it is read, except the count copies, which the top-k
+  // blocks add into; faults (NaN score, index out of range) go to the caller's status word
   CK(cudaMemsetAsync(counts32, 0, (size_t)kCountCopies * E * sizeof(int), st));
   TopkArgs ta{scores, bias, T, E, k, idx, rank, blkcnt, counts32, gates, nullptr, 0, TopkRefine{}, status};
   CK(launch_topk(ta, st));

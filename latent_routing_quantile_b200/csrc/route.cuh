@@ -70,7 +70,8 @@ struct TopkRefine {
   const float* cz;    // router column offsets [E]
   float eps, tau;
 };
-constexpr int kRefineExtra = 8;  // candidates beyond the k-th that an exact decision considers
+constexpr int kRefineExtra = 8;  // candidates beyond the k-th that an exact decision lists
+constexpr int kOverflow = 1 << 30;  // deferred-token flag: more candidates than the list holds
 
 // The exact decision of a token whose fp32 top-k is ambiguous (two of its top k+1 biased scores
 // within tau of each other, so the scores' fp32 rounding could order them either way).  Its
@@ -85,6 +86,14 @@ constexpr int kRefineExtra = 8;  // candidates beyond the k-th that an exact dec
 // (u descending, expert ascending).  The whole block computes each such token's dot products
 // together (one memory round trip instead of one per 32 elements), after its warps have ranked
 // every other token.
+//
+// A token can have more experts within tau of its k-th than the candidate list holds (at most
+// kRefineExtra beyond the k-th, and 32 in all): many scores that saturate the sigmoid to exactly
+// 1.0f in fp32 do that, and at k = 32 the list has no room beyond the k-th at all.  Such a token
+// ("overflow") is decided from every expert whose fp32 biased score lies within tau of the k-th:
+// any other expert trails the k experts above it by more than tau in fp32, hence by more than
+// tau / 2 exactly, so the exact top k lies among them.  Each of them is rescored in fp64 as above
+// and the k best (u descending, expert ascending) are taken in that order.
 
 // One warp per token; a block of W warps ranks kTokBlock = 32 tokens (32 / W per warp; W = 16
 // for E <= 256, whose registers allow two such blocks per SM, else 8).  Lane L holds the scores
@@ -122,7 +131,9 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 
   __shared__ int def_e[kTokBlock][32];
   __shared__ unsigned char def_mi[kTokBlock][32];  // candidate positions of the cluster members
   __shared__ unsigned def_lp[kTokBlock];           // bit c: candidate c is linked to candidate c-1
-  __shared__ int def_info[kTokBlock];              // token | candidates << 8 | members << 16
+  __shared__ int def_info[kTokBlock];              // token | candidates << 8 | members << 16 (| kOverflow)
+  __shared__ float def_thr[kTokBlock];             // overflow: the fp32 threshold u_(k) - tau
+  __shared__ double ovf_u[NJ * 32];                // overflow: fp64 biased score of each candidate
   __shared__ int def_n;
   __shared__ double red[W][9];
   __shared__ double def_z[48];  // [0, 32): candidate dot products; [32, 41): first group's sums; 40: x^2
@@ -245,6 +256,26 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 
         int slot = 0;
         if (lane == 0) slot = atomicAdd(&def_n, 1);
         slot = __shfl_sync(kFull, slot, 0);
+        // overflow: the list is full and the next expert is still within tau of the k-th
+        bool ovf = false;
+        if (nc == kmax && kmax < E) {
+          uint32_t nk = 0u;
+#pragma unroll
+          for (int j = 0; j < NJ; ++j) nk = max(nk, key[j]);
+          nk = __reduce_max_sync(kFull, nk);
+          ovf = nk >= 2u && key_value(nk) >= u_k1 - rf.tau;
+        }
+        if (ovf) {
+          if (lane == 0) {
+            def_info[slot] = tl | kOverflow;
+            def_thr[slot] = u_k1 - rf.tau;
+          }
+          const char* xr = reinterpret_cast<const char*>(rf.x) + (size_t)t * rf.d * (rf.x_bf16 ? 2 : 4);
+          for (int b = lane * 128; b < rf.d * (rf.x_bf16 ? 2 : 4); b += 32 * 128) prefetch_l2(xr + b);
+          deferred |= 1u << (q0 + p);
+          slot_q[q0 + p] = slot;
+          continue;
+        }
         // clusters: candidate c is linked to c-1 when their fp32 scores are within tau (every
         // candidate is, when one of them has no numeric score)
         const float u_up = __shfl_up_sync(kFull, my_u, 1);
@@ -277,7 +308,8 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 
   __syncthreads();  // every deferred token is listed
   const int ndef = def_n;
   for (int di = 0; di < ndef; ++di) {  // block-uniform
-    const int tl = def_info[di] & 255, nc = (def_info[di] >> 8) & 255, nm = def_info[di] >> 16, t = t0 + tl;
+    const int tl = def_info[di] & 255, nc = (def_info[di] >> 8) & 255, nm = (def_info[di] >> 16) & 255,
+              t = t0 + tl;
     const size_t xoff = (size_t)t * rf.d;
     auto xval = [&](int j) -> double {
       return rf.x_bf16 ? (double)__bfloat162float(reinterpret_cast<const bf16*>(rf.x)[xoff + j])
@@ -300,6 +332,63 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 
       }
       __syncthreads();
     };
+    if (def_info[di] & kOverflow) {
+      // every expert within tau of the k-th, rescored in fp64 (one warp per expert), then the k
+      // best in order; other experts hold -inf
+      double v[9];
+      v[0] = 0.0;
+      for (int j = threadIdx.x; j < rf.d; j += blockDim.x) {
+        const double xv = xval(j);
+        v[0] = fma(xv, xv, v[0]);
+      }
+      block_sum(v, 1, def_z + 40);
+      const double r = 1.0 / sqrt(def_z[40] / rf.d + (double)rf.eps);
+      const float thr = def_thr[di];
+      for (int e = warp; e < E; e += W) {  // warp-uniform
+        const float uf = s[(size_t)t * E + e] + bias[e];  // the fp32 biased score top-k ranked
+        double u = -INFINITY;
+        if (uf >= thr) {  // false for NaN
+          const double* wr = rf.wc + (size_t)e * rf.d;
+          double z = 0.0;
+          for (int j = lane; j < rf.d; j += 32) z = fma(xval(j), wr[j], z);
+          z = warp_sum_d(z);
+          u = 1.0 / (1.0 + exp(-(r * z + (double)rf.cz[e]))) + (double)bias[e];
+        }
+        if (lane == 0) ovf_u[e] = u;
+      }
+      __syncthreads();
+      if (warp == 0) {
+        int sel = -1;
+        for (int i = 0; i < k; ++i) {
+          double bu = -INFINITY;
+          int be = INT_MAX;
+          for (int e = lane; e < E; e += 32) {  // ascending e: a strict > keeps the lower index
+            const double uv = ovf_u[e];
+            if (uv > bu) {
+              bu = uv;
+              be = e;
+            }
+          }
+#pragma unroll
+          for (int off = 16; off; off >>= 1) {
+            const double ou = __shfl_xor_sync(kFull, bu, off);
+            const int oe = __shfl_xor_sync(kFull, be, off);
+            if (ou > bu || (ou == bu && oe < be)) {
+              bu = ou;
+              be = oe;
+            }
+          }
+          if (lane == i) sel = be < E ? be : -1;
+          __syncwarp();
+          if (be < E && lane == (be & 31)) ovf_u[be] = -INFINITY;  // taken
+          __syncwarp();
+        }
+        commit(t, tl, sel);
+        def_e[di][lane] = sel;  // the owning warp reads its choice back for the ranks
+      }
+      __syncthreads();
+      continue;
+    }
     // group g sums x . W_comb[e] for members 8g..8g+7 (group 0 also sums x^2 for r)
     double v[9];
     for (int c0 = 0; c0 < nm; c0 += 8) {

@@ -77,3 +77,89 @@ def test_two_ranks_sum_to_the_single_rank_statistics():
     half = oracle.expert_counts(oracle.layer_routing(datagen.tokens(SHAPE, rows=np.arange(0, SHAPE.T, 2)), w,
                                                      np.zeros(SHAPE.E), SHAPE.k)["idx"], SHAPE.E)
     assert not np.array_equal(oracle.sign_rule_update(np.zeros(SHAPE.E), half, 1e-2), b_sign)
+
+
+class OracleLayer:
+    """A stand-in for lq.Layer on the CPU with the calls dp_qb_update makes (hist, load, set_hist,
+    set_load, qb_update): its statistics are those of the oracle's routing of this rank's tokens,
+    and its update is the oracle's.  It records the order of the calls."""
+
+    def __init__(self, x, w, b):
+        r = oracle.layer_routing(x, w, b, SHAPE.k)
+        self._hist = torch.from_numpy(oracle.score_histogram(r["s"]).astype(np.int32))
+        self._n = torch.tensor([x.shape[0]], dtype=torch.int64)
+        self._load = torch.from_numpy(oracle.expert_counts(r["idx"], SHAPE.E).astype(np.int64))
+        self.b = np.asarray(b, dtype=np.float64)
+        self.calls = []
+
+    def hist(self, stream=None):
+        self.calls.append("hist")
+        return self._hist.clone(), self._n.clone()
+
+    def load(self, stream=None):
+        self.calls.append("load")
+        return self._load.clone()
+
+    def set_hist(self, hist, n, stream=None):
+        self.calls.append("set_hist")
+        self._hist, self._n = hist.clone(), n.clone()
+
+    def set_load(self, load, stream=None):
+        self.calls.append("set_load")
+        self._load = load.clone()
+
+    def qb_update(self, beta, literal=False, sign_rule=False, stream=None):
+        self.calls.append("qb_update")
+        if sign_rule:
+            self.b = oracle.sign_rule_update(self.b, self._load.numpy(), beta)
+        else:
+            self.b = oracle.qb_update(self.b, self._hist.numpy().astype(np.int64), int(self._n.item()), SHAPE.k, beta,
+                                      literal=literal)
+
+
+def _rank_update(rank, world, port, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = datagen.layer_weights(SHAPE)
+        x = datagen.tokens(SHAPE, rows=np.arange(SHAPE.T)[rank::world])
+        res = {}
+        for rule in ("qb", "sign"):
+            layer = OracleLayer(x, w, np.zeros(SHAPE.E))
+            lq.dp_qb_update(layer, SHAPE.beta if rule == "qb" else 1e-2, sign_rule=(rule == "sign"))
+            res[rule] = (layer.b, layer.calls)
+        out[rank] = res
+    finally:
+        dist.destroy_process_group()
+
+
+def test_dp_qb_update_sums_before_the_update_on_every_rank():
+    """lq.dp_qb_update, the step bench.py runs between ranks: each rank reads its statistics,
+    the ranks sum them, each sets the sums back and updates.  Driven on two gloo ranks through
+    a CPU stand-in layer, both ranks end with the bias of one rank that saw every token, for
+    QB and for the sign rule, and the calls come in the order read -> sum -> set -> update."""
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        out = mgr.dict()
+        port = _free_port()
+        procs = [ctx.Process(target=_rank_update, args=(r, 2, port, out)) for r in range(2)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(timeout=300)
+            assert p.exitcode == 0
+        res = dict(out)
+    w = datagen.layer_weights(SHAPE)
+    r_all = oracle.layer_routing(datagen.tokens(SHAPE), w, np.zeros(SHAPE.E), SHAPE.k)
+    b_qb = oracle.qb_update(np.zeros(SHAPE.E), oracle.score_histogram(r_all["s"]), SHAPE.T, SHAPE.k, SHAPE.beta)
+    b_sign = oracle.sign_rule_update(np.zeros(SHAPE.E), oracle.expert_counts(r_all["idx"], SHAPE.E), 1e-2)
+    for r in range(2):
+        assert np.array_equal(res[r]["qb"][0], b_qb)
+        assert np.array_equal(res[r]["sign"][0], b_sign)
+        assert res[r]["qb"][1] == ["hist", "set_hist", "qb_update"]
+        assert res[r]["sign"][1] == ["hist", "load", "set_hist", "set_load", "qb_update"]
+    # a rank that updated from its own statistics alone would have another bias
+    own = OracleLayer(datagen.tokens(SHAPE, rows=np.arange(0, SHAPE.T, 2)), w, np.zeros(SHAPE.E))
+    own.qb_update(SHAPE.beta)
+    assert not np.array_equal(own.b, b_qb)

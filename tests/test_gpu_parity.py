@@ -183,7 +183,16 @@ def test_qb_update_stage(literal):
 
 
 # --------------------------------------------------------------------------- whole layer
-def run_layer_check(shape, w, x, b=None, sample=None, record=True):
+def oracle_routing(x, w, b64, k, eps, chunk=None):
+    """oracle.layer_routing on every token, in token chunks of `chunk` rows (None: at once) so the
+    fp64 intermediates of a large workload stay within a few hundred MB of host memory."""
+    if chunk is None or x.shape[0] <= chunk:
+        return oracle.layer_routing(x, w, b64, k, eps)
+    parts = [oracle.layer_routing(x[c0:c0 + chunk], w, b64, k, eps) for c0 in range(0, x.shape[0], chunk)]
+    return {n: np.concatenate([p[n] for p in parts]) for n in parts[0]}
+
+
+def run_layer_check(shape, w, x, b=None, sample=None, record=True, route_chunk=None):
     """Forward on the GPU, oracle on all tokens (routing) and on `sample` rows (outputs)."""
     T, E, k = shape.T, shape.E, shape.k
     layer = make_layer(shape, w, max_tokens=T)
@@ -194,7 +203,7 @@ def run_layer_check(shape, w, x, b=None, sample=None, record=True):
     r = layer.routing()
     torch.cuda.synchronize()
     b64 = np.zeros(E) if b is None else b.astype(np.float64)
-    ro = oracle.layer_routing(x, w, b64, k, shape.rms_eps)
+    ro = oracle_routing(x, w, b64, k, shape.rms_eps, route_chunk)
     s_gpu = r["scores"].cpu().numpy()
     s_err = float(np.max(np.abs(s_gpu - ro["s"])))
     s_tol = score_tolerance(shape)
@@ -243,15 +252,44 @@ def test_small_bf16_layer_ragged(gain, E):
     layer.close()
 
 
-def test_sweep_65536_tokens_sampled():
-    """The token sweep's 65536-token point (the sweep workload's seeded inputs, as bench.py --workload
-    sweep --tokens 65536 uses them; mini_replica widths): routing parity on every token,
-    outputs on every 64th (1024 tokens), as the sweep's parity check asks for T >= 16384."""
-    shape = dataclasses.replace(datagen.WORKLOADS["sweep"], T=65536)
+@pytest.mark.parametrize("T", datagen.SWEEP_T)
+def test_sweep_point_matches_oracle(T):
+    """Every point of the token sweep (the sweep workload's seeded inputs, seed 4, as bench.py
+    --workload sweep --tokens T uses them; mini_replica widths): routing, counts, offsets and the
+    permutation on every token; outputs on every token up to 4096 and on 1024 tokens spread over
+    the batch above that.  262144 tokens run the largest grids (8192 top-k blocks, about 12,300
+    tile-table entries, 1.57 M permuted rows); the oracle routes them in 8192-token chunks."""
+    shape = dataclasses.replace(datagen.WORKLOADS["sweep"], T=T)
     w = datagen.layer_weights(shape)
     x = datagen.tokens(shape)
-    layer, y, ro, stats = run_layer_check(shape, w, x, sample=np.arange(0, shape.T, 64))
-    print("sweep_65536", json.dumps(stats))
+    sample = None if T <= 4096 else np.arange(0, T, T // 1024)
+    layer, y, ro, stats = run_layer_check(shape, w, x, sample=sample, route_chunk=8192)
+    print(f"sweep_{T}", json.dumps(stats))
+    layer.close()
+
+
+@pytest.mark.parametrize("name,E,k,nsat", [("saturated_k6", 256, 6, 40), ("saturated_k32", 64, 32, 48)])
+def test_saturated_router_ties_are_decided_exactly(name, E, k, nsat):
+    """Router column offsets of 18 and up on nsat experts saturate their sigmoid: in fp32 most of
+    their scores are exactly 1.0f (all within the near-tie width of each other), far more of them
+    than the exact decision's candidate list holds beyond the k-th (8; none at k = 32), while in
+    fp64 they still differ.  Every token then takes the overflow decision, which rescores every
+    expert within the near-tie width in fp64; routing must equal the fp64 oracle's on every token
+    (set and rank order), and outputs stay within tolerance."""
+    d, l = (512, 128) if E == 256 else (256, 64)
+    shape = datagen.LayerShape(name, 1000, d, l, E, k, 128, 256, "bf16", seed=61)
+    sat = (np.arange(nsat) * E) // nsat
+    c = np.zeros(E, dtype=np.float32)
+    c[sat] = 18.0 + 0.1 * np.arange(nsat, dtype=np.float32)
+    w = datagen.layer_weights(shape, router_offsets=c)
+    x = datagen.tokens(shape)
+    layer, y, ro, stats = run_layer_check(shape, w, x)
+    s = layer.routing()["scores"].cpu().numpy()
+    ones = (s[:, sat] == 1.0).sum(1)
+    print(name, json.dumps(dict(stats, exact_ones_per_token=float(ones.mean()))))
+    # the fp32 ties are there: more experts at exactly 1.0f than the candidate list holds
+    assert np.all(ones > min(k + 8, 32))
+    assert np.all(np.isin(ro["idx"], sat))
     layer.close()
 
 
