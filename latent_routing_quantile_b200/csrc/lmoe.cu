@@ -16,8 +16,15 @@
 #include "simt_gemm.cuh"
 #include "tc_gemm.cuh"
 #include "k1_router.cuh"
+#include "expert_gemm.cuh"
 
 using namespace lmoe;
+
+// The routed-expert GEMMs run on the 128-row tile engine (tc_gemm.cuh, grouped mode) unless this
+// is 1: then shapes with h % 128 == 0 and l % 256 == 0 run the CTA-pair kernel of expert_gemm.cuh.
+#ifndef LMOE_PAIR_EXPERTS
+#define LMOE_PAIR_EXPERTS 0
+#endif
 
 namespace {
 
@@ -327,6 +334,12 @@ struct lmoe_handle {
   long long rows_pad = 0;                     // rows of that layout (upper bound)
   float* gates = nullptr;
   int2* mtiles = nullptr;
+  // pair expert GEMMs (bf16, h % 128 == 0, l % 256 == 0): token tiles of up to 256 tokens
+  bool xgemm = false;
+  int4* ttiles = nullptr;
+  int* num_ttiles = nullptr;
+  int max_ttiles = 0;
+  CUtensorMap tm_xw13, tm_xaperm, tm_xact_out, tm_xw2, tm_xact, tm_xo_out;
   void *a_perm = nullptr, *act = nullptr, *o = nullptr, *z = nullptr, *a_s = nullptr;
   void *x_stage = nullptr, *y_stage = nullptr;
   // lmoe_forward_host: two input staging buffers, so the next call's host-to-device copy (on its
@@ -427,6 +440,8 @@ void plan_layout(lmoe_handle* h, Arena& a) {
   a.add((void**)&h->offsets, (E + 1) * 4);
   a.add((void**)&h->num_mtiles, 4);
   a.add((void**)&h->mtiles, (size_t)h->max_mtiles * 8);
+  a.add((void**)&h->ttiles, (size_t)h->max_ttiles * 16);
+  a.add((void**)&h->num_ttiles, 4);
   a.add((void**)&h->perm, TK * 4);
   a.add((void**)&h->inv, TK * 4);
   a.add((void**)&h->prow, TK * 4);
@@ -500,6 +515,14 @@ int build_maps(lmoe_handle* h) {
   (void)TK;
   ok &= make_map(&h->tm_aperm, h->a_perm, RP, l, l, 128);
   ok &= make_map(&h->tm_w13, h->w13, E * 2 * hh, l, l, h->bn_e1);
+  if (h->xgemm) {
+    ok &= make_map(&h->tm_xw13, h->w13, E * 2 * hh, l, l, 128);
+    ok &= make_map(&h->tm_xaperm, h->a_perm, RP, l, l, 16);
+    ok &= make_map(&h->tm_xact_out, h->act, RP, hh, hh, 32);
+    ok &= make_map(&h->tm_xw2, h->w2, E * l, hh, hh, 128);
+    ok &= make_map(&h->tm_xact, h->act, RP, hh, hh, 16);
+    ok &= make_map(&h->tm_xo_out, h->o, RP, l, l, 32);
+  }
   ok &= make_map(&h->tm_act, h->act, RP, hh, hh, 128);
   ok &= make_map(&h->tm_o, h->o, RP, l, l, 128);
   for (int i = 0; i < 3; ++i) {
@@ -645,7 +668,8 @@ int route_from_scores(lmoe_handle* h, int T, uint32_t flags, const StatsState& p
   CK(launch_k(plan_kernel, dim3((c.E + 31) / 32), dim3(1024), 0, st, 1, (const int*)h->counts32, h->counts,
               (const int*)h->blkcnt, nblk, c.E, h->offsets, h->pad_delta, h->blkbase, h->mtiles, h->num_mtiles,
               // an update already forked clears the loads itself, which equals adding them first
-              ((flags & LMOE_RECORD_STATS) && !early) ? h->load : (long long*)nullptr));
+              ((flags & LMOE_RECORD_STATS) && !early) ? h->load : (long long*)nullptr,
+              h->xgemm ? h->ttiles : (int4*)nullptr, h->num_ttiles));
   const int pairs = T * c.k;
   const dim3 ggrid((pairs + 8 * kGatherPairs - 1) / (8 * kGatherPairs));
   int4* clear = reinterpret_cast<int4*>(h->counts32);
@@ -781,6 +805,32 @@ int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, 
   }
   // routed experts, grouped over the permuted rows
   mark(h, ST_EXPERT1, st);
+  if (h->xgemm) {
+    static unsigned done1 = 0, done2 = 0;
+    CK(ensure_smem_attr(expert_gemm_kernel<XEPI_SWIGLU>, kXSmemBytes, done1));
+    CK(ensure_smem_attr(expert_gemm_kernel<XEPI_STORE>, kXSmemBytes, done2));
+    const int grid = h->sms & ~1;
+    XParams p;
+    memset(&p, 0, sizeof(p));
+    p.status = h->status;
+    p.tiles = h->ttiles;
+    p.num_tiles = h->num_ttiles;
+    // act = silu(A W1_e^T) * (A W3_e^T): weight slices of the interleaved gate/linear rows
+    p.tmW = h->tm_xw13;
+    p.tmX = h->tm_xaperm;
+    p.tmOut = h->tm_xact_out;
+    p.w_rows = 2 * c.h;
+    p.nkb = c.l / 64;
+    CK(launch_k(expert_gemm_kernel<XEPI_SWIGLU>, dim3(grid), dim3(kTcThreads), kXSmemBytes, st, 2, p));
+    mark(h, ST_EXPERT2, st);
+    // o = act W2_e^T
+    p.tmW = h->tm_xw2;
+    p.tmX = h->tm_xact;
+    p.tmOut = h->tm_xo_out;
+    p.w_rows = c.l;
+    p.nkb = c.h / 64;
+    CK(launch_k(expert_gemm_kernel<XEPI_STORE>, dim3(grid), dim3(kTcThreads), kXSmemBytes, st, 2, p));
+  } else {
   {
     TcParams p = tc_base(h);
     p.tmA[0] = h->tm_aperm;
@@ -826,6 +876,7 @@ int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, 
     p.hint_b = 1;
     p.hint_out = 1;  // o is read by the combine kernel
     CK(launch_tc(p, EPI_BF16, h->bn_e2, h->sms, st));
+  }
   }
   mark(h, ST_COMBINE, st);
   CK(launch_combine((const bf16*)h->o, h->gates, h->prow, T, c.k, c.l, (bf16*)h->z, st));
@@ -953,8 +1004,12 @@ int repack(lmoe_handle* h, const lmoe_weights* w, cudaStream_t st) {
     if (hs)
       interleave_kernel<bf16><<<grid_1d(hs * d, TPB), TPB, 0, st>>>((const bf16*)w->ws1, (const bf16*)w->ws3, g, 1,
                                                                     hs, d, (bf16*)h->ws13);
-    interleave_kernel<bf16><<<grid_1d(E * hh * l, TPB), TPB, 0, st>>>((const bf16*)w->w1, (const bf16*)w->w3,
-                                                                      nullptr, E, hh, l, (bf16*)h->w13);
+    if (h->xgemm)
+      pair_pack_kernel<bf16><<<grid_1d(2 * E * hh * l, TPB), TPB, 0, st>>>((const bf16*)w->w1, (const bf16*)w->w3,
+                                                                          E, hh, l, (bf16*)h->w13);
+    else
+      interleave_kernel<bf16><<<grid_1d(E * hh * l, TPB), TPB, 0, st>>>((const bf16*)w->w1, (const bf16*)w->w3,
+                                                                        nullptr, E, hh, l, (bf16*)h->w13);
     CK(cudaMemcpyAsync(h->w2, w->w2, E * l * hh * 2, cudaMemcpyDeviceToDevice, st));
     fold_gain_kernel<bf16><<<grid_1d(d * l, TPB), TPB, 0, st>>>((const bf16*)w->w_up, nullptr, d, l,
                                                                 (bf16*)h->wy, l + hs, 0);
@@ -1086,6 +1141,8 @@ static void size_handle(lmoe_handle* h, const lmoe_config* cfg) {
   h->max_mtiles = (int)(((long long)cfg->max_tokens * cfg->k + kTileRows - 1) / kTileRows) + cfg->E;
   h->ld_bins = (cfg->max_tokens + 31) / 32 * 32;
   h->rows_pad = (long long)cfg->max_tokens * cfg->k + (long long)kTileRows * cfg->E;
+  h->max_ttiles = (int)(((long long)cfg->max_tokens * cfg->k + kTokTile - 1) / kTokTile) + cfg->E;
+  h->xgemm = LMOE_PAIR_EXPERTS && cfg->dtype == LMOE_BF16 && cfg->h % 128 == 0 && cfg->l % 256 == 0;
 }
 
 int lmoe_workspace_bytes(const lmoe_config* cfg, size_t* bytes) {
@@ -1539,7 +1596,7 @@ int lmoe_route_noalloc(const float* scores, const float* bias, int32_t T, int32_
   CK(launch_topk(ta, st));
   const int nblk = (T + kTokBlock - 1) / kTokBlock;
   plan_kernel<<<(E + 31) / 32, 1024, 0, st>>>(counts32, counts, blkcnt, nblk, E, offsets, delta, blkbase, tiles,
-                                               ntiles, nullptr);
+                                               ntiles, nullptr, nullptr, nullptr);
   CK(cudaGetLastError());
   const int pairs = T * k;
   gather_kernel<float><<<(pairs + 8 * kGatherPairs - 1) / (8 * kGatherPairs), 256, 0, st>>>(

@@ -12,6 +12,7 @@ namespace lmoe {
 constexpr int kTokBlock = 32;      // tokens per routing block: one rank-mask word per expert
 constexpr int kCountCopies = 32;   // per-expert counts are summed into this many copies (block % 32)
 constexpr int kTileRows = 128;     // rows per grouped-GEMM M-tile
+constexpr int kTokTile = 256;      // tokens per tile of the pair expert GEMMs
 constexpr unsigned kFull = 0xffffffffu;
 
 // --------------------------------------------------------------------------- RMSNorm
@@ -121,6 +122,9 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 
   constexpr int W = topk_warps(NJ);
   constexpr int TPW = kTokBlock / W;  // tokens per warp
   constexpr int PF = topk_prefetch(NJ);
+  // fp64 rescoring reads four elements per thread and step where the registers allow it (the
+  // 8-warp blocks of E > 256, whose wide d makes the rescoring loop latency-bound)
+  constexpr bool kQuad = W == 8;
   extern __shared__ uint32_t smem_topk[];
   uint32_t* mask = smem_topk;                                    // [E]
   uint16_t* sbins = reinterpret_cast<uint16_t*>(smem_topk + E);  // [32 tokens][E + 2] (padded rows)
@@ -315,6 +319,22 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 
       return rf.x_bf16 ? (double)__bfloat162float(reinterpret_cast<const bf16*>(rf.x)[xoff + j])
                        : (double)reinterpret_cast<const float*>(rf.x)[xoff + j];
     };
+    // x[t, 4q .. 4q+3] widened to fp64 (one 8- or 16-byte load)
+    auto xquad = [&](int q, double (&xv)[4]) {
+      if (rf.x_bf16) {
+        const uint2 pr = reinterpret_cast<const uint2*>(reinterpret_cast<const bf16*>(rf.x) + xoff)[q];
+        xv[0] = (double)__uint_as_float(pr.x << 16);
+        xv[1] = (double)__uint_as_float(pr.x & 0xFFFF0000u);
+        xv[2] = (double)__uint_as_float(pr.y << 16);
+        xv[3] = (double)__uint_as_float(pr.y & 0xFFFF0000u);
+      } else {
+        const float4 f = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(rf.x) + xoff)[q];
+        xv[0] = f.x;
+        xv[1] = f.y;
+        xv[2] = f.z;
+        xv[3] = f.w;
+      }
+    };
     // block sums: warp shuffles, then one partial per warp in red[][u]
     auto block_sum = [&](double (&v)[9], int nv, double* out) {
 #pragma unroll
@@ -350,7 +370,17 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 
         if (uf >= thr) {  // false for NaN
           const double* wr = rf.wc + (size_t)e * rf.d;
           double z = 0.0;
-          for (int j = lane; j < rf.d; j += 32) z = fma(xval(j), wr[j], z);
+          if constexpr (kQuad) {
+            for (int q = lane; q < (rf.d >> 2); q += 32) {
+              double xv[4];
+              xquad(q, xv);
+              const double2 a = reinterpret_cast<const double2*>(wr)[2 * q];
+              const double2 b = reinterpret_cast<const double2*>(wr)[2 * q + 1];
+              z = fma(xv[3], b.y, fma(xv[2], b.x, fma(xv[1], a.y, fma(xv[0], a.x, z))));
+            }
+          } else {
+            for (int j = lane; j < rf.d; j += 32) z = fma(xval(j), wr[j], z);
+          }
           z = warp_sum_d(z);
           u = 1.0 / (1.0 + exp(-(r * z + (double)rf.cz[e]))) + (double)bias[e];
         }
@@ -400,11 +430,38 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 
         wrow[u] = rf.wc + (size_t)def_e[di][def_mi[di][min(c0 + u, nm - 1)]] * rf.d;
       }
       v[8] = 0.0;
-      for (int j = threadIdx.x; j < rf.d; j += blockDim.x) {
-        const double xv = xval(j);
-        v[8] = fma(xv, xv, v[8]);
+      if constexpr (!kQuad) {
+        for (int j = threadIdx.x; j < rf.d; j += blockDim.x) {
+          const double xv = xval(j);
+          v[8] = fma(xv, xv, v[8]);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) v[u] = fma(xv, wrow[u][j], v[u]);
+          for (int u = 0; u < 8; ++u) v[u] = fma(xv, wrow[u][j], v[u]);
+        }
+      }
+      // four consecutive elements per thread and step (d is a multiple of 64): each step issues
+      // the rows' 32 bytes before any product, so their latencies overlap
+      for (int q = threadIdx.x; kQuad && q < (rf.d >> 2); q += blockDim.x) {
+        double xv[4];
+        xquad(q, xv);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[8] = fma(xv[i], xv[i], v[8]);
+#pragma unroll
+        for (int u0 = 0; u0 < 8; u0 += 4) {  // four rows at a time bounds the registers in flight
+          if (u0 < ng) {  // block-uniform
+            double2 a[4], b[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              if (u0 + u < ng) {
+                a[u] = reinterpret_cast<const double2*>(wrow[u0 + u])[2 * q];
+                b[u] = reinterpret_cast<const double2*>(wrow[u0 + u])[2 * q + 1];
+              }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              if (u0 + u < ng)
+                v[u0 + u] = fma(xv[3], b[u].y, fma(xv[2], b[u].x, fma(xv[1], a[u].y, fma(xv[0], a[u].x, v[u0 + u]))));
+          }
+        }
       }
       if (c0 == 0) {
 #pragma unroll
@@ -518,7 +575,8 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ coun
                                                     const int* __restrict__ blkcnt, int nblk, int E,
                                                     int* __restrict__ offsets, int* __restrict__ pad_delta,
                                                     int* __restrict__ blkbase, int2* __restrict__ mtiles,
-                                                    int* __restrict__ num_mtiles, long long* __restrict__ load) {
+                                                    int* __restrict__ num_mtiles, long long* __restrict__ load,
+                                                    int4* __restrict__ ttiles, int* __restrict__ num_ttiles) {
   __shared__ int sh[32];
   __shared__ int s_off[1024];
   __shared__ int part[32][33];
@@ -552,6 +610,16 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ coun
     for (int j = 0; j < mt; ++j)
       mtiles[mt_start + j] = make_int2(tid | (min(kTileRows, c - j * kTileRows) << 16), poff + j * kTileRows);
     if (tid == 0) *num_mtiles = mt_total;
+    if (ttiles) {
+      // token tiles of the pair expert GEMMs: up to kTokTile tokens of one expert each,
+      // (expert, first row in the padded layout, valid tokens)
+      const int nt = (c + kTokTile - 1) / kTokTile;
+      int nt_total;
+      const int nt_start = block_exclusive_scan_1024(nt, sh, &nt_total);
+      for (int j = 0; j < nt; ++j)
+        ttiles[nt_start + j] = make_int4(tid, poff + j * kTokTile, min(kTokTile, c - j * kTokTile), 0);
+      if (tid == 0) *num_ttiles = nt_total;
+    }
   }
   __syncthreads();
   const int tx = tid & 31, ty = tid >> 5;
@@ -956,6 +1024,26 @@ __global__ void interleave_kernel(const T* __restrict__ w1, const T* __restrict_
     const long long o1 = base + (long long)((r / 64) * 128 + (r % 64)) * cols + c;
     out[o1] = from_f<T>(gv * to_f<T>(w1[i]));
     out[o1 + 64LL * cols] = from_f<T>(gv * to_f<T>(w3[i]));
+  }
+}
+
+// Gate (w1) and linear (w3) rows of `groups` experts [groups, rows, cols] in the order of the pair
+// expert GEMM: in each 256-row slice s, CTA half r, row 32q + j holds feature
+// 128 s + 64 r + 16 q + (j & 15), from w1 when j < 16 and from w3 otherwise.
+template <typename T>
+__global__ void pair_pack_kernel(const T* __restrict__ w1, const T* __restrict__ w3, int groups, int rows, int cols,
+                                 T* __restrict__ out) {
+  const long long n = (long long)groups * 2 * rows * cols;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long rc = 2LL * rows * cols;
+    const int grp = (int)(i / rc);
+    const long long rem = i - grp * rc;
+    const int orow = (int)(rem / cols), c = (int)(rem - (long long)orow * cols);
+    const int sl = orow >> 8, r = (orow >> 7) & 1, q = (orow >> 5) & 3, j = orow & 31;
+    const int f = sl * 128 + r * 64 + q * 16 + (j & 15);
+    const T* src = j < 16 ? w1 : w3;
+    out[i] = src[((long long)grp * rows + f) * cols + c];
   }
 }
 
