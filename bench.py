@@ -151,7 +151,7 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------------------- ours
-def measure(shape, args, rank, world, local_rank, e2e=True):
+def measure(shape, args, rank, world, local_rank, e2e=True, experts=0):
     """Device-timed steps (the headline), per-stage times (a second, eager pass) and, with e2e,
     the host-buffer entry point, for one workload on this rank.  Returns (summary on rank 0, or
     None; the number of kernels launched in the timed region)."""
@@ -164,7 +164,7 @@ def measure(shape, args, rank, world, local_rank, e2e=True):
     T = shape.T
     w = datagen.layer_weights(shape)
     x_cpu = datagen.tokens(shape, seed=shape.seed + 1000 * rank)
-    layer = lq.layer_from_weights(shape, w)
+    layer = lq.layer_from_weights(shape, w, experts=experts)
     del w
     stream = torch.cuda.current_stream()
     x = x_cpu.cuda()
@@ -300,6 +300,8 @@ def measure(shape, args, rank, world, local_rank, e2e=True):
     rpc_ms = sum(per_launch[n] for n in rpc)
     ex_flops = work["expert_swiglu"][0] + work["expert_down"][0]
     ex_ms = per_launch["expert_swiglu"] + per_launch["expert_down"]
+    # 8-bit experts run at twice the bf16 tensor rate (the dense fp8 rate is twice bf16's)
+    ex_peak = peaks["bf16_tflops"] * (2 if experts else 1)
     summary = {
         "workload": shape.name, "T": T, "ms_per_step": round(ms_max, 5),
         "value": round(T * world / (ms_max / 1e3), 1),
@@ -310,6 +312,9 @@ def measure(shape, args, rank, world, local_rank, e2e=True):
         "router_permute_combine_frac_of_hbm":
             round(rpc_bytes / (rpc_ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4) if rpc_ms > 0 else None,
         "expert_gemm_frac_of_bf16_peak": round(ex_flops / (ex_ms / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
+        "expert_gemm_tflops": round(ex_flops / (ex_ms / 1e3) / 1e12, 1),
+        "expert_gemm_frac_of_format_peak": round(ex_flops / (ex_ms / 1e3) / 1e12 / ex_peak, 4),
+        "experts": "mxfp8" if experts else "bf16",
         "clocks": clk.summary(),
         "e2e_ms": e2e_ms, "e2e_steps": e2e_steps, "stage_ms": per_launch, "work": work,
         "peaks": (peaks, peak_src),
@@ -353,10 +358,11 @@ def run_ours(args, rank, world, local_rank):
     also = {}
     if world == 1 and args.also and not args.tokens:
         for spec in args.also.split(","):
-            wl, t = spec.split(":")
-            sh = datagen.WORKLOADS[wl].with_tokens(int(t))
-            s2, _ = measure(sh, args, rank, world, local_rank, e2e=False)
-            also[sh.name] = s2
+            parts = spec.split(":")
+            sh = datagen.WORKLOADS[parts[0]].with_tokens(int(parts[1]))
+            mx = len(parts) > 2 and parts[2] == "mxfp8"
+            s2, _ = measure(sh, args, rank, world, local_rank, e2e=False, experts=1 if mx else 0)
+            also[sh.name + ("_mxfp8" if mx else "")] = s2
     if rank != 0:
         return None
     m = main_s
@@ -398,6 +404,8 @@ def run_ours(args, rank, world, local_rank):
                 "gpu_launches": a["gpu_launches"], "router_permute_gbs": a["router_permute_gbs"],
                 "router_permute_combine_frac_of_hbm": a["router_permute_combine_frac_of_hbm"],
                 "expert_gemm_frac_of_bf16_peak": a["expert_gemm_frac_of_bf16_peak"],
+                "experts": a["experts"], "expert_gemm_tflops": a["expert_gemm_tflops"],
+                "expert_gemm_frac_of_format_peak": a["expert_gemm_frac_of_format_peak"],
                 "tensor_peak_frac_step": a["tensor_peak_frac_step"], "kernels": a["kernels"], "clocks": a["clocks"]}
             for n, a in also.items()}
     return out
@@ -508,7 +516,8 @@ def main():
     ap.add_argument("--workload", default="wide_stress")
     ap.add_argument("--tokens", type=int, default=0)
     ap.add_argument("--also", default="sweep:262144",
-                    help="extra workloads (name:T, comma-separated) measured in the same call on one GPU; '' for none")
+                    help="extra workloads (name:T[:mxfp8], comma-separated) measured in the same call on one GPU, "
+                         "':mxfp8' with 8-bit routed experts; '' for none")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)

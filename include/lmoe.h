@@ -53,9 +53,24 @@ extern "C" {
 
 /* lmoe_config.dtype: storage and arithmetic type of activations and of all weights except the
  * router (always fp32).  BF16 runs the GEMMs on tcgen05 tensor cores with fp32 accumulation;
- * F32 runs them as fp32 FFMA (tensor-core tf32 would not meet fp32 accuracy). */
+ * F32 runs them on the tensor cores too, as split-precision products: each fp32 operand held as three
+ * bf16 parts, six exact part products accumulated in fp32 (tf32 alone would not meet fp32 accuracy). */
 #define LMOE_F32 0
 #define LMOE_BF16 1
+
+/* lmoe_config.experts: the operand format of the routed experts' two GEMMs.
+ * BF16: bf16 operands, fp32 accumulation (as the rest of the layer).
+ * MXFP8: block-scaled 8-bit operands on tcgen05.mma.kind::mxf8f6f4 (the pages give K3's experts
+ * 4-bit weights and 8-bit activations after quantisation-aware training, "Kimi K3登顶开源第一..."
+ * (cge.wang), and report FP8 at 0.19x of the bf16 replica's MFU on H200, the wink.run summary of
+ * "Pretraining a Mini Kimi K3"; they fix no format, so the reading here is MXFP8): E4M3 elements
+ * (round to nearest even, saturating at 448) with one power-of-two scale per 32 elements along K,
+ * 2^X with X = floor(log2 max|v|) - 8 clamped to [-127, 127].  The expert weights are quantised
+ * once at lmoe_create; the gathered latent rows (from the fp32 value of h) and the SwiGLU
+ * activations (in the first GEMM's epilogue) in every forward; products accumulate in fp32 and
+ * the expert outputs are bf16.  Needs dtype BF16 and l and h multiples of 128. */
+#define LMOE_EXPERTS_BF16 0
+#define LMOE_EXPERTS_MXFP8 1
 
 /* lmoe_forward flags */
 #define LMOE_RECORD_STATS 1u    /* add this forward's scores to the QB histogram and its expert
@@ -93,6 +108,7 @@ typedef struct {
   int32_t nbins;      /* QB histogram bins; must be LMOE_NBINS */
   float rms_eps;      /* RMSNorm epsilon (1e-6) */
   int32_t max_tokens; /* largest T any forward will pass; sizes the workspace */
+  int32_t experts;    /* LMOE_EXPERTS_BF16 or LMOE_EXPERTS_MXFP8 (routed-expert operand format) */
 } lmoe_config;
 
 /* Weights, all device pointers, row-major (out, in).  "dtype" means lmoe_config.dtype.

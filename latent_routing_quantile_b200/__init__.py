@@ -16,6 +16,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "liblmoe.so")
 
 F32, BF16 = 0, 1
+EXPERTS_BF16, EXPERTS_MXFP8 = 0, 1
 RECORD_STATS = 1
 UPDATE_BIAS = 4
 ASYNC_OUTPUT = 8
@@ -41,7 +42,7 @@ class LmoeError(RuntimeError):
 class lmoe_config(ctypes.Structure):
     _fields_ = [("d", c_int32), ("l", c_int32), ("E", c_int32), ("k", c_int32), ("h", c_int32),
                 ("hs", c_int32), ("dtype", c_int32), ("nbins", c_int32), ("rms_eps", c_float),
-                ("max_tokens", c_int32)]
+                ("max_tokens", c_int32), ("experts", c_int32)]
 
 
 class lmoe_weights(ctypes.Structure):
@@ -128,8 +129,9 @@ class Layer:
     router_bias, w1, w3, w2, w_up, ws1, ws3, ws2), layouts (out, in).
     """
 
-    def __init__(self, d, l, E, k, h, hs, dtype, max_tokens, weights, rms_eps=1e-6, stream=None):
-        self.cfg = lmoe_config(d, l, E, k, h, hs, dtype, NBINS, rms_eps, max_tokens)
+    def __init__(self, d, l, E, k, h, hs, dtype, max_tokens, weights, rms_eps=1e-6, stream=None,
+                 experts=EXPERTS_BF16):
+        self.cfg = lmoe_config(d, l, E, k, h, hs, dtype, NBINS, rms_eps, max_tokens, experts)
         self.dtype = torch.float32 if dtype == F32 else torch.bfloat16
         dt = self.dtype
         shapes = {"rms_gain": ((d,), dt), "w_down": ((l, d), dt), "w_router": ((E, l), torch.float32),
@@ -294,8 +296,8 @@ def stage_name(i: int) -> str:
     return lib().lmoe_stage_name(i).decode()
 
 
-def workspace_bytes(d, l, E, k, h, hs, dtype, max_tokens, rms_eps=1e-6) -> int:
-    cfg = lmoe_config(d, l, E, k, h, hs, dtype, NBINS, rms_eps, max_tokens)
+def workspace_bytes(d, l, E, k, h, hs, dtype, max_tokens, rms_eps=1e-6, experts=EXPERTS_BF16) -> int:
+    cfg = lmoe_config(d, l, E, k, h, hs, dtype, NBINS, rms_eps, max_tokens, experts)
     n = c_size_t(0)
     _check(lib().lmoe_workspace_bytes(ctypes.byref(cfg), ctypes.byref(n)), "lmoe_workspace_bytes")
     return n.value
@@ -365,9 +367,10 @@ def route_noalloc(scores, bias, k, out=None, stream=None):
     return out
 
 
-def layer_from_weights(shape, weights_cpu: dict, max_tokens=None, device="cuda", stream=None) -> Layer:
+def layer_from_weights(shape, weights_cpu: dict, max_tokens=None, device="cuda", stream=None,
+                       experts=EXPERTS_BF16) -> Layer:
     """Creates a Layer from the CPU weight dict of the seeded generator (copied to the device)."""
     w = {n: t.to(device) for n, t in weights_cpu.items()}
     return Layer(shape.d, shape.l, shape.E, shape.k, shape.h, shape.hs,
                  F32 if shape.dtype == "f32" else BF16, max_tokens or shape.T, w,
-                 rms_eps=shape.rms_eps, stream=stream)
+                 rms_eps=shape.rms_eps, stream=stream, experts=experts)

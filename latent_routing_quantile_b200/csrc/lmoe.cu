@@ -13,18 +13,11 @@
 
 #include "common.cuh"
 #include "route.cuh"
-#include "simt_gemm.cuh"
 #include "tc_gemm.cuh"
 #include "k1_router.cuh"
-#include "expert_gemm.cuh"
+#include "q8_gemm.cuh"
 
 using namespace lmoe;
-
-// The routed-expert GEMMs run on the 128-row tile engine (tc_gemm.cuh, grouped mode) unless this
-// is 1: then shapes with h % 128 == 0 and l % 256 == 0 run the CTA-pair kernel of expert_gemm.cuh.
-#ifndef LMOE_PAIR_EXPERTS
-#define LMOE_PAIR_EXPERTS 0
-#endif
 
 namespace {
 
@@ -64,6 +57,19 @@ bool make_map_t(CUtensorMap* m, const void* base, long long rows, long long cols
 // bf16 matrix [rows, cols], row pitch `pitch` elements; box = 64 columns (128 bytes) x box_rows.
 bool make_map(CUtensorMap* m, const void* base, long long rows, long long cols, long long pitch, int box_rows) {
   return make_map_t(m, base, rows, cols, pitch, box_rows, false);
+}
+// 8-bit matrix [rows, cols]; box = 128 columns (128 bytes) x box_rows, 128-byte swizzle.
+bool make_map_u8(CUtensorMap* m, const void* base, long long rows, long long cols, long long pitch, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  if (((uintptr_t)base & 15) || (pitch & 15) || rows <= 0 || cols <= 0) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)pitch};
+  cuuint32_t box[2] = {128u, (cuuint32_t)box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 // fp32 matrix; box = 32 columns (128 bytes) x box_rows.
 bool make_map_f32(CUtensorMap* m, const void* base, long long rows, long long cols, long long pitch, int box_rows) {
@@ -154,7 +160,7 @@ cudaError_t launch_tc_e(const TcParams& p, int bn, int grid, cudaStream_t st) {
       else return launch_tc_t<256, EPI>(p, grid, st);
     case 128: return launch_tc_t<128, EPI>(p, grid, st);
     default:
-      if constexpr (EPI == EPI_SWIGLU) return cudaErrorInvalidValue;
+      if constexpr (EPI == EPI_SWIGLU || EPI == EPI_SWIGLU3) return cudaErrorInvalidValue;
       else return launch_tc_t<64, EPI>(p, grid, st);
   }
 }
@@ -165,6 +171,7 @@ cudaError_t launch_tc(const TcParams& p, int epi, int bn, int grid, cudaStream_t
     case EPI_BF16: return launch_tc_e<EPI_BF16>(p, bn, grid, st);
     case EPI_SWIGLU: return launch_tc_e<EPI_SWIGLU>(p, bn, grid, st);
     case EPI_DOWN3: return launch_tc_e<EPI_DOWN3>(p, bn, grid, st);
+    case EPI_SWIGLU3: return launch_tc_e<EPI_SWIGLU3>(p, bn, grid, st);
     default: return launch_tc_e<EPI_ROUTER>(p, bn, grid, st);
   }
 }
@@ -223,11 +230,6 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st) {
   if (nj <= 8) return launch_topk_t<8>(a, st);
   if (nj <= 16) return launch_topk_t<16>(a, st);
   return launch_topk_t<32>(a, st);
-}
-
-template <int EPI>
-cudaError_t launch_simt(const SimtParams& p, int mtiles, cudaStream_t st) {
-  return launch_k(simt_gemm_kernel<EPI>, dim3(p.N / 32, mtiles), dim3(256), 0, st, 1, p);
 }
 
 template <typename T>
@@ -308,21 +310,19 @@ struct lmoe_handle {
   int nblk_max = 0, max_mtiles = 0, ld_bins = 0;
   uint8_t* arena = nullptr;
   size_t arena_bytes = 0;
-  // repacked weights
-  void* w_down = nullptr;   // bf16 [l, d] or [l, 2d] (hi|lo); f32 [l, d]
-  void* w_r = nullptr;      // bf16 [E, 3l] (hi|mid|lo); f32 [E, l]
+  // repacked weights; an fp32 layer keeps each as three bf16 parts along K ([.., 3K])
+  void* w_down = nullptr;   // bf16 [l, d] or [l, 2d] (hi|lo); f32 [l, 3d]
+  void* w_r = nullptr;      // [E_pad, 3l] (hi|mid|lo of the fp32 router)
   float* c = nullptr;       // [E]
   double* wc = nullptr;     // W_comb [E, d] fp64 (exact decision of ambiguous top-k)
   float tau = 0.f;          // near-tie width below which a token's top-k is decided in fp64
-  void* ws13 = nullptr;     // bf16 [2hs, d] interleaved; f32: ws1 [hs, d]
-  void* ws3f = nullptr;     // f32 only: ws3 [hs, d]
-  void* w13 = nullptr;      // bf16 [E, 2h, l] interleaved; f32: w1 [E, h, l]
-  void* w3f = nullptr;      // f32 only: w3 [E, h, l]
-  void* w2 = nullptr;       // [E, l, h]
-  void* wy = nullptr;       // [d, l + hs]
+  void* ws13 = nullptr;     // [2hs, d] interleaved (f32: [2hs, 3d])
+  void* w13 = nullptr;      // [E, 2h, l] interleaved (f32: [E, 2h, 3l])
+  void* w2 = nullptr;       // [E, l, h] (f32: [E, l, 3h])
+  void* wy = nullptr;       // [d, l + hs] (f32: [d, 3l + 3hs])
   // workspace
   float* r = nullptr;
-  void* hx = nullptr;       // bf16 [Tm, 3l] (hi|mid|lo of h); f32 [Tm, l]
+  void* hx = nullptr;       // [Tm, 3l] (hi|mid|lo of h)
   float* s = nullptr;
   uint16_t* bins = nullptr;  // 2 x [E, ld_bins] histogram bin of every score, expert-major
   StatsState ss;
@@ -334,17 +334,22 @@ struct lmoe_handle {
   long long rows_pad = 0;                     // rows of that layout (upper bound)
   float* gates = nullptr;
   int2* mtiles = nullptr;
-  // pair expert GEMMs (bf16, h % 128 == 0, l % 256 == 0): token tiles of up to 256 tokens
-  bool xgemm = false;
-  int4* ttiles = nullptr;
-  int* num_ttiles = nullptr;
-  int max_ttiles = 0;
-  CUtensorMap tm_xw13, tm_xaperm, tm_xact_out, tm_xw2, tm_xact, tm_xo_out;
+  // MXFP8 routed experts: 8-bit elements and scale bytes of the weights, of h, of the gathered
+  // rows and of the activations
+  bool q8 = false;
+  uint8_t *w13q = nullptr, *w13sf = nullptr, *w2q = nullptr, *w2sf = nullptr;
+  uint8_t *hq = nullptr, *hsf = nullptr, *aq = nullptr, *aqsf = nullptr, *actq = nullptr, *actsf = nullptr;
+  CUtensorMap tm_aq, tm_aq_part[3], tm_w13q, tm_actq, tm_actq_part[3], tm_w2q;
   void *a_perm = nullptr, *act = nullptr, *o = nullptr, *z = nullptr, *a_s = nullptr;
   void *x_stage = nullptr, *y_stage = nullptr;
   // lmoe_forward_host: two input staging buffers, so the next call's host-to-device copy (on its
   // own stream) overlaps this call's forward
   void* x_stage2 = nullptr;
+  // fp32 layers: the three bf16 parts of x and of z for the split-precision products, and E
+  // rounded up to 64 (the router's weight rows and column offsets are padded with zeros)
+  void *x3 = nullptr, *z3 = nullptr;
+  int E_pad = 0;
+  CUtensorMap tm_x3, tm_z3;
   void* y_stage2 = nullptr;
   int host_slot = 0;
   cudaStream_t cp_in = nullptr;
@@ -412,22 +417,30 @@ void plan_layout(lmoe_handle* h, Arena& a) {
   const size_t es = h->es;
   const size_t Tm = c.max_tokens, TK = (size_t)c.max_tokens * c.k;
   const size_t d = c.d, l = c.l, E = c.E, hh = c.h, hs = c.hs;
-  // weights
-  a.add(&h->w_down, (h->bf && !h->unit_gain ? 2 : 1) * l * d * es);
-  a.add(&h->w_r, h->bf ? E * 3 * l * 2 : E * l * 4);
-  a.add((void**)&h->c, E * 4);
+  // weights (an fp32 layer keeps every GEMM operand as three bf16 parts along K)
+  const size_t Ep = (size_t)h->E_pad;
+  a.add(&h->w_down, h->bf ? (h->unit_gain ? 1 : 2) * l * d * es : 3 * l * d * 2);
+  a.add(&h->w_r, Ep * 3 * l * 2);
+  a.add((void**)&h->c, Ep * 4);
   a.add((void**)&h->wc, E * d * 8);
-  if (hs) {
-    a.add(&h->ws13, 2 * hs * d * es);
-    if (!h->bf) a.add(&h->ws3f, hs * d * es);
+  if (hs) a.add(&h->ws13, h->bf ? 2 * hs * d * es : 2 * hs * 3 * d * 2);
+  if (h->q8) {
+    a.add((void**)&h->w13q, 2 * E * hh * l);
+    a.add((void**)&h->w13sf, 2 * E * hh * l / 32);
+    a.add((void**)&h->w2q, E * l * hh);
+    a.add((void**)&h->w2sf, E * l * hh / 32);
+  } else {
+    a.add(&h->w13, h->bf ? 2 * E * hh * l * es : 2 * E * hh * 3 * l * 2);
+    a.add(&h->w2, h->bf ? E * l * hh * es : E * l * 3 * hh * 2);
   }
-  a.add(&h->w13, 2 * E * hh * l * es);
-  if (!h->bf) a.add(&h->w3f, E * hh * l * es);
-  a.add(&h->w2, E * l * hh * es);
-  a.add(&h->wy, d * (l + hs) * es);
+  a.add(&h->wy, h->bf ? d * (l + hs) * es : d * 3 * (l + hs) * 2);
   // workspace
   a.add((void**)&h->r, Tm * 4);
-  a.add(&h->hx, h->bf ? Tm * 3 * l * 2 : Tm * l * 4);
+  a.add(&h->hx, Tm * 3 * l * 2);
+  if (!h->bf) {
+    a.add(&h->x3, Tm * 3 * d * 2);
+    a.add(&h->z3, Tm * 3 * l * 2);
+  }
   a.add((void**)&h->s, Tm * E * 4);
   a.add((void**)&h->bins, 2 * (size_t)h->ld_bins * E * 2);
   a.add((void**)&h->idx, TK * 4);
@@ -440,18 +453,26 @@ void plan_layout(lmoe_handle* h, Arena& a) {
   a.add((void**)&h->offsets, (E + 1) * 4);
   a.add((void**)&h->num_mtiles, 4);
   a.add((void**)&h->mtiles, (size_t)h->max_mtiles * 8);
-  a.add((void**)&h->ttiles, (size_t)h->max_ttiles * 16);
-  a.add((void**)&h->num_ttiles, 4);
   a.add((void**)&h->perm, TK * 4);
   a.add((void**)&h->inv, TK * 4);
   a.add((void**)&h->prow, TK * 4);
   a.add((void**)&h->pad_delta, E * 4);
   const size_t RP = (size_t)h->rows_pad;
-  a.add(&h->a_perm, RP * l * es);
-  a.add(&h->act, RP * hh * es);
+  if (h->q8) {
+    a.add((void**)&h->hq, Tm * l);
+    a.add((void**)&h->hsf, Tm * l / 32);
+    a.add((void**)&h->aq, RP * l);
+    const size_t RP128 = (RP + 127) / 128 * 128;  // scale atoms cover whole 128-row tiles
+    a.add((void**)&h->aqsf, RP128 * l / 32);
+    a.add((void**)&h->actq, RP * hh);
+    a.add((void**)&h->actsf, RP128 * hh / 32);
+  } else {
+    a.add(&h->a_perm, h->bf ? RP * l * es : RP * 3 * l * 2);
+    a.add(&h->act, h->bf ? RP * hh * es : RP * 3 * hh * 2);
+  }
   a.add(&h->o, RP * l * es);
   a.add(&h->z, Tm * l * es);
-  if (hs) a.add(&h->a_s, Tm * hs * es);
+  if (hs) a.add(&h->a_s, h->bf ? Tm * hs * es : Tm * 3 * hs * 2);
   a.add(&h->x_stage, Tm * d * es);
   a.add(&h->x_stage2, Tm * d * es);
   a.add(&h->y_stage, Tm * d * es);
@@ -477,6 +498,9 @@ int validate(const lmoe_config* c) {
   if (c->dtype == LMOE_BF16 && c->E % 64) return LMOE_EUNSUPPORTED;
   if (c->dtype == LMOE_F32 && c->E % 32) return LMOE_EUNSUPPORTED;
   if ((long long)c->max_tokens * c->k > (1LL << 30)) return LMOE_EUNSUPPORTED;
+  if (c->experts != LMOE_EXPERTS_BF16 && c->experts != LMOE_EXPERTS_MXFP8) return LMOE_EINVAL;
+  if (c->experts == LMOE_EXPERTS_MXFP8 && (c->dtype != LMOE_BF16 || c->l % 128 || c->h % 128))
+    return LMOE_EUNSUPPORTED;
   return LMOE_OK;
 }
 
@@ -513,16 +537,18 @@ int build_maps(lmoe_handle* h) {
   if (hs) ok &= make_weight_maps(h->tm_ws13, h->ws13, 2 * hs, d);
   const long long RP = h->rows_pad;
   (void)TK;
+  if (h->q8) {
+    ok &= make_map_u8(&h->tm_aq, h->aq, RP, l, l, 128);
+    ok &= make_map_u8(&h->tm_actq, h->actq, RP, hh, hh, 128);
+    for (int i = 0; i < 3; ++i) {
+      ok &= make_map_u8(&h->tm_aq_part[i], h->aq, RP, l, l, 32 * (i + 1));
+      ok &= make_map_u8(&h->tm_actq_part[i], h->actq, RP, hh, hh, 32 * (i + 1));
+    }
+    ok &= make_map_u8(&h->tm_w13q, h->w13q, E * 2 * hh, l, l, 128);
+    ok &= make_map_u8(&h->tm_w2q, h->w2q, E * l, hh, hh, 128);
+  } else {
   ok &= make_map(&h->tm_aperm, h->a_perm, RP, l, l, 128);
   ok &= make_map(&h->tm_w13, h->w13, E * 2 * hh, l, l, h->bn_e1);
-  if (h->xgemm) {
-    ok &= make_map(&h->tm_xw13, h->w13, E * 2 * hh, l, l, 128);
-    ok &= make_map(&h->tm_xaperm, h->a_perm, RP, l, l, 16);
-    ok &= make_map(&h->tm_xact_out, h->act, RP, hh, hh, 32);
-    ok &= make_map(&h->tm_xw2, h->w2, E * l, hh, hh, 128);
-    ok &= make_map(&h->tm_xact, h->act, RP, hh, hh, 16);
-    ok &= make_map(&h->tm_xo_out, h->o, RP, l, l, 32);
-  }
   ok &= make_map(&h->tm_act, h->act, RP, hh, hh, 128);
   ok &= make_map(&h->tm_o, h->o, RP, l, l, 128);
   for (int i = 0; i < 3; ++i) {
@@ -530,8 +556,9 @@ int build_maps(lmoe_handle* h) {
     ok &= make_map(&h->tm_act_part[i], h->act, RP, hh, hh, 32 * (i + 1));
     ok &= make_map(&h->tm_o_part[i], h->o, RP, l, l, 32 * (i + 1));
   }
-  ok &= make_map_f32(&h->tm_s, h->s, Tm, E, E, 128);
   ok &= make_map(&h->tm_w2, h->w2, E * l, hh, hh, h->bn_e2);
+  }
+  ok &= make_map_f32(&h->tm_s, h->s, Tm, E, E, 128);
   ok &= make_map(&h->tm_z, h->z, Tm, l, l, 128);
   if (hs) ok &= make_map(&h->tm_as, h->a_s, Tm, hs, hs, 128);
   ok &= make_weight_maps(h->tm_wy, h->wy, d, l + hs);
@@ -545,6 +572,39 @@ int build_maps(lmoe_handle* h) {
       ok &= make_map(&h->tm_k1_wr2, h->w_r, E, 3 * l, 3 * l, (int)E / 2);
     }
   }
+  return ok ? LMOE_OK : LMOE_ECUDA;
+}
+
+// Maps of an fp32 layer: every GEMM operand is three bf16 parts along K (weights split at create,
+// x and z in each forward, h, a_s and act written that way by the epilogues); o and y are fp32.
+int build_maps_f32(lmoe_handle* h) {
+  const lmoe_config& c = h->cfg;
+  const long long Tm = c.max_tokens, d = c.d, l = c.l, E = c.E, hh = c.h, hs = c.hs, Ep = h->E_pad;
+  const long long RP = h->rows_pad;
+  h->bn_e1 = (2 * c.h) % 256 == 0 ? 256 : 128;
+  h->bn_e2 = pick_bn(c.l);
+  bool ok = true;
+  ok &= make_map(&h->tm_x3, h->x3, Tm, 3 * d, 3 * d, 128);
+  ok &= make_weight_maps(h->tm_wdown, h->w_down, l, 3 * d);
+  ok &= make_map(&h->tm_hx, h->hx, Tm, 3 * l, 3 * l, 128);
+  ok &= make_weight_maps(h->tm_wr, h->w_r, Ep, 3 * l);
+  ok &= make_map_f32(&h->tm_s, h->s, Tm, E, E, 128);
+  if (hs) {
+    ok &= make_weight_maps(h->tm_ws13, h->ws13, 2 * hs, 3 * d);
+    ok &= make_map(&h->tm_as, h->a_s, Tm, 3 * hs, 3 * hs, 128);
+  }
+  ok &= make_map(&h->tm_aperm, h->a_perm, RP, 3 * l, 3 * l, 128);
+  ok &= make_map(&h->tm_w13, h->w13, E * 2 * hh, 3 * l, 3 * l, h->bn_e1);
+  ok &= make_map(&h->tm_act, h->act, RP, 3 * hh, 3 * hh, 128);
+  ok &= make_map(&h->tm_w2, h->w2, E * l, 3 * hh, 3 * hh, h->bn_e2);
+  ok &= make_map_f32(&h->tm_o, h->o, RP, l, l, 128);
+  for (int i = 0; i < 3; ++i) {
+    ok &= make_map(&h->tm_aperm_part[i], h->a_perm, RP, 3 * l, 3 * l, 32 * (i + 1));
+    ok &= make_map(&h->tm_act_part[i], h->act, RP, 3 * hh, 3 * hh, 32 * (i + 1));
+    ok &= make_map_f32(&h->tm_o_part[i], h->o, RP, l, l, 32 * (i + 1));
+  }
+  ok &= make_map(&h->tm_z3, h->z3, Tm, 3 * l, 3 * l, 128);
+  ok &= make_weight_maps(h->tm_wy, h->wy, d, 3 * (l + hs));
   return ok ? LMOE_OK : LMOE_ECUDA;
 }
 
@@ -668,8 +728,7 @@ int route_from_scores(lmoe_handle* h, int T, uint32_t flags, const StatsState& p
   CK(launch_k(plan_kernel, dim3((c.E + 31) / 32), dim3(1024), 0, st, 1, (const int*)h->counts32, h->counts,
               (const int*)h->blkcnt, nblk, c.E, h->offsets, h->pad_delta, h->blkbase, h->mtiles, h->num_mtiles,
               // an update already forked clears the loads itself, which equals adding them first
-              ((flags & LMOE_RECORD_STATS) && !early) ? h->load : (long long*)nullptr,
-              h->xgemm ? h->ttiles : (int4*)nullptr, h->num_ttiles));
+              ((flags & LMOE_RECORD_STATS) && !early) ? h->load : (long long*)nullptr));
   const int pairs = T * c.k;
   const dim3 ggrid((pairs + 8 * kGatherPairs - 1) / (8 * kGatherPairs));
   int4* clear = reinterpret_cast<int4*>(h->counts32);
@@ -679,10 +738,20 @@ int route_from_scores(lmoe_handle* h, int T, uint32_t flags, const StatsState& p
     CK(launch_k(gather_kernel<bf16>, ggrid, dim3(256), 0, st, 1, (const bf16*)h->hx, 3 * c.l, c.l,
                 (const int*)h->idx, (const int*)h->rank, (const int*)h->blkbase, (const int*)h->pad_delta, T, c.E,
                 c.k, h->perm, h->inv, h->prow, (bf16*)h->a_perm, clear, nclear, h->status));
+    if (h->q8 && x) {
+      // MXFP8 experts: h (fp32, from its hi | mid | lo parts) quantised once per token, then each
+      // pair's 8-bit row and scale bytes copied into the padded expert layout
+      CK(launch_k(mx_quant_rows_kernel, dim3(grid_1d((long long)T * c.l / 32, 256)), dim3(256), 0, st, 1,
+                  (const bf16*)h->hx, 3, (long long)T, c.l, h->hq, h->hsf, 0));
+      CK(launch_k(gather_q8_kernel, dim3((pairs + 7) / 8), dim3(256), 0, st, 1, (const uint8_t*)h->hq,
+                  (const uint8_t*)h->hsf, c.l, (const int*)h->prow, pairs, c.k, h->aq, h->aqsf));
+      h->launches += 2;
+    }
   } else {
-    CK(launch_k(gather_kernel<float>, ggrid, dim3(256), 0, st, 1, (const float*)h->hx, c.l, c.l,
+    // fp32 layer: all three parts of h travel with each row (the experts' split-precision products)
+    CK(launch_k(gather_kernel<bf16>, ggrid, dim3(256), 0, st, 1, (const bf16*)h->hx, 3 * c.l, 3 * c.l,
                 (const int*)h->idx, (const int*)h->rank, (const int*)h->blkbase, (const int*)h->pad_delta, T, c.E,
-                c.k, h->perm, h->inv, h->prow, (float*)h->a_perm, clear, nclear, h->status));
+                c.k, h->perm, h->inv, h->prow, (bf16*)h->a_perm, clear, nclear, h->status));
   }
   h->counts32_dirty = false;
   mark(h, ST_HIST, st);
@@ -805,33 +874,45 @@ int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, 
   }
   // routed experts, grouped over the permuted rows
   mark(h, ST_EXPERT1, st);
-  if (h->xgemm) {
+  if (h->q8) {
     static unsigned done1 = 0, done2 = 0;
-    CK(ensure_smem_attr(expert_gemm_kernel<XEPI_SWIGLU>, kXSmemBytes, done1));
-    CK(ensure_smem_attr(expert_gemm_kernel<XEPI_STORE>, kXSmemBytes, done2));
-    const int grid = h->sms & ~1;
-    XParams p;
+    CK(ensure_smem_attr(q8_gemm_kernel<Q8_SWIGLU>, kQ8SmemBytes, done1));
+    CK(ensure_smem_attr(q8_gemm_kernel<Q8_BF16>, kQ8SmemBytes, done2));
+    Q8Params p;
     memset(&p, 0, sizeof(p));
     p.status = h->status;
-    p.tiles = h->ttiles;
-    p.num_tiles = h->num_ttiles;
-    // act = silu(A W1_e^T) * (A W3_e^T): weight slices of the interleaved gate/linear rows
-    p.tmW = h->tm_xw13;
-    p.tmX = h->tm_xaperm;
-    p.tmOut = h->tm_xact_out;
-    p.w_rows = 2 * c.h;
-    p.nkb = c.l / 64;
-    CK(launch_k(expert_gemm_kernel<XEPI_SWIGLU>, dim3(grid), dim3(kTcThreads), kXSmemBytes, st, 2, p));
+    p.mtile_table = h->mtiles;
+    p.num_mtiles = h->num_mtiles;
+    // act (MXFP8) = silu(A W1_e^T) * (A W3_e^T)
+    p.tmA = h->tm_aq;
+    for (int i = 0; i < 3; ++i) p.tmA_part[i] = h->tm_aq_part[i];
+    p.tmB = h->tm_w13q;
+    p.a_sf = h->aqsf;
+    p.b_sf = h->w13sf;
+    p.n_tiles = 2 * c.h / 128;
+    p.b_rows = 2 * c.h;
+    p.nkb = c.l / 128;
+    p.out_q = h->actq;
+    p.out_sf = h->actsf;
+    p.n_out = c.h;
+    CK(launch_k(q8_gemm_kernel<Q8_SWIGLU>, dim3(h->sms), dim3(kQ8Threads), kQ8SmemBytes, st, 1, p));
     mark(h, ST_EXPERT2, st);
-    // o = act W2_e^T
-    p.tmW = h->tm_xw2;
-    p.tmX = h->tm_xact;
-    p.tmOut = h->tm_xo_out;
-    p.w_rows = c.l;
-    p.nkb = c.h / 64;
-    CK(launch_k(expert_gemm_kernel<XEPI_STORE>, dim3(grid), dim3(kTcThreads), kXSmemBytes, st, 2, p));
+    // o (bf16) = act W2_e^T
+    p.tmA = h->tm_actq;
+    for (int i = 0; i < 3; ++i) p.tmA_part[i] = h->tm_actq_part[i];
+    p.tmB = h->tm_w2q;
+    p.a_sf = h->actsf;
+    p.b_sf = h->w2sf;
+    p.n_tiles = c.l / 128;
+    p.b_rows = c.l;
+    p.nkb = c.h / 128;
+    p.out_q = nullptr;
+    p.out_sf = nullptr;
+    p.out_bf = (bf16*)h->o;
+    p.n_out = c.l;
+    CK(launch_k(q8_gemm_kernel<Q8_BF16>, dim3(h->sms), dim3(kQ8Threads), kQ8SmemBytes, st, 1, p));
   } else {
-  {
+    {
     TcParams p = tc_base(h);
     p.tmA[0] = h->tm_aperm;
     p.tmA[1] = h->tm_aperm;
@@ -852,9 +933,8 @@ int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, 
     p.hint_b = 1;    // each expert's weights serve its few tiles, then not again this step
     p.hint_out = 1;  // act is read by the next GEMM
     CK(launch_tc(p, EPI_SWIGLU, h->bn_e1, h->sms, st));
-  }
-  mark(h, ST_EXPERT2, st);
-  {
+    }
+    mark(h, ST_EXPERT2, st);
     TcParams p = tc_base(h);
     p.tmA[0] = h->tm_act;
     p.tmA[1] = h->tm_act;
@@ -876,7 +956,6 @@ int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, 
     p.hint_b = 1;
     p.hint_out = 1;  // o is read by the combine kernel
     CK(launch_tc(p, EPI_BF16, h->bn_e2, h->sms, st));
-  }
   }
   mark(h, ST_COMBINE, st);
   CK(launch_combine((const bf16*)h->o, h->gates, h->prow, T, c.k, c.l, (bf16*)h->z, st));
@@ -909,82 +988,140 @@ int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, 
   return join_update(h, flags, st);
 }
 
+// The six significant products of A = [hi | mid | lo] and B = [hi | mid | lo] (three bf16 parts of
+// fp32 values along K each): part pairs (a, b), smallest first, as K segments of the engine.
+constexpr int kSplitA[6] = {1, 2, 0, 1, 0, 0}, kSplitB[6] = {1, 0, 2, 0, 1, 0};
+void split_segments(TcParams& p, int first, int a_map, int b_off, int K) {
+  for (int i = 0; i < 6; ++i) p.seg[first + i] = KSeg{a_map, kSplitA[i] * K, b_off + kSplitB[i] * K, K / 64};
+}
+
+// fp32 layer: the same stages as forward_bf16, every product split-precision on the tensor cores.
 int forward_f32(lmoe_handle* h, const void* xv, void* yv, int T, uint32_t flags, const StatsState& pre,
                 cudaStream_t st) {
   const lmoe_config& c = h->cfg;
   const float* x = (const float*)xv;
   const int mt = (T + 127) / 128;
+  const int d = c.d, l = c.l, hh = c.h, hs = c.hs;
   mark(h, ST_RMS, st);
-  CK(launch_k(rms_kernel<float>, dim3((T + 7) / 8), dim3(256), 0, st, 1, x, T, c.d, c.rms_eps, h->r));
-  SimtParams b;
-  memset(&b, 0, sizeof(b));
-  b.status = h->status;
+  CK(launch_k(rms_kernel<float>, dim3((T + 7) / 8), dim3(256), 0, st, 1, x, T, d, c.rms_eps, h->r));
+  CK(launch_k(split3_kernel, dim3(grid_1d((long long)T * d, 256)), dim3(256), 0, st, 1, x, (const float*)nullptr, T, d,
+              (bf16*)h->x3, 3 * d, 0));
   mark(h, ST_DOWN, st);
-  {  // h = r * (x Wdown'^T)
-    SimtParams p = b;
-    p.A0 = x; p.lda0 = c.d; p.K0 = c.d; p.a_rows = T;
-    p.B0 = (const float*)h->w_down; p.ldb = c.d;
-    p.M = T; p.N = c.l;
-    p.out = (float*)h->hx; p.ldo = c.l; p.row_scale = h->r;
-    CK(launch_simt<SE_STORE>(p, mt, st));
+  {  // h = r * (x W_down'^T), stored as hi | mid | lo parts
+    TcParams p = tc_base(h);
+    p.tmA[0] = p.tmA[1] = h->tm_x3;
+    const int bn = pick_bn_for(T, l, h->sms, 64);
+    p.tmB = h->tm_wdown[bn_index(bn)];
+    p.nseg = 6;
+    split_segments(p, 0, 0, 0, d);
+    p.M = T;
+    p.M_rows = T;
+    p.n_tiles = l / bn;
+    p.tmOut = h->tm_hx;
+    p.split = l;
+    p.row_scale = h->r;
+    CK(launch_tc(p, EPI_DOWN3, bn, std::min(mt * p.n_tiles, h->sms), st));
   }
   mark(h, ST_ROUTER, st);
-  {  // s = sigmoid(h Wr^T + c)
-    SimtParams p = b;
-    p.A0 = (const float*)h->hx; p.lda0 = c.l; p.K0 = c.l; p.a_rows = T;
-    p.B0 = (const float*)h->w_r; p.ldb = c.l;
-    p.M = T; p.N = c.E;
-    p.out = h->s; p.ldo = c.E; p.col_bias = h->c;
-    CK(launch_simt<SE_ROUTER>(p, mt, st));
+  {  // s = sigmoid(h W_r^T + c), chunk by chunk over the three parts (the engine's split-router mode)
+    TcParams p = tc_base(h);
+    p.tmA[0] = p.tmA[1] = h->tm_hx;
+    const int bn = std::min(pick_bn_for(T, h->E_pad, h->sms, 64), 128);
+    p.tmB = h->tm_wr[bn_index(bn)];
+    const int nk = l / 64;
+    p.nseg = 3;
+    p.seg[0] = {0, 0, 0, nk};
+    p.seg[1] = {0, l, l, nk};
+    p.seg[2] = {0, 2 * l, 2 * l, nk};
+    p.M = T;
+    p.M_rows = T;
+    p.n_tiles = h->E_pad / bn;
+    p.tmOut = h->tm_s;
+    p.col_bias = h->c;
+    CK(launch_tc(p, EPI_ROUTER, bn, std::min(mt * p.n_tiles, h->sms), st));
   }
   mark(h, ST_K1, st);
+  h->launches += 4;
   int rc = route_from_scores(h, T, flags, pre, xv, st);
   if (rc) return rc;
   mark(h, ST_SHARED, st);
-  if (c.hs) {  // a_s = silu(r x Ws1'^T) * (r x Ws3'^T)
-    SimtParams p = b;
-    p.A0 = x; p.lda0 = c.d; p.K0 = c.d; p.a_rows = T;
-    p.B0 = (const float*)h->ws13; p.B1 = (const float*)h->ws3f; p.ldb = c.d;
-    p.M = T; p.N = c.hs;
-    p.out = (float*)h->a_s; p.ldo = c.hs; p.row_scale = h->r;
-    CK(launch_simt<SE_SWIGLU>(p, mt, st));
+  if (hs) {  // a_s = silu(r x Ws1'^T) * (r x Ws3'^T), stored as three parts
+    TcParams p = tc_base(h);
+    p.tmA[0] = p.tmA[1] = h->tm_x3;
+    const int bn = pick_bn_for(T, 2 * hs, h->sms, 128);
+    p.tmB = h->tm_ws13[bn_index(bn)];
+    p.nseg = 6;
+    split_segments(p, 0, 0, 0, d);
+    p.M = T;
+    p.M_rows = T;
+    p.n_tiles = 2 * hs / bn;
+    p.tmOut = h->tm_as;
+    p.split = hs;
+    p.row_scale = h->r;
+    CK(launch_tc(p, EPI_SWIGLU3, bn, std::min(mt * p.n_tiles, h->sms), st));
   }
-  const int gm = (T * c.k + 127) / 128 + c.E;
   mark(h, ST_EXPERT1, st);
-  {  // act = silu(A W1_e^T) * (A W3_e^T)
-    SimtParams p = b;
-    p.A0 = (const float*)h->a_perm; p.lda0 = c.l; p.K0 = c.l; p.a_rows = (int)h->rows_pad;
-    p.B0 = (const float*)h->w13; p.B1 = (const float*)h->w3f; p.ldb = c.l;
-    p.b_group_stride = (long long)c.h * c.l;
-    p.N = c.h; p.grouped = 1;
-    p.mtile_table = h->mtiles; p.num_mtiles = h->num_mtiles;
-    p.out = (float*)h->act; p.ldo = c.h;
-    CK(launch_simt<SE_SWIGLU>(p, gm, st));
+  {  // act = silu(A W1_e^T) * (A W3_e^T) over each expert's rows, stored as three parts
+    TcParams p = tc_base(h);
+    p.tmA[0] = p.tmA[1] = h->tm_aperm;
+    p.tmB = h->tm_w13;
+    p.nseg = 6;
+    split_segments(p, 0, 0, 0, l);
+    p.grouped = 1;
+    p.n_tiles = 2 * hh / h->bn_e1;
+    p.mtile_table = h->mtiles;
+    p.num_mtiles = h->num_mtiles;
+    p.b_rows_per_group = 2 * hh;
+    p.tmOut = h->tm_act;
+    p.split = hh;
+    p.trim = 1;
+    for (int i = 0; i < 3; ++i) {
+      p.tmA_part[i] = h->tm_aperm_part[i];
+      p.tmOut_part[i] = h->tm_act_part[i];
+    }
+    CK(launch_tc(p, EPI_SWIGLU3, h->bn_e1, h->sms, st));
   }
   mark(h, ST_EXPERT2, st);
-  {  // o = act W2_e^T
-    SimtParams p = b;
-    p.A0 = (const float*)h->act; p.lda0 = c.h; p.K0 = c.h; p.a_rows = (int)h->rows_pad;
-    p.B0 = (const float*)h->w2; p.ldb = c.h;
-    p.b_group_stride = (long long)c.l * c.h;
-    p.N = c.l; p.grouped = 1;
-    p.mtile_table = h->mtiles; p.num_mtiles = h->num_mtiles;
-    p.out = (float*)h->o; p.ldo = c.l;
-    CK(launch_simt<SE_STORE>(p, gm, st));
+  {  // o = act W2_e^T, fp32
+    TcParams p = tc_base(h);
+    p.tmA[0] = p.tmA[1] = h->tm_act;
+    p.tmB = h->tm_w2;
+    p.nseg = 6;
+    split_segments(p, 0, 0, 0, hh);
+    p.grouped = 1;
+    p.n_tiles = l / h->bn_e2;
+    p.mtile_table = h->mtiles;
+    p.num_mtiles = h->num_mtiles;
+    p.b_rows_per_group = l;
+    p.tmOut = h->tm_o;
+    p.trim = 1;
+    for (int i = 0; i < 3; ++i) {
+      p.tmA_part[i] = h->tm_act_part[i];
+      p.tmOut_part[i] = h->tm_o_part[i];
+    }
+    CK(launch_tc(p, EPI_F32, h->bn_e2, h->sms, st));
   }
   mark(h, ST_COMBINE, st);
-  CK(launch_combine((const float*)h->o, h->gates, h->prow, T, c.k, c.l, (float*)h->z, st));
+  CK(launch_combine((const float*)h->o, h->gates, h->prow, T, c.k, l, (float*)h->z, st));
+  CK(launch_k(split3_kernel, dim3(grid_1d((long long)T * l, 256)), dim3(256), 0, st, 1, (const float*)h->z,
+              (const float*)nullptr, T, l, (bf16*)h->z3, 3 * l, 0));
   mark(h, ST_UP, st);
-  {  // y = [z | a_s] [W_up | Ws2]^T
-    SimtParams p = b;
-    p.A0 = (const float*)h->z; p.lda0 = c.l; p.K0 = c.l;
-    p.A1 = (const float*)h->a_s; p.lda1 = c.hs; p.K1 = c.hs; p.a_rows = T;
-    p.B0 = (const float*)h->wy; p.ldb = c.l + c.hs;
-    p.M = T; p.N = c.d;
-    p.out = (float*)yv; p.ldo = c.d;
-    CK(launch_simt<SE_STORE>(p, mt, st));
+  {  // y = [z | a_s] [W_up | Ws2]^T: six part products of z, then six of a_s
+    TcParams p = tc_base(h);
+    p.tmA[0] = h->tm_z3;
+    p.tmA[1] = hs ? h->tm_as : h->tm_z3;
+    p.nseg = hs ? 12 : 6;
+    split_segments(p, 0, 0, 0, l);
+    if (hs) split_segments(p, 6, 1, 3 * l, hs);
+    p.M = T;
+    p.M_rows = T;
+    if (!make_map_f32(&p.tmOut, yv, T, d, d, 128)) return LMOE_EINVAL;
+    const int bn = pick_bn_for(T, d, h->sms, 64);
+    p.tmB = h->tm_wy[bn_index(bn)];
+    p.n_tiles = d / bn;
+    CK(launch_tc(p, EPI_F32, bn, std::min(mt * p.n_tiles, h->sms), st));
   }
-  h->launches += 4 + (c.hs ? 2 : 1) + 2;
+  h->launches += (hs ? 1 : 0) + 5;
   return join_update(h, flags, st);
 }
 
@@ -1000,41 +1137,47 @@ int repack(lmoe_handle* h, const lmoe_weights* w, cudaStream_t st) {
     else
       fold_gain_split_kernel<<<grid_1d(l * d, TPB), TPB, 0, st>>>((const bf16*)w->w_down, g, l, d,
                                                                   (bf16*)h->w_down);
-    split3_kernel<<<grid_1d(E * l, TPB), TPB, 0, st>>>(w->w_router, E, l, (bf16*)h->w_r);
+    split3_kernel<<<grid_1d(E * l, TPB), TPB, 0, st>>>(w->w_router, nullptr, (int)E, (int)l, (bf16*)h->w_r,
+                                                       (int)(3 * l), 0);
     if (hs)
       interleave_kernel<bf16><<<grid_1d(hs * d, TPB), TPB, 0, st>>>((const bf16*)w->ws1, (const bf16*)w->ws3, g, 1,
                                                                     hs, d, (bf16*)h->ws13);
-    if (h->xgemm)
-      pair_pack_kernel<bf16><<<grid_1d(2 * E * hh * l, TPB), TPB, 0, st>>>((const bf16*)w->w1, (const bf16*)w->w3,
-                                                                          E, hh, l, (bf16*)h->w13);
-    else
+    if (h->q8) {
+      mx_quant_w13_kernel<<<grid_1d(2 * E * hh * l / 32, TPB), TPB, 0, st>>>(
+          (const bf16*)w->w1, (const bf16*)w->w3, (int)E, (int)hh, (int)l, h->w13q, h->w13sf);
+      mx_quant_rows_kernel<<<grid_1d(E * l * hh / 32, TPB), TPB, 0, st>>>((const bf16*)w->w2, 1, E * l, (int)hh,
+                                                                         h->w2q, h->w2sf, 1);
+    } else
       interleave_kernel<bf16><<<grid_1d(E * hh * l, TPB), TPB, 0, st>>>((const bf16*)w->w1, (const bf16*)w->w3,
                                                                         nullptr, E, hh, l, (bf16*)h->w13);
-    CK(cudaMemcpyAsync(h->w2, w->w2, E * l * hh * 2, cudaMemcpyDeviceToDevice, st));
+    if (!h->q8) CK(cudaMemcpyAsync(h->w2, w->w2, E * l * hh * 2, cudaMemcpyDeviceToDevice, st));
     fold_gain_kernel<bf16><<<grid_1d(d * l, TPB), TPB, 0, st>>>((const bf16*)w->w_up, nullptr, d, l,
                                                                 (bf16*)h->wy, l + hs, 0);
     if (hs)
       fold_gain_kernel<bf16><<<grid_1d(d * hs, TPB), TPB, 0, st>>>((const bf16*)w->ws2, nullptr, d, hs,
                                                                    (bf16*)h->wy, l + hs, l);
   } else {
+    // every GEMM operand as three bf16 parts along K (the gain folded into W_down and Ws1/Ws3 in
+    // fp32 first); the router weights padded to E_pad rows of zeros
     const float* g = (const float*)w->rms_gain;
-    fold_gain_kernel<float><<<grid_1d(l * d, TPB), TPB, 0, st>>>((const float*)w->w_down, g, l, d,
-                                                                 (float*)h->w_down, d, 0);
-    CK(cudaMemcpyAsync(h->w_r, w->w_router, E * l * 4, cudaMemcpyDeviceToDevice, st));
-    if (hs) {
-      fold_gain_kernel<float><<<grid_1d(hs * d, TPB), TPB, 0, st>>>((const float*)w->ws1, g, hs, d,
-                                                                    (float*)h->ws13, d, 0);
-      fold_gain_kernel<float><<<grid_1d(hs * d, TPB), TPB, 0, st>>>((const float*)w->ws3, g, hs, d,
-                                                                    (float*)h->ws3f, d, 0);
-    }
-    CK(cudaMemcpyAsync(h->w13, w->w1, E * hh * l * 4, cudaMemcpyDeviceToDevice, st));
-    CK(cudaMemcpyAsync(h->w3f, w->w3, E * hh * l * 4, cudaMemcpyDeviceToDevice, st));
-    CK(cudaMemcpyAsync(h->w2, w->w2, E * l * hh * 4, cudaMemcpyDeviceToDevice, st));
-    fold_gain_kernel<float><<<grid_1d(d * l, TPB), TPB, 0, st>>>((const float*)w->w_up, nullptr, d, l,
-                                                                 (float*)h->wy, l + hs, 0);
+    split3_kernel<<<grid_1d(l * d, TPB), TPB, 0, st>>>((const float*)w->w_down, g, (int)l, (int)d, (bf16*)h->w_down,
+                                                       (int)(3 * d), 0);
+    CK(cudaMemsetAsync(h->w_r, 0, (size_t)h->E_pad * 3 * l * 2, st));
+    split3_kernel<<<grid_1d(E * l, TPB), TPB, 0, st>>>(w->w_router, nullptr, (int)E, (int)l, (bf16*)h->w_r,
+                                                       (int)(3 * l), 0);
     if (hs)
-      fold_gain_kernel<float><<<grid_1d(d * hs, TPB), TPB, 0, st>>>((const float*)w->ws2, nullptr, d, hs,
-                                                                    (float*)h->wy, l + hs, l);
+      interleave_split3_kernel<<<grid_1d(hs * d, TPB), TPB, 0, st>>>((const float*)w->ws1, (const float*)w->ws3, g, 1,
+                                                                     (int)hs, (int)d, (bf16*)h->ws13);
+    interleave_split3_kernel<<<grid_1d(E * hh * l, TPB), TPB, 0, st>>>((const float*)w->w1, (const float*)w->w3,
+                                                                       nullptr, (int)E, (int)hh, (int)l,
+                                                                       (bf16*)h->w13);
+    split3_kernel<<<grid_1d(E * l * hh, TPB), TPB, 0, st>>>((const float*)w->w2, nullptr, (int)(E * l), (int)hh,
+                                                            (bf16*)h->w2, (int)(3 * hh), 0);
+    split3_kernel<<<grid_1d(d * l, TPB), TPB, 0, st>>>((const float*)w->w_up, nullptr, (int)d, (int)l, (bf16*)h->wy,
+                                                       (int)(3 * (l + hs)), 0);
+    if (hs)
+      split3_kernel<<<grid_1d(d * hs, TPB), TPB, 0, st>>>((const float*)w->ws2, nullptr, (int)d, (int)hs,
+                                                          (bf16*)h->wy, (int)(3 * (l + hs)), (int)(3 * l));
   }
   {  // W_comb = W_r (W_down g) in fp64, for the exact decision of ambiguous top-k choices
     const dim3 grid((unsigned)((d + 255) / 256), (unsigned)E);
@@ -1047,10 +1190,8 @@ int repack(lmoe_handle* h, const lmoe_weights* w, cudaStream_t st) {
                                                          (const float*)w->rms_gain, (int)l, (int)d, h->wc);
   }
   CK(cudaGetLastError());
-  if (w->router_bias)
-    CK(cudaMemcpyAsync(h->c, w->router_bias, E * 4, cudaMemcpyDeviceToDevice, st));
-  else
-    CK(cudaMemsetAsync(h->c, 0, E * 4, st));
+  CK(cudaMemsetAsync(h->c, 0, (size_t)h->E_pad * 4, st));
+  if (w->router_bias) CK(cudaMemcpyAsync(h->c, w->router_bias, E * 4, cudaMemcpyDeviceToDevice, st));
   return LMOE_OK;
 }
 
@@ -1141,8 +1282,8 @@ static void size_handle(lmoe_handle* h, const lmoe_config* cfg) {
   h->max_mtiles = (int)(((long long)cfg->max_tokens * cfg->k + kTileRows - 1) / kTileRows) + cfg->E;
   h->ld_bins = (cfg->max_tokens + 31) / 32 * 32;
   h->rows_pad = (long long)cfg->max_tokens * cfg->k + (long long)kTileRows * cfg->E;
-  h->max_ttiles = (int)(((long long)cfg->max_tokens * cfg->k + kTokTile - 1) / kTokTile) + cfg->E;
-  h->xgemm = LMOE_PAIR_EXPERTS && cfg->dtype == LMOE_BF16 && cfg->h % 128 == 0 && cfg->l % 256 == 0;
+  h->q8 = cfg->experts == LMOE_EXPERTS_MXFP8;
+  h->E_pad = h->bf ? cfg->E : (cfg->E + 63) / 64 * 64;
 }
 
 int lmoe_workspace_bytes(const lmoe_config* cfg, size_t* bytes) {
@@ -1198,7 +1339,7 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, void* stream, lmo
   if (!rc && cudaMemsetAsync(h->load, 0, (size_t)cfg->E * 8, st) != cudaSuccess) rc = LMOE_ECUDA;
   if (!rc && cudaMemsetAsync(h->status, 0, 4, st) != cudaSuccess) rc = LMOE_ECUDA;
   if (!rc && cudaMemsetAsync(h->qb_done, 0, 4, st) != cudaSuccess) rc = LMOE_ECUDA;
-  if (!rc && h->bf) rc = build_maps(h);
+  if (!rc) rc = h->bf ? build_maps(h) : build_maps_f32(h);
   if (!rc && cudaStreamCreateWithFlags(&h->cap, cudaStreamNonBlocking) != cudaSuccess) rc = LMOE_ECUDA;
   if (!rc && cudaStreamCreateWithFlags(&h->cp_in, cudaStreamNonBlocking) != cudaSuccess) rc = LMOE_ECUDA;
   if (!rc && cudaStreamCreateWithFlags(&h->cp_out, cudaStreamNonBlocking) != cudaSuccess) rc = LMOE_ECUDA;
@@ -1596,7 +1737,7 @@ int lmoe_route_noalloc(const float* scores, const float* bias, int32_t T, int32_
   CK(launch_topk(ta, st));
   const int nblk = (T + kTokBlock - 1) / kTokBlock;
   plan_kernel<<<(E + 31) / 32, 1024, 0, st>>>(counts32, counts, blkcnt, nblk, E, offsets, delta, blkbase, tiles,
-                                               ntiles, nullptr, nullptr, nullptr);
+                                               ntiles, nullptr);
   CK(cudaGetLastError());
   const int pairs = T * k;
   gather_kernel<float><<<(pairs + 8 * kGatherPairs - 1) / (8 * kGatherPairs), 256, 0, st>>>(

@@ -8,16 +8,23 @@
 // products by its two operands' scales and accumulates in fp32 (one instruction of shape
 // 128 x N x 32 per scale block).
 //
+// Scale layout.  The scales of a 128-row tile and a 128-element K-block (4 blocks of 32) form a
+// 512-byte atom: byte 16 i + 4 j + b is the scale of row i + 32 j, 32-element block b
+// (i < 32, j < 4, b < 4).  In global memory the atoms of a matrix are stored tile-major, then by
+// K-block: atom (t, kb) at byte ((t * nkb) + kb) * 512.  A tcgen05.cp of shape 32x128b.warpx4
+// copies an atom into four TMEM columns of all four lane quarters (lane 32 q + i, column j, byte
+// b), where the MMA reads the scale of row m from column m / 32, lane m % 32 and byte sf_id.
+//
 // Grouped like the engine's bf16 grouped mode: M-tiles of 128 gathered token rows (every expert's
 // rows start on a multiple of 128; an expert's last tile loads only its valid rows, rounded up to
 // 32), N-tiles of 128 weight rows, K-blocks of 128 elements (one 128-byte swizzle atom, four MMAs).
-// CTA = 14 warps: warp 0 issues TMA loads into a 6-stage ring (16 KB A + 16 KB B per stage), warp
-// 1 issues the MMAs into one of two TMEM accumulators, warps 2-9 drain the other accumulator,
-// warps 10-13 write each tile's scale bytes (A rows and B rows, all of K) into one of two TMEM
-// scale buffers with tcgen05.st before the MMA issuer starts the tile.
+// CTA = 10 warps: warp 0 issues TMA loads of the two operand tiles and bulk copies of their two
+// scale atoms into a 6-stage ring, warp 1 copies each stage's atoms into TMEM (two buffers,
+// alternating by K-block, at 32-column-aligned addresses) and issues the four MMAs that read
+// them, warps 2-9 drain the other accumulator.
 //  Q8_SWIGLU (gate/up, N columns interleaved in groups of 64 gate + 64 linear): act = silu(g) * u
 //    for 32 features per thread, quantised to MXFP8 right there (the thread holds exactly one
-//    32-element block of its row) and stored as 32 element bytes and one scale byte.
+//    32-element block of its row) and stored as 32 element bytes and one scale byte (atom layout).
 //  Q8_BF16 (down): out bf16.
 // Every wait is bounded as in the engine.
 #pragma once
@@ -34,26 +41,31 @@ struct Q8Params {
   CUtensorMap tmA;          // A elements [rows, K] u8, box 128 x 128
   CUtensorMap tmA_part[3];  // the same with boxes of 32, 64, 96 rows
   CUtensorMap tmB;          // B elements [groups * b_rows, K] u8, box 128 x 128
-  const uint8_t* a_sf;      // [rows, K / 32] scale bytes
-  const uint8_t* b_sf;      // [groups * b_rows, K / 32]
+  const uint8_t* a_sf;      // A scale atoms (rows / 128 tiles x K / 128 blocks x 512 bytes)
+  const uint8_t* b_sf;      // B scale atoms
   const int2* mtile_table;  // (expert | valid rows << 16, first row)
   const int* num_mtiles;
   int n_tiles;              // N / 128
   int b_rows;               // B rows per expert
   int nkb;                  // K / 128 (at most 32)
   uint8_t* out_q;           // Q8_SWIGLU: act elements [rows, N / 2]
-  uint8_t* out_sf;          //            act scales [rows, N / 64]
+  uint8_t* out_sf;          //            act scale atoms (K-blocks of N / 2)
   bf16* out_bf;             // Q8_BF16: [rows, N]
   int n_out;                // output columns of the whole GEMM (N, or N / 2 for SwiGLU)
   uint32_t* status;
 };
 
 constexpr int kQ8Stages = 6;
-constexpr int kQ8StageBytes = 32768;
+constexpr int kQ8StageBytes = 32768 + 1024;  // A tile, B tile, A scale atom, B scale atom
 constexpr int kQ8BarOffset = kQ8Stages * kQ8StageBytes;
 constexpr int kQ8SmemBytes = kQ8BarOffset + 256 + 1024;
-constexpr int kQ8Threads = 14 * 32;
-constexpr int kQ8SfCols = 32;  // TMEM columns of one operand's scales (K / 128 <= 32)
+constexpr int kQ8Threads = kTcThreads;
+
+// Byte offset of the scale of row r, 32-element block c (of K) in a matrix's atom layout with nkb
+// K-blocks of 128.
+__host__ __device__ __forceinline__ long long mx_atom_offset(long long r, int c, int nkb) {
+  return ((r >> 7) * nkb + (c >> 2)) * 512 + 16 * (r & 31) + 4 * ((r & 127) >> 5) + (c & 3);
+}
 
 // MXFP8 scale exponent of a block whose largest magnitude is amax: floor(log2 amax) - 8, clamped
 // to [-127, 127]; -127 for a zero block (or one below fp32's normal range).
@@ -104,10 +116,28 @@ __device__ __forceinline__ void tc_mma_mxf8(uint32_t d_tmem, uint64_t adesc, uin
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate));
 }
 
-__device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t v) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v));
+// Shared-memory descriptor of a 32-row x 16-byte matrix stored row after row, without swizzle:
+// core matrices of 8 rows x 16 bytes, 128 bytes apart.
+__device__ __forceinline__ uint64_t smem_desc_rows16(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)(128u >> 4) << 16;
+  d |= (uint64_t)(128u >> 4) << 32;
+  d |= (uint64_t)1u << 46;
+  return d;
 }
-__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// Copies a 512-byte scale atom from shared memory into TMEM columns [taddr, taddr + 4) of all four
+// lane quarters (ordered with this thread's later MMAs).
+__device__ __forceinline__ void tc_cp_atom(uint32_t taddr, uint32_t saddr) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(smem_desc_rows16(saddr)));
+}
+// Bulk copy (no tensor map) of `bytes` from global to shared memory, completing on `bar`.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
 
 template <int EPI>
 __global__ void __launch_bounds__(kQ8Threads, 1) q8_gemm_kernel(const __grid_constant__ Q8Params p) {
@@ -119,9 +149,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1) q8_gemm_kernel(const __grid_con
   uint64_t* empty = full + S;
   uint64_t* tfull = empty + S;
   uint64_t* tempty = tfull + 2;
-  uint64_t* sfull = tempty + 2;  // a tile's scales are in TMEM buffer i
-  uint64_t* sempty = sfull + 2;  // the MMAs that read buffer i have completed
-  uint64_t* drain = sempty + 2;
+  uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -134,8 +162,6 @@ __global__ void __launch_bounds__(kQ8Threads, 1) q8_gemm_kernel(const __grid_con
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], kEpiWarps);
-      mbar_init(&sfull[i], 4);
-      mbar_init(&sempty[i], 1);
     }
     mbar_init(drain, 1);
     *abort = 0;
@@ -152,12 +178,12 @@ __global__ void __launch_bounds__(kQ8Threads, 1) q8_gemm_kernel(const __grid_con
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  // TMEM columns: accumulators [0, 256); scale buffer i: A at 256 + 64 i, B at 256 + 64 i + 32
+  // TMEM columns: accumulators [0, 256); scale buffer i (by K-block parity): A at 256 + 64 i,
+  // B at 288 + 64 i (four columns each, at 32-column-aligned addresses)
   const uint32_t sf_base = tmem_base + 256;
   pdl_wait();
   pdl_trigger();
   const int num_tiles = *p.num_mtiles * p.n_tiles;
-  const int ksf = p.nkb * 4;  // scale bytes per row
 
   if (warp == 0) {
     if (lane == 0) {
@@ -179,9 +205,11 @@ __global__ void __launch_bounds__(kQ8Threads, 1) q8_gemm_kernel(const __grid_con
             break;
           }
           uint8_t* a_dst = smem + stage * kQ8StageBytes;
-          mbar_expect_tx(&full[stage], (uint32_t)(q * 32 * 128 + 16384));
+          mbar_expect_tx(&full[stage], (uint32_t)(q * 32 * 128 + 16384 + 1024));
           tma_load_2d(a_dst, amap, &full[stage], kb * 128, row0);
           tma_load_2d_hint(a_dst + 16384, &p.tmB, &full[stage], kb * 128, brow0, pol_first);
+          bulk_load(a_dst + 32768, p.a_sf + ((size_t)(row0 >> 7) * p.nkb + kb) * 512, 512, &full[stage]);
+          bulk_load(a_dst + 32768 + 512, p.b_sf + ((size_t)(brow0 >> 7) * p.nkb + kb) * 512, 512, &full[stage]);
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == S) {
@@ -204,13 +232,12 @@ __global__ void __launch_bounds__(kQ8Threads, 1) q8_gemm_kernel(const __grid_con
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++it) {
         const int acc = it & 1;
         const uint32_t par = (it >> 1) & 1;
-        if (!mbar_wait(&tempty[acc], par ^ 1u, abort, p.status) || !mbar_wait(&sfull[acc], par, abort, p.status)) {
+        if (!mbar_wait(&tempty[acc], par ^ 1u, abort, p.status)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * 128;
-        const uint32_t sfa = sf_base + acc * 64, sfb = sfa + 32;
         for (int kb = 0; kb < p.nkb; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort, p.status)) {
             ok = false;
@@ -219,57 +246,26 @@ __global__ void __launch_bounds__(kQ8Threads, 1) q8_gemm_kernel(const __grid_con
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + stage * kQ8StageBytes);
           const uint32_t b_addr = a_addr + 16384;
+          // this K-block's scale atoms into the scale buffer of its parity, then its four MMAs
+          const uint32_t sfa = sf_base + (kb & 1) * 64, sfb = sfa + 32;
+          tc_cp_atom(sfa, a_addr + 32768);
+          tc_cp_atom(sfb, a_addr + 32768 + 512);
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             tc_mma_mxf8(d_tmem, smem_desc_sw128(a_addr + k * 32), smem_desc_sw128(b_addr + k * 32),
-                        idesc_mxf8(128, k, k), sfa + kb, sfb + kb, (kb | k) != 0);
+                        idesc_mxf8(128, k, k), sfa, sfb, (kb | k) != 0);
           tc_commit(&empty[stage]);
           if (++stage == S) {
             stage = 0;
             phase ^= 1u;
           }
         }
-        if (ok) {
-          tc_commit(&tfull[acc]);
-          tc_commit(&sempty[acc]);
-        }
+        if (ok) tc_commit(&tfull[acc]);
       }
       if (!ok) {
         tc_commit(drain);
         mbar_drain(drain, 0);
       }
-    }
-  } else if (warp >= 10) {
-    // ---------------- scale writers: lane quarter warp % 4, one row of A and one of B per thread
-    const int wq = warp & 3;
-    int it = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++it) {
-      const int mt = tile / p.n_tiles, nt = tile - mt * p.n_tiles;
-      const int2 e_r = p.mtile_table[mt];
-      const int r = wq * 32 + lane;
-      const uint32_t* arow = reinterpret_cast<const uint32_t*>(p.a_sf + (size_t)(e_r.y + r) * ksf);
-      const uint32_t* brow =
-          reinterpret_cast<const uint32_t*>(p.b_sf + (size_t)((e_r.x & 0xFFFF) * p.b_rows + nt * 128 + r) * ksf);
-      const int buf = it & 1;
-      ok = mbar_wait(&sempty[buf], ((it >> 1) & 1) ^ 1u, abort, p.status);
-      __syncwarp();
-      if (__any_sync(0xffffffffu, !ok)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t lanes = (uint32_t)(wq * 32) << 16;
-      const uint32_t ta = sf_base + buf * 64 + lanes, tb = ta + 32;
-      // word c of a row holds the scales of K-block c (bytes 4c .. 4c + 3 of the row)
-      for (int c = 0; c < p.nkb; ++c) {
-        tmem_st1(ta + c, arow[c]);
-        tmem_st1(tb + c, brow[c]);
-      }
-      tc_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sfull[buf]);
     }
   } else {
     // ---------------- epilogue warps 2..9: TMEM lane quarter (warp % 4), column half (warp - 2) / 4
@@ -305,7 +301,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1) q8_gemm_kernel(const __grid_con
         uint4* dst = reinterpret_cast<uint4*>(p.out_q + (size_t)row * p.n_out + col);
         dst[0] = make_uint4(qw[0], qw[1], qw[2], qw[3]);
         dst[1] = make_uint4(qw[4], qw[5], qw[6], qw[7]);
-        p.out_sf[(size_t)row * (p.n_out / 32) + col / 32] = (uint8_t)sfb;
+        p.out_sf[mx_atom_offset(row, col >> 5, p.n_out >> 7)] = (uint8_t)sfb;
       } else {
         // columns [64 half, +64) of this N-tile, bf16
 #pragma unroll 1
@@ -337,11 +333,11 @@ __global__ void __launch_bounds__(kQ8Threads, 1) q8_gemm_kernel(const __grid_con
 // --------------------------------------------------------------------------- quantisation kernels
 // MXFP8 of rows of a matrix along its columns (the GEMM's K): one thread per 32-element block.
 // Source: bf16 [rows, cols] (parts == 1), or the hi | mid | lo bf16 parts of fp32 values
-// ([rows, 3 cols], parts == 3), summed back to fp32 first.  out: [rows, cols] elements and
-// [rows, cols / 32] scale bytes.
+// ([rows, 3 cols], parts == 3), summed back to fp32 first.  out: [rows, cols] elements; scale
+// bytes row after row ([rows, cols / 32], atom == 0) or in the atom layout (atom == 1).
 __global__ void __launch_bounds__(256) mx_quant_rows_kernel(const bf16* __restrict__ src, int parts, long long rows,
                                                             int cols, uint8_t* __restrict__ out,
-                                                            uint8_t* __restrict__ out_sf) {
+                                                            uint8_t* __restrict__ out_sf, int atom) {
   pdl_wait();
   pdl_trigger();
   const int nb = cols / 32;
@@ -375,12 +371,44 @@ __global__ void __launch_bounds__(256) mx_quant_rows_kernel(const bf16* __restri
     uint4* d = reinterpret_cast<uint4*>(out + r * cols + b * 32);
     d[0] = make_uint4(q[0], q[1], q[2], q[3]);
     d[1] = make_uint4(q[4], q[5], q[6], q[7]);
-    out_sf[r * nb + b] = (uint8_t)sf;
+    out_sf[atom ? mx_atom_offset(r, b, cols / 128) : r * nb + b] = (uint8_t)sf;
   }
 }
 
-// Copies each (token, slot) pair's MXFP8 row (cols elements, cols / 32 scale bytes) into row
-// prow[pair] of the padded expert layout; one warp per pair.
+// MXFP8 of the routed experts' gate and linear projections, rows interleaved in groups of 64 as
+// the SwiGLU epilogue reads them (out row (j / 64) 128 + j % 64 = w1[j], 64 further = w3[j], per
+// expert), along l, scales in the atom layout; one thread per 32-element block.
+__global__ void __launch_bounds__(256) mx_quant_w13_kernel(const bf16* __restrict__ w1, const bf16* __restrict__ w3,
+                                                           int E, int h, int l, uint8_t* __restrict__ out,
+                                                           uint8_t* __restrict__ out_sf) {
+  const int nb = l / 32;
+  const long long n = (long long)E * 2 * h * nb;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const long long orow = i / nb;
+    const int b = (int)(i - orow * nb);
+    const int e = (int)(orow / (2 * h)), r = (int)(orow - (long long)e * 2 * h);
+    const int within = r & 127, j = (r >> 7) * 64 + (within & 63);
+    const bf16* s = (within < 64 ? w1 : w3) + ((long long)e * h + j) * l + b * 32;
+    float v[32];
+#pragma unroll
+    for (int q = 0; q < 32; q += 8) {
+      const uint4 hv = *reinterpret_cast<const uint4*>(s + q);
+      const bf16* he = reinterpret_cast<const bf16*>(&hv);
+#pragma unroll
+      for (int t = 0; t < 8; ++t) v[q + t] = __bfloat162float(he[t]);
+    }
+    uint32_t qw[8];
+    const uint32_t sf = mx_quant32(v, qw);
+    uint4* d = reinterpret_cast<uint4*>(out + orow * l + b * 32);
+    d[0] = make_uint4(qw[0], qw[1], qw[2], qw[3]);
+    d[1] = make_uint4(qw[4], qw[5], qw[6], qw[7]);
+    out_sf[mx_atom_offset(orow, b, l / 128)] = (uint8_t)sf;
+  }
+}
+
+// Copies each (token, slot) pair's MXFP8 row (cols elements, cols / 32 scale bytes stored row
+// after row) into row prow[pair] of the padded expert layout, its scales into the atom layout;
+// one warp per pair.
 __global__ void __launch_bounds__(256) gather_q8_kernel(const uint8_t* __restrict__ src, const uint8_t* __restrict__ src_sf,
                                                         int cols, const int* __restrict__ prow, int npairs, int k,
                                                         uint8_t* __restrict__ dst, uint8_t* __restrict__ dst_sf) {
@@ -392,9 +420,8 @@ __global__ void __launch_bounds__(256) gather_q8_kernel(const uint8_t* __restric
   const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)t * cols);
   uint4* d = reinterpret_cast<uint4*>(dst + (size_t)r * cols);
   for (int v = lane; v < cols / 16; v += 32) d[v] = s[v];
-  const uint32_t* ss = reinterpret_cast<const uint32_t*>(src_sf + (size_t)t * (cols / 32));
-  uint32_t* ds = reinterpret_cast<uint32_t*>(dst_sf + (size_t)r * (cols / 32));
-  for (int v = lane; v < cols / 128; v += 32) ds[v] = ss[v];
+  const uint8_t* ss = src_sf + (size_t)t * (cols / 32);
+  for (int c = lane; c < cols / 32; c += 32) dst_sf[mx_atom_offset(r, c, cols / 128)] = ss[c];
 }
 
 }  // namespace lmoe

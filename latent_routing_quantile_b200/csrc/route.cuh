@@ -12,7 +12,6 @@ namespace lmoe {
 constexpr int kTokBlock = 32;      // tokens per routing block: one rank-mask word per expert
 constexpr int kCountCopies = 32;   // per-expert counts are summed into this many copies (block % 32)
 constexpr int kTileRows = 128;     // rows per grouped-GEMM M-tile
-constexpr int kTokTile = 256;      // tokens per tile of the pair expert GEMMs
 constexpr unsigned kFull = 0xffffffffu;
 
 // --------------------------------------------------------------------------- RMSNorm
@@ -219,24 +218,50 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 
       float u_prev = 0.f, u_k1 = 0.f, my_u = 0.f;
       bool amb = false, odd = false;  // odd: a candidate without a numeric score
       int nc = 0, lim = k;
-      for (int i = 0; i < lim; ++i) {
-        uint32_t bk = 0u;
-        int bjx = 0;
+      // each lane keeps its best remaining key h1 (slot j1) and, while hv, the next one h2 (slot
+      // j2); a round takes the warp's best h1 (ties to the lower expert), and the lane it came from
+      // moves up its second, re-scanning its keys (minus the taken ones, bits of tk) only when the
+      // second was used up already
+      uint32_t h1 = 0u, h2 = 0u, tk = 0u;
+      int j1 = 0, j2 = 0;
+      bool hv = true;
+      auto best_two = [&]() {
+        h1 = 0u;
+        h2 = 0u;
+        j1 = 0;
+        j2 = 0;
 #pragma unroll
         for (int j = 0; j < NJ; ++j) {
-          if (key[j] > bk) {
-            bk = key[j];
-            bjx = j;
+          const uint32_t kj = ((tk >> j) & 1u) ? 0u : key[j];
+          if (kj > h1) {
+            h2 = h1;
+            j2 = j1;
+            h1 = kj;
+            j1 = j;
+          } else if (kj > h2) {
+            h2 = kj;
+            j2 = j;
           }
         }
-        const uint32_t wmax = __reduce_max_sync(kFull, bk);
+        hv = true;
+      };
+      best_two();
+      for (int i = 0; i < lim; ++i) {
+        const uint32_t wmax = __reduce_max_sync(kFull, h1);
         if (i >= k) {  // an extra candidate: only within tau of the k-th, and only a number
           if (wmax < 2u || !(key_value(wmax) >= u_k1 - rf.tau)) break;
         }
-        const uint32_t emin = __reduce_min_sync(kFull, bk == wmax ? (uint32_t)(bjx * 32 + lane) : 0xffffffffu);
-#pragma unroll
-        for (int j = 0; j < NJ; ++j)
-          if ((uint32_t)(j * 32 + lane) == emin) key[j] = 0u;
+        const uint32_t emin = __reduce_min_sync(kFull, h1 == wmax ? (uint32_t)(j1 * 32 + lane) : 0xffffffffu);
+        if ((emin & 31u) == (uint32_t)lane) {  // this lane's best was taken
+          tk |= 1u << j1;
+          if (hv) {
+            h1 = h2;
+            j1 = j2;
+            hv = false;
+          } else {
+            best_two();
+          }
+        }
         if (lane == i) my_sel = (int)emin;
         if (rf.x) {
           const float ui = wmax >= 2u ? key_value(wmax) : 0.f;
@@ -245,10 +270,7 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 
           if (i > 0 && wmax >= 2u && u_prev - ui < rf.tau) amb = true;
           if (i == k - 1) {
             u_k1 = ui;
-            uint32_t nk = 0u;  // best remaining key
-#pragma unroll
-            for (int j = 0; j < NJ; ++j) nk = max(nk, key[j]);
-            nk = __reduce_max_sync(kFull, nk);
+            const uint32_t nk = __reduce_max_sync(kFull, h1);  // best remaining key
             if (nk >= 2u && ui - key_value(nk) < rf.tau) amb = true;
             if (amb) lim = kmax;
           }
@@ -263,10 +285,7 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 
         // overflow: the list is full and the next expert is still within tau of the k-th
         bool ovf = false;
         if (nc == kmax && kmax < E) {
-          uint32_t nk = 0u;
-#pragma unroll
-          for (int j = 0; j < NJ; ++j) nk = max(nk, key[j]);
-          nk = __reduce_max_sync(kFull, nk);
+          const uint32_t nk = __reduce_max_sync(kFull, h1);
           ovf = nk >= 2u && key_value(nk) >= u_k1 - rf.tau;
         }
         if (ovf) {
@@ -575,8 +594,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ coun
                                                     const int* __restrict__ blkcnt, int nblk, int E,
                                                     int* __restrict__ offsets, int* __restrict__ pad_delta,
                                                     int* __restrict__ blkbase, int2* __restrict__ mtiles,
-                                                    int* __restrict__ num_mtiles, long long* __restrict__ load,
-                                                    int4* __restrict__ ttiles, int* __restrict__ num_ttiles) {
+                                                    int* __restrict__ num_mtiles, long long* __restrict__ load) {
   __shared__ int sh[32];
   __shared__ int s_off[1024];
   __shared__ int part[32][33];
@@ -610,16 +628,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ coun
     for (int j = 0; j < mt; ++j)
       mtiles[mt_start + j] = make_int2(tid | (min(kTileRows, c - j * kTileRows) << 16), poff + j * kTileRows);
     if (tid == 0) *num_mtiles = mt_total;
-    if (ttiles) {
-      // token tiles of the pair expert GEMMs: up to kTokTile tokens of one expert each,
-      // (expert, first row in the padded layout, valid tokens)
-      const int nt = (c + kTokTile - 1) / kTokTile;
-      int nt_total;
-      const int nt_start = block_exclusive_scan_1024(nt, sh, &nt_total);
-      for (int j = 0; j < nt; ++j)
-        ttiles[nt_start + j] = make_int4(tid, poff + j * kTokTile, min(kTokTile, c - j * kTokTile), 0);
-      if (tid == 0) *num_ttiles = nt_total;
-    }
+
   }
   __syncthreads();
   const int tx = tid & 31, ty = tid >> 5;
@@ -1027,41 +1036,55 @@ __global__ void interleave_kernel(const T* __restrict__ w1, const T* __restrict_
   }
 }
 
-// Gate (w1) and linear (w3) rows of `groups` experts [groups, rows, cols] in the order of the pair
-// expert GEMM: in each 256-row slice s, CTA half r, row 32q + j holds feature
-// 128 s + 64 r + 16 q + (j & 15), from w1 when j < 16 and from w3 otherwise.
-template <typename T>
-__global__ void pair_pack_kernel(const T* __restrict__ w1, const T* __restrict__ w3, int groups, int rows, int cols,
-                                 T* __restrict__ out) {
-  const long long n = (long long)groups * 2 * rows * cols;
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
-       i += (long long)gridDim.x * blockDim.x) {
-    const long long rc = 2LL * rows * cols;
-    const int grp = (int)(i / rc);
-    const long long rem = i - grp * rc;
-    const int orow = (int)(rem / cols), c = (int)(rem - (long long)orow * cols);
-    const int sl = orow >> 8, r = (orow >> 7) & 1, q = (orow >> 5) & 3, j = orow & 31;
-    const int f = sl * 128 + r * 64 + q * 16 + (j & 15);
-    const T* src = j < 16 ? w1 : w3;
-    out[i] = src[((long long)grp * rows + f) * cols + c];
-  }
-}
-
-// fp32 router weights as three bf16 parts [hi | mid | lo] per row (sum exact to 24 bits).
-__global__ void split3_kernel(const float* __restrict__ w, int rows, int cols, bf16* __restrict__ out) {
+// fp32 values as three bf16 parts hi, mid, lo (hi = bf16(v), mid = bf16(v - hi), lo = bf16(v - hi
+// - mid); their sum is v to fp32's 24 bits): out[r, col_off + part * cols + c] for v = g[c] w[r, c]
+// (g = null: v = w[r, c]; the product rounded to fp32 once), ld_out elements per output row.
+__global__ void split3_kernel(const float* __restrict__ w, const float* __restrict__ g, int rows, int cols,
+                              bf16* __restrict__ out, int ld_out, int col_off) {
+  pdl_wait();
+  pdl_trigger();
   const long long n = (long long)rows * cols;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
        i += (long long)gridDim.x * blockDim.x) {
     const int r = (int)(i / cols), c = (int)(i - (long long)r * cols);
-    const float v = w[i];
+    const float v = g ? g[c] * w[i] : w[i];
     const bf16 hi = __float2bfloat16_rn(v);
     const float r1 = v - __bfloat162float(hi);
     const bf16 mid = __float2bfloat16_rn(r1);
     const bf16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
-    bf16* o = out + (long long)r * 3 * cols + c;
+    bf16* o = out + (long long)r * ld_out + col_off + c;
     o[0] = hi;
     o[cols] = mid;
     o[2 * cols] = lo;
+  }
+}
+
+// Gate (w1) and linear (w3) rows of `groups` fp32 matrices [groups, rows, cols] interleaved in
+// blocks of 64 as interleave_kernel does, each row (times the gain g, when given) split into
+// three bf16 parts along cols: out [groups * 2 rows, 3 cols].
+__global__ void interleave_split3_kernel(const float* __restrict__ w1, const float* __restrict__ w3,
+                                         const float* __restrict__ g, int groups, int rows, int cols,
+                                         bf16* __restrict__ out) {
+  const long long n = (long long)groups * rows * cols;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long rc = (long long)rows * cols;
+    const int grp = (int)(i / rc);
+    const long long rem = i - grp * rc;
+    const int r = (int)(rem / cols), c = (int)(rem - (long long)r * cols);
+    const long long orow = (long long)grp * 2 * rows + (r / 64) * 128 + (r % 64);
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {
+      const float v = (g ? g[c] : 1.f) * (which ? w3[i] : w1[i]);
+      const bf16 hi = __float2bfloat16_rn(v);
+      const float r1 = v - __bfloat162float(hi);
+      const bf16 mid = __float2bfloat16_rn(r1);
+      const bf16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+      bf16* o = out + (orow + which * 64) * 3 * cols + c;
+      o[0] = hi;
+      o[cols] = mid;
+      o[2 * cols] = lo;
+    }
   }
 }
 

@@ -20,9 +20,12 @@
 // 128 rows; rows past the load hold stale shared memory, and only their own output rows, which
 // are never stored, depend on them.
 //
-// K is described by up to 6 segments, each naming which A tensor map and which A and B columns
+// K is described by up to 12 segments, each naming which A tensor map and which A and B columns
 // its k-blocks read; this expresses concatenated-K products ([z | a_s] [W_up | Ws2]^T) without
-// copying operands.
+// copying operands, and the split-precision products of the fp32 layer: an fp32 operand is held
+// as three bf16 parts [hi | mid | lo] along K (hi + mid + lo = the value to fp32's 24 bits) and
+// A B^T is the sum of the six significant part products (lo lo, mid lo and lo mid fall below
+// fp32's rounding), one segment each, all accumulated in fp32 in TMEM.
 //
 // EPI_ROUTER (the split-precision router, not paired) reads three segments, the hi, mid and lo
 // parts of h and of the router weights, chunk by chunk: the three stages of a 64-column chunk
@@ -43,6 +46,8 @@ enum TcEpilogue : int {
                    // both scaled by row_scale[row] first when row_scale != null
   EPI_DOWN3 = 3,   // v = row_scale[row]*acc; out bf16 [.., 3*split]: hi, mid, lo parts of v
   EPI_ROUTER = 4,  // out fp32 = sigmoid(acc + col_bias[col])
+  EPI_SWIGLU3 = 5, // as EPI_SWIGLU with an accurate SiLU, the fp32 result stored as hi, mid, lo bf16
+                   // parts (columns part * split + c) for the next split-precision product
 };
 
 struct KSeg {
@@ -58,7 +63,7 @@ struct TcParams {
   CUtensorMap tmOut;          // output: box 64 x 128 (bf16) or 32 x 128 (fp32), 128-byte swizzle
   CUtensorMap tmA_part[3];    // trim: tmA[0] with boxes of 32, 64, 96 rows
   CUtensorMap tmOut_part[3];  // trim: tmOut with boxes of 32, 64, 96 rows
-  KSeg seg[6];
+  KSeg seg[12];
   int nseg;
   int grouped;
   int M;                      // rows (non-grouped)
@@ -448,6 +453,29 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             w[q] = pack_bf16x2(silu_fast(g0) * u0, silu_fast(g1) * u1);
           }
           ok = emit(w, (ti.n0 >> 1) + j * 64, ti.row0);
+        }
+      } else if constexpr (EPI == EPI_SWIGLU3) {
+#pragma unroll 1
+        for (int j = 0; ok && j < BN / 128; ++j) {
+          uint32_t gv[32], uv[32];
+          tmem_ld32(tbase + j * 128 + half_id * 32, gv);
+          tmem_ld32(tbase + j * 128 + 64 + half_id * 32, uv);
+          tc_wait_ld();
+          float a[32];
+#pragma unroll
+          for (int q = 0; q < 32; ++q) a[q] = siluf(__uint_as_float(gv[q]) * rs) * (__uint_as_float(uv[q]) * rs);
+#pragma unroll 1
+          for (int part = 0; ok && part < 3; ++part) {
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+              const bf16 h0 = __float2bfloat16_rn(a[2 * q]), h1 = __float2bfloat16_rn(a[2 * q + 1]);
+              __nv_bfloat162 ph = __halves2bfloat162(h0, h1);
+              w[q] = *reinterpret_cast<uint32_t*>(&ph);
+              a[2 * q] -= __bfloat162float(h0);  // remainder for the next part
+              a[2 * q + 1] -= __bfloat162float(h1);
+            }
+            ok = emit(w, part * p.split + (ti.n0 >> 1) + j * 64, ti.row0);
+          }
         }
       } else if constexpr (EPI == EPI_BF16) {
 #pragma unroll 1

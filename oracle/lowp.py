@@ -112,18 +112,43 @@ def routed_outputs_mxfp8(h, idx, w1, w3, w2, block: int = MX_BLOCK) -> np.ndarra
     with 8-bit operands: the expert's rows of h and its W1, W3 are quantised along l (their K),
     act = silu(p1) * p3 and W2 along h; each product is the float64 product of the dequantised
     operands, and silu and the elementwise product are float64 as well."""
-    h = np.asarray(h, dtype=np.float64)
+    h = _f64(h)
     T, k = idx.shape
     o = np.zeros((T, k, np.shape(w2)[1]), dtype=np.float64)
     for e in np.unique(idx):
         t, i = np.nonzero(idx == e)
         a = h[t]
-        p1 = mxfp8_matmul(a, np.asarray(w1[e], dtype=np.float64), block)
-        p3 = mxfp8_matmul(a, np.asarray(w3[e], dtype=np.float64), block)
+        p1 = mxfp8_matmul(a, _f64(w1[e]), block)
+        p3 = mxfp8_matmul(a, _f64(w3[e]), block)
         act = p1 / (1.0 + np.exp(-p1)) * p3
-        o[t, i] = mxfp8_matmul(act, np.asarray(w2[e], dtype=np.float64), block)
+        o[t, i] = mxfp8_matmul(act, _f64(w2[e]), block)
     return o
 
 
+def _f64(a) -> np.ndarray:
+    """An input (numpy array, or a CPU torch tensor of any float type) widened exactly to float64."""
+    if hasattr(a, "detach"):
+        import torch
+        return a.detach().to(torch.float64).numpy()
+    return np.asarray(a, dtype=np.float64)
+
+
+def layer_forward_mxfp8(x, w: dict, b, k: int, eps: float = 1e-6, block: int = MX_BLOCK) -> dict:
+    """The whole layer with MXFP8 routed experts: the forward oracle's steps in its order, with
+    routed_outputs replaced by routed_outputs_mxfp8 (the routing, the gates, the combine, the
+    up-projection and the shared expert stay float64).  Returns y and the routing."""
+    import oracle
+    xf = oracle.f64(x)
+    x_hat = oracle.rmsnorm(xf, oracle.f64(w["rms_gain"]), eps)
+    r = oracle.layer_routing(x, w, b, k, eps)
+    o = routed_outputs_mxfp8(r["h"], r["idx"], w["w1"], w["w3"], w["w2"], block)
+    z = oracle.combine(r["gates"], o)
+    y = oracle.up_projection(z, oracle.f64(w["w_up"]))
+    if "ws1" in w:
+        y = y + oracle.shared_expert(x_hat, oracle.f64(w["ws1"]), oracle.f64(w["ws3"]), oracle.f64(w["ws2"]))
+    return dict(r, o=o, z=z, y=y)
+
+
 __all__ = ["E4M3_MAX", "MX_BLOCK", "e4m3_decode", "round_e4m3", "mx_scale_exponent", "mxfp8_quantize",
-           "mxfp8_dequantize", "mxfp8_matmul", "e4m3_half_step", "routed_outputs_mxfp8"]
+           "mxfp8_dequantize", "mxfp8_matmul", "e4m3_half_step", "routed_outputs_mxfp8",
+           "layer_forward_mxfp8"]

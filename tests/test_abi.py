@@ -59,6 +59,15 @@ def test_workspace_query_and_validation(built):
         lq.workspace_bytes(1024, 256, 256, 300, 256, 2048, lq.BF16, 8192)  # k > E
     with pytest.raises(lq.LmoeError, match="unsupported"):
         lq.workspace_bytes(1024, 256, 96, 6, 256, 2048, lq.BF16, 8192)    # E not a multiple of 64
+    # MXFP8 experts: bf16 layers with l and h multiples of 128; the 8-bit expert weights need less
+    n8 = lq.workspace_bytes(1024, 256, 256, 6, 256, 2048, lq.BF16, 8192, experts=lq.EXPERTS_MXFP8)
+    assert 0 < n8 < n
+    with pytest.raises(lq.LmoeError, match="unsupported"):
+        lq.workspace_bytes(256, 64, 32, 4, 128, 512, lq.F32, 256, experts=lq.EXPERTS_MXFP8)
+    with pytest.raises(lq.LmoeError, match="unsupported"):
+        lq.workspace_bytes(1024, 192, 256, 6, 256, 2048, lq.BF16, 8192, experts=lq.EXPERTS_MXFP8)
+    with pytest.raises(lq.LmoeError, match="invalid"):
+        lq.workspace_bytes(1024, 256, 256, 6, 256, 2048, lq.BF16, 8192, experts=2)
 
 
 def test_product_path_never_imports_the_oracle():
@@ -78,7 +87,8 @@ def test_binding_constants_match_the_header():
     pairs = {"F32": lq.F32, "BF16": lq.BF16, "RECORD_STATS": lq.RECORD_STATS, "UPDATE_BIAS": lq.UPDATE_BIAS,
              "ASYNC_OUTPUT": lq.ASYNC_OUTPUT, "QB_LITERAL": lq.QB_LITERAL, "BIAS_SIGN": lq.BIAS_SIGN,
              "STATUS_NAN_SCORE": lq.STATUS_NAN_SCORE, "STATUS_WATCHDOG": lq.STATUS_WATCHDOG,
-             "STATUS_BAD_INDEX": lq.STATUS_BAD_INDEX, "NBINS": lq.NBINS}
+             "STATUS_BAD_INDEX": lq.STATUS_BAD_INDEX, "NBINS": lq.NBINS,
+             "EXPERTS_BF16": lq.EXPERTS_BF16, "EXPERTS_MXFP8": lq.EXPERTS_MXFP8}
     for name, value in pairs.items():
         assert defs.get(name) == value, (name, defs.get(name), value)
     # the forward flags are distinct bits, and the update's rule flags stay out of their way

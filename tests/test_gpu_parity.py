@@ -17,6 +17,7 @@ import torch
 
 import datagen
 import oracle
+import oracle.lowp as lowp
 import latent_routing_quantile_b200 as lq
 
 pytestmark = pytest.mark.gpu
@@ -671,4 +672,38 @@ def test_degenerate_layers_match_oracle(name, T, d, l, E, k, h, hs, dtype):
     if E == k:
         assert np.array_equal(np.sort(r["idx"].cpu().numpy(), 1), np.tile(np.arange(E), (T, 1)))
     np.testing.assert_allclose(gates.sum(1), 1.0, rtol=0, atol=1e-5 * k)
+    layer.close()
+
+
+@pytest.mark.parametrize("name,T,d,l,E,k,h,hs", [
+    ("mx_small", 1000, 256, 128, 64, 4, 128, 256),      # ragged tiles, two N-tiles of W13
+    ("mx_mini", 8192, 1024, 256, 256, 6, 256, 2048),    # mini_replica widths
+])
+def test_mxfp8_experts_match_the_8bit_oracle(name, T, d, l, E, k, h, hs):
+    """Routed experts with MXFP8 operands (LMOE_EXPERTS_MXFP8: weights quantised at create, the
+    gathered latent rows and the SwiGLU activations in every forward, tcgen05 block-scaled MMAs):
+    routing identical to the oracle's; outputs within 1e-2 normwise of the oracle's 8-bit layer
+    (oracle.lowp.layer_forward_mxfp8), and at least twice as far from the bf16-expert oracle, so
+    the 8-bit path is the one that ran (the two oracles differ by about 4% at these shapes)."""
+    shape = datagen.LayerShape(name, T, d, l, E, k, h, hs, "bf16", seed=81, offset_var=0.5)
+    w = datagen.layer_weights(shape)
+    x = datagen.tokens(shape)
+    layer = lq.layer_from_weights(shape, w, experts=lq.EXPERTS_MXFP8)
+    y = layer.forward(x.cuda(), record_stats=True)
+    r = layer.routing()
+    torch.cuda.synchronize()
+    ro = oracle.layer_routing(x, w, np.zeros(E), k, shape.rms_eps)
+    frac = check_routing(r["idx"].cpu().numpy(), ro, score_tolerance(shape))
+    assert frac == 0.0
+    check_permutation(r, T, k, E)
+    rows = np.arange(T) if T <= 1000 else np.arange(0, T, 16)
+    xs = x[torch.from_numpy(rows)]
+    yg = y.float().cpu().numpy()[rows]
+    y8 = lowp.layer_forward_mxfp8(xs, w, np.zeros(E), k, shape.rms_eps)["y"]
+    y16 = oracle.layer_forward(xs, w, np.zeros(E), k, shape.rms_eps)["y"]
+    err8, err16 = normwise(yg, y8), normwise(yg, y16)
+    print(name, json.dumps(dict(err_vs_8bit_oracle=err8, err_vs_bf16_oracle=err16)))
+    assert err8 <= 1e-2, err8
+    assert err16 >= 2 * err8, (err8, err16)
+    assert layer.status() == 0
     layer.close()

@@ -174,3 +174,29 @@ def test_mxfp8_experts_stay_near_the_full_precision_experts():
     o = oracle.routed_outputs(hid, idx, w1, w3, w2)
     rel = np.max(np.abs(o8 - o)) / np.max(np.abs(o))
     assert 0 < rel < 0.3, rel
+
+
+def test_layer_forward_mxfp8_with_an_identity_quantiser_is_the_forward_oracle():
+    """With the quantiser replaced by the identity (elements = values, every scale 2^0), the
+    8-bit layer is the forward oracle's layer: routing, combine, up-projection and shared expert
+    are wired exactly as there, and only the experts' operands change with the format."""
+    import datagen
+    import oracle
+    shape = datagen.LayerShape("mx_pin", 24, 64, 64, 8, 2, 64, 96, "f32", seed=77, offset_var=0.5)
+    w = datagen.layer_weights(shape, gain="random")
+    x = datagen.tokens(shape)
+    b = datagen.normal_bias(shape.E, seed=77, std=0.1).astype(np.float64)
+    real = lp.mxfp8_quantize
+    try:
+        lp.mxfp8_quantize = lambda a, block=32: (np.asarray(a, dtype=np.float64),
+                                                 np.zeros(np.shape(a)[:-1] + (np.shape(a)[-1] // block,), int))
+        y8 = lp.layer_forward_mxfp8(x, w, b, shape.k)
+    finally:
+        lp.mxfp8_quantize = real
+    ref = oracle.layer_forward(x, w, b, shape.k)
+    assert np.array_equal(y8["idx"], ref["idx"])
+    np.testing.assert_allclose(y8["y"], ref["y"], rtol=1e-12, atol=1e-12)
+    # and with the real quantiser it moves, within the 8-bit bound of the experts' part
+    y8 = lp.layer_forward_mxfp8(x, w, b, shape.k)["y"]
+    rel = np.max(np.abs(y8 - ref["y"])) / np.max(np.abs(ref["y"]))
+    assert 0 < rel < 0.2, rel
