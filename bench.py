@@ -515,7 +515,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="wide_stress")
     ap.add_argument("--tokens", type=int, default=0)
-    ap.add_argument("--also", default="sweep:262144",
+    ap.add_argument("--also", default="sweep:262144,wide_stress:16384:mxfp8",
                     help="extra workloads (name:T[:mxfp8], comma-separated) measured in the same call on one GPU, "
                          "':mxfp8' with 8-bit routed experts; '' for none")
     ap.add_argument("--no-cpu-baseline", action="store_true")
