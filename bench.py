@@ -354,7 +354,7 @@ def run_ours(args, rank, world, local_rank):
     shape = datagen.WORKLOADS[args.workload]
     if args.tokens:
         shape = shape.with_tokens(args.tokens)
-    main_s, launches = measure(shape, args, rank, world, local_rank)
+    main_s, launches = measure(shape, args, rank, world, local_rank, experts=1 if args.experts == "mxfp8" else 0)
     also = {}
     if world == 1 and args.also and not args.tokens:
         for spec in args.also.split(","):
@@ -373,7 +373,7 @@ def run_ours(args, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": m["ms_per_step"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": shape.dtype, "data": "synthetic (seeded; x ~ N(0,1), weights ~ N(0,1/fan_in))",
         "config": {"workload": shape.name, "T": T, "d": shape.d, "l": shape.l, "E": shape.E, "k": shape.k,
-                   "h": shape.h, "hs": shape.hs, "tokens_per_gpu": T, "global_tokens": T * world,
+                   "h": shape.h, "hs": shape.hs, "experts": args.experts, "tokens_per_gpu": T, "global_tokens": T * world,
                    "step": "forward with QB statistics + QB update"
                            + (" (update inside the forward, after routing)" if world == 1 else ""), "beta": BETA,
                    "l2": "flushed between steps (256 MiB write outside the timed events)",
@@ -518,6 +518,8 @@ def main():
     ap.add_argument("--also", default="sweep:262144,wide_stress:16384:mxfp8",
                     help="extra workloads (name:T[:mxfp8], comma-separated) measured in the same call on one GPU, "
                          "':mxfp8' with 8-bit routed experts; '' for none")
+    ap.add_argument("--experts", choices=["bf16", "mxfp8"], default="bf16",
+                    help="operand format of the routed experts of the main workload")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)

@@ -77,6 +77,9 @@ WORKLOADS = {
     # QB convergence run on a skewed router: 50 steps, beta 0.05, fresh x from seed 3+step.
     "qb_skewed": LayerShape("qb_skewed", 4096, 1024, 256, 128, 8, 256, 2048, "bf16",
                             seed=3, beta=0.05, steps=50),
+    # the wide layer's routed-expert shape (l = 2048, h = 512, k = 16, about 292 rows per expert)
+    # with 128 experts and d = 1024: the small case on which ncu captures the expert GEMMs.
+    "wide_experts": LayerShape("wide_experts", 2336, 1024, 2048, 128, 16, 512, 1024, "bf16", seed=2),
     # large-batch sweep, T in SWEEP_T.
     "sweep": LayerShape("sweep", 262144, 1024, 256, 256, 6, 256, 2048, "bf16", seed=4, offset_var=0.5),
 }
