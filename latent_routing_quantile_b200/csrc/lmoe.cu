@@ -78,6 +78,15 @@ bool make_map_f32(CUtensorMap* m, const void* base, long long rows, long long co
 
 int pick_bn(int n) { return n % 256 == 0 ? 256 : (n % 128 == 0 ? 128 : 64); }
 
+// N-tiles per band of a non-grouped GEMM's tile order (tc_tile): B's band (bn columns x K bf16
+// elements per N-tile) at most 32 MB, so that it and the A rows of the tiles running beside it
+// stay in the 126 MB L2; 0 (row-major order) when all of B fits.
+int pick_band(int n_tiles, int bn, long long k_elems) {
+  const long long per_tile = (long long)bn * k_elems * 2;
+  const long long fit = (32ll << 20) / per_tile;
+  return fit >= n_tiles ? 0 : (int)std::max(1ll, fit);
+}
+
 // Tile width for a non-grouped GEMM of M rows and N columns: the widest that divides N and still
 // gives every SM a tile (min_bn = 128 for the SwiGLU epilogue, whose column groups are 128 wide).
 int pick_bn_for(long long M, int N, int sms, int min_bn) {
@@ -816,6 +825,7 @@ int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, 
       p.M = T;
       p.M_rows = T;
       p.n_tiles = c.l / bn;
+      p.band_n = pick_band(p.n_tiles, bn, (h->unit_gain ? 1 : 2) * (long long)c.d);
       p.tmOut = h->tm_hx;
       p.split = c.l;
       p.row_scale = h->r;
@@ -863,12 +873,14 @@ int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, 
     if (pbn) {  // two-CTA tiles: each CTA loads BN/2 rows of the weights
       p.tmB = h->tm_ws13[bn_index(pbn / 2)];
       p.n_tiles = 2 * c.hs / pbn;
+      p.band_n = pick_band(p.n_tiles, pbn, c.d);
       const int tiles = (T + 255) / 256 * p.n_tiles;
       CK(launch_tc_pair(p, EPI_SWIGLU, pbn, 2 * std::min(tiles, h->sms / 2), st));
     } else {
       const int bn = pick_bn_for(T, 2 * c.hs, h->sms, 128);
       p.tmB = h->tm_ws13[bn_index(bn)];
       p.n_tiles = 2 * c.hs / bn;
+      p.band_n = pick_band(p.n_tiles, bn, c.d);
       CK(launch_tc(p, EPI_SWIGLU, bn, std::min(mt * p.n_tiles, h->sms), st));
     }
   }
@@ -975,12 +987,14 @@ int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, 
     if (pbn) {
       p.tmB = h->tm_wy[bn_index(pbn / 2)];
       p.n_tiles = c.d / pbn;
+      p.band_n = pick_band(p.n_tiles, pbn, c.l + c.hs);
       const int tiles = (T + 255) / 256 * p.n_tiles;
       CK(launch_tc_pair(p, EPI_BF16, pbn, 2 * std::min(tiles, h->sms / 2), st));
     } else {
       const int bn = pick_bn_for(T, c.d, h->sms, 64);
       p.tmB = h->tm_wy[bn_index(bn)];
       p.n_tiles = c.d / bn;
+      p.band_n = pick_band(p.n_tiles, bn, c.l + c.hs);
       CK(launch_tc(p, EPI_BF16, bn, std::min(mt * p.n_tiles, h->sms), st));
     }
   }

@@ -78,6 +78,7 @@ struct TcParams {
   int trim;                   // grouped: move only the valid rows of a tile, rounded up to 32
   int hint_a, hint_b;         // 1: load A / B with L2 evict_first (read once, not again soon)
   int hint_out;               // 1: store the output with L2 evict_last (the next kernel reads it)
+  int band_n;                 // non-grouped: N-tiles per band of the tile order (0: row-major order)
   uint32_t* status;
 };
 
@@ -100,9 +101,24 @@ struct TileInfo {
   int q;  // 32-row quarters of the tile that are loaded and stored (4 = all)
 };
 
+// Tile order: row-major over (M-tile, N-tile), or, with band_n > 0 (non-grouped), band by band:
+// all M-tiles of N-tiles [b band_n, (b+1) band_n) before the next band, so the tiles that run at
+// the same time share a band of B that stays in L2 instead of streaming all of B per M-tile.
 __device__ __forceinline__ TileInfo tc_tile(const TcParams& p, int tile, int BN, int pair, uint32_t rank) {
   TileInfo ti;
-  int mt = tile / p.n_tiles, nt = tile - mt * p.n_tiles;
+  int mt, nt;
+  if (p.band_n > 0 && !p.grouped) {
+    const int m_tiles = pair ? (p.M + 255) / 256 : (p.M + 127) / 128;
+    const int per_band = m_tiles * p.band_n;
+    const int band = tile / per_band;
+    const int idx = tile - band * per_band;
+    const int nb = min(p.band_n, p.n_tiles - band * p.band_n);  // the last band may be narrower
+    mt = idx / nb;
+    nt = band * p.band_n + (idx - mt * nb);
+  } else {
+    mt = tile / p.n_tiles;
+    nt = tile - mt * p.n_tiles;
+  }
   ti.n0 = nt * BN;
   ti.q = 4;
   if (pair) {  // 256-row tiles; this CTA owns rows 128*rank.. and B rows BN/2*rank..
@@ -415,7 +431,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       const uint32_t acc_phase = (it >> 1) & 1;
       float c_lane[BN / 32];  // router column offsets of this tile, one per lane and step
       if constexpr (EPI == EPI_ROUTER) {
-        const int n0 = (tile % p.n_tiles) * BN;
+        const int n0 = tc_tile(p, tile, BN, PAIR, rank).n0;
 #pragma unroll
         for (int j = 0; j < BN / 32; ++j) c_lane[j] = p.col_bias[n0 + j * 32 + lane];
       } else {
