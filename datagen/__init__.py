@@ -32,7 +32,7 @@ TOKEN_CHUNK = 1024  # rows of x drawn from one stream
 _TID = {
     "w_down": 1, "w_router": 2, "w1": 3, "w3": 4, "w2": 5, "w_up": 6,
     "ws1": 7, "ws3": 8, "ws2": 9, "router_bias": 10, "x": 11, "rms_gain": 12,
-    "bias": 13, "scores": 14,
+    "bias": 13, "scores": 14, "dy": 15,
 }
 
 
@@ -187,6 +187,22 @@ def tokens(shape: LayerShape, seed: int | None = None, rows=None, T: int | None 
         sel = np.nonzero(rows // TOKEN_CHUNK == c)[0]
         out[sel] = blk[rows[sel] - c * TOKEN_CHUNK]
     return _store(out, dt)
+
+
+def output_grad(shape: LayerShape, seed: int | None = None, T: int | None = None,
+                scale: float = 1.0) -> torch.Tensor:
+    """dL/dy ~ scale * N(0,1) of shape [T, d] in the layer's dtype (the output gradient of a
+    backward pass), drawn in chunks of TOKEN_CHUNK rows like tokens()."""
+    s = shape.seed if seed is None else seed
+    T = shape.T if T is None else T
+    d = shape.d
+    out = np.empty((T, d), dtype=np.float32)
+    for c0 in range(0, T, TOKEN_CHUNK):
+        n = min(TOKEN_CHUNK, T - c0)
+        out[c0:c0 + n] = _normal(s, _TID["dy"], c0 // TOKEN_CHUNK, TOKEN_CHUNK * d).reshape(TOKEN_CHUNK, d)[:n]
+    if scale != 1.0:
+        out *= np.float32(scale)
+    return _store(out, torch_dtype(shape))
 
 
 def uniform_scores(T: int, E: int, seed: int, quantise: int = 0) -> np.ndarray:

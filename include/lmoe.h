@@ -277,6 +277,54 @@ const char *lmoe_strerror(int code);
 int lmoe_gemm_bf16(const void *a_dev, const void *b_dev, float *c_dev, int32_t M, int32_t N,
                    int32_t K, void *stream);
 
+/* C = op(A) op(B)^T (fp32) on the tensor-core engine with either operand stored MN-major:
+ * a_mn = 0: A is [M, K] row-major; a_mn = 1: A is stored [K, M] (the product reads A^T).
+ * b_mn = 0: B is [N, K]; b_mn = 1: B is stored [K, N].  N a multiple of 64, K of 8, M of 8 when
+ * a_mn.  k_split > 1 (at most ceil(K/64)) cuts K into that many ranges whose products are added
+ * into C by TMA reductions (C is zeroed first; the sum order then varies between runs).  The
+ * products of the layer backward use these forms.  For tests. */
+int lmoe_gemm_bf16_ex(const void *a_dev, int32_t a_mn, const void *b_dev, int32_t b_mn, float *c_dev,
+                      int32_t M, int32_t N, int32_t K, int32_t k_split, void *stream);
+
+/* ---- Layer backward (training) -------------------------------------------------------------
+ * Gradients of the loss L = sum(y * dy) with respect to x and every weight, for y the layer's
+ * forward ("Pretraining a Mini Kimi K3" builds the training step by hand: forward, backward,
+ * optimiser; "KimiK3MoE 架构轻量化复刻演示上线", Tab 6, shows the sparse expert gradients).
+ * The expert choice is piecewise constant, so no gradient flows through the top-k selection or
+ * into the balancing bias b; the gate weights g_i = s_i / sum_j s_j pass theirs to the chosen
+ * scores through the renormalisation, and the scores to the router logits through the sigmoid
+ * (unchosen scores get none).  Each expert's weight gradient sums over the (token, slot) pairs
+ * routed to it only; an expert that received none gets a zero gradient.
+ * All buffers fp32 device memory in the layouts of lmoe_weights; rms_gain may be NULL. */
+typedef struct {
+  float *dx;          /* [T, d] dL/dx */
+  float *rms_gain;    /* [d] (also when the layer has no gain tensor: the gradient at gain = 1) */
+  float *w_down;      /* [l, d] */
+  float *w_router;    /* [E, l] */
+  float *router_bias; /* [E] column offsets c */
+  float *w1;          /* [E, h, l] */
+  float *w3;          /* [E, h, l] */
+  float *w2;          /* [E, l, h] */
+  float *w_up;        /* [d, l] */
+  float *ws1;         /* [hs, d] (unused when hs == 0) */
+  float *ws3;         /* [hs, d] */
+  float *ws2;         /* [d, hs] */
+} lmoe_grads;
+
+/* One training step's layer work on `stream`: the forward of x [T, d] into y (exactly
+ * lmoe_forward with `flags`, which may record statistics but not update the bias), then every
+ * gradient of lmoe_grads for the output gradient dy [T, d] (bf16, 16-byte aligned).
+ * `w` must hold the weights the handle was created from, still on the device (the backward
+ * reads the caller's layouts: their transposes are read in place by MN-major tensor-core
+ * operands).  BF16 layers with BF16 experts only (LMOE_EUNSUPPORTED otherwise).  Operands of
+ * the backward's products are bf16 (gradients are rounded to bf16 before each product),
+ * accumulation fp32.  The first call allocates the backward's workspace (about
+ * max_tokens * (4 d + 8 hs + 12 l + 2 E) + rows * (10 h + 4 l + 4) bytes, rows = max_tokens k +
+ * 128 E); lmoe_destroy frees it.  Gradients of GEMMs whose output tiles cannot fill the GPU are
+ * summed over K ranges by atomic tensor reductions, so their last bits vary between runs. */
+int lmoe_forward_backward(lmoe_handle *h, const lmoe_weights *w, const void *x, const void *dy, void *y,
+                          int32_t T, uint32_t flags, const lmoe_grads *g, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

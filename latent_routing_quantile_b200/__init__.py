@@ -30,7 +30,7 @@ EXPORTED = (
     "lmoe_qb_update", "lmoe_set_update", "lmoe_route_scores", "lmoe_get_routing", "lmoe_get_bias", "lmoe_set_bias",
     "lmoe_get_hist", "lmoe_set_hist", "lmoe_get_load", "lmoe_set_load", "lmoe_get_status", "lmoe_strerror", "lmoe_gemm_bf16",
     "lmoe_profile_enable", "lmoe_profile_read", "lmoe_stage_name", "lmoe_launch_count",
-    "lmoe_route_noalloc", "lmoe_watchdog_selftest",
+    "lmoe_route_noalloc", "lmoe_watchdog_selftest", "lmoe_gemm_bf16_ex", "lmoe_forward_backward",
 )
 NUM_STAGES = 14
 
@@ -48,6 +48,11 @@ class lmoe_config(ctypes.Structure):
 class lmoe_weights(ctypes.Structure):
     _fields_ = [(n, c_void_p) for n in ("rms_gain", "w_down", "w_router", "router_bias", "w1", "w3",
                                          "w2", "w_up", "ws1", "ws3", "ws2")]
+
+
+class lmoe_grads(ctypes.Structure):
+    _fields_ = [(n, c_void_p) for n in ("dx", "rms_gain", "w_down", "w_router", "router_bias", "w1", "w3", "w2",
+                                         "w_up", "ws1", "ws3", "ws2")]
 
 
 _lib = None
@@ -80,6 +85,8 @@ def lib() -> ctypes.CDLL:
             "lmoe_set_load": [vp, vp, vp],
             "lmoe_get_status": [vp, POINTER(u32)],
             "lmoe_gemm_bf16": [vp, vp, vp, i32, i32, i32, vp],
+            "lmoe_gemm_bf16_ex": [vp, i32, vp, i32, vp, i32, i32, i32, i32, vp],
+            "lmoe_forward_backward": [vp, POINTER(lmoe_weights), vp, vp, vp, i32, u32, POINTER(lmoe_grads), vp],
             "lmoe_profile_enable": [vp, i32],
             "lmoe_profile_read": [vp, POINTER(c_float), i32, POINTER(i32)],
             "lmoe_launch_count": [vp, POINTER(ctypes.c_int64)],
@@ -170,6 +177,45 @@ class Layer:
                                   _stream(stream)), "lmoe_forward")
         self.last_T = T
         return y
+
+    GRAD_NAMES = ("x", "rms_gain", "w_down", "w_router", "router_bias", "w1", "w3", "w2", "w_up", "ws1", "ws3",
+                  "ws2")
+
+    def forward_backward(self, x, dy, weights, y=None, record_stats=False, grads=None, stream=None):
+        """One training step's layer work (lmoe_forward_backward): y = forward(x) and the fp32
+        gradients of sum(y * dy) with respect to x and every weight, returned as a dict keyed like
+        the weights (plus "x").  `weights` are the device tensors the layer was created from.
+        `grads` may pass preallocated fp32 buffers."""
+        c = self.cfg
+        T = x.shape[0]
+        _dev(x, self.dtype, (T, c.d), "x")
+        _dev(dy, self.dtype, (T, c.d), "dy")
+        if y is None:
+            y = torch.empty_like(x)
+        _dev(y, self.dtype, (T, c.d), "y")
+        shapes = {"x": (T, c.d), "rms_gain": (c.d,), "w_down": (c.l, c.d), "w_router": (c.E, c.l),
+                  "router_bias": (c.E,), "w1": (c.E, c.h, c.l), "w3": (c.E, c.h, c.l), "w2": (c.E, c.l, c.h),
+                  "w_up": (c.d, c.l)}
+        if c.hs:
+            shapes.update({"ws1": (c.hs, c.d), "ws3": (c.hs, c.d), "ws2": (c.d, c.hs)})
+        g = dict(grads or {})
+        for n, shp in shapes.items():
+            if n not in g:
+                g[n] = torch.empty(shp, dtype=torch.float32, device=x.device)
+            _dev(g[n], torch.float32, shp, "grad " + n)
+        w = lmoe_weights()
+        for n in ("rms_gain", "w_down", "w_router", "router_bias", "w1", "w3", "w2", "w_up", "ws1", "ws3", "ws2"):
+            t = weights.get(n)
+            if t is not None:
+                setattr(w, n, _dev(t, None, None, n).data_ptr())
+        gs = lmoe_grads()
+        for n in shapes:
+            setattr(gs, "dx" if n == "x" else n, g[n].data_ptr())
+        _check(lib().lmoe_forward_backward(self.handle, ctypes.byref(w), _ptr(x), _ptr(dy), _ptr(y), T,
+                                           self._fwd_flags(record_stats, False), ctypes.byref(gs), _stream(stream)),
+               "lmoe_forward_backward")
+        self.last_T = T
+        return y, g
 
     def forward_host(self, x_host, y_host, record_stats=False, update_bias=False, async_output=False,
                      stream=None):
@@ -311,6 +357,22 @@ def gemm_bf16(a, b, stream=None):
     _dev(b, torch.bfloat16, (N, K), "b")
     c = torch.empty((M, N), dtype=torch.float32, device=a.device)
     _check(lib().lmoe_gemm_bf16(_ptr(a), _ptr(b), _ptr(c), M, N, K, _stream(stream)), "lmoe_gemm_bf16")
+    return c
+
+
+def gemm_bf16_ex(a, b, a_mn=False, b_mn=False, k_split=1, stream=None):
+    """C = op(A) op(B)^T with op(A) = A ([M, K]) or, a_mn, A^T of A stored [K, M]; likewise B
+    ([N, K], or stored [K, N] with b_mn).  k_split > 1 adds K-range partial products by TMA
+    reductions.  For checks of the engine's MN-major operands and split K."""
+    M, K = (a.shape[1], a.shape[0]) if a_mn else a.shape
+    N = b.shape[1] if b_mn else b.shape[0]
+    _dev(a, torch.bfloat16, None, "a")
+    _dev(b, torch.bfloat16, None, "b")
+    if (b.shape[0] if b_mn else b.shape[1]) != K:
+        raise LmoeError("A and B disagree on K")
+    c = torch.empty((M, N), dtype=torch.float32, device=a.device)
+    _check(lib().lmoe_gemm_bf16_ex(_ptr(a), int(a_mn), _ptr(b), int(b_mn), _ptr(c), M, N, K, k_split,
+                                   _stream(stream)), "lmoe_gemm_bf16_ex")
     return c
 
 

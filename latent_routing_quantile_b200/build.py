@@ -14,7 +14,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "liblmoe.so")
 SOURCES = ["lmoe.cu"]
-HEADERS = ["common.cuh", "k1_router.cuh", "q8_gemm.cuh", "route.cuh", "tc_gemm.cuh"]
+HEADERS = ["bwd.cuh", "common.cuh", "k1_router.cuh", "q8_gemm.cuh", "route.cuh", "tc_gemm.cuh"]
 
 
 def nvcc() -> str:

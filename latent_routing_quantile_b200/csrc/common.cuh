@@ -129,6 +129,13 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* s
                "r"(smem_u32(src)), "r"(x), "r"(y)
                : "memory");
 }
+// Adds a shared-memory box into global memory element by element (the tensor map's element type;
+// fp32 here), at a non-negative coordinate.
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* m, const void* src, int x, int y) {
+  asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(m),
+               "r"(x), "r"(y), "r"(smem_u32(src))
+               : "memory");
+}
 // L2 eviction priority for TMA traffic (createpolicy): evict_first for data read once and not
 // needed again soon (streamed expert weights, last reads), evict_last for outputs the next kernel
 // reads, so streams of weights do not push those out of L2.
@@ -306,6 +313,27 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
   d |= (uint64_t)1u << 46;            // version
   d |= (uint64_t)2u << 61;            // SWIZZLE_128B
   return d;
+}
+
+// Descriptor of an MN-major bf16 operand staged as 64 x 64 TMA boxes with the 128-byte swizzle:
+// each box holds 64 K rows of 64 M (or N) elements, one 128-byte row per K; 8-row groups are
+// 1024 bytes apart (stride byte offset) and the next 64 elements of M (N) sit one 8 KB box
+// further (leading byte offset).
+__device__ __forceinline__ uint64_t smem_desc_mn128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)(8192u >> 4) << 16;  // leading byte offset: next 64 elements of M (N)
+  d |= (uint64_t)(1024u >> 4) << 32;  // stride byte offset: next 8 K rows
+  d |= (uint64_t)1u << 46;            // version
+  d |= (uint64_t)2u << 61;            // SWIZZLE_128B
+  return d;
+}
+
+// 16 bytes from global memory through the non-coherent path (data no kernel of the launch writes).
+__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
 }
 
 // Instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major, M = m (128 or 256), N = n.

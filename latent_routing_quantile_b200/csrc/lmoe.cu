@@ -13,6 +13,7 @@
 
 #include "common.cuh"
 #include "route.cuh"
+#include "bwd.cuh"
 #include "tc_gemm.cuh"
 #include "k1_router.cuh"
 #include "q8_gemm.cuh"
@@ -181,6 +182,7 @@ cudaError_t launch_tc(const TcParams& p, int epi, int bn, int grid, cudaStream_t
     case EPI_SWIGLU: return launch_tc_e<EPI_SWIGLU>(p, bn, grid, st);
     case EPI_DOWN3: return launch_tc_e<EPI_DOWN3>(p, bn, grid, st);
     case EPI_SWIGLU3: return launch_tc_e<EPI_SWIGLU3>(p, bn, grid, st);
+    case EPI_SWIGLU_BWD: return launch_tc_e<EPI_SWIGLU_BWD>(p, bn, grid, st);
     default: return launch_tc_e<EPI_ROUTER>(p, bn, grid, st);
   }
 }
@@ -310,6 +312,18 @@ struct ProfRecord {
 }  // namespace
 
 // ---------------------------------------------------------------------- handle
+// Workspace of lmoe_forward_backward, allocated by its first call (sized for max_tokens).
+struct BwdWork {
+  void* mem = nullptr;
+  bf16 *xh = nullptr, *ps = nullptr, *dps = nullptr, *dz = nullptr;  // token rows
+  bf16 *pe = nullptr, *dpe = nullptr, *d_o = nullptr, *dhe = nullptr;  // padded expert rows
+  bf16 *dlogit = nullptr, *dh = nullptr;
+  float *dlp = nullptr, *dhr = nullptr, *dxh = nullptr, *gpart = nullptr;
+  long long RP = 0;  // rows of the padded expert layout, a multiple of 128
+  // maps of the padded expert-row buffers (fixed addresses)
+  CUtensorMap pe_out, dpe_out, dpe_k, dpe_mn, do_k, do_mn, dhe_out, aperm_mn, act_mn;
+};
+
 struct lmoe_handle {
   lmoe_config cfg;
   int device = 0, sms = 148;
@@ -408,6 +422,7 @@ struct lmoe_handle {
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
   long long g_tick = 0;
   long long g_used[2] = {0, 0};
+  BwdWork* bw = nullptr;
 };
 
 namespace {
@@ -1271,6 +1286,391 @@ int run_cached(lmoe_handle* h, GraphCache& g, const void* x, void* y, int T, uin
   return LMOE_OK;
 }
 
+// ---------------------------------------------------------------------- layer backward
+// Allocates the backward's workspace on first use.
+int bwd_alloc(lmoe_handle* h) {
+  if (h->bw) return LMOE_OK;
+  const lmoe_config& c = h->cfg;
+  const size_t Tm = c.max_tokens, d = c.d, l = c.l, E = c.E, hh = c.h, hs = c.hs;
+  BwdWork* b = new (std::nothrow) BwdWork();
+  if (!b) return LMOE_ENOMEM;
+  b->RP = (h->rows_pad + 127) / 128 * 128;
+  const size_t RP = (size_t)b->RP;
+  Arena a;
+  a.add((void**)&b->xh, Tm * d * 2);
+  a.add((void**)&b->ps, Tm * 2 * hs * 2);
+  a.add((void**)&b->dps, Tm * 2 * hs * 2);
+  a.add((void**)&b->dz, Tm * l * 2);
+  a.add((void**)&b->pe, RP * 2 * hh * 2);
+  a.add((void**)&b->dpe, RP * 2 * hh * 2);
+  a.add((void**)&b->d_o, RP * l * 2);
+  a.add((void**)&b->dhe, RP * l * 2);
+  a.add((void**)&b->dlogit, Tm * E * 2);
+  a.add((void**)&b->dh, Tm * l * 2);
+  a.add((void**)&b->dlp, RP * 4);
+  a.add((void**)&b->dhr, Tm * l * 4);
+  a.add((void**)&b->dxh, Tm * d * 4);
+  a.add((void**)&b->gpart, (Tm + kRmsRows - 1) / kRmsRows * d * 4);
+  if (cudaMalloc(&b->mem, a.off) != cudaSuccess) {
+    delete b;
+    return LMOE_ENOMEM;
+  }
+  for (auto& it : a.items) *it.first = (uint8_t*)b->mem + it.second;
+  const long long R = b->RP;
+  bool ok = true;
+  ok &= make_map(&b->pe_out, b->pe, R, 2 * hh, 2 * hh, 128);
+  ok &= make_map(&b->dpe_out, b->dpe, R, 2 * hh, 2 * hh, 128);
+  ok &= make_map(&b->dpe_k, b->dpe, R, 2 * hh, 2 * hh, 128);
+  ok &= make_map(&b->dpe_mn, b->dpe, R, 2 * hh, 2 * hh, 64);
+  ok &= make_map(&b->do_k, b->d_o, R, l, l, 128);
+  ok &= make_map(&b->do_mn, b->d_o, R, l, l, 64);
+  ok &= make_map(&b->dhe_out, b->dhe, R, l, l, 128);
+  ok &= make_map(&b->aperm_mn, h->a_perm, h->rows_pad, l, l, 64);
+  ok &= make_map(&b->act_mn, h->act, h->rows_pad, hh, hh, 64);
+  h->bw = b;
+  return ok ? LMOE_OK : LMOE_EINVAL;
+}
+
+void bwd_free(lmoe_handle* h) {
+  if (!h->bw) return;
+  cudaFree(h->bw->mem);
+  delete h->bw;
+  h->bw = nullptr;
+}
+
+// A weight gradient G [M, N] (fp32) = A^T B over K rows (both operands MN-major: A stored [K, M],
+// B stored [K, N]).  When the output tiles cannot fill the SMs, K is cut into ranges whose partial
+// products are added into the zeroed output by TMA reductions.
+int wgrad_gemm(lmoe_handle* h, TcParams& p, int M, int N, long long K, size_t out_bytes, void* out,
+               size_t out2_bytes, void* out2, cudaStream_t st) {
+  const int bn = N % 256 == 0 ? 256 : (N % 128 == 0 ? 128 : 64);
+  p.a_mn = 1;
+  p.b_mn = 1;
+  p.M = M;
+  p.M_rows = M;
+  p.n_tiles = N / bn;
+  p.nseg = 1;
+  p.seg[0] = KSeg{0, 0, 0, (int)((K + 63) / 64), 0};
+  const long long base = (long long)((M + 127) / 128) * p.n_tiles;
+  const int nkb = p.seg[0].nkb;
+  int S = 1;
+  if (base < h->sms) S = (int)std::min<long long>((h->sms + base - 1) / base, std::max(1, nkb / 4));
+  p.k_split = S;
+  if (S > 1) {
+    CK(cudaMemsetAsync(out, 0, out_bytes, st));
+    if (out2) CK(cudaMemsetAsync(out2, 0, out2_bytes, st));
+  }
+  const long long tiles = base * S;
+  CK(launch_tc(p, EPI_F32, bn, (int)std::min<long long>(tiles, h->sms), st));
+  h->launches += 1;
+  return LMOE_OK;
+}
+
+// The backward of a bf16 layer with bf16 experts, right after the forward of the same x on the
+// same stream (the forward's routing, gathered rows, activations and expert outputs are still in
+// the workspace).  Operands are bf16 (the gradients flowing back are rounded to bf16 before each
+// product), accumulation fp32; every gradient is written in fp32.
+int backward_bf16(lmoe_handle* h, const lmoe_weights* w, const void* x, const void* dy, int T, const lmoe_grads* g,
+                  cudaStream_t st) {
+  const lmoe_config& c = h->cfg;
+  BwdWork* b = h->bw;
+  const long long d = c.d, l = c.l, E = c.E, hh = c.h, hs = c.hs;
+  const int mt = (T + 127) / 128;
+  const int sms = h->sms;
+  bool ok = true;
+  // per-call maps of the token-row buffers (their row extent is T, so K = T products read zeros
+  // past the last token)
+  CUtensorMap x_k, dy_k, dy_mn, xh_mn, ps_out, dps_out, dps_k, dps_mn, dz_out, as_mn, z_mn, dlg_k, dlg_mn, hx_mn, dhr_out,
+      dh_k, dh_mn, dxh_out;
+  ok &= make_map(&x_k, x, T, d, d, 128);
+  ok &= make_map(&dy_k, dy, T, d, d, 128);
+  ok &= make_map(&dy_mn, dy, T, d, d, 64);
+  ok &= make_map(&xh_mn, b->xh, T, d, d, 64);
+  if (hs) {
+    ok &= make_map(&ps_out, b->ps, T, 2 * hs, 2 * hs, 128);
+    ok &= make_map(&dps_out, b->dps, T, 2 * hs, 2 * hs, 128);
+    ok &= make_map(&dps_k, b->dps, T, 2 * hs, 2 * hs, 128);
+    ok &= make_map(&dps_mn, b->dps, T, 2 * hs, 2 * hs, 64);
+    ok &= make_map(&as_mn, h->a_s, T, hs, hs, 64);
+  }
+  ok &= make_map(&dz_out, b->dz, T, l, l, 128);
+  ok &= make_map(&z_mn, h->z, T, l, l, 64);
+  ok &= make_map(&dlg_k, b->dlogit, T, E, E, 128);
+  ok &= make_map(&dlg_mn, b->dlogit, T, E, E, 64);
+  ok &= make_map(&hx_mn, h->hx, T, l, 3 * l, 64);
+  ok &= make_map_f32(&dhr_out, b->dhr, T, l, l, 128);
+  ok &= make_map(&dh_k, b->dh, T, l, l, 128);
+  ok &= make_map(&dh_mn, b->dh, T, l, l, 64);
+  ok &= make_map_f32(&dxh_out, b->dxh, T, d, d, 128);
+  // the caller's weights, MN-major (rows = the product's K)
+  CUtensorMap wup_mn, ws2_mn, ws1_mn, ws3_mn, w2_mn, w1_mn, w3_mn, wd_mn, wr_hi_mn, wr_mid_mn;
+  ok &= make_map(&wup_mn, w->w_up, d, l, l, 64);
+  if (hs) {
+    ok &= make_map(&ws2_mn, w->ws2, d, hs, hs, 64);
+    ok &= make_map(&ws1_mn, w->ws1, hs, d, d, 64);
+    ok &= make_map(&ws3_mn, w->ws3, hs, d, d, 64);
+  }
+  ok &= make_map(&w2_mn, w->w2, E * l, hh, hh, 64);
+  ok &= make_map(&w1_mn, w->w1, E * hh, l, l, 64);
+  ok &= make_map(&w3_mn, w->w3, E * hh, l, l, 64);
+  ok &= make_map(&wd_mn, w->w_down, l, d, d, 64);
+  // the router weights: the hi and mid bf16 parts of the fp32 values the handle holds
+  ok &= make_map(&wr_hi_mn, h->w_r, E, l, 3 * l, 64);
+  ok &= make_map(&wr_mid_mn, (const bf16*)h->w_r + l, E, l, 3 * l, 64);
+  // gradient outputs (fp32, boxes of 32 columns x 128 rows)
+  CUtensorMap gw1, gw3, gw2, gwr, gwd, gws1, gws3, gws2, gwup;
+  ok &= make_map_f32(&gw1, g->w1, E * hh, l, l, 128);
+  ok &= make_map_f32(&gw3, g->w3, E * hh, l, l, 128);
+  ok &= make_map_f32(&gw2, g->w2, E * l, hh, hh, 128);
+  ok &= make_map_f32(&gwr, g->w_router, E, l, l, 128);
+  ok &= make_map_f32(&gwd, g->w_down, l, d, d, 128);
+  ok &= make_map_f32(&gwup, g->w_up, d, l, l, 128);
+  if (hs) {
+    ok &= make_map_f32(&gws1, g->ws1, hs, d, d, 128);
+    ok &= make_map_f32(&gws3, g->ws3, hs, d, d, 128);
+    ok &= make_map_f32(&gws2, g->ws2, d, hs, hs, 128);
+  }
+  if (!ok) return LMOE_EINVAL;
+
+  // x_hat, the operand of the W_down and shared-expert weight gradients
+  CK(launch_k(xhat_kernel, dim3(grid_1d((long long)T * d / 8, 256)), dim3(256), 0, st, 1, (const bf16*)x,
+              (const bf16*)w->rms_gain, (const float*)h->r, (long long)T, (int)d, b->xh));
+  h->launches += 1;
+  if (hs) {
+    // the shared expert's pre-activations again: [p1 | p3] = r x (gain Ws13)^T, interleaved
+    TcParams p = tc_base(h);
+    p.tmA[0] = p.tmA[1] = x_k;
+    const int bn = pick_bn_for(T, 2 * hs, sms, 128);
+    p.tmB = h->tm_ws13[bn_index(bn)];
+    p.nseg = 1;
+    p.seg[0] = KSeg{0, 0, 0, (int)(d / 64), 0};
+    p.M = T;
+    p.M_rows = T;
+    p.n_tiles = 2 * hs / bn;
+    p.tmOut = ps_out;
+    p.row_scale = h->r;
+    CK(launch_tc(p, EPI_BF16, bn, std::min(mt * p.n_tiles, sms), st));
+    // dL/d act_s = dy Ws2 and through the SwiGLU: [dL/dp1 | dL/dp3] of the shared expert
+    p = tc_base(h);
+    p.tmA[0] = p.tmA[1] = dy_k;
+    p.tmB = ws2_mn;
+    p.b_mn = 1;
+    p.nseg = 1;
+    p.seg[0] = KSeg{0, 0, 0, (int)(d / 64), 0};
+    p.M = T;
+    p.M_rows = T;
+    const int bn3 = pick_bn_for(T, hs, sms, 64);
+    p.n_tiles = hs / bn3;
+    p.tmOut = dps_out;
+    p.aux = b->ps;
+    p.ld_aux = 2 * hs;
+    p.split = hs;
+    CK(launch_tc(p, EPI_SWIGLU_BWD, bn3, std::min(mt * p.n_tiles, sms), st));
+    h->launches += 2;
+  }
+  {  // dL/dz = dy W_up
+    TcParams p = tc_base(h);
+    p.tmA[0] = p.tmA[1] = dy_k;
+    p.tmB = wup_mn;
+    p.b_mn = 1;
+    p.nseg = 1;
+    p.seg[0] = KSeg{0, 0, 0, (int)(d / 64), 0};
+    p.M = T;
+    p.M_rows = T;
+    const int bn = pick_bn_for(T, l, sms, 64);
+    p.n_tiles = l / bn;
+    p.tmOut = dz_out;
+    CK(launch_tc(p, EPI_BF16, bn, std::min(mt * p.n_tiles, sms), st));
+    h->launches += 1;
+  }
+  // combine and gates: dL/do of every pair, dL/dlogit
+  CK(launch_k(combine_bwd_kernel, dim3((T + 7) / 8), dim3(256), 0, st, 1, (const bf16*)b->dz, (const bf16*)h->o,
+              (const int*)h->prow, (const float*)h->gates, (const int*)h->idx, (const float*)h->s, T, c.k, (int)l,
+              (int)E, b->d_o, b->dlogit, b->dlp));
+  h->launches += 1;
+  {  // routed experts: pre-activations again, [p1 | p3] = A_perm W13_e^T (interleaved)
+    TcParams p = tc_base(h);
+    p.tmA[0] = p.tmA[1] = h->tm_aperm;
+    p.tmB = h->tm_w13;
+    p.nseg = 1;
+    p.seg[0] = KSeg{0, 0, 0, (int)(l / 64), 0};
+    p.grouped = 1;
+    p.n_tiles = 2 * hh / h->bn_e1;
+    p.mtile_table = h->mtiles;
+    p.num_mtiles = h->num_mtiles;
+    p.b_rows_per_group = 2 * hh;
+    p.tmOut = b->pe_out;
+    CK(launch_tc(p, EPI_BF16, h->bn_e1, sms, st));
+    // dL/d act_e = dL/do W2_e, through the SwiGLU: [dL/dp1 | dL/dp3] (zero past each expert's rows)
+    p = tc_base(h);
+    p.tmA[0] = p.tmA[1] = b->do_k;
+    p.tmB = w2_mn;
+    p.b_mn = 1;
+    p.nseg = 1;
+    p.seg[0] = KSeg{0, 0, 0, (int)(l / 64), 0};
+    p.grouped = 1;
+    const int bn5 = hh % 256 == 0 ? 256 : (hh % 128 == 0 ? 128 : 64);
+    p.n_tiles = (int)(hh / bn5);
+    p.mtile_table = h->mtiles;
+    p.num_mtiles = h->num_mtiles;
+    p.b_rows_per_group = (int)l;
+    p.tmOut = b->dpe_out;
+    p.aux = b->pe;
+    p.ld_aux = 2 * hh;
+    p.split = hh;
+    CK(launch_tc(p, EPI_SWIGLU_BWD, bn5, sms, st));
+    // dL/dh of each pair = dL/dp1 W1_e + dL/dp3 W3_e
+    p = tc_base(h);
+    p.tmA[0] = p.tmA[1] = b->dpe_k;
+    p.tmB = w1_mn;
+    p.tmB2[0] = w3_mn;
+    p.b_mn = 1;
+    p.nseg = 2;
+    p.seg[0] = KSeg{0, 0, 0, (int)(hh / 64), 0};
+    p.seg[1] = KSeg{0, (int)hh, 0, (int)(hh / 64), 1};
+    p.grouped = 1;
+    const int bn6 = l % 256 == 0 ? 256 : (l % 128 == 0 ? 128 : 64);
+    p.n_tiles = (int)(l / bn6);
+    p.mtile_table = h->mtiles;
+    p.num_mtiles = h->num_mtiles;
+    p.b_rows_per_group = (int)hh;
+    p.tmOut = b->dhe_out;
+    CK(launch_tc(p, EPI_BF16, bn6, sms, st));
+    h->launches += 3;
+  }
+  // rows past each expert's last pair, up to its next 64-row boundary: zero in A_perm, act and
+  // dL/do, the operands of the expert weight gradients
+  CK(launch_k(pad_zero_kernel, dim3((unsigned)E), dim3(256), 0, st, 1, (const int*)h->offsets,
+              (const int*)h->pad_delta, (const int*)h->counts, (bf16*)h->a_perm, (int)l, (bf16*)h->act, (int)hh,
+              b->d_o, (int)l));
+  h->launches += 1;
+  {  // dW1_e, dW3_e = [dL/dp1 | dL/dp3]^T A_perm and dW2_e = (dL/do)^T act over each expert's rows
+    TcParams p = tc_base(h);
+    p.tmA[0] = p.tmA[1] = b->dpe_mn;
+    p.tmB = b->aperm_mn;
+    p.a_mn = p.b_mn = 1;
+    p.grouped_k = 1;
+    p.k_groups = (int)E;
+    p.k_first = h->offsets;
+    p.k_pad = h->pad_delta;
+    p.k_rows = h->counts;
+    p.M = (int)(2 * hh);
+    p.M_rows = p.M;
+    const int bn7 = l % 256 == 0 ? 256 : (l % 128 == 0 ? 128 : 64);
+    p.n_tiles = (int)(l / bn7);
+    p.nseg = 1;
+    p.seg[0] = KSeg{0, 0, 0, 0, 0};
+    p.tmOut = gw1;
+    p.tmOut2 = gw3;
+    p.out_split = (int)hh;
+    CK(launch_tc(p, EPI_F32, bn7, sms, st));
+    p.tmA[0] = p.tmA[1] = b->do_mn;
+    p.tmB = b->act_mn;
+    p.M = (int)l;
+    p.M_rows = p.M;
+    const int bn8 = hh % 256 == 0 ? 256 : (hh % 128 == 0 ? 128 : 64);
+    p.n_tiles = (int)(hh / bn8);
+    p.tmOut = gw2;
+    p.out_split = 0;
+    CK(launch_tc(p, EPI_F32, bn8, sms, st));
+    h->launches += 2;
+  }
+  // router: dL/dc, dW_r = dlogit^T h, and its part of dL/dh = dlogit W_r
+  CK(launch_k(bias_grad_kernel, dim3((unsigned)((E + 7) / 8)), dim3(256), 0, st, 1, (const int*)h->offsets,
+              (const int*)h->pad_delta, (const int*)h->counts, (const float*)b->dlp, (int)E, g->router_bias));
+  h->launches += 1;
+  {
+    TcParams p = tc_base(h);
+    p.tmA[0] = p.tmA[1] = dlg_mn;
+    p.tmB = hx_mn;
+    p.tmOut = gwr;
+    int rc = wgrad_gemm(h, p, (int)E, (int)l, T, (size_t)E * l * 4, g->w_router, 0, nullptr, st);
+    if (rc) return rc;
+    p = tc_base(h);
+    p.tmA[0] = p.tmA[1] = dlg_k;
+    p.tmB = wr_hi_mn;
+    p.tmB2[0] = wr_mid_mn;
+    p.b_mn = 1;
+    p.nseg = 2;
+    p.seg[0] = KSeg{0, 0, 0, (int)(E / 64), 0};
+    p.seg[1] = KSeg{0, 0, 0, (int)(E / 64), 1};
+    p.M = T;
+    p.M_rows = T;
+    const int bn = pick_bn_for(T, l, sms, 64);
+    p.n_tiles = l / bn;
+    p.tmOut = dhr_out;
+    CK(launch_tc(p, EPI_F32, bn, std::min(mt * p.n_tiles, sms), st));
+    h->launches += 1;
+  }
+  // dL/dh = the router's part + the experts' parts of the token's pairs
+  CK(launch_k(scatter_dh_kernel, dim3((T + 7) / 8), dim3(256), 0, st, 1, (const float*)b->dhr, (const bf16*)b->dhe,
+              (const int*)h->prow, T, c.k, (int)l, b->dh));
+  h->launches += 1;
+  {  // dW_down = (dL/dh)^T x_hat
+    TcParams p = tc_base(h);
+    p.tmA[0] = p.tmA[1] = dh_mn;
+    p.tmB = xh_mn;
+    p.tmOut = gwd;
+    int rc = wgrad_gemm(h, p, (int)l, (int)d, T, (size_t)l * d * 4, g->w_down, 0, nullptr, st);
+    if (rc) return rc;
+  }
+  {  // dL/dx_hat = dL/dh W_down + dL/dp1_s Ws1 + dL/dp3_s Ws3
+    TcParams p = tc_base(h);
+    p.tmA[0] = dh_k;
+    p.tmA[1] = hs ? dps_k : dh_k;
+    p.tmB = wd_mn;
+    if (hs) {
+      p.tmB2[0] = ws1_mn;
+      p.tmB2[1] = ws3_mn;
+    }
+    p.b_mn = 1;
+    p.nseg = hs ? 3 : 1;
+    p.seg[0] = KSeg{0, 0, 0, (int)(l / 64), 0};
+    p.seg[1] = KSeg{1, 0, 0, (int)(hs / 64), 1};
+    p.seg[2] = KSeg{1, (int)hs, 0, (int)(hs / 64), 2};
+    p.M = T;
+    p.M_rows = T;
+    const int bn = pick_bn_for(T, d, sms, 64);
+    p.n_tiles = d / bn;
+    p.tmOut = dxh_out;
+    CK(launch_tc(p, EPI_F32, bn, std::min(mt * p.n_tiles, sms), st));
+    h->launches += 1;
+  }
+  if (hs) {  // dWs1, dWs3 = [dL/dp1_s | dL/dp3_s]^T x_hat;  dWs2 = dy^T act_s
+    TcParams p = tc_base(h);
+    p.tmA[0] = p.tmA[1] = dps_mn;
+    p.tmB = xh_mn;
+    p.tmOut = gws1;
+    p.tmOut2 = gws3;
+    p.out_split = (int)hs;
+    int rc = wgrad_gemm(h, p, (int)(2 * hs), (int)d, T, (size_t)hs * d * 4, g->ws1, (size_t)hs * d * 4, g->ws3, st);
+    if (rc) return rc;
+    p = tc_base(h);
+    p.tmA[0] = p.tmA[1] = dy_mn;
+    p.tmB = as_mn;
+    p.tmOut = gws2;
+    rc = wgrad_gemm(h, p, (int)d, (int)hs, T, (size_t)d * hs * 4, g->ws2, 0, nullptr, st);
+    if (rc) return rc;
+  }
+  {  // dW_up = dy^T z
+    TcParams p = tc_base(h);
+    p.tmA[0] = p.tmA[1] = dy_mn;
+    p.tmB = z_mn;
+    p.tmOut = gwup;
+    int rc = wgrad_gemm(h, p, (int)d, (int)l, T, (size_t)d * l * 4, g->w_up, 0, nullptr, st);
+    if (rc) return rc;
+  }
+  // RMSNorm: dL/dx and dL/dgain
+  const int nrb = (T + kRmsRows - 1) / kRmsRows;
+  CK(launch_k(rms_bwd_kernel, dim3(nrb), dim3(256), 0, st, 1, (const bf16*)x, (const bf16*)w->rms_gain,
+              (const float*)h->r, (const float*)b->dxh, T, (int)d, g->dx, b->gpart));
+  if (g->rms_gain)
+    CK(launch_k(colsum_kernel, dim3((unsigned)((d + 255) / 256)), dim3(256), 0, st, 1, (const float*)b->gpart, nrb,
+                (int)d, g->rms_gain));
+  h->launches += 2;
+  return LMOE_OK;
+}
+
 }  // namespace
 
 // ======================================================================= C ABI
@@ -1379,6 +1779,7 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, void* stream, lmo
 int lmoe_destroy(lmoe_handle* h) {
   if (!h) return LMOE_EINVAL;
   cudaDeviceSynchronize();
+  bwd_free(h);
   for (auto& r : h->prof)
     for (auto& e : r.ev) cudaEventDestroy(e);
   for (auto& g : h->g_fwd) g.reset(nullptr, nullptr, -1, 0, 0.f, 0);
@@ -1439,6 +1840,30 @@ int lmoe_forward(lmoe_handle* h, const void* x, void* y, int32_t T, uint32_t fla
     }
   }
   return rc;
+}
+
+int lmoe_forward_backward(lmoe_handle* h, const lmoe_weights* w, const void* x, const void* dy, void* y, int32_t T,
+                          uint32_t flags, const lmoe_grads* g, void* stream) {
+  if (!h || !w || !g || T < 0 || T > h->cfg.max_tokens) return LMOE_EINVAL;
+  if (!h->bf || h->q8) return LMOE_EUNSUPPORTED;
+  if (flags & (LMOE_UPDATE_BIAS | LMOE_ASYNC_OUTPUT)) return LMOE_EINVAL;
+  const lmoe_config& c = h->cfg;
+  // 128-row tiles of the weight gradients never straddle two experts or the W1 / W3 (Ws1 / Ws3)
+  // boundary
+  if (c.l % 128 || c.h % 128 || c.hs % 128) return LMOE_EUNSUPPORTED;
+  if (!w->w_down || !w->w_router || !w->w1 || !w->w3 || !w->w2 || !w->w_up) return LMOE_EINVAL;
+  if (c.hs && (!w->ws1 || !w->ws3 || !w->ws2)) return LMOE_EINVAL;
+  if (!g->dx || !g->w_down || !g->w_router || !g->router_bias || !g->w1 || !g->w3 || !g->w2 || !g->w_up)
+    return LMOE_EINVAL;
+  if (c.hs && (!g->ws1 || !g->ws3 || !g->ws2)) return LMOE_EINVAL;
+  if (!dy || ((uintptr_t)dy & 15)) return LMOE_EINVAL;
+  if (T == 0) return LMOE_OK;
+  int rc = bwd_alloc(h);
+  if (rc) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  rc = lmoe_forward(h, x, y, T, flags, stream);
+  if (rc) return rc;
+  return backward_bf16(h, w, x, dy, T, g, st);
 }
 
 int lmoe_forward_host(lmoe_handle* h, const void* x_host, void* y_host, int32_t T, uint32_t flags, void* stream) {
@@ -1669,6 +2094,37 @@ int lmoe_gemm_bf16(const void* a, const void* b, float* c, int32_t M, int32_t N,
     const int tiles = ((M + 127) / 128) * p.n_tiles;
     CK(launch_tc(p, EPI_F32, bn, tiles < sms ? tiles : sms, (cudaStream_t)stream));
   }
+  return LMOE_OK;
+}
+
+int lmoe_gemm_bf16_ex(const void* a, int32_t a_mn, const void* b, int32_t b_mn, float* c, int32_t M, int32_t N,
+                      int32_t K, int32_t k_split, void* stream) {
+  if (!a || !b || !c || M <= 0 || N <= 0 || K <= 0 || N % 64 || K % 8 || k_split < 1) return LMOE_EINVAL;
+  if ((a_mn && M % 8) || (b_mn && N % 8)) return LMOE_EINVAL;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int bn = pick_bn(N);
+  TcParams p;
+  memset(&p, 0, sizeof(p));
+  bool ok = a_mn ? make_map(&p.tmA[0], a, K, M, M, 64) : make_map(&p.tmA[0], a, M, K, K, 128);
+  ok &= b_mn ? make_map(&p.tmB, b, K, N, N, 64) : make_map(&p.tmB, b, N, K, K, bn);
+  ok &= make_map_f32(&p.tmOut, c, M, N, N, 128);
+  if (!ok) return LMOE_EINVAL;
+  p.tmA[1] = p.tmA[0];
+  p.a_mn = a_mn ? 1 : 0;
+  p.b_mn = b_mn ? 1 : 0;
+  p.nseg = 1;
+  p.seg[0] = KSeg{0, 0, 0, (K + 63) / 64, 0};
+  if (k_split > p.seg[0].nkb) return LMOE_EINVAL;
+  p.k_split = k_split;
+  p.M = M;
+  p.M_rows = M;
+  p.n_tiles = N / bn;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (k_split > 1) CK(cudaMemsetAsync(c, 0, (size_t)M * N * 4, st));
+  const long long tiles = (long long)((M + 127) / 128) * p.n_tiles * k_split;
+  CK(launch_tc(p, EPI_F32, bn, (int)(tiles < sms ? tiles : sms), st));
   return LMOE_OK;
 }
 

@@ -48,13 +48,17 @@ enum TcEpilogue : int {
   EPI_ROUTER = 4,  // out fp32 = sigmoid(acc + col_bias[col])
   EPI_SWIGLU3 = 5, // as EPI_SWIGLU with an accurate SiLU, the fp32 result stored as hi, mid, lo bf16
                    // parts (columns part * split + c) for the next split-precision product
+  EPI_SWIGLU_BWD = 6,  // acc = dL/d act of a SwiGLU; with its pre-activations p1 (gate) and p3
+                       // (linear) read from aux, out bf16: dL/dp1 = acc p3 silu'(p1) at column c and
+                       // dL/dp3 = acc silu(p1) at column split + c; rows past the tile's valid rows 0
 };
 
 struct KSeg {
   int a_map;  // 0 or 1
-  int a_col;  // first A column of the segment
-  int b_col;  // first B column of the segment
+  int a_col;  // first A column of the segment (MN-major A: first K row)
+  int b_col;  // first B column of the segment (MN-major B: first K row)
   int nkb;    // k-blocks of 64
+  int b_map;  // 0: tmB, 1 / 2: tmB2[0] / tmB2[1]
 };
 
 struct TcParams {
@@ -80,6 +84,21 @@ struct TcParams {
   int hint_out;               // 1: store the output with L2 evict_last (the next kernel reads it)
   int band_n;                 // non-grouped: N-tiles per band of the tile order (0: row-major order)
   uint32_t* status;
+  // ---- the layer backward's products
+  CUtensorMap tmB2[2];        // B maps of segments with b_map 1 and 2
+  CUtensorMap tmOut2;         // output of the rows at or past out_split (re-based to row 0)
+  int out_split;              // 0: one output map
+  int a_mn, b_mn;             // operand stored MN-major: A as [K, M], B as [K, N] (64 x 64 boxes)
+  int grouped_k;              // expert weight gradients: K runs over one expert's rows
+  int k_groups;               // grouped_k: experts (tiles = k_groups x M-tiles x N-tiles)
+  const int* k_first;         // grouped_k: first row of each expert, unpadded ...
+  const int* k_pad;           // ... plus this: its first row in the padded layout
+  const int* k_rows;          // grouped_k: rows of each expert
+  const bf16* aux;            // EPI_SWIGLU_BWD: [rows, 2 split] pre-activations, gate and linear
+  int ld_aux;                 // columns interleaved in groups of 64 (as the forward's weights)
+  int k_split;                // > 1 (non-grouped, one segment, EPI_F32): the k-blocks are cut into
+                              // k_split ranges, one tile each, whose results are added into the
+                              // output (zeroed first) by TMA reductions
 };
 
 // PAIR = 1: a cluster of two CTAs computes one 256 x BN tile with tcgen05.mma.cta_group::2; each
@@ -98,7 +117,13 @@ struct TcCfg {
 
 struct TileInfo {
   int row0, b_row0, n0;
-  int q;  // 32-row quarters of the tile that are loaded and stored (4 = all)
+  int q;         // 32-row quarters of the tile that are loaded and stored (4 = all)
+  int out_y;     // first output row of the tile
+  int sel;       // output map: 0 tmOut (or its trimmed forms), 1 tmOut2
+  int valid;     // rows of the tile that hold data (grouped: the expert's rows; else up to M)
+  int ak0, bk0;  // first K row of an MN-major A / B operand (grouped modes: the expert's)
+  int kb0, nkb;  // grouped_k / k_split: first k-block and k-blocks of the tile; nkb -1: the
+                 // segments' own counts
 };
 
 // Tile order: row-major over (M-tile, N-tile), or, with band_n > 0 (non-grouped), band by band:
@@ -107,6 +132,42 @@ struct TileInfo {
 __device__ __forceinline__ TileInfo tc_tile(const TcParams& p, int tile, int BN, int pair, uint32_t rank) {
   TileInfo ti;
   int mt, nt;
+  ti.q = 4;
+  ti.sel = 0;
+  ti.valid = 128;
+  ti.ak0 = 0;
+  ti.bk0 = 0;
+  ti.kb0 = 0;
+  ti.nkb = -1;
+  if (p.k_split > 1) {
+    // split s of a one-segment K: tiles [s*base, (s+1)*base) cover k-blocks [s*nkb/S, (s+1)*nkb/S)
+    const int base = ((p.M + 127) >> 7) * p.n_tiles;
+    const int sp = tile / base;
+    tile -= sp * base;
+    const int nk = p.seg[0].nkb;
+    ti.kb0 = (int)(((long long)sp * nk) / p.k_split);
+    ti.nkb = (int)(((long long)(sp + 1) * nk) / p.k_split) - ti.kb0;
+  }
+  if (p.grouped_k) {
+    // expert-major: all (M-tile, N-tile) pairs of one expert's gradient, then the next expert's
+    const int per = ((p.M + 127) >> 7) * p.n_tiles;
+    const int e = tile / per;
+    const int idx = tile - e * per;
+    mt = idx / p.n_tiles;
+    nt = idx - mt * p.n_tiles;
+    ti.n0 = nt * BN;
+    ti.row0 = mt * 128;
+    ti.b_row0 = ti.n0;
+    ti.ak0 = ti.bk0 = p.k_first[e] + p.k_pad[e];
+    ti.nkb = (p.k_rows[e] + 63) >> 6;
+    int m = ti.row0;
+    if (p.out_split && m >= p.out_split) {
+      ti.sel = 1;
+      m -= p.out_split;
+    }
+    ti.out_y = e * (p.out_split ? p.out_split : p.M) + m;
+    return ti;
+  }
   if (p.band_n > 0 && !p.grouped) {
     const int m_tiles = pair ? (p.M + 255) / 256 : (p.M + 127) / 128;
     const int per_band = m_tiles * p.band_n;
@@ -120,7 +181,6 @@ __device__ __forceinline__ TileInfo tc_tile(const TcParams& p, int tile, int BN,
     nt = tile - mt * p.n_tiles;
   }
   ti.n0 = nt * BN;
-  ti.q = 4;
   if (pair) {  // 256-row tiles; this CTA owns rows 128*rank.. and B rows BN/2*rank..
     ti.row0 = mt * 256 + (int)rank * 128;
     ti.b_row0 = ti.n0 + (int)rank * (BN / 2);
@@ -128,15 +188,25 @@ __device__ __forceinline__ TileInfo tc_tile(const TcParams& p, int tile, int BN,
     int2 e_r = p.mtile_table[mt];
     ti.row0 = e_r.y;
     ti.b_row0 = (e_r.x & 0xFFFF) * p.b_rows_per_group + ti.n0;
+    ti.bk0 = (e_r.x & 0xFFFF) * p.b_rows_per_group;
+    ti.valid = e_r.x >> 16;
     if (p.trim) ti.q = ((e_r.x >> 16) + 31) >> 5;
   } else {
     ti.row0 = mt * 128;
     ti.b_row0 = ti.n0;
+    ti.valid = min(128, p.M - ti.row0);
+  }
+  ti.out_y = ti.row0;
+  if (p.out_split && ti.row0 >= p.out_split) {
+    ti.sel = 1;
+    ti.out_y -= p.out_split;
   }
   return ti;
 }
 
 __device__ __forceinline__ int tc_num_tiles(const TcParams& p, int pair) {
+  if (p.grouped_k) return p.k_groups * ((p.M + 127) >> 7) * p.n_tiles;
+  if (p.k_split > 1) return p.k_split * ((p.M + 127) >> 7) * p.n_tiles;
   int mt = p.grouped ? *p.num_mtiles : (pair ? (p.M + 255) / 256 : (p.M + 127) / 128);
   return mt * p.n_tiles;
 }
@@ -231,10 +301,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         // k-blocks segment by segment, or (split router) chunk by chunk over the three segments
         const int nouter = kSplit3 ? p.seg[0].nkb : p.nseg;
         for (int o = 0; ok && o < nouter; ++o) {
-          const int ninner = kSplit3 ? 3 : p.seg[o].nkb;
+          const int ninner = kSplit3 ? 3 : (ti.nkb >= 0 ? ti.nkb : p.seg[o].nkb);
           for (int in = 0; in < ninner; ++in) {
             const KSeg sg = p.seg[kSplit3 ? in : o];
-            const int kb = kSplit3 ? o : in;
+            const int kb = kSplit3 ? o : ti.kb0 + in;
             if (!mbar_wait(&empty[stage], phase ^ 1u, abort, p.status)) {
               ok = false;
               break;
@@ -247,17 +317,36 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
               if (leader) mbar_expect_tx(&full[stage], 2 * C::kStageBytes);
               tma_load_2d_pair(a_dst, &p.tmA[sg.a_map], bar0, sg.a_col + kb * 64, ti.row0);
               tma_load_2d_pair(b_dst, &p.tmB, bar0, sg.b_col + kb * 64, ti.b_row0);
+            } else if (p.a_mn | p.b_mn) {
+              // MN-major operands: one 64 x 64 box per 64 columns of M (N), 64 K rows each
+              const CUtensorMap* bmap = sg.b_map ? &p.tmB2[sg.b_map - 1] : &p.tmB;
+              mbar_expect_tx(&full[stage], (uint32_t)(C::kABytes + C::kBBytes));
+              if (p.a_mn) {
+                const int ky = ti.ak0 + sg.a_col + kb * 64;
+                tma_load_2d(a_dst, &p.tmA[sg.a_map], &full[stage], ti.row0, ky);
+                tma_load_2d(a_dst + 8192, &p.tmA[sg.a_map], &full[stage], ti.row0 + 64, ky);
+              } else {
+                tma_load_2d(a_dst, &p.tmA[sg.a_map], &full[stage], sg.a_col + kb * 64, ti.row0);
+              }
+              if (p.b_mn) {
+                const int ky = ti.bk0 + sg.b_col + kb * 64;
+#pragma unroll
+                for (int c = 0; c < BN / 64; ++c) tma_load_2d(b_dst + c * 8192, bmap, &full[stage], ti.n0 + 64 * c, ky);
+              } else {
+                tma_load_2d(b_dst, bmap, &full[stage], sg.b_col + kb * 64, ti.b_row0);
+              }
             } else {
               const CUtensorMap* amap = ti.q < 4 ? &p.tmA_part[ti.q - 1] : &p.tmA[sg.a_map];
+              const CUtensorMap* bmap = sg.b_map ? &p.tmB2[sg.b_map - 1] : &p.tmB;
               mbar_expect_tx(&full[stage], (uint32_t)(ti.q * 32 * 128 + C::kBBytes));
               if (p.hint_a)
                 tma_load_2d_hint(a_dst, amap, &full[stage], sg.a_col + kb * 64, ti.row0, pol_first);
               else
                 tma_load_2d(a_dst, amap, &full[stage], sg.a_col + kb * 64, ti.row0);
               if (p.hint_b)
-                tma_load_2d_hint(b_dst, &p.tmB, &full[stage], sg.b_col + kb * 64, ti.b_row0, pol_first);
+                tma_load_2d_hint(b_dst, bmap, &full[stage], sg.b_col + kb * 64, ti.b_row0, pol_first);
               else
-                tma_load_2d(b_dst, &p.tmB, &full[stage], sg.b_col + kb * 64, ti.b_row0);
+                tma_load_2d(b_dst, bmap, &full[stage], sg.b_col + kb * 64, ti.b_row0);
             }
             armed |= 1u << stage;
             armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
@@ -279,6 +368,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     if (lane == 0 && leader) {
       // ---------------- MMA issuer (the even CTA of a pair issues for both)
       constexpr uint32_t idesc = idesc_bf16_f32(BN, PAIR ? 256 : 128);
+      // MN-major operands (not in pairs): transpose bits of the instruction descriptor
+      const uint32_t idesc_t = idesc | (p.a_mn ? 1u << 15 : 0u) | (p.b_mn ? 1u << 16 : 0u);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
@@ -336,8 +427,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
           continue;
         }
         int kbi = 0;
+        const int tnkb = (p.grouped_k || p.k_split > 1) ? tc_tile(p, tile, BN, PAIR, rank).nkb : -1;
         for (int s = 0; ok && s < p.nseg; ++s) {
-          const int nkb = p.seg[s].nkb;
+          const int nkb = tnkb >= 0 ? tnkb : p.seg[s].nkb;
           for (int kb = 0; kb < nkb; ++kb, ++kbi) {
             if (!mbar_wait(&full[stage], phase, abort, p.status)) {
               ok = false;
@@ -348,12 +440,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             const uint32_t b_addr = a_addr + C::kABytes;
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              if constexpr (PAIR)
+              if constexpr (PAIR) {
                 tc_mma_bf16_pair(d_tmem, smem_desc_sw128(a_addr + k * 32), smem_desc_sw128(b_addr + k * 32), idesc,
                                  (kbi | k) != 0);
-              else
-                tc_mma_bf16(d_tmem, smem_desc_sw128(a_addr + k * 32), smem_desc_sw128(b_addr + k * 32), idesc,
-                            (kbi | k) != 0);
+              } else {
+                // K-major: the next 16 K columns are 32 bytes on in each 128-byte row; MN-major: 16
+                // K rows of 128 bytes further
+                const uint64_t ad = p.a_mn ? smem_desc_mn128(a_addr + k * 2048) : smem_desc_sw128(a_addr + k * 32);
+                const uint64_t bd = p.b_mn ? smem_desc_mn128(b_addr + k * 2048) : smem_desc_sw128(b_addr + k * 32);
+                tc_mma_bf16(d_tmem, ad, bd, idesc_t, (kbi | k) != 0);
+              }
             }
             if constexpr (PAIR)
               tc_commit_pair(&empty[stage]);
@@ -411,7 +507,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         __syncwarp();
         if (__any_sync(0xffffffffu, !good)) return false;
         if (lane == 0) {
-          if (p.hint_out)
+          if (p.k_split > 1)
+            tma_reduce_add_2d(omap, box, x, y);
+          else if (p.hint_out)
             tma_store_2d_hint(omap, box, x, y, l2_evict_last());
           else
             tma_store_2d(omap, box, x, y);
@@ -449,7 +547,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         break;
       }
       tc_fence_after();
-      omap = ti.q < 4 ? &p.tmOut_part[ti.q - 1] : &p.tmOut;
+      omap = ti.sel ? &p.tmOut2 : (ti.q < 4 ? &p.tmOut_part[ti.q - 1] : &p.tmOut);
+      const bool zero_acc = ti.nkb == 0;  // grouped_k: an expert without rows has a zero gradient
       const uint32_t tbase = tmem_base + ((uint32_t)(wq * 32) << 16) + acc * kAccCols;
       uint32_t w[16];
 
@@ -468,7 +567,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             const float u0 = __uint_as_float(uv[2 * q]) * rs, u1 = __uint_as_float(uv[2 * q + 1]) * rs;
             w[q] = pack_bf16x2(silu_fast(g0) * u0, silu_fast(g1) * u1);
           }
-          ok = emit(w, (ti.n0 >> 1) + j * 64, ti.row0);
+          ok = emit(w, (ti.n0 >> 1) + j * 64, ti.out_y);
         }
       } else if constexpr (EPI == EPI_SWIGLU3) {
 #pragma unroll 1
@@ -490,7 +589,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
               a[2 * q] -= __bfloat162float(h0);  // remainder for the next part
               a[2 * q + 1] -= __bfloat162float(h1);
             }
-            ok = emit(w, part * p.split + (ti.n0 >> 1) + j * 64, ti.row0);
+            ok = emit(w, part * p.split + (ti.n0 >> 1) + j * 64, ti.out_y);
           }
         }
       } else if constexpr (EPI == EPI_BF16) {
@@ -500,8 +599,47 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
           tmem_ld32(tbase + j * 64 + half_id * 32, v);
           tc_wait_ld();
 #pragma unroll
-          for (int q = 0; q < 16; ++q) w[q] = pack_bf16x2(__uint_as_float(v[2 * q]), __uint_as_float(v[2 * q + 1]));
-          ok = emit(w, ti.n0 + j * 64, ti.row0);
+          for (int q = 0; q < 16; ++q)
+            w[q] = pack_bf16x2(__uint_as_float(v[2 * q]) * rs, __uint_as_float(v[2 * q + 1]) * rs);
+          ok = emit(w, ti.n0 + j * 64, ti.out_y);
+        }
+      } else if constexpr (EPI == EPI_SWIGLU_BWD) {
+        // step j: accumulator columns c = n0 + j*64 + half*32 + q hold dL/d act; the gate and linear
+        // pre-activations of column c sit at aux columns (c/64)*128 + c%64 and 64 further
+        const bool live = rl < ti.valid;
+        const bf16* arow = p.aux + (size_t)(live ? row : 0) * p.ld_aux;
+#pragma unroll 1
+        for (int j = 0; ok && j < BN / 64; ++j) {
+          uint32_t v[32];
+          tmem_ld32(tbase + j * 64 + half_id * 32, v);
+          const int c0 = ti.n0 + j * 64 + half_id * 32;
+          const int g0 = ((c0 >> 6) << 7) + (c0 & 63);
+          uint4 pg[4], pu[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            pg[i] = live ? ldg_nc_v4(arow + g0 + 8 * i) : make_uint4(0, 0, 0, 0);
+            pu[i] = live ? ldg_nc_v4(arow + g0 + 64 + 8 * i) : make_uint4(0, 0, 0, 0);
+          }
+          tc_wait_ld();
+          uint32_t w3[16];
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            const uint32_t gw = (&pg[q >> 2].x)[q & 3], uw = (&pu[q >> 2].x)[q & 3];
+            float d1[2], d3[2];
+#pragma unroll
+            for (int hlf = 0; hlf < 2; ++hlf) {
+              const float g = __uint_as_float(hlf ? (gw & 0xFFFF0000u) : (gw << 16));
+              const float u = __uint_as_float(hlf ? (uw & 0xFFFF0000u) : (uw << 16));
+              const float a = __uint_as_float(v[2 * q + hlf]);
+              const float sg = sigmoidf_acc(g);
+              d1[hlf] = live ? a * u * sg * (1.0f + g * (1.0f - sg)) : 0.0f;
+              d3[hlf] = live ? a * g * sg : 0.0f;
+            }
+            w[q] = pack_bf16x2(d1[0], d1[1]);
+            w3[q] = pack_bf16x2(d3[0], d3[1]);
+          }
+          ok = emit(w, c0 - half_id * 32, ti.out_y);
+          if (ok) ok = emit(w3, p.split + c0 - half_id * 32, ti.out_y);
         }
       } else if constexpr (EPI == EPI_DOWN3) {
         // v = r * acc, stored as hi + mid + lo bf16 parts (exact to fp32's 24 bits), one box each
@@ -523,7 +661,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
               a[2 * q] -= __bfloat162float(h0);   // remainder for the next part
               a[2 * q + 1] -= __bfloat162float(h1);
             }
-            ok = emit(w, part * p.split + ti.n0 + j * 64, ti.row0);
+            ok = emit(w, part * p.split + ti.n0 + j * 64, ti.out_y);
           }
         }
       } else {
@@ -536,6 +674,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
           if constexpr (kSplit3) {
             tmem_ld16(tbase + BN + j * 32 + half_id * 16, v);  // (hi, hi)
             tmem_ld16(tbase + j * 32 + half_id * 16, vs);      // the five small products
+          } else if (zero_acc) {
+#pragma unroll
+            for (int q = 0; q < 16; ++q) v[q] = 0u;
           } else {
             tmem_ld16(tbase + j * 32 + half_id * 16, v);
           }
@@ -559,7 +700,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
 #pragma unroll
             for (int q = 0; q < 16; ++q) w[q] = v[q];
           }
-          ok = emit(w, ti.n0 + j * 32, ti.row0);
+          ok = emit(w, ti.n0 + j * 32, ti.out_y);
         }
         if (nan && row < p.M_rows) set_status(p.status, LMOE_STATUS_NAN_SCORE);
       }
