@@ -322,6 +322,69 @@ def measure(shape, args, rank, world, local_rank, e2e=True, experts=0):
     return summary, launches
 
 
+def train_flops(shape, T):
+    """Algorithmic FLOPs of one training step's layer products: every forward product and its two
+    backward products (the data gradient and the weight gradient), three times the forward's."""
+    d, l, E, k, h, hs = shape.d, shape.l, shape.E, shape.k, shape.h, shape.hs
+    fwd = 2 * T * d * l + 2 * T * l * E + 6 * T * k * l * h + 4 * T * d * hs + 2 * T * d * (l + hs)
+    return 3 * fwd
+
+
+def measure_train(shape, args, local_rank):
+    """Device-timed training steps of one layer: lmoe_forward_backward (the forward, then every
+    gradient for a fixed output gradient dy), L2 flushed between steps outside the events; and the
+    forward alone the same way, so the backward's share is known."""
+    import torch
+
+    import datagen
+    import latent_routing_quantile_b200 as lq
+
+    T = shape.T
+    w_dev = {n: t.cuda() for n, t in datagen.layer_weights(shape).items()}
+    layer = lq.Layer(shape.d, shape.l, shape.E, shape.k, shape.h, shape.hs, lq.BF16, T, w_dev,
+                     rms_eps=shape.rms_eps)
+    x = datagen.tokens(shape).cuda()
+    dy = datagen.output_grad(shape, seed=shape.seed + 100).cuda()
+    y = torch.empty_like(x)
+    _, g = layer.forward_backward(x, dy, w_dev, y=y)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            flush.zero_()
+            fn()
+        torch.cuda.synchronize()
+        st = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        en = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush.zero_()
+            st[i].record(stream)
+            fn()
+            en[i].record(stream)
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in zip(st, en)) / args.steps
+
+    l0 = layer.launches()
+    with ClockSampler(local_rank) as clk:
+        ms = timed(lambda: layer.forward_backward(x, dy, w_dev, y=y, grads=g))
+    launches = (layer.launches() - l0) // (args.warmup + args.steps)
+    ms_fwd = timed(lambda: layer.forward(x, y))
+    assert layer.status() == 0, "device status word set during the training bench"
+    layer.close()
+    del g, w_dev, flush
+    torch.cuda.empty_cache()
+    peaks, peak_src = load_peaks()
+    fl = train_flops(shape, T)
+    return {"workload": shape.name, "T": T, "ms_per_step": round(ms, 5), "value": round(T / (ms / 1e3), 1),
+            "unit": "tokens/s", "forward_ms": round(ms_fwd, 5), "backward_ms": round(ms - ms_fwd, 5),
+            "gpu_launches_per_step": launches, "algorithmic_tflop": round(fl / 1e12, 4),
+            "tflops": round(fl / (ms / 1e3) / 1e12, 1),
+            "frac_of_bf16_peak": round(fl / (ms / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
+            "peak_source": f"{peak_src}, burst", "clocks": clk.summary(),
+            "step": "lmoe_forward_backward: forward, then dL/dx and every weight gradient (fp32) for a fixed dy"}
+
+
 def roofline(summary, shape, name):
     """The roofline object of one kernel (stage) of a measured workload."""
     peaks, peak_src = summary["peaks"]
@@ -355,11 +418,14 @@ def run_ours(args, rank, world, local_rank):
     if args.tokens:
         shape = shape.with_tokens(args.tokens)
     main_s, launches = measure(shape, args, rank, world, local_rank, experts=1 if args.experts == "mxfp8" else 0)
-    also = {}
+    also, train = {}, {}
     if world == 1 and args.also and not args.tokens:
         for spec in args.also.split(","):
             parts = spec.split(":")
             sh = datagen.WORKLOADS[parts[0]].with_tokens(int(parts[1]))
+            if len(parts) > 2 and parts[2] == "train":
+                train[sh.name] = measure_train(sh, args, local_rank)
+                continue
             mx = len(parts) > 2 and parts[2] == "mxfp8"
             s2, _ = measure(sh, args, rank, world, local_rank, e2e=False, experts=1 if mx else 0)
             also[sh.name + ("_mxfp8" if mx else "")] = s2
@@ -408,6 +474,8 @@ def run_ours(args, rank, world, local_rank):
                 "expert_gemm_frac_of_format_peak": a["expert_gemm_frac_of_format_peak"],
                 "tensor_peak_frac_step": a["tensor_peak_frac_step"], "kernels": a["kernels"], "clocks": a["clocks"]}
             for n, a in also.items()}
+    if train:
+        out["train"] = train
     return out
 
 
@@ -515,12 +583,16 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="wide_stress")
     ap.add_argument("--tokens", type=int, default=0)
-    ap.add_argument("--also", default="sweep:262144,wide_stress:16384:mxfp8",
-                    help="extra workloads (name:T[:mxfp8], comma-separated) measured in the same call on one GPU, "
-                         "':mxfp8' with 8-bit routed experts; '' for none")
+    ap.add_argument("--also", default="sweep:262144,wide_stress:16384:mxfp8,mini_replica:8192:train",
+                    help="extra workloads (name:T[:mxfp8|:train], comma-separated) measured in the same call on one "
+                         "GPU, ':mxfp8' with 8-bit routed experts, ':train' as training steps (forward + backward); "
+                         "'' for none")
     ap.add_argument("--experts", choices=["bf16", "mxfp8"], default="bf16",
                     help="operand format of the routed experts of the main workload")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--train-only", default="",
+                    help="name:T: time only training steps (lmoe_forward_backward) of that workload on one GPU and "
+                         "print their summary (for profiling the backward)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     world_env = os.environ.get("WORLD_SIZE")
@@ -540,6 +612,16 @@ def main():
         out = run_reference(args, rank)
         if out is not None:
             print(json.dumps(out), flush=True)
+        return
+
+    if args.train_only:
+        import torch
+
+        import datagen
+        name, t = args.train_only.split(":")
+        torch.cuda.set_device(local_rank)
+        print(json.dumps({"train": {name: measure_train(datagen.WORKLOADS[name].with_tokens(int(t)), args,
+                                                        local_rank)}}), flush=True)
         return
 
     import datetime

@@ -185,9 +185,20 @@ __global__ void __launch_bounds__(256) scatter_dh_kernel(const float* __restrict
 
 // RMSNorm backward over a block of kRmsRows tokens.  With gdx = gain * dL/dx_hat:
 //   dL/dx = gdx r - x r^3 / d * sum_m gdx_m x_m;   dL/dgain_m = sum_t dL/dx_hat_m x_m r.
-// Phase 1 (a warp per token) forms each row's sum; phase 2 (threads over columns, tokens in
-// order) writes dL/dx and this block's partial dL/dgain, so the sums need no atomics.
-constexpr int kRmsRows = 64;
+// Phase 1 (a warp per token, 16-byte loads) forms each row's sum; phase 2 (a thread per 8
+// columns, the block's tokens in order) writes dL/dx and this block's partial dL/dgain, so the
+// sums need no atomics and come out the same every run.
+constexpr int kRmsRows = 32;
+__device__ __forceinline__ void load8_f32(const float* p, float (&v)[8]) {
+  const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void load8_bf16(const bf16* p, float (&v)[8]) {
+  const uint4 q = *reinterpret_cast<const uint4*>(p);
+  const bf16* e = reinterpret_cast<const bf16*>(&q);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) v[j] = bf2f(e[j]);
+}
 __global__ void __launch_bounds__(256) rms_bwd_kernel(const bf16* __restrict__ x, const bf16* __restrict__ gain,
                                                       const float* __restrict__ r, const float* __restrict__ dxh,
                                                       int ntok, int d, float* __restrict__ dx,
@@ -197,13 +208,18 @@ __global__ void __launch_bounds__(256) rms_bwd_kernel(const bf16* __restrict__ x
   __shared__ float dot[kRmsRows];
   const int t0 = blockIdx.x * kRmsRows;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nv = d / 8;
   for (int tt = warp; tt < kRmsRows; tt += 8) {
     const int t = t0 + tt;
     float acc = 0.f;
     if (t < ntok)
-      for (int c = lane; c < d; c += 32) {
-        const float gm = gain ? bf2f(gain[c]) : 1.f;
-        acc = fmaf(gm * dxh[(size_t)t * d + c], bf2f(x[(size_t)t * d + c]), acc);
+      for (int v = lane; v < nv; v += 32) {
+        float xv[8], gv[8], gm[8];
+        load8_bf16(x + (size_t)t * d + 8 * v, xv);
+        load8_f32(dxh + (size_t)t * d + 8 * v, gv);
+        if (gain) load8_bf16(gain + 8 * v, gm);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc = fmaf((gain ? gm[j] : 1.f) * gv[j], xv[j], acc);
       }
 #pragma unroll
     for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(kFull, acc, off);
@@ -211,32 +227,60 @@ __global__ void __launch_bounds__(256) rms_bwd_kernel(const bf16* __restrict__ x
   }
   __syncthreads();
   const float inv_d = 1.f / (float)d;
-  for (int c = threadIdx.x; c < d; c += blockDim.x) {
-    const float gm = gain ? bf2f(gain[c]) : 1.f;
-    float ga = 0.f;
-    for (int tt = 0; tt < kRmsRows; ++tt) {
+  const int nt = min(kRmsRows, ntok - t0);
+  for (int v = threadIdx.x; v < nv; v += blockDim.x) {
+    float gm[8], ga[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) ga[j] = 0.f;
+    if (gain) load8_bf16(gain + 8 * v, gm);
+    else
+#pragma unroll
+      for (int j = 0; j < 8; ++j) gm[j] = 1.f;
+#pragma unroll 4
+    for (int tt = 0; tt < nt; ++tt) {
       const int t = t0 + tt;
-      if (t >= ntok) break;
       const float rt = r[t];
-      const float xv = bf2f(x[(size_t)t * d + c]);
-      const float g = dxh[(size_t)t * d + c];
-      dx[(size_t)t * d + c] = gm * g * rt - xv * rt * rt * rt * inv_d * dot[tt];
-      ga = fmaf(g * xv, rt, ga);
+      const float cr = rt * rt * rt * inv_d * dot[tt];
+      float xv[8], gv[8];
+      load8_bf16(x + (size_t)t * d + 8 * v, xv);
+      load8_f32(dxh + (size_t)t * d + 8 * v, gv);
+      float o[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        o[j] = gm[j] * gv[j] * rt - xv[j] * cr;
+        ga[j] = fmaf(gv[j] * xv[j], rt, ga[j]);
+      }
+      float4* dst = reinterpret_cast<float4*>(dx + (size_t)t * d + 8 * v);
+      dst[0] = make_float4(o[0], o[1], o[2], o[3]);
+      dst[1] = make_float4(o[4], o[5], o[6], o[7]);
     }
-    gpart[(size_t)blockIdx.x * d + c] = ga;
+    float4* gp = reinterpret_cast<float4*>(gpart + (size_t)blockIdx.x * d + 8 * v);
+    gp[0] = make_float4(ga[0], ga[1], ga[2], ga[3]);
+    gp[1] = make_float4(ga[4], ga[5], ga[6], ga[7]);
   }
 }
 
-// dL/dgain = the sum of the blocks' partial sums, in block order.
+// dL/dgain = the sum of the blocks' partial sums: a block per 32 columns, its 8 warps summing
+// interleaved rows, then the 8 sums added in a fixed order.
 __global__ void __launch_bounds__(256) colsum_kernel(const float* __restrict__ part, int nrows, int d,
                                                      float* __restrict__ out) {
   pdl_wait();
   pdl_trigger();
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  if (c >= d) return;
+  __shared__ float sm[8][33];
+  const int c = blockIdx.x * 32 + (threadIdx.x & 31), y = threadIdx.x >> 5;
   float acc = 0.f;
-  for (int i = 0; i < nrows; ++i) acc += part[(size_t)i * d + c];
-  out[c] = acc;
+  if (c < d) {
+#pragma unroll 8
+    for (int i = y; i < nrows; i += 8) acc += part[(size_t)i * d + c];
+  }
+  sm[y][threadIdx.x & 31] = acc;
+  __syncthreads();
+  if (y == 0 && c < d) {
+    float s = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) s += sm[j][threadIdx.x];
+    out[c] = s;
+  }
 }
 
 }  // namespace lmoe

@@ -147,9 +147,10 @@ template <int BN, int EPI>
 cudaError_t launch_tc_t(const TcParams& p, int grid, cudaStream_t st) {
   auto kern = tc_gemm_kernel<BN, EPI, 0>;
   static unsigned done = 0;
-  cudaError_t e = ensure_smem_attr(kern, TcCfg<BN>::kSmemBytes, done);
+  constexpr int smem = TcCfgFor<BN, EPI, 0>::kSmemBytes;
+  cudaError_t e = ensure_smem_attr(kern, smem, done);
   if (e != cudaSuccess) return e;
-  return launch_k(kern, dim3(grid), dim3(kTcThreads), TcCfg<BN>::kSmemBytes, st, 1, p);
+  return launch_k(kern, dim3(grid), dim3(kTcThreads), smem, st, 1, p);
 }
 
 // Two-CTA (cta_group::2) variant: clusters of 2 along x, grid even.
@@ -157,9 +158,10 @@ template <int BN, int EPI>
 cudaError_t launch_tc_pair_t(const TcParams& p, int grid, cudaStream_t st) {
   auto kern = tc_gemm_kernel<BN, EPI, 1>;
   static unsigned done = 0;
-  cudaError_t e = ensure_smem_attr(kern, TcCfg<BN, 1>::kSmemBytes, done);
+  constexpr int smem = TcCfgFor<BN, EPI, 1>::kSmemBytes;
+  cudaError_t e = ensure_smem_attr(kern, smem, done);
   if (e != cudaSuccess) return e;
-  return launch_k(kern, dim3((unsigned)(grid & ~1)), dim3(kTcThreads), TcCfg<BN, 1>::kSmemBytes, st, 2, p);
+  return launch_k(kern, dim3((unsigned)(grid & ~1)), dim3(kTcThreads), smem, st, 2, p);
 }
 
 template <int EPI>
@@ -322,6 +324,7 @@ struct BwdWork {
   long long RP = 0;  // rows of the padded expert layout, a multiple of 128
   // maps of the padded expert-row buffers (fixed addresses)
   CUtensorMap pe_out, dpe_out, dpe_k, dpe_mn, do_k, do_mn, dhe_out, aperm_mn, act_mn;
+  CUtensorMap ps_out;  // the shared expert's pre-activations [max_tokens, 2 hs]
 };
 
 struct lmoe_handle {
@@ -791,7 +794,7 @@ int route_from_scores(lmoe_handle* h, int T, uint32_t flags, const StatsState& p
 }
 
 int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, const StatsState& pre,
-                 cudaStream_t st) {
+                 cudaStream_t st, bool save_pre = false) {
   const lmoe_config& c = h->cfg;
   const int mt = (T + 127) / 128;
   CUtensorMap tm_x;
@@ -884,6 +887,10 @@ int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, 
     p.M_rows = T;
     p.tmOut = h->tm_as;
     p.row_scale = h->r;
+    if (save_pre) {  // a training step: the backward reads the pre-activations
+      p.out_pre = 1;
+      p.tmOut2 = h->bw->ps_out;
+    }
     const int pbn = T >= 256 * 8 ? pick_pair_bn(T, 2 * c.hs, h->sms) : 0;
     if (pbn) {  // two-CTA tiles: each CTA loads BN/2 rows of the weights
       p.tmB = h->tm_ws13[bn_index(pbn / 2)];
@@ -959,6 +966,11 @@ int forward_bf16(lmoe_handle* h, const void* x, void* y, int T, uint32_t flags, 
     }
     p.hint_b = 1;    // each expert's weights serve its few tiles, then not again this step
     p.hint_out = 1;  // act is read by the next GEMM
+    if (save_pre) {
+      p.out_pre = 1;
+      p.tmOut2 = h->bw->pe_out;
+      p.trim = 0;
+    }
     CK(launch_tc(p, EPI_SWIGLU, h->bn_e1, h->sms, st));
     }
     mark(h, ST_EXPERT2, st);
@@ -1327,6 +1339,7 @@ int bwd_alloc(lmoe_handle* h) {
   ok &= make_map(&b->dhe_out, b->dhe, R, l, l, 128);
   ok &= make_map(&b->aperm_mn, h->a_perm, h->rows_pad, l, l, 64);
   ok &= make_map(&b->act_mn, h->act, h->rows_pad, hh, hh, 64);
+  if (hs) ok &= make_map(&b->ps_out, b->ps, (long long)Tm, 2 * hs, 2 * hs, 128);
   h->bw = b;
   return ok ? LMOE_OK : LMOE_EINVAL;
 }
@@ -1353,8 +1366,17 @@ int wgrad_gemm(lmoe_handle* h, TcParams& p, int M, int N, long long K, size_t ou
   p.seg[0] = KSeg{0, 0, 0, (int)((K + 63) / 64), 0};
   const long long base = (long long)((M + 127) / 128) * p.n_tiles;
   const int nkb = p.seg[0].nkb;
+  // K ranges (at least 4 k-blocks each): the count whose waves of tiles finish first, the work of
+  // a tile falling as 1/S (the fewest ranges among equals: each adds a pass of reductions)
   int S = 1;
-  if (base < h->sms) S = (int)std::min<long long>((h->sms + base - 1) / base, std::max(1, nkb / 4));
+  double best = (double)((base + h->sms - 1) / h->sms);
+  for (int s = 2; s <= std::min(64, nkb / 4); ++s) {
+    const double t = (double)((base * s + h->sms - 1) / h->sms) / s;
+    if (t < best - 1e-9) {
+      best = t;
+      S = s;
+    }
+  }
   p.k_split = S;
   if (S > 1) {
     CK(cudaMemsetAsync(out, 0, out_bytes, st));
@@ -1380,14 +1402,12 @@ int backward_bf16(lmoe_handle* h, const lmoe_weights* w, const void* x, const vo
   bool ok = true;
   // per-call maps of the token-row buffers (their row extent is T, so K = T products read zeros
   // past the last token)
-  CUtensorMap x_k, dy_k, dy_mn, xh_mn, ps_out, dps_out, dps_k, dps_mn, dz_out, as_mn, z_mn, dlg_k, dlg_mn, hx_mn, dhr_out,
+  CUtensorMap dy_k, dy_mn, xh_mn, dps_out, dps_k, dps_mn, dz_out, as_mn, z_mn, dlg_k, dlg_mn, hx_mn, dhr_out,
       dh_k, dh_mn, dxh_out;
-  ok &= make_map(&x_k, x, T, d, d, 128);
   ok &= make_map(&dy_k, dy, T, d, d, 128);
   ok &= make_map(&dy_mn, dy, T, d, d, 64);
   ok &= make_map(&xh_mn, b->xh, T, d, d, 64);
   if (hs) {
-    ok &= make_map(&ps_out, b->ps, T, 2 * hs, 2 * hs, 128);
     ok &= make_map(&dps_out, b->dps, T, 2 * hs, 2 * hs, 128);
     ok &= make_map(&dps_k, b->dps, T, 2 * hs, 2 * hs, 128);
     ok &= make_map(&dps_mn, b->dps, T, 2 * hs, 2 * hs, 64);
@@ -1437,21 +1457,9 @@ int backward_bf16(lmoe_handle* h, const lmoe_weights* w, const void* x, const vo
               (const bf16*)w->rms_gain, (const float*)h->r, (long long)T, (int)d, b->xh));
   h->launches += 1;
   if (hs) {
-    // the shared expert's pre-activations again: [p1 | p3] = r x (gain Ws13)^T, interleaved
+    // dL/d act_s = dy Ws2 and through the SwiGLU (pre-activations saved by the forward):
+    // [dL/dp1 | dL/dp3] of the shared expert
     TcParams p = tc_base(h);
-    p.tmA[0] = p.tmA[1] = x_k;
-    const int bn = pick_bn_for(T, 2 * hs, sms, 128);
-    p.tmB = h->tm_ws13[bn_index(bn)];
-    p.nseg = 1;
-    p.seg[0] = KSeg{0, 0, 0, (int)(d / 64), 0};
-    p.M = T;
-    p.M_rows = T;
-    p.n_tiles = 2 * hs / bn;
-    p.tmOut = ps_out;
-    p.row_scale = h->r;
-    CK(launch_tc(p, EPI_BF16, bn, std::min(mt * p.n_tiles, sms), st));
-    // dL/d act_s = dy Ws2 and through the SwiGLU: [dL/dp1 | dL/dp3] of the shared expert
-    p = tc_base(h);
     p.tmA[0] = p.tmA[1] = dy_k;
     p.tmB = ws2_mn;
     p.b_mn = 1;
@@ -1466,7 +1474,7 @@ int backward_bf16(lmoe_handle* h, const lmoe_weights* w, const void* x, const vo
     p.ld_aux = 2 * hs;
     p.split = hs;
     CK(launch_tc(p, EPI_SWIGLU_BWD, bn3, std::min(mt * p.n_tiles, sms), st));
-    h->launches += 2;
+    h->launches += 1;
   }
   {  // dL/dz = dy W_up
     TcParams p = tc_base(h);
@@ -1488,21 +1496,9 @@ int backward_bf16(lmoe_handle* h, const lmoe_weights* w, const void* x, const vo
               (const int*)h->prow, (const float*)h->gates, (const int*)h->idx, (const float*)h->s, T, c.k, (int)l,
               (int)E, b->d_o, b->dlogit, b->dlp));
   h->launches += 1;
-  {  // routed experts: pre-activations again, [p1 | p3] = A_perm W13_e^T (interleaved)
+  {  // routed experts: dL/d act_e = dL/do W2_e, through the SwiGLU (pre-activations saved by the
+     // forward): [dL/dp1 | dL/dp3] (zero past each expert's rows)
     TcParams p = tc_base(h);
-    p.tmA[0] = p.tmA[1] = h->tm_aperm;
-    p.tmB = h->tm_w13;
-    p.nseg = 1;
-    p.seg[0] = KSeg{0, 0, 0, (int)(l / 64), 0};
-    p.grouped = 1;
-    p.n_tiles = 2 * hh / h->bn_e1;
-    p.mtile_table = h->mtiles;
-    p.num_mtiles = h->num_mtiles;
-    p.b_rows_per_group = 2 * hh;
-    p.tmOut = b->pe_out;
-    CK(launch_tc(p, EPI_BF16, h->bn_e1, sms, st));
-    // dL/d act_e = dL/do W2_e, through the SwiGLU: [dL/dp1 | dL/dp3] (zero past each expert's rows)
-    p = tc_base(h);
     p.tmA[0] = p.tmA[1] = b->do_k;
     p.tmB = w2_mn;
     p.b_mn = 1;
@@ -1536,7 +1532,7 @@ int backward_bf16(lmoe_handle* h, const lmoe_weights* w, const void* x, const vo
     p.b_rows_per_group = (int)hh;
     p.tmOut = b->dhe_out;
     CK(launch_tc(p, EPI_BF16, bn6, sms, st));
-    h->launches += 3;
+    h->launches += 2;
   }
   // rows past each expert's last pair, up to its next 64-row boundary: zero in A_perm, act and
   // dL/do, the operands of the expert weight gradients
@@ -1665,7 +1661,7 @@ int backward_bf16(lmoe_handle* h, const lmoe_weights* w, const void* x, const vo
   CK(launch_k(rms_bwd_kernel, dim3(nrb), dim3(256), 0, st, 1, (const bf16*)x, (const bf16*)w->rms_gain,
               (const float*)h->r, (const float*)b->dxh, T, (int)d, g->dx, b->gpart));
   if (g->rms_gain)
-    CK(launch_k(colsum_kernel, dim3((unsigned)((d + 255) / 256)), dim3(256), 0, st, 1, (const float*)b->gpart, nrb,
+    CK(launch_k(colsum_kernel, dim3((unsigned)((d + 31) / 32)), dim3(256), 0, st, 1, (const float*)b->gpart, nrb,
                 (int)d, g->rms_gain));
   h->launches += 2;
   return LMOE_OK;
@@ -1800,7 +1796,18 @@ int lmoe_destroy(lmoe_handle* h) {
   return LMOE_OK;
 }
 
+// Forward of lmoe_forward; save_pre (a training step) also stores the SwiGLU pre-activations for
+// the backward (a separate graph: its key carries kSavePre).
+constexpr uint32_t kSavePre = 1u << 15;
+static int forward_impl(lmoe_handle* h, const void* x, void* y, int32_t T, uint32_t flags, bool save_pre,
+                        void* stream);
+
 int lmoe_forward(lmoe_handle* h, const void* x, void* y, int32_t T, uint32_t flags, void* stream) {
+  return forward_impl(h, x, y, T, flags & ~kSavePre, false, stream);
+}
+
+static int forward_impl(lmoe_handle* h, const void* x, void* y, int32_t T, uint32_t flags, bool save_pre,
+                        void* stream) {
   if (!h || T < 0 || T > h->cfg.max_tokens) return LMOE_EINVAL;
   if (T == 0) return LMOE_OK;
   if (!x || !y || ((uintptr_t)x & 15) || ((uintptr_t)y & 15)) return LMOE_EINVAL;
@@ -1813,7 +1820,7 @@ int lmoe_forward(lmoe_handle* h, const void* x, void* y, int32_t T, uint32_t fla
   if (upd && (!(flags & LMOE_RECORD_STATS) || !h->upd_set)) return LMOE_EINVAL;
   const StatsState pre = h->ss;
   // graph key: the arguments, the update's step and flags, the statistics state
-  const uint32_t kflags = flags | (upd ? h->upd_flags << 16 : 0u);
+  const uint32_t kflags = flags | (upd ? h->upd_flags << 16 : 0u) | (save_pre ? kSavePre : 0u);
   const float kbeta = upd ? h->upd_beta : 0.f;
   // the cached graph of these arguments, else the least recently used one
   int gi = h->g_fwd[0].same(x, y, T, kflags, kbeta, pre.key()) ? 0
@@ -1822,7 +1829,7 @@ int lmoe_forward(lmoe_handle* h, const void* x, void* y, int32_t T, uint32_t fla
   h->g_used[gi] = ++h->g_tick;
   int rc = run_cached(h, h->g_fwd[gi], x, y, T, kflags, kbeta, pre.key(), st, [&](cudaStream_t s) {
     prof_open(h, ST_RMS, ST_UP - ST_RMS + 1);
-    int r = h->bf ? forward_bf16(h, x, y, T, flags, pre, s) : forward_f32(h, x, y, T, flags, pre, s);
+    int r = h->bf ? forward_bf16(h, x, y, T, flags, pre, s, save_pre) : forward_f32(h, x, y, T, flags, pre, s);
     prof_close(h, s);
     if (!r && upd && h->profiling) {  // profiled: the update after the forward, timed as its own stage
       prof_open(h, ST_QB_UPDATE, 1);
@@ -1861,7 +1868,7 @@ int lmoe_forward_backward(lmoe_handle* h, const lmoe_weights* w, const void* x, 
   int rc = bwd_alloc(h);
   if (rc) return rc;
   cudaStream_t st = (cudaStream_t)stream;
-  rc = lmoe_forward(h, x, y, T, flags, stream);
+  rc = forward_impl(h, x, y, T, flags, true, stream);
   if (rc) return rc;
   return backward_bf16(h, w, x, dy, T, g, st);
 }

@@ -96,6 +96,9 @@ struct TcParams {
   const int* k_rows;          // grouped_k: rows of each expert
   const bf16* aux;            // EPI_SWIGLU_BWD: [rows, 2 split] pre-activations, gate and linear
   int ld_aux;                 // columns interleaved in groups of 64 (as the forward's weights)
+  int out_pre;                // EPI_SWIGLU: also store the bf16 pre-activations (the accumulator
+                              // scaled by row_scale, gate and linear columns as accumulated) to
+                              // tmOut2, for a backward pass (no trim)
   int k_split;                // > 1 (non-grouped, one segment, EPI_F32): the k-blocks are cut into
                               // k_split ranges, one tile each, whose results are added into the
                               // output (zeroed first) by TMA reductions
@@ -103,17 +106,33 @@ struct TcParams {
 
 // PAIR = 1: a cluster of two CTAs computes one 256 x BN tile with tcgen05.mma.cta_group::2; each
 // CTA holds 128 rows of A and BN/2 rows of B per stage.
-template <int BN, int PAIR = 0>
+// EXTRA: shared memory the epilogue keeps for itself, taken from the load ring.
+template <int BN, int PAIR = 0, int EXTRA = 0>
 struct TcCfg {
   static constexpr int kABytes = 128 * 128;              // 128 rows x 64 bf16
   static constexpr int kBBytes = (PAIR ? BN / 2 : BN) * 128;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = (192 * 1024) / kStageBytes;
+  static constexpr int kStages = (192 * 1024 - EXTRA) / kStageBytes;
   static constexpr int kTmemCols = 2 * BN;
   static constexpr int kOutOffset = kStages * kStageBytes;    // two 16 KB output boxes
-  static constexpr int kBarOffset = kOutOffset + 2 * 16384;
+  static constexpr int kAuxOffset = kOutOffset + 2 * 16384;   // the epilogue's own (EXTRA bytes)
+  static constexpr int kBarOffset = kAuxOffset + EXTRA;
   static constexpr int kSmemBytes = kBarOffset + 256 + 1024;  // barriers + alignment slack
 };
+
+// EPI_SWIGLU_BWD stages the pre-activations each epilogue warp reads: per warp, gate and linear
+// values of its 32 rows x 32 columns, rows 80 bytes apart (64 bytes of data + 16 of padding, so
+// that eight lanes reading eight rows hit distinct banks).
+constexpr int kAuxWarpBytes = 2 * 32 * 80;
+// Output staging boxes of an epilogue (boxes past two would live in its EXTRA bytes).  Four for
+// the fp32 outputs of short-K weight gradients were measured slower than two: they cost a stage
+// of the load ring and the stores were not what limited those tiles.
+__host__ __device__ constexpr int tc_out_boxes(int) { return 2; }
+__host__ __device__ constexpr int tc_epi_extra(int epi) {
+  return epi == EPI_SWIGLU_BWD ? 8 * kAuxWarpBytes : (tc_out_boxes(epi) - 2) * 16384;
+}
+template <int BN, int EPI, int PAIR>
+using TcCfgFor = TcCfg<BN, PAIR, tc_epi_extra(EPI)>;
 
 struct TileInfo {
   int row0, b_row0, n0;
@@ -216,8 +235,9 @@ constexpr int kTcThreads = 64 + 32 * kEpiWarps;
 
 template <int BN, int EPI, int PAIR>
 __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_constant__ TcParams p) {
-  using C = TcCfg<BN, PAIR>;
+  using C = TcCfgFor<BN, EPI, PAIR>;
   constexpr int S = C::kStages;
+  constexpr int NB = tc_out_boxes(EPI);  // output staging boxes (the ones past two in the EXTRA bytes)
   constexpr bool kSplit3 = EPI == EPI_ROUTER && !PAIR;  // chunk-major split-precision products
   constexpr int kAccCols = kSplit3 ? 2 * BN : BN;       // TMEM columns of one accumulator buffer
   constexpr uint32_t kTmemCols = 2 * kAccCols;
@@ -230,8 +250,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
   uint64_t* tfull = empty + S;
   uint64_t* tempty = tfull + 2;
   uint64_t* bfull = tempty + 2;   // output box written by all epilogue warps
-  uint64_t* bfree = bfull + 2;    // output box read by its TMA store
-  uint64_t* drain = bfree + 2;
+  uint64_t* bfree = bfull + NB;   // output box read by its TMA store
+  uint64_t* drain = bfree + NB;
   uint8_t* obox = smem + C::kOutOffset;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -250,6 +270,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], PAIR ? 2 * kEpiWarps : kEpiWarps);
+    }
+    for (int i = 0; i < NB; ++i) {
       mbar_init(&bfull[i], kEpiWarps);
       mbar_init(&bfree[i], 1);
     }
@@ -488,9 +510,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     bool ok = true;
     // Writes this thread's 64 bytes into the current box, then (storer) stores the box.
     const CUtensorMap* omap = &p.tmOut;  // this tile's output map (trim: only its valid rows)
-    auto emit = [&](const uint32_t (&w)[16], int x, int y) -> bool {
-      const int buf = step & 1;
-      const uint32_t par = (step >> 1) & 1u;
+    auto emit = [&](const uint32_t (&w)[16], int x, int y, const CUtensorMap* to = nullptr) -> bool {
+      const int buf = (int)(step % NB);
+      const uint32_t par = (step / NB) & 1u;
       bool good = mbar_wait(&bfree[buf], par ^ 1u, abort, p.status);
       __syncwarp();
       if (__any_sync(0xffffffffu, !good)) return false;
@@ -507,16 +529,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         __syncwarp();
         if (__any_sync(0xffffffffu, !good)) return false;
         if (lane == 0) {
-          if (p.k_split > 1)
+          if (to)
+            tma_store_2d(to, box, x, y);
+          else if (p.k_split > 1)
             tma_reduce_add_2d(omap, box, x, y);
           else if (p.hint_out)
             tma_store_2d_hint(omap, box, x, y, l2_evict_last());
           else
             tma_store_2d(omap, box, x, y);
           bulk_commit();
-          if (step > 0) {
-            bulk_wait_read<1>();  // the previous box has been read: its buffer is free
-            mbar_arrive(&bfree[(step - 1) & 1]);
+          if (step >= NB - 1) {
+            bulk_wait_read<NB - 1>();  // the box stored NB - 1 steps ago has been read: it is free
+            mbar_arrive(&bfree[(step - (NB - 1)) % NB]);
           }
         }
         __syncwarp();
@@ -568,6 +592,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             w[q] = pack_bf16x2(silu_fast(g0) * u0, silu_fast(g1) * u1);
           }
           ok = emit(w, (ti.n0 >> 1) + j * 64, ti.out_y);
+          if (p.out_pre) {
+            // the pre-activations, in the accumulator's own column order
+#pragma unroll
+            for (int q = 0; q < 16; ++q)
+              w[q] = pack_bf16x2(__uint_as_float(gv[2 * q]) * rs, __uint_as_float(gv[2 * q + 1]) * rs);
+            if (ok) ok = emit(w, ti.n0 + j * 128, ti.out_y, &p.tmOut2);
+#pragma unroll
+            for (int q = 0; q < 16; ++q)
+              w[q] = pack_bf16x2(__uint_as_float(uv[2 * q]) * rs, __uint_as_float(uv[2 * q + 1]) * rs);
+            if (ok) ok = emit(w, ti.n0 + j * 128 + 64, ti.out_y, &p.tmOut2);
+          }
         }
       } else if constexpr (EPI == EPI_SWIGLU3) {
 #pragma unroll 1
@@ -605,20 +640,44 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         }
       } else if constexpr (EPI == EPI_SWIGLU_BWD) {
         // step j: accumulator columns c = n0 + j*64 + half*32 + q hold dL/d act; the gate and linear
-        // pre-activations of column c sit at aux columns (c/64)*128 + c%64 and 64 further
+        // pre-activations of column c sit at aux columns (c/64)*128 + c%64 and 64 further.  Each
+        // warp copies the 32 x 32 gate and linear values of its rows and columns with whole
+        // 64-byte row pieces (8 rows per load instruction) into its staging rows, one step ahead,
+        // then every lane reads its own row from there.
         const bool live = rl < ti.valid;
-        const bf16* arow = p.aux + (size_t)(live ? row : 0) * p.ld_aux;
+        uint8_t* stg = smem + C::kAuxOffset + (warp - 2) * kAuxWarpBytes;
+        const int rbase = ti.row0 + wq * 32;
+        const int nlive = ti.valid - wq * 32;  // rows of this warp's quarter that hold data
+        uint4 pf[8];
+        auto fetch = [&](int j) {
+          const int c0 = ti.n0 + j * 64 + half_id * 32;
+          const int g0 = ((c0 >> 6) << 7) + (c0 & 63);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int c = lane + 32 * i, which = c >> 7, rr = (c >> 2) & 31, cc = c & 3;
+            pf[i] = rr < nlive ? ldg_nc_v4(p.aux + (size_t)(rbase + rr) * p.ld_aux + g0 + which * 64 + cc * 8)
+                               : make_uint4(0, 0, 0, 0);
+          }
+        };
+        fetch(0);
 #pragma unroll 1
         for (int j = 0; ok && j < BN / 64; ++j) {
           uint32_t v[32];
           tmem_ld32(tbase + j * 64 + half_id * 32, v);
           const int c0 = ti.n0 + j * 64 + half_id * 32;
-          const int g0 = ((c0 >> 6) << 7) + (c0 & 63);
+          __syncwarp();  // every lane has read the previous step's staging rows
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int c = lane + 32 * i, which = c >> 7, rr = (c >> 2) & 31, cc = c & 3;
+            *reinterpret_cast<uint4*>(stg + which * (kAuxWarpBytes / 2) + rr * 80 + cc * 16) = pf[i];
+          }
+          __syncwarp();
+          if (j + 1 < BN / 64) fetch(j + 1);
           uint4 pg[4], pu[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            pg[i] = live ? ldg_nc_v4(arow + g0 + 8 * i) : make_uint4(0, 0, 0, 0);
-            pu[i] = live ? ldg_nc_v4(arow + g0 + 64 + 8 * i) : make_uint4(0, 0, 0, 0);
+            pg[i] = *reinterpret_cast<const uint4*>(stg + lane * 80 + i * 16);
+            pu[i] = *reinterpret_cast<const uint4*>(stg + kAuxWarpBytes / 2 + lane * 80 + i * 16);
           }
           tc_wait_ld();
           uint32_t w3[16];
