@@ -1366,17 +1366,9 @@ int wgrad_gemm(lmoe_handle* h, TcParams& p, int M, int N, long long K, size_t ou
   p.seg[0] = KSeg{0, 0, 0, (int)((K + 63) / 64), 0};
   const long long base = (long long)((M + 127) / 128) * p.n_tiles;
   const int nkb = p.seg[0].nkb;
-  // K ranges (at least 4 k-blocks each): the count whose waves of tiles finish first, the work of
-  // a tile falling as 1/S (the fewest ranges among equals: each adds a pass of reductions)
-  int S = 1;
-  double best = (double)((base + h->sms - 1) / h->sms);
-  for (int s = 2; s <= std::min(64, nkb / 4); ++s) {
-    const double t = (double)((base * s + h->sms - 1) / h->sms) / s;
-    if (t < best - 1e-9) {
-      best = t;
-      S = s;
-    }
-  }
+  // K ranges (at least 4 k-blocks each): as many as fill one wave of tiles.  Measured on a B200
+  // with L2-resident operands, a second partial wave cost more than the reductions it saved.
+  const int S = (int)std::max<long long>(1, std::min<long long>(h->sms / base, std::max(1, nkb / 4)));
   p.k_split = S;
   if (S > 1) {
     CK(cudaMemsetAsync(out, 0, out_bytes, st));

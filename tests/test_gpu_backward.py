@@ -137,3 +137,13 @@ def test_backward_rejects_unsupported_layers():
     with pytest.raises(lq.LmoeError):
         layer.forward_backward(x, x.clone(), w)
     layer.close()
+
+
+def test_backward_at_the_training_bench_size():
+    """mini_replica at full size (T = 8192, d = 1024, l = 256, E = 256, k = 6, h = 256,
+    hs = 2048), the workload and launch configuration bench.py times as its training step: every
+    gradient against the oracle on all tokens (the weight gradients sum over all of them)."""
+    shape = datagen.WORKLOADS["mini_replica"]
+    g, ref, r, _ = run_backward(shape, gain="ones")
+    errs = check_grads(shape, g, ref, r)
+    print("max error / max|ref| per gradient:", {n: f"{v:.2e}" for n, v in errs.items()})
