@@ -281,8 +281,9 @@ int lmoe_gemm_bf16(const void *a_dev, const void *b_dev, float *c_dev, int32_t M
  * a_mn = 0: A is [M, K] row-major; a_mn = 1: A is stored [K, M] (the product reads A^T).
  * b_mn = 0: B is [N, K]; b_mn = 1: B is stored [K, N].  N a multiple of 64, K of 8, M of 8 when
  * a_mn.  k_split > 1 (at most ceil(K/64)) cuts K into that many ranges whose products are added
- * into C by TMA reductions (C is zeroed first; the sum order then varies between runs).  The
- * products of the layer backward use these forms.  For tests. */
+ * into C by TMA reductions (C is zeroed first; the sum order then varies between runs).  M >= 256
+ * with N a multiple of 128 runs the two-CTA (256-row tile) variant.  The products of the layer
+ * backward use these forms.  For tests. */
 int lmoe_gemm_bf16_ex(const void *a_dev, int32_t a_mn, const void *b_dev, int32_t b_mn, float *c_dev,
                       int32_t M, int32_t N, int32_t K, int32_t k_split, void *stream);
 

@@ -1352,10 +1352,12 @@ void bwd_free(lmoe_handle* h) {
 }
 
 // A weight gradient G [M, N] (fp32) = A^T B over K rows (both operands MN-major: A stored [K, M],
-// B stored [K, N]).  When the output tiles cannot fill the SMs, K is cut into ranges whose partial
-// products are added into the zeroed output by TMA reductions.
+// B stored [K, N]), on two-CTA 256-row tiles where M allows.  When the output tiles cannot fill the
+// GPU, K is cut into ranges whose partial products are added into the zeroed output by TMA
+// reductions.
 int wgrad_gemm(lmoe_handle* h, TcParams& p, int M, int N, long long K, size_t out_bytes, void* out,
                size_t out2_bytes, void* out2, cudaStream_t st) {
+  const bool pair = M >= 256 && N % 128 == 0;
   const int bn = N % 256 == 0 ? 256 : (N % 128 == 0 ? 128 : 64);
   p.a_mn = 1;
   p.b_mn = 1;
@@ -1364,18 +1366,43 @@ int wgrad_gemm(lmoe_handle* h, TcParams& p, int M, int N, long long K, size_t ou
   p.n_tiles = N / bn;
   p.nseg = 1;
   p.seg[0] = KSeg{0, 0, 0, (int)((K + 63) / 64), 0};
-  const long long base = (long long)((M + 127) / 128) * p.n_tiles;
+  const int units = pair ? h->sms / 2 : h->sms;  // CTAs, or CTA pairs
+  const long long base = (long long)(pair ? (M + 255) / 256 : (M + 127) / 128) * p.n_tiles;
   const int nkb = p.seg[0].nkb;
   // K ranges (at least 4 k-blocks each): as many as fill one wave of tiles.  Measured on a B200
   // with L2-resident operands, a second partial wave cost more than the reductions it saved.
-  const int S = (int)std::max<long long>(1, std::min<long long>(h->sms / base, std::max(1, nkb / 4)));
+  const int S = (int)std::max<long long>(1, std::min<long long>(units / base, std::max(1, nkb / 4)));
   p.k_split = S;
   if (S > 1) {
     CK(cudaMemsetAsync(out, 0, out_bytes, st));
     if (out2) CK(cudaMemsetAsync(out2, 0, out2_bytes, st));
   }
   const long long tiles = base * S;
-  CK(launch_tc(p, EPI_F32, bn, (int)std::min<long long>(tiles, h->sms), st));
+  if (pair)
+    CK(launch_tc_pair(p, EPI_F32, bn, 2 * (int)std::min<long long>(tiles, units), st));
+  else
+    CK(launch_tc(p, EPI_F32, bn, (int)std::min<long long>(tiles, units), st));
+  h->launches += 1;
+  return LMOE_OK;
+}
+
+// A dense product of T rows (fp32 or bf16 out) on two-CTA 256-row tiles where T and N allow, else
+// on 128-row tiles.  The caller sets the operands, segments and output; this picks the tile width
+// and the grid.
+int dense_gemm(lmoe_handle* h, TcParams& p, int epi, int T, int N, cudaStream_t st) {
+  p.M = T;
+  p.M_rows = T;
+  const int pbn = (T >= 256 * 8 && (epi == EPI_F32 || epi == EPI_BF16)) ? pick_pair_bn(T, N, h->sms) : 0;
+  if (pbn) {
+    p.n_tiles = N / pbn;
+    const long long tiles = (long long)((T + 255) / 256) * p.n_tiles;
+    CK(launch_tc_pair(p, epi, pbn, 2 * (int)std::min<long long>(tiles, h->sms / 2), st));
+  } else {
+    const int bn = pick_bn_for(T, N, h->sms, 64);
+    p.n_tiles = N / bn;
+    const long long tiles = (long long)((T + 127) / 128) * p.n_tiles;
+    CK(launch_tc(p, epi, bn, (int)std::min<long long>(tiles, h->sms), st));
+  }
   h->launches += 1;
   return LMOE_OK;
 }
@@ -1475,13 +1502,9 @@ int backward_bf16(lmoe_handle* h, const lmoe_weights* w, const void* x, const vo
     p.b_mn = 1;
     p.nseg = 1;
     p.seg[0] = KSeg{0, 0, 0, (int)(d / 64), 0};
-    p.M = T;
-    p.M_rows = T;
-    const int bn = pick_bn_for(T, l, sms, 64);
-    p.n_tiles = l / bn;
     p.tmOut = dz_out;
-    CK(launch_tc(p, EPI_BF16, bn, std::min(mt * p.n_tiles, sms), st));
-    h->launches += 1;
+    int rc = dense_gemm(h, p, EPI_BF16, T, (int)l, st);
+    if (rc) return rc;
   }
   // combine and gates: dL/do of every pair, dL/dlogit
   CK(launch_k(combine_bwd_kernel, dim3((T + 7) / 8), dim3(256), 0, st, 1, (const bf16*)b->dz, (const bf16*)h->o,
@@ -1582,13 +1605,9 @@ int backward_bf16(lmoe_handle* h, const lmoe_weights* w, const void* x, const vo
     p.nseg = 2;
     p.seg[0] = KSeg{0, 0, 0, (int)(E / 64), 0};
     p.seg[1] = KSeg{0, 0, 0, (int)(E / 64), 1};
-    p.M = T;
-    p.M_rows = T;
-    const int bn = pick_bn_for(T, l, sms, 64);
-    p.n_tiles = l / bn;
     p.tmOut = dhr_out;
-    CK(launch_tc(p, EPI_F32, bn, std::min(mt * p.n_tiles, sms), st));
-    h->launches += 1;
+    rc = dense_gemm(h, p, EPI_F32, T, (int)l, st);
+    if (rc) return rc;
   }
   // dL/dh = the router's part + the experts' parts of the token's pairs
   CK(launch_k(scatter_dh_kernel, dim3((T + 7) / 8), dim3(256), 0, st, 1, (const float*)b->dhr, (const bf16*)b->dhe,
@@ -1616,13 +1635,9 @@ int backward_bf16(lmoe_handle* h, const lmoe_weights* w, const void* x, const vo
     p.seg[0] = KSeg{0, 0, 0, (int)(l / 64), 0};
     p.seg[1] = KSeg{1, 0, 0, (int)(hs / 64), 1};
     p.seg[2] = KSeg{1, (int)hs, 0, (int)(hs / 64), 2};
-    p.M = T;
-    p.M_rows = T;
-    const int bn = pick_bn_for(T, d, sms, 64);
-    p.n_tiles = d / bn;
     p.tmOut = dxh_out;
-    CK(launch_tc(p, EPI_F32, bn, std::min(mt * p.n_tiles, sms), st));
-    h->launches += 1;
+    int rc = dense_gemm(h, p, EPI_F32, T, (int)d, st);
+    if (rc) return rc;
   }
   if (hs) {  // dWs1, dWs3 = [dL/dp1_s | dL/dp3_s]^T x_hat;  dWs2 = dy^T act_s
     TcParams p = tc_base(h);
@@ -2104,10 +2119,11 @@ int lmoe_gemm_bf16_ex(const void* a, int32_t a_mn, const void* b, int32_t b_mn, 
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int bn = pick_bn(N);
+  const bool pair = M >= 256 && bn >= 128;  // the two-CTA variant, so tests exercise it
   TcParams p;
   memset(&p, 0, sizeof(p));
   bool ok = a_mn ? make_map(&p.tmA[0], a, K, M, M, 64) : make_map(&p.tmA[0], a, M, K, K, 128);
-  ok &= b_mn ? make_map(&p.tmB, b, K, N, N, 64) : make_map(&p.tmB, b, N, K, K, bn);
+  ok &= b_mn ? make_map(&p.tmB, b, K, N, N, 64) : make_map(&p.tmB, b, N, K, K, pair ? bn / 2 : bn);
   ok &= make_map_f32(&p.tmOut, c, M, N, N, 128);
   if (!ok) return LMOE_EINVAL;
   p.tmA[1] = p.tmA[0];
@@ -2122,8 +2138,13 @@ int lmoe_gemm_bf16_ex(const void* a, int32_t a_mn, const void* b, int32_t b_mn, 
   p.n_tiles = N / bn;
   cudaStream_t st = (cudaStream_t)stream;
   if (k_split > 1) CK(cudaMemsetAsync(c, 0, (size_t)M * N * 4, st));
-  const long long tiles = (long long)((M + 127) / 128) * p.n_tiles * k_split;
-  CK(launch_tc(p, EPI_F32, bn, (int)(tiles < sms ? tiles : sms), st));
+  if (pair) {
+    const long long tiles = (long long)((M + 255) / 256) * p.n_tiles * k_split;
+    CK(launch_tc_pair(p, EPI_F32, bn, 2 * (int)(tiles < sms / 2 ? tiles : sms / 2), st));
+  } else {
+    const long long tiles = (long long)((M + 127) / 128) * p.n_tiles * k_split;
+    CK(launch_tc(p, EPI_F32, bn, (int)(tiles < sms ? tiles : sms), st));
+  }
   return LMOE_OK;
 }
 

@@ -160,7 +160,7 @@ __device__ __forceinline__ TileInfo tc_tile(const TcParams& p, int tile, int BN,
   ti.nkb = -1;
   if (p.k_split > 1) {
     // split s of a one-segment K: tiles [s*base, (s+1)*base) cover k-blocks [s*nkb/S, (s+1)*nkb/S)
-    const int base = ((p.M + 127) >> 7) * p.n_tiles;
+    const int base = (pair ? (p.M + 255) >> 8 : (p.M + 127) >> 7) * p.n_tiles;
     const int sp = tile / base;
     tile -= sp * base;
     const int nk = p.seg[0].nkb;
@@ -225,7 +225,7 @@ __device__ __forceinline__ TileInfo tc_tile(const TcParams& p, int tile, int BN,
 
 __device__ __forceinline__ int tc_num_tiles(const TcParams& p, int pair) {
   if (p.grouped_k) return p.k_groups * ((p.M + 127) >> 7) * p.n_tiles;
-  if (p.k_split > 1) return p.k_split * ((p.M + 127) >> 7) * p.n_tiles;
+  if (p.k_split > 1) return p.k_split * (pair ? (p.M + 255) >> 8 : (p.M + 127) >> 7) * p.n_tiles;
   int mt = p.grouped ? *p.num_mtiles : (pair ? (p.M + 255) / 256 : (p.M + 127) / 128);
   return mt * p.n_tiles;
 }
@@ -337,8 +337,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
               // both CTAs' bytes complete the leader's full barrier; the leader expects all of them
               const uint32_t bar0 = mapa_shared(smem_u32(&full[stage]), 0);
               if (leader) mbar_expect_tx(&full[stage], 2 * C::kStageBytes);
-              tma_load_2d_pair(a_dst, &p.tmA[sg.a_map], bar0, sg.a_col + kb * 64, ti.row0);
-              tma_load_2d_pair(b_dst, &p.tmB, bar0, sg.b_col + kb * 64, ti.b_row0);
+              const CUtensorMap* bmap = sg.b_map ? &p.tmB2[sg.b_map - 1] : &p.tmB;
+              if (p.a_mn) {  // this CTA's 128 rows of M as two 64 x 64 boxes
+                const int ky = ti.ak0 + sg.a_col + kb * 64;
+                tma_load_2d_pair(a_dst, &p.tmA[sg.a_map], bar0, ti.row0, ky);
+                tma_load_2d_pair(a_dst + 8192, &p.tmA[sg.a_map], bar0, ti.row0 + 64, ky);
+              } else {
+                tma_load_2d_pair(a_dst, &p.tmA[sg.a_map], bar0, sg.a_col + kb * 64, ti.row0);
+              }
+              if (p.b_mn) {  // this CTA's BN/2 columns of N, 64 at a time
+                const int ky = ti.bk0 + sg.b_col + kb * 64;
+#pragma unroll
+                for (int c = 0; c < BN / 128; ++c) tma_load_2d_pair(b_dst + c * 8192, bmap, bar0, ti.b_row0 + 64 * c, ky);
+              } else {
+                tma_load_2d_pair(b_dst, bmap, bar0, sg.b_col + kb * 64, ti.b_row0);
+              }
             } else if (p.a_mn | p.b_mn) {
               // MN-major operands: one 64 x 64 box per 64 columns of M (N), 64 K rows each
               const CUtensorMap* bmap = sg.b_map ? &p.tmB2[sg.b_map - 1] : &p.tmB;
@@ -390,7 +403,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     if (lane == 0 && leader) {
       // ---------------- MMA issuer (the even CTA of a pair issues for both)
       constexpr uint32_t idesc = idesc_bf16_f32(BN, PAIR ? 256 : 128);
-      // MN-major operands (not in pairs): transpose bits of the instruction descriptor
+      // MN-major operands: transpose bits of the instruction descriptor
       const uint32_t idesc_t = idesc | (p.a_mn ? 1u << 15 : 0u) | (p.b_mn ? 1u << 16 : 0u);
       int stage = 0;
       uint32_t phase = 0;
@@ -462,16 +475,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             const uint32_t b_addr = a_addr + C::kABytes;
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              if constexpr (PAIR) {
-                tc_mma_bf16_pair(d_tmem, smem_desc_sw128(a_addr + k * 32), smem_desc_sw128(b_addr + k * 32), idesc,
-                                 (kbi | k) != 0);
-              } else {
-                // K-major: the next 16 K columns are 32 bytes on in each 128-byte row; MN-major: 16
-                // K rows of 128 bytes further
-                const uint64_t ad = p.a_mn ? smem_desc_mn128(a_addr + k * 2048) : smem_desc_sw128(a_addr + k * 32);
-                const uint64_t bd = p.b_mn ? smem_desc_mn128(b_addr + k * 2048) : smem_desc_sw128(b_addr + k * 32);
+              // K-major: the next 16 K columns are 32 bytes on in each 128-byte row; MN-major: 16
+              // K rows of 128 bytes further
+              const uint64_t ad = p.a_mn ? smem_desc_mn128(a_addr + k * 2048) : smem_desc_sw128(a_addr + k * 32);
+              const uint64_t bd = p.b_mn ? smem_desc_mn128(b_addr + k * 2048) : smem_desc_sw128(b_addr + k * 32);
+              if constexpr (PAIR)
+                tc_mma_bf16_pair(d_tmem, ad, bd, idesc_t, (kbi | k) != 0);
+              else
                 tc_mma_bf16(d_tmem, ad, bd, idesc_t, (kbi | k) != 0);
-              }
             }
             if constexpr (PAIR)
               tc_commit_pair(&empty[stage]);

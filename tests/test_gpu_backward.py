@@ -39,11 +39,13 @@ def _rel(g, ref):
 
 @pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (1, 0), (0, 1), (1, 1)])
 @pytest.mark.parametrize("k_split", [1, 3])
-def test_engine_operand_layouts_and_split_k(a_mn, b_mn, k_split):
+@pytest.mark.parametrize("M,N", [(200, 192), (392, 256)])
+def test_engine_operand_layouts_and_split_k(a_mn, b_mn, k_split, M, N):
     """C = op(A) op(B)^T with either operand stored MN-major (the transposed reads of the
     backward's products), ragged M, N and K, against the float64 product of the same bf16
-    values.  fp32 accumulation over K = 200 terms: the error stays below 1e-5 of max|C|."""
-    M, N, K = 200, 192, 200
+    values; M = 392 runs the two-CTA 256-row tiles.  fp32 accumulation over K = 200 terms: the
+    error stays below 1e-5 of max|C|."""
+    K = 200
     g = torch.Generator().manual_seed(7 + 2 * a_mn + b_mn)
     A = torch.randn(M, K, generator=g).to(torch.bfloat16)
     B = torch.randn(N, K, generator=g).to(torch.bfloat16)
