@@ -189,7 +189,8 @@ cudaError_t launch_tc(const TcParams& p, int epi, int bn, int grid, cudaStream_t
   }
 }
 
-// Pair launches exist for tile widths 128 and 256 and the bf16 / SwiGLU / fp32 epilogues.
+// Pair launches exist for tile widths 128 and 256 and the bf16 / SwiGLU / fp32 / SwiGLU-backward
+// epilogues.
 cudaError_t launch_tc_pair(const TcParams& p, int epi, int bn, int grid, cudaStream_t st) {
   if (epi == EPI_SWIGLU) return bn == 256 ? launch_tc_pair_t<256, EPI_SWIGLU>(p, grid, st)
                                           : launch_tc_pair_t<128, EPI_SWIGLU>(p, grid, st);
@@ -197,6 +198,8 @@ cudaError_t launch_tc_pair(const TcParams& p, int epi, int bn, int grid, cudaStr
                                         : launch_tc_pair_t<128, EPI_BF16>(p, grid, st);
   if (epi == EPI_F32) return bn == 256 ? launch_tc_pair_t<256, EPI_F32>(p, grid, st)
                                        : launch_tc_pair_t<128, EPI_F32>(p, grid, st);
+  if (epi == EPI_SWIGLU_BWD) return bn == 256 ? launch_tc_pair_t<256, EPI_SWIGLU_BWD>(p, grid, st)
+                                              : launch_tc_pair_t<128, EPI_SWIGLU_BWD>(p, grid, st);
   return cudaErrorInvalidValue;
 }
 
@@ -1392,7 +1395,9 @@ int wgrad_gemm(lmoe_handle* h, TcParams& p, int M, int N, long long K, size_t ou
 int dense_gemm(lmoe_handle* h, TcParams& p, int epi, int T, int N, cudaStream_t st) {
   p.M = T;
   p.M_rows = T;
-  const int pbn = (T >= 256 * 8 && (epi == EPI_F32 || epi == EPI_BF16)) ? pick_pair_bn(T, N, h->sms) : 0;
+  const int pbn = (T >= 256 * 8 && epi != EPI_SWIGLU && epi != EPI_SWIGLU3 && epi != EPI_ROUTER && epi != EPI_DOWN3)
+                      ? pick_pair_bn(T, N, h->sms)
+                      : 0;
   if (pbn) {
     p.n_tiles = N / pbn;
     const long long tiles = (long long)((T + 255) / 256) * p.n_tiles;
@@ -1484,16 +1489,12 @@ int backward_bf16(lmoe_handle* h, const lmoe_weights* w, const void* x, const vo
     p.b_mn = 1;
     p.nseg = 1;
     p.seg[0] = KSeg{0, 0, 0, (int)(d / 64), 0};
-    p.M = T;
-    p.M_rows = T;
-    const int bn3 = pick_bn_for(T, hs, sms, 64);
-    p.n_tiles = hs / bn3;
     p.tmOut = dps_out;
     p.aux = b->ps;
     p.ld_aux = 2 * hs;
     p.split = hs;
-    CK(launch_tc(p, EPI_SWIGLU_BWD, bn3, std::min(mt * p.n_tiles, sms), st));
-    h->launches += 1;
+    int rc = dense_gemm(h, p, EPI_SWIGLU_BWD, T, (int)hs, st);
+    if (rc) return rc;
   }
   {  // dL/dz = dy W_up
     TcParams p = tc_base(h);

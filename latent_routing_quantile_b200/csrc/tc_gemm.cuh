@@ -203,6 +203,7 @@ __device__ __forceinline__ TileInfo tc_tile(const TcParams& p, int tile, int BN,
   if (pair) {  // 256-row tiles; this CTA owns rows 128*rank.. and B rows BN/2*rank..
     ti.row0 = mt * 256 + (int)rank * 128;
     ti.b_row0 = ti.n0 + (int)rank * (BN / 2);
+    ti.valid = min(128, p.M - ti.row0);  // may be 0 or less: no row of this CTA holds data
   } else if (p.grouped) {
     int2 e_r = p.mtile_table[mt];
     ti.row0 = e_r.y;
