@@ -1421,7 +1421,6 @@ int backward_bf16(lmoe_handle* h, const lmoe_weights* w, const void* x, const vo
   const lmoe_config& c = h->cfg;
   BwdWork* b = h->bw;
   const long long d = c.d, l = c.l, E = c.E, hh = c.h, hs = c.hs;
-  const int mt = (T + 127) / 128;
   const int sms = h->sms;
   bool ok = true;
   // per-call maps of the token-row buffers (their row extent is T, so K = T products read zeros
