@@ -560,6 +560,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       ++step;
       return true;
     };
+    uint4 pf[8];           // EPI_SWIGLU_BWD: pre-activations fetched ahead
+    bool pf_next = false;  // EPI_SWIGLU_BWD: pf holds the next tile's first step
     for (int tile = first; ok && tile < num_tiles; tile += stride, ++it) {
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
@@ -658,12 +660,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         // then every lane reads its own row from there.
         const bool live = rl < ti.valid;
         uint8_t* stg = smem + C::kAuxOffset + (warp - 2) * kAuxWarpBytes;
-        const int rbase = ti.row0 + wq * 32;
-        const int nlive = ti.valid - wq * 32;  // rows of this warp's quarter that hold data
-        uint4 pf[8];
-        auto fetch = [&](int j) {
-          const int c0 = ti.n0 + j * 64 + half_id * 32;
+        // copies step j of tile t's pre-activations for this warp's 32 rows and columns into pf
+        auto fetch = [&](const TileInfo& t, int j) {
+          const int c0 = t.n0 + j * 64 + half_id * 32;
           const int g0 = ((c0 >> 6) << 7) + (c0 & 63);
+          const int rbase = t.row0 + wq * 32;
+          const int nlive = t.valid - wq * 32;  // rows of this warp's quarter that hold data
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const int c = lane + 32 * i, which = c >> 7, rr = (c >> 2) & 31, cc = c & 3;
@@ -671,7 +673,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                                : make_uint4(0, 0, 0, 0);
           }
         };
-        fetch(0);
+        if (!pf_next) fetch(ti, 0);  // else the previous tile's last step fetched it
 #pragma unroll 1
         for (int j = 0; ok && j < BN / 64; ++j) {
           uint32_t v[32];
@@ -684,7 +686,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             *reinterpret_cast<uint4*>(stg + which * (kAuxWarpBytes / 2) + rr * 80 + cc * 16) = pf[i];
           }
           __syncwarp();
-          if (j + 1 < BN / 64) fetch(j + 1);
+          // the next step's values, or the next tile's first step's, load while this step computes
+          if (j + 1 < BN / 64) {
+            fetch(ti, j + 1);
+          } else {
+            pf_next = tile + stride < num_tiles;
+            if (pf_next) fetch(tc_tile(p, tile + stride, BN, PAIR, rank), 0);
+          }
           uint4 pg[4], pu[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
@@ -701,10 +709,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             for (int hlf = 0; hlf < 2; ++hlf) {
               const float g = __uint_as_float(hlf ? (gw & 0xFFFF0000u) : (gw << 16));
               const float u = __uint_as_float(hlf ? (uw & 0xFFFF0000u) : (uw << 16));
-              const float a = __uint_as_float(v[2 * q + hlf]);
               const float sg = sigmoidf_acc(g);
-              d1[hlf] = live ? a * u * sg * (1.0f + g * (1.0f - sg)) : 0.0f;
-              d3[hlf] = live ? a * g * sg : 0.0f;
+              const float as = __uint_as_float(v[2 * q + hlf]) * sg;  // dL/dact * sigmoid(g)
+              d1[hlf] = live ? as * u * fmaf(g, 1.0f - sg, 1.0f) : 0.0f;
+              d3[hlf] = live ? as * g : 0.0f;
             }
             w[q] = pack_bf16x2(d1[0], d1[1]);
             w3[q] = pack_bf16x2(d3[0], d3[1]);
