@@ -59,6 +59,8 @@ def load_peaks():
 # a recorded figure counts only while these files are the ones it was measured on
 TRAFFIC_SOURCES = {
     "shared_swiglu": ("common.cuh", "tc_gemm.cuh", "lmoe.cu"),
+    "expert_swiglu": ("common.cuh", "tc_gemm.cuh", "lmoe.cu"),
+    "expert_down": ("common.cuh", "tc_gemm.cuh", "lmoe.cu"),
     "norm_down_router": ("common.cuh", "k1_router.cuh", "lmoe.cu"),
 }
 
@@ -394,9 +396,8 @@ def roofline(summary, shape, name):
     tpath = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tpath):
         tj = json.load(open(tpath))
-        ent = tj.get("kernels", {}).get(name)
-        if (ent and name in TRAFFIC_SOURCES and ent.get("src_digest") == csrc_digest(TRAFFIC_SOURCES[name])
-                and tj.get("workload") == shape.name):
+        ent = tj.get("workloads", {}).get(shape.name, {}).get("kernels", {}).get(name)
+        if ent and name in TRAFFIC_SOURCES and ent.get("src_digest") == csrc_digest(TRAFFIC_SOURCES[name]):
             traffic = ent["dram_bytes_per_launch"]
     if kd["bound"] == "tensor":
         roof = {"bound": "tensor", "achieved": kd["tflops"], "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
