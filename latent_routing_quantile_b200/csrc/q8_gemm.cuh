@@ -191,7 +191,6 @@ __global__ void __launch_bounds__(kQ8Threads, 1) q8_gemm_kernel(const __grid_con
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed = 0, armed_parity = 0;
-      const uint64_t pol_first = l2_evict_first();
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
         const int mt = tile / p.n_tiles, nt = tile - mt * p.n_tiles;
@@ -207,7 +206,9 @@ __global__ void __launch_bounds__(kQ8Threads, 1) q8_gemm_kernel(const __grid_con
           uint8_t* a_dst = smem + stage * kQ8StageBytes;
           mbar_expect_tx(&full[stage], (uint32_t)(q * 32 * 128 + 16384 + 1024));
           tma_load_2d(a_dst, amap, &full[stage], kb * 128, row0);
-          tma_load_2d_hint(a_dst + 16384, &p.tmB, &full[stage], kb * 128, brow0, pol_first);
+          // no L2 evict-first hint on the weights: an expert's slice serves row tiles that run at
+          // about the same time (the hint made the wide layer's 8-bit experts slower)
+          tma_load_2d(a_dst + 16384, &p.tmB, &full[stage], kb * 128, brow0);
           bulk_load(a_dst + 32768, p.a_sf + ((size_t)(row0 >> 7) * p.nkb + kb) * 512, 512, &full[stage]);
           bulk_load(a_dst + 32768 + 512, p.b_sf + ((size_t)(brow0 >> 7) * p.nkb + kb) * 512, 512, &full[stage]);
           armed |= 1u << stage;
