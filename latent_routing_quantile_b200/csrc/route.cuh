@@ -113,7 +113,10 @@ __host__ __device__ constexpr int topk_prefetch(int nj) {
 }
 
 template <int NJ>
-__global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 : 1)
+// Blocks per SM: 2 of 16 warps for E <= 256; 3 of 8 warps above (registers capped at 80, a few
+// spilled): at E = 896 the rescoring of near-tie tokens is latency-bound, and one block per SM
+// (153 registers) took 290 us per 16384 tokens against 188 us with three.
+__global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 : 3)
     topk_kernel(const float* __restrict__ s, const float* __restrict__ bias, int ntok, int E, int k,
                 int* __restrict__ idx, float* __restrict__ gates, int* __restrict__ rank,
                 int* __restrict__ blkcnt, int* __restrict__ counts32, uint16_t* __restrict__ bins, int ld_bins,
