@@ -755,7 +755,7 @@ int route_from_scores(lmoe_handle* h, int T, uint32_t flags, const StatsState& p
     if (rc) return rc;
   }
   mark(h, ST_PLAN, st);
-  CK(launch_k(plan_kernel, dim3((c.E + 31) / 32), dim3(1024), 0, st, 1, (const int*)h->counts32, h->counts,
+  CK(launch_k(plan_kernel, dim3((c.E + kPlanExperts - 1) / kPlanExperts), dim3(1024), 0, st, 1, (const int*)h->counts32, h->counts,
               (const int*)h->blkcnt, nblk, c.E, h->offsets, h->pad_delta, h->blkbase, h->mtiles, h->num_mtiles,
               // an update already forked clears the loads itself, which equals adding them first
               ((flags & LMOE_RECORD_STATS) && !early) ? h->load : (long long*)nullptr));
@@ -2226,7 +2226,7 @@ int lmoe_route_noalloc(const float* scores, const float* bias, int32_t T, int32_
   TopkArgs ta{scores, bias, T, E, k, idx, rank, blkcnt, counts32, gates, nullptr, 0, TopkRefine{}, status};
   CK(launch_topk(ta, st));
   const int nblk = (T + kTokBlock - 1) / kTokBlock;
-  plan_kernel<<<(E + 31) / 32, 1024, 0, st>>>(counts32, counts, blkcnt, nblk, E, offsets, delta, blkbase, tiles,
+  plan_kernel<<<(E + kPlanExperts - 1) / kPlanExperts, 1024, 0, st>>>(counts32, counts, blkcnt, nblk, E, offsets, delta, blkbase, tiles,
                                                ntiles, nullptr);
   CK(cudaGetLastError());
   const int pairs = T * k;
