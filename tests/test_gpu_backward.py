@@ -10,6 +10,8 @@ so max|G - G_ref| / max|G_ref| <= 8 * 2^-9 = 1.6e-2 to first order; the bound as
 (a wrong expert cannot hide behind the others' larger values), and an expert that received no
 pair must get exactly zero.
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -149,3 +151,32 @@ def test_backward_at_the_training_bench_size():
     g, ref, r, _ = run_backward(shape, gain="ones")
     errs = check_grads(shape, g, ref, r)
     print("max error / max|ref| per gradient:", {n: f"{v:.2e}" for n, v in errs.items()})
+
+
+def test_training_and_inference_calls_share_a_handle():
+    """One handle, three calls: a training step on 300 tokens, an inference forward on the same
+    tokens (its own cached graph; the output must equal the training step's bit for bit, since both
+    run the same forward arithmetic), and a training step on the first 128 tokens only (the
+    backward's per-call tensor maps and row extents follow T; its gradients must match the oracle
+    on those 128 tokens)."""
+    shape = SMALL
+    w_cpu = datagen.layer_weights(shape, gain="random")
+    x = datagen.tokens(shape)
+    dy = datagen.output_grad(shape, seed=shape.seed + 100)
+    w_dev = {n: t.cuda() for n, t in w_cpu.items()}
+    layer = lq.Layer(shape.d, shape.l, shape.E, shape.k, shape.h, shape.hs, lq.BF16, shape.T, w_dev,
+                     rms_eps=shape.rms_eps)
+    y_train, _ = layer.forward_backward(x.cuda(), dy.cuda(), w_dev)
+    y_inf = layer.forward(x.cuda())
+    y_inf2 = layer.forward(x.cuda())  # the replay of the cached inference graph
+    torch.cuda.synchronize()
+    assert torch.equal(y_train, y_inf) and torch.equal(y_inf, y_inf2)
+    T2 = 128
+    sub = dataclasses.replace(shape, T=T2)
+    _, g = layer.forward_backward(x[:T2].contiguous().cuda(), dy[:T2].contiguous().cuda(), w_dev)
+    torch.cuda.synchronize()
+    assert layer.status() == 0
+    r = layer.routing()
+    layer.close()
+    ref = ob.layer_backward(x[:T2], w_cpu, np.zeros(shape.E), shape.k, dy[:T2], shape.rms_eps)
+    check_grads(sub, {n: t.cpu().double().numpy() for n, t in g.items()}, ref, r)
