@@ -405,6 +405,23 @@ def dp_qb_update(layer, beta, literal=False, sign_rule=False, group=None, stream
     layer.qb_update(beta, literal=literal, sign_rule=sign_rule, stream=stream)
 
 
+def dp_train_step(layer, x, dy, weights, beta=None, literal=False, sign_rule=False, group=None, grads=None,
+                  stream=None):
+    """One data-parallel training step's layer work on every rank of `group`: forward_backward of
+    this rank's tokens (QB statistics recorded), then the exchange: every weight gradient summed
+    over the ranks with one all-reduce each (the loss is the sum over all ranks' tokens, so its
+    gradient is the sum of the ranks' own; dL/dx stays per rank), and, when beta is given, the
+    ranks' QB statistics summed and the bias updated (dp_qb_update).  Returns (y, grads)."""
+    import torch.distributed as dist
+    y, g = layer.forward_backward(x, dy, weights, record_stats=True, grads=grads, stream=stream)
+    for name, t in g.items():
+        if name != "x":
+            dist.all_reduce(t, group=group)
+    if beta is not None:
+        dp_qb_update(layer, beta, literal=literal, sign_rule=sign_rule, group=group, stream=stream)
+    return y, g
+
+
 def route_noalloc(scores, bias, k, out=None, stream=None):
     """Routing of fp32 scores [T, E] with bias [E] through lmoe_route_noalloc, which allocates no
     device memory (its scratch is a static array in the library).  `out` may pass preallocated
