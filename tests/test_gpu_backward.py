@@ -141,6 +141,15 @@ def test_backward_rejects_unsupported_layers():
     with pytest.raises(lq.LmoeError):
         layer.forward_backward(x, x.clone(), w)
     layer.close()
+    # bf16 layer with 8-bit (MXFP8) routed experts: no backward either
+    shape = datagen.LayerShape("bwd_mx", 64, 256, 128, 64, 4, 128, 256, "bf16", seed=74)
+    w = {n: t.cuda() for n, t in datagen.layer_weights(shape).items()}
+    layer = lq.Layer(shape.d, shape.l, shape.E, shape.k, shape.h, shape.hs, lq.BF16, shape.T, w,
+                     experts=lq.EXPERTS_MXFP8)
+    x = datagen.tokens(shape).cuda()
+    with pytest.raises(lq.LmoeError):
+        layer.forward_backward(x, x.clone(), w)
+    layer.close()
 
 
 def test_backward_at_the_training_bench_size():
