@@ -185,6 +185,7 @@ cudaError_t launch_tc(const TcParams& p, int epi, int bn, int grid, cudaStream_t
     case EPI_DOWN3: return launch_tc_e<EPI_DOWN3>(p, bn, grid, st);
     case EPI_SWIGLU3: return launch_tc_e<EPI_SWIGLU3>(p, bn, grid, st);
     case EPI_SWIGLU_BWD: return launch_tc_e<EPI_SWIGLU_BWD>(p, bn, grid, st);
+    case EPI_F32_DEEP: return launch_tc_e<EPI_F32_DEEP>(p, bn, grid, st);
     default: return launch_tc_e<EPI_ROUTER>(p, bn, grid, st);
   }
 }
@@ -1587,7 +1588,11 @@ int backward_bf16(lmoe_handle* h, const lmoe_weights* w, const void* x, const vo
     p.tmOut = gw1;
     p.tmOut2 = gw3;
     p.out_split = (int)hh;
-    CK(launch_tc(p, EPI_F32, bn7, sms, st));
+    // four output boxes in flight when the experts average 256 rows or more (4+ k-blocks per tile:
+    // the fp32 stream of gradients limits them; wide layer's backward 14.6-15.2 -> 13.9-14.0 ms),
+    // two below (mini_replica, 192 rows: the ring stage they cost mattered more, +10 us)
+    const int wepi = (long long)T * c.k >= 256LL * E ? EPI_F32_DEEP : EPI_F32;
+    CK(launch_tc(p, wepi, bn7, sms, st));
     p.tmA[0] = p.tmA[1] = b->do_mn;
     p.tmB = b->act_mn;
     p.M = (int)l;
@@ -1596,7 +1601,7 @@ int backward_bf16(lmoe_handle* h, const lmoe_weights* w, const void* x, const vo
     p.n_tiles = (int)(hh / bn8);
     p.tmOut = gw2;
     p.out_split = 0;
-    CK(launch_tc(p, EPI_F32, bn8, sms, st));
+    CK(launch_tc(p, wepi, bn8, sms, st));
     h->launches += 2;
   }
   // router: dL/dc, dW_r = dlogit^T h, and its part of dL/dh = dlogit W_r

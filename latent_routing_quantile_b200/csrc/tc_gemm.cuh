@@ -48,6 +48,8 @@ enum TcEpilogue : int {
   EPI_ROUTER = 4,  // out fp32 = sigmoid(acc + col_bias[col])
   EPI_SWIGLU3 = 5, // as EPI_SWIGLU with an accurate SiLU, the fp32 result stored as hi, mid, lo bf16
                    // parts (columns part * split + c) for the next split-precision product
+  EPI_F32_DEEP = 7,    // as EPI_F32 with four output staging boxes (for streams of fp32 results:
+                       // the experts' weight gradients)
   EPI_SWIGLU_BWD = 6,  // acc = dL/d act of a SwiGLU; with its pre-activations p1 (gate) and p3
                        // (linear) read from aux, out bf16: dL/dp1 = acc p3 silu'(p1) at column c and
                        // dL/dp3 = acc silu(p1) at column split + c; rows past the tile's valid rows 0
@@ -124,10 +126,9 @@ struct TcCfg {
 // values of its 32 rows x 32 columns, rows 80 bytes apart (64 bytes of data + 16 of padding, so
 // that eight lanes reading eight rows hit distinct banks).
 constexpr int kAuxWarpBytes = 2 * 32 * 80;
-// Output staging boxes of an epilogue (boxes past two would live in its EXTRA bytes).  Four for
-// the fp32 outputs of short-K weight gradients were measured slower than two: they cost a stage
-// of the load ring and the stores were not what limited those tiles.
-__host__ __device__ constexpr int tc_out_boxes(int) { return 2; }
+// Output staging boxes of an epilogue (boxes past two live in its EXTRA bytes).  Four cost a stage
+// of the load ring; they pay only where the output stream is what limits a kernel.
+__host__ __device__ constexpr int tc_out_boxes(int epi) { return epi == EPI_F32_DEEP ? 4 : 2; }
 __host__ __device__ constexpr int tc_epi_extra(int epi) {
   return epi == EPI_SWIGLU_BWD ? 8 * kAuxWarpBytes : (tc_out_boxes(epi) - 2) * 16384;
 }
