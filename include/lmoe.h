@@ -321,9 +321,13 @@ typedef struct {
  * the backward's products are bf16 (gradients are rounded to bf16 before each product),
  * accumulation fp32.  The first call allocates the backward's workspace (about
  * max_tokens * (4 d + 8 hs + 12 l + 2 E) + rows * (10 h + 4 l + 4) bytes, rows = max_tokens k +
- * 128 E) with cudaMalloc, so make it outside any stream capture; lmoe_destroy frees it.  The
- * forward of a training step is cached as its own graph, beside lmoe_forward's.  Gradients of GEMMs whose output tiles cannot fill the GPU are
- * summed over K ranges by atomic tensor reductions, so their last bits vary between runs. */
+ * 128 E) with cudaMalloc, so make it outside any stream capture; lmoe_destroy frees it.  Outside
+ * a caller's stream capture, repeated calls replay CUDA graphs the handle caches: the training
+ * forward has its own (beside lmoe_forward's), the backward one keyed by x, dy, T and every
+ * pointer in w and g (a call that changes any of them runs eagerly, the next identical one is
+ * captured, later ones replay it).  Gradients
+ * of GEMMs whose output tiles cannot fill the GPU are summed over K ranges by atomic tensor
+ * reductions, so their last bits vary between runs. */
 int lmoe_forward_backward(lmoe_handle *h, const lmoe_weights *w, const void *x, const void *dy, void *y,
                           int32_t T, uint32_t flags, const lmoe_grads *g, void *stream);
 

@@ -423,6 +423,10 @@ struct lmoe_handle {
   // graph replay of repeated calls
   cudaStream_t cap = nullptr;
   GraphCache g_fwd[2], g_qb;  // two forward graphs (the host path alternates input buffers)
+  // the backward of lmoe_forward_backward, and the buffers its graph was captured with besides x,
+  // dy and the handle's own: the weights' and the gradients' pointers
+  GraphCache g_bwd;
+  const void* bwd_ptrs[23] = {};
   // LMOE_UPDATE_BIAS: the update's step and flags, and the branch it runs on
   bool upd_set = false;
   float upd_beta = 0.f;
@@ -1805,6 +1809,7 @@ int lmoe_destroy(lmoe_handle* h) {
     for (auto& e : r.ev) cudaEventDestroy(e);
   for (auto& g : h->g_fwd) g.reset(nullptr, nullptr, -1, 0, 0.f, 0);
   h->g_qb.reset(nullptr, nullptr, -1, 0, 0.f, 0);
+  h->g_bwd.reset(nullptr, nullptr, -1, 0, 0.f, 0);
   if (h->cap) cudaStreamDestroy(h->cap);
   if (h->cp_in) cudaStreamDestroy(h->cp_in);
   if (h->cp_out) cudaStreamDestroy(h->cp_out);
@@ -1895,7 +1900,19 @@ int lmoe_forward_backward(lmoe_handle* h, const lmoe_weights* w, const void* x, 
   cudaStream_t st = (cudaStream_t)stream;
   rc = forward_impl(h, x, y, T, flags, true, stream);
   if (rc) return rc;
-  return backward_bf16(h, w, x, dy, T, g, st);
+  // the backward is cached as a graph of its own (its host work, 40-odd tensor maps and 25-odd
+  // launches, is then one replay): its key is x, dy, T and every pointer of w and g, since the
+  // captured tensor maps and kernel arguments hold them
+  const void* ptrs[23] = {w->rms_gain, w->w_down, w->w_router, w->router_bias, w->w1, w->w3, w->w2, w->w_up,
+                          w->ws1, w->ws3, w->ws2, g->dx, g->rms_gain, g->w_down, g->w_router, g->router_bias,
+                          g->w1, g->w3, g->w2, g->w_up, g->ws1, g->ws3, g->ws2};
+  static_assert(sizeof ptrs == sizeof h->bwd_ptrs, "backward graph key");
+  if (memcmp(ptrs, h->bwd_ptrs, sizeof ptrs) != 0) {
+    memcpy(h->bwd_ptrs, ptrs, sizeof ptrs);
+    h->g_bwd.reset(nullptr, nullptr, -1, 0, 0.f, 0);
+  }
+  return run_cached(h, h->g_bwd, x, const_cast<void*>(dy), T, 0, 0.f, 0, st,
+                    [&](cudaStream_t s) { return backward_bf16(h, w, x, dy, T, g, s); });
 }
 
 int lmoe_forward_host(lmoe_handle* h, const void* x_host, void* y_host, int32_t T, uint32_t flags, void* stream) {

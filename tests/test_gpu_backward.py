@@ -189,3 +189,46 @@ def test_training_and_inference_calls_share_a_handle():
     layer.close()
     ref = ob.layer_backward(x[:T2], w_cpu, np.zeros(shape.E), shape.k, dy[:T2], shape.rms_eps)
     check_grads(sub, {n: t.cpu().double().numpy() for n, t in g.items()}, ref, r)
+
+
+def test_repeated_training_steps_replay_the_backward_graph():
+    """A training loop with fixed buffers: the first step runs eagerly, the second captures the
+    forward and the backward as graphs, the third replays them (same kernel count, same y bit for
+    bit, gradients on the oracle).  Then new gradient buffers: the backward's graph is keyed by
+    every pointer it writes, so steps with them run, capture and replay afresh, fill the new
+    buffers, and leave the old ones as they were."""
+    shape = SMALL
+    w_cpu = datagen.layer_weights(shape, gain="random")
+    x = datagen.tokens(shape).cuda()
+    dy = datagen.output_grad(shape, seed=shape.seed + 100).cuda()
+    w_dev = {n: t.cuda() for n, t in w_cpu.items()}
+    layer = lq.Layer(shape.d, shape.l, shape.E, shape.k, shape.h, shape.hs, lq.BF16, shape.T, w_dev,
+                     rms_eps=shape.rms_eps)
+    y = torch.empty_like(x)
+    _, ga = layer.forward_backward(x, dy, w_dev, y=y)
+    grads_a = dict(ga)
+    ys, counts = [], []
+    for _ in range(3):
+        before = layer.launches()
+        layer.forward_backward(x, dy, w_dev, y=y, grads=grads_a)
+        torch.cuda.synchronize()
+        counts.append(layer.launches() - before)
+        ys.append(y.clone())
+    assert layer.status() == 0
+    assert counts[0] == counts[1] == counts[2] > 0, counts
+    assert torch.equal(ys[0], ys[1]) and torch.equal(ys[1], ys[2])
+    r = layer.routing()
+    ref = ob.layer_backward(datagen.tokens(shape), w_cpu, np.zeros(shape.E), shape.k,
+                            datagen.output_grad(shape, seed=shape.seed + 100), shape.rms_eps)
+    check_grads(shape, {n: t.cpu().double().numpy() for n, t in grads_a.items()}, ref, r)
+    # new gradient buffers (the old ones zeroed: they must stay zero)
+    for t in grads_a.values():
+        t.zero_()
+    grads_b = {n: torch.full_like(t, float("nan")) for n, t in grads_a.items()}
+    for _ in range(3):
+        layer.forward_backward(x, dy, w_dev, y=y, grads=grads_b)
+    torch.cuda.synchronize()
+    assert layer.status() == 0
+    assert all(not torch.any(t) for t in grads_a.values()), "a stale graph wrote the old gradient buffers"
+    check_grads(shape, {n: t.cpu().double().numpy() for n, t in grads_b.items()}, ref, layer.routing())
+    layer.close()
