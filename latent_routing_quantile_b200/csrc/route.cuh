@@ -95,8 +95,8 @@ constexpr int kOverflow = 1 << 30;  // deferred-token flag: more candidates than
 // tau / 2 exactly, so the exact top k lies among them.  Each of them is rescored in fp64 as above
 // and the k best (u descending, expert ascending) are taken in that order.
 
-// One warp per token; a block of W warps ranks kTokBlock = 32 tokens (32 / W per warp; W = 16
-// for E <= 256, whose registers allow two such blocks per SM, else 8).  Lane L holds the scores
+// One warp per token; a block of W = 16 warps ranks kTokBlock = 32 tokens (two per warp), two
+// blocks per SM (registers capped at 64).  Lane L holds the scores
 // of experts L, L+32, ...; the scores of up to PF tokens are loaded before any of them is ranked,
 // so their memory latency overlaps.  k rounds of: local best (larger key, then lower index),
 // warp max of the keys (redux), warp min of the expert index among the lanes holding that key
@@ -107,16 +107,16 @@ constexpr int kOverflow = 1 << 30;  // deferred-token flag: more candidates than
 // stable (token ascending) with no order-dependent atomics.  With bins != null it also stores
 // each score's histogram bin, min(floor(s * 4096), 4095) as uint16, expert-major
 // (bins[e * ld_bins + t]).
-__host__ __device__ constexpr int topk_warps(int nj) { return nj <= 8 ? 16 : 8; }
-__host__ __device__ constexpr int topk_prefetch(int nj) {
-  return nj <= 8 ? kTokBlock / topk_warps(nj) : (nj <= 16 ? 2 : 1);
-}
+__host__ __device__ constexpr int topk_warps(int) { return 16; }
+__host__ __device__ constexpr int topk_prefetch(int nj) { return nj <= 16 ? 2 : 1; }
 
 template <int NJ>
-// Blocks per SM: 2 of 16 warps for E <= 256; 3 of 8 warps above (registers capped at 80, a few
-// spilled): at E = 896 the rescoring of near-tie tokens is latency-bound, and one block per SM
-// (153 registers) took 290 us per 16384 tokens against 188 us with three.
-__global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 : 3)
+// Above E = 256 the registers spill a little at the cap (364 bytes at E <= 1024), and the
+// rescoring of near-tie tokens is latency-bound: at E = 896 (16384 tokens) one 8-warp block per
+// SM (153 registers) took 290 us, three 8-warp blocks (80 registers) 183-273 us, two 16-warp
+// blocks 243-247 us against 268-273 us for three 8-warp ones in the same runs (its 512 blocks
+// fill 1.7 waves of 296 instead of 1.15 waves of 444: less of a tail).
+__global__ void __launch_bounds__(32 * topk_warps(NJ), 2)
     topk_kernel(const float* __restrict__ s, const float* __restrict__ bias, int ntok, int E, int k,
                 int* __restrict__ idx, float* __restrict__ gates, int* __restrict__ rank,
                 int* __restrict__ blkcnt, int* __restrict__ counts32, uint16_t* __restrict__ bins, int ld_bins,
@@ -124,9 +124,9 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), topk_warps(NJ) == 16 ? 2 
   constexpr int W = topk_warps(NJ);
   constexpr int TPW = kTokBlock / W;  // tokens per warp
   constexpr int PF = topk_prefetch(NJ);
-  // fp64 rescoring reads four elements per thread and step where the registers allow it (the
-  // 8-warp blocks of E > 256, whose wide d makes the rescoring loop latency-bound)
-  constexpr bool kQuad = W == 8;
+  // fp64 rescoring reads four elements per thread and step above E = 256 (the wide layers, whose
+  // d makes the rescoring loop latency-bound)
+  constexpr bool kQuad = NJ > 8;
   extern __shared__ uint32_t smem_topk[];
   uint32_t* mask = smem_topk;                                    // [E]
   uint16_t* sbins = reinterpret_cast<uint16_t*>(smem_topk + E);  // [32 tokens][E + 2] (padded rows)
