@@ -143,25 +143,58 @@ cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-template <int BN, int EPI>
-cudaError_t launch_tc_t(const TcParams& p, int grid, cudaStream_t st) {
-  auto kern = tc_gemm_kernel<BN, EPI, 0>;
+// Whether a launch uses the engine's general modes (MN-major operands, per-segment B maps,
+// grouped or split K, a second output map): only the backward's products do, and they run the
+// kernel compiled with them; the forward's products run the one without.
+bool tc_general(const TcParams& p) {
+  if (p.a_mn || p.b_mn || p.grouped_k || p.k_split > 1 || p.out_split) return true;
+  for (int s = 0; s < p.nseg; ++s)
+    if (p.seg[s].b_map) return true;
+  return false;
+}
+
+// Forms an epilogue is compiled in: 0 without the general modes, 1 with them, 2 both.
+constexpr int tc_forms(int epi) {
+  return (epi == EPI_BF16 || epi == EPI_F32) ? 2 : ((epi == EPI_SWIGLU_BWD || epi == EPI_F32_DEEP) ? 1 : 0);
+}
+
+template <int BN, int EPI, int PAIR, int GEN>
+cudaError_t launch_tc_g(const TcParams& p, int grid, cudaStream_t st) {
+  auto kern = tc_gemm_kernel<BN, EPI, PAIR, GEN>;
   static unsigned done = 0;
-  constexpr int smem = TcCfgFor<BN, EPI, 0>::kSmemBytes;
+  constexpr int smem = TcCfgFor<BN, EPI, PAIR>::kSmemBytes;
   cudaError_t e = ensure_smem_attr(kern, smem, done);
   if (e != cudaSuccess) return e;
-  return launch_k(kern, dim3(grid), dim3(kTcThreads), smem, st, 1, p);
+  // pairs: clusters of 2 along x, grid even
+  return launch_k(kern, dim3(PAIR ? (unsigned)(grid & ~1) : (unsigned)grid), dim3(kTcThreads), smem, st,
+                  PAIR ? 2 : 1, p);
+}
+
+// The form the parameters need; a general launch of an epilogue compiled only without the general
+// modes is refused.
+template <int BN, int EPI, int PAIR>
+cudaError_t launch_tc_f(const TcParams& p, int grid, cudaStream_t st) {
+  constexpr int f = tc_forms(EPI);
+  const bool gen = tc_general(p);
+  if constexpr (f == 2) {
+    return gen ? launch_tc_g<BN, EPI, PAIR, 1>(p, grid, st) : launch_tc_g<BN, EPI, PAIR, 0>(p, grid, st);
+  } else if constexpr (f == 1) {
+    return launch_tc_g<BN, EPI, PAIR, 1>(p, grid, st);
+  } else {
+    if (gen) return cudaErrorInvalidValue;
+    return launch_tc_g<BN, EPI, PAIR, 0>(p, grid, st);
+  }
+}
+
+template <int BN, int EPI>
+cudaError_t launch_tc_t(const TcParams& p, int grid, cudaStream_t st) {
+  return launch_tc_f<BN, EPI, 0>(p, grid, st);
 }
 
 // Two-CTA (cta_group::2) variant: clusters of 2 along x, grid even.
 template <int BN, int EPI>
 cudaError_t launch_tc_pair_t(const TcParams& p, int grid, cudaStream_t st) {
-  auto kern = tc_gemm_kernel<BN, EPI, 1>;
-  static unsigned done = 0;
-  constexpr int smem = TcCfgFor<BN, EPI, 1>::kSmemBytes;
-  cudaError_t e = ensure_smem_attr(kern, smem, done);
-  if (e != cudaSuccess) return e;
-  return launch_k(kern, dim3((unsigned)(grid & ~1)), dim3(kTcThreads), smem, st, 2, p);
+  return launch_tc_f<BN, EPI, 1>(p, grid, st);
 }
 
 template <int EPI>

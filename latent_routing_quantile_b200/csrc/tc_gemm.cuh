@@ -149,6 +149,9 @@ struct TileInfo {
 // Tile order: row-major over (M-tile, N-tile), or, with band_n > 0 (non-grouped), band by band:
 // all M-tiles of N-tiles [b band_n, (b+1) band_n) before the next band, so the tiles that run at
 // the same time share a band of B that stays in L2 instead of streaming all of B per M-tile.
+// GEN: the general modes (split K, grouped K, a second output map) exist; the forward's products
+// are compiled without them.
+template <bool GEN>
 __device__ __forceinline__ TileInfo tc_tile(const TcParams& p, int tile, int BN, int pair, uint32_t rank) {
   TileInfo ti;
   int mt, nt;
@@ -159,7 +162,7 @@ __device__ __forceinline__ TileInfo tc_tile(const TcParams& p, int tile, int BN,
   ti.bk0 = 0;
   ti.kb0 = 0;
   ti.nkb = -1;
-  if (p.k_split > 1) {
+  if (GEN && p.k_split > 1) {
     // split s of a one-segment K: tiles [s*base, (s+1)*base) cover k-blocks [s*nkb/S, (s+1)*nkb/S)
     const int base = (pair ? (p.M + 255) >> 8 : (p.M + 127) >> 7) * p.n_tiles;
     const int sp = tile / base;
@@ -168,7 +171,7 @@ __device__ __forceinline__ TileInfo tc_tile(const TcParams& p, int tile, int BN,
     ti.kb0 = (int)(((long long)sp * nk) / p.k_split);
     ti.nkb = (int)(((long long)(sp + 1) * nk) / p.k_split) - ti.kb0;
   }
-  if (p.grouped_k) {
+  if (GEN && p.grouped_k) {
     // expert-major: all (M-tile, N-tile) pairs of one expert's gradient, then the next expert's
     const int per = ((p.M + 127) >> 7) * p.n_tiles;
     const int e = tile / per;
@@ -218,16 +221,17 @@ __device__ __forceinline__ TileInfo tc_tile(const TcParams& p, int tile, int BN,
     ti.valid = min(128, p.M - ti.row0);
   }
   ti.out_y = ti.row0;
-  if (p.out_split && ti.row0 >= p.out_split) {
+  if (GEN && p.out_split && ti.row0 >= p.out_split) {
     ti.sel = 1;
     ti.out_y -= p.out_split;
   }
   return ti;
 }
 
+template <bool GEN>
 __device__ __forceinline__ int tc_num_tiles(const TcParams& p, int pair) {
-  if (p.grouped_k) return p.k_groups * ((p.M + 127) >> 7) * p.n_tiles;
-  if (p.k_split > 1) return p.k_split * (pair ? (p.M + 255) >> 8 : (p.M + 127) >> 7) * p.n_tiles;
+  if (GEN && p.grouped_k) return p.k_groups * ((p.M + 127) >> 7) * p.n_tiles;
+  if (GEN && p.k_split > 1) return p.k_split * (pair ? (p.M + 255) >> 8 : (p.M + 127) >> 7) * p.n_tiles;
   int mt = p.grouped ? *p.num_mtiles : (pair ? (p.M + 255) / 256 : (p.M + 127) / 128);
   return mt * p.n_tiles;
 }
@@ -235,8 +239,12 @@ __device__ __forceinline__ int tc_num_tiles(const TcParams& p, int pair) {
 constexpr int kEpiWarps = 8;
 constexpr int kTcThreads = 64 + 32 * kEpiWarps;
 
-template <int BN, int EPI, int PAIR>
+// GEN = 0: without the backward's modes (MN-major operands, per-segment B maps, grouped or split
+// K, a second output map), whose runtime branches in the producer, MMA and epilogue loops cost the
+// forward's products 3-7% at the replica's width; the host picks the form from the parameters.
+template <int BN, int EPI, int PAIR, int GEN>
 __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_constant__ TcParams p) {
+  constexpr bool G = GEN != 0;
   using C = TcCfgFor<BN, EPI, PAIR>;
   constexpr int S = C::kStages;
   constexpr int NB = tc_out_boxes(EPI);  // output staging boxes (the ones past two in the EXTRA bytes)
@@ -306,7 +314,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
   const uint32_t tmem_base = *tmem_slot;
   pdl_wait();  // operands, tile table and row scales come from earlier kernels
   pdl_trigger();
-  const int num_tiles = tc_num_tiles(p, PAIR);
+  const int num_tiles = tc_num_tiles<G>(p, PAIR);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -318,17 +326,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       bool ok = true;
       // the tile after this one is looked up one tile ahead: in grouped mode that is a global load
       // whose latency would otherwise stall the issue of every tile's first loads
-      TileInfo ti_next = tc_tile(p, first < num_tiles ? first : 0, BN, PAIR, rank);
+      TileInfo ti_next = tc_tile<G>(p, first < num_tiles ? first : 0, BN, PAIR, rank);
       for (int tile = first; ok && tile < num_tiles; tile += stride) {
         const TileInfo ti = ti_next;
-        if (tile + stride < num_tiles) ti_next = tc_tile(p, tile + stride, BN, PAIR, rank);
+        if (tile + stride < num_tiles) ti_next = tc_tile<G>(p, tile + stride, BN, PAIR, rank);
         // k-blocks segment by segment, or (split router) chunk by chunk over the three segments
         const int nouter = kSplit3 ? p.seg[0].nkb : p.nseg;
         for (int o = 0; ok && o < nouter; ++o) {
-          const int ninner = kSplit3 ? 3 : (ti.nkb >= 0 ? ti.nkb : p.seg[o].nkb);
+          const int ninner = kSplit3 ? 3 : ((G && ti.nkb >= 0) ? ti.nkb : p.seg[o].nkb);
           for (int in = 0; in < ninner; ++in) {
             const KSeg sg = p.seg[kSplit3 ? in : o];
-            const int kb = kSplit3 ? o : ti.kb0 + in;
+            const int kb = kSplit3 ? o : (G ? ti.kb0 + in : in);
             if (!mbar_wait(&empty[stage], phase ^ 1u, abort, p.status)) {
               ok = false;
               break;
@@ -339,24 +347,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
               // both CTAs' bytes complete the leader's full barrier; the leader expects all of them
               const uint32_t bar0 = mapa_shared(smem_u32(&full[stage]), 0);
               if (leader) mbar_expect_tx(&full[stage], 2 * C::kStageBytes);
-              const CUtensorMap* bmap = sg.b_map ? &p.tmB2[sg.b_map - 1] : &p.tmB;
-              if (p.a_mn) {  // this CTA's 128 rows of M as two 64 x 64 boxes
+              const CUtensorMap* bmap = (G && sg.b_map) ? &p.tmB2[sg.b_map - 1] : &p.tmB;
+              if (G && p.a_mn) {  // this CTA's 128 rows of M as two 64 x 64 boxes
                 const int ky = ti.ak0 + sg.a_col + kb * 64;
                 tma_load_2d_pair(a_dst, &p.tmA[sg.a_map], bar0, ti.row0, ky);
                 tma_load_2d_pair(a_dst + 8192, &p.tmA[sg.a_map], bar0, ti.row0 + 64, ky);
               } else {
                 tma_load_2d_pair(a_dst, &p.tmA[sg.a_map], bar0, sg.a_col + kb * 64, ti.row0);
               }
-              if (p.b_mn) {  // this CTA's BN/2 columns of N, 64 at a time
+              if (G && p.b_mn) {  // this CTA's BN/2 columns of N, 64 at a time
                 const int ky = ti.bk0 + sg.b_col + kb * 64;
 #pragma unroll
                 for (int c = 0; c < BN / 128; ++c) tma_load_2d_pair(b_dst + c * 8192, bmap, bar0, ti.b_row0 + 64 * c, ky);
               } else {
                 tma_load_2d_pair(b_dst, bmap, bar0, sg.b_col + kb * 64, ti.b_row0);
               }
-            } else if (p.a_mn | p.b_mn) {
+            } else if (G && (p.a_mn | p.b_mn)) {
               // MN-major operands: one 64 x 64 box per 64 columns of M (N), 64 K rows each
-              const CUtensorMap* bmap = sg.b_map ? &p.tmB2[sg.b_map - 1] : &p.tmB;
+              const CUtensorMap* bmap = (G && sg.b_map) ? &p.tmB2[sg.b_map - 1] : &p.tmB;
               mbar_expect_tx(&full[stage], (uint32_t)(C::kABytes + C::kBBytes));
               if (p.a_mn) {
                 const int ky = ti.ak0 + sg.a_col + kb * 64;
@@ -374,7 +382,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
               }
             } else {
               const CUtensorMap* amap = ti.q < 4 ? &p.tmA_part[ti.q - 1] : &p.tmA[sg.a_map];
-              const CUtensorMap* bmap = sg.b_map ? &p.tmB2[sg.b_map - 1] : &p.tmB;
+              const CUtensorMap* bmap = (G && sg.b_map) ? &p.tmB2[sg.b_map - 1] : &p.tmB;
               mbar_expect_tx(&full[stage], (uint32_t)(ti.q * 32 * 128 + C::kBBytes));
               if (p.hint_a)
                 tma_load_2d_hint(a_dst, amap, &full[stage], sg.a_col + kb * 64, ti.row0, pol_first);
@@ -406,7 +414,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       // ---------------- MMA issuer (the even CTA of a pair issues for both)
       constexpr uint32_t idesc = idesc_bf16_f32(BN, PAIR ? 256 : 128);
       // MN-major operands: transpose bits of the instruction descriptor
-      const uint32_t idesc_t = idesc | (p.a_mn ? 1u << 15 : 0u) | (p.b_mn ? 1u << 16 : 0u);
+      const uint32_t idesc_t = G ? idesc | (p.a_mn ? 1u << 15 : 0u) | (p.b_mn ? 1u << 16 : 0u) : idesc;
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
@@ -464,7 +472,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
           continue;
         }
         int kbi = 0;
-        const int tnkb = (p.grouped_k || p.k_split > 1) ? tc_tile(p, tile, BN, PAIR, rank).nkb : -1;
+        const int tnkb = (G && (p.grouped_k || p.k_split > 1)) ? tc_tile<G>(p, tile, BN, PAIR, rank).nkb : -1;
         for (int s = 0; ok && s < p.nseg; ++s) {
           const int nkb = tnkb >= 0 ? tnkb : p.seg[s].nkb;
           for (int kb = 0; kb < nkb; ++kb, ++kbi) {
@@ -479,8 +487,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             for (int k = 0; k < 4; ++k) {
               // K-major: the next 16 K columns are 32 bytes on in each 128-byte row; MN-major: 16
               // K rows of 128 bytes further
-              const uint64_t ad = p.a_mn ? smem_desc_mn128(a_addr + k * 2048) : smem_desc_sw128(a_addr + k * 32);
-              const uint64_t bd = p.b_mn ? smem_desc_mn128(b_addr + k * 2048) : smem_desc_sw128(b_addr + k * 32);
+              const uint64_t ad = (G && p.a_mn) ? smem_desc_mn128(a_addr + k * 2048) : smem_desc_sw128(a_addr + k * 32);
+              const uint64_t bd = (G && p.b_mn) ? smem_desc_mn128(b_addr + k * 2048) : smem_desc_sw128(b_addr + k * 32);
               if constexpr (PAIR)
                 tc_mma_bf16_pair(d_tmem, ad, bd, idesc_t, (kbi | k) != 0);
               else
@@ -544,7 +552,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         if (lane == 0) {
           if (to)
             tma_store_2d(to, box, x, y);
-          else if (p.k_split > 1)
+          else if (G && p.k_split > 1)
             tma_reduce_add_2d(omap, box, x, y);
           else if (p.hint_out)
             tma_store_2d_hint(omap, box, x, y, l2_evict_last());
@@ -568,7 +576,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       const uint32_t acc_phase = (it >> 1) & 1;
       float c_lane[BN / 32];  // router column offsets of this tile, one per lane and step
       if constexpr (EPI == EPI_ROUTER) {
-        const int n0 = tc_tile(p, tile, BN, PAIR, rank).n0;
+        const int n0 = tc_tile<G>(p, tile, BN, PAIR, rank).n0;
 #pragma unroll
         for (int j = 0; j < BN / 32; ++j) c_lane[j] = p.col_bias[n0 + j * 32 + lane];
       } else {
@@ -576,7 +584,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         for (int j = 0; j < BN / 32; ++j) c_lane[j] = 0.f;
       }
       // tile table entry and row scale are loaded before the wait, so their latency overlaps it
-      const TileInfo ti = tc_tile(p, tile, BN, PAIR, rank);
+      const TileInfo ti = tc_tile<G>(p, tile, BN, PAIR, rank);
       const int row = ti.row0 + rl;
       const float rs = (p.row_scale != nullptr && row < p.M_rows) ? p.row_scale[row] : 1.0f;
       ok = mbar_wait(&tfull[acc], acc_phase, abort, p.status);
@@ -586,8 +594,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         break;
       }
       tc_fence_after();
-      omap = ti.sel ? &p.tmOut2 : (ti.q < 4 ? &p.tmOut_part[ti.q - 1] : &p.tmOut);
-      const bool zero_acc = ti.nkb == 0;  // grouped_k: an expert without rows has a zero gradient
+      omap = (G && ti.sel) ? &p.tmOut2 : (ti.q < 4 ? &p.tmOut_part[ti.q - 1] : &p.tmOut);
+      const bool zero_acc = G && ti.nkb == 0;  // grouped_k: an expert without rows has a zero gradient
       const uint32_t tbase = tmem_base + ((uint32_t)(wq * 32) << 16) + acc * kAccCols;
       uint32_t w[16];
 
@@ -692,7 +700,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             fetch(ti, j + 1);
           } else {
             pf_next = tile + stride < num_tiles;
-            if (pf_next) fetch(tc_tile(p, tile + stride, BN, PAIR, rank), 0);
+            if (pf_next) fetch(tc_tile<G>(p, tile + stride, BN, PAIR, rank), 0);
           }
           uint4 pg[4], pu[4];
 #pragma unroll
