@@ -46,10 +46,10 @@ __global__ void __launch_bounds__(256) rms_kernel(const T* __restrict__ x, int n
 __device__ __forceinline__ uint32_t order_key(float f) {
   // -0 + 0 = +0 under round-to-nearest (every other value is unchanged), so -0 and +0, which
   // compare equal, get one key; negative numbers have all bits flipped, the others the sign bit
+  // (an XOR with the sign spread over the word, and the sign bit)
   if (f != f) return 1u;
-  if (f == 0.f) f = 0.f;
-  const uint32_t b = __float_as_uint(f);
-  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+  const uint32_t b = __float_as_uint(f + 0.0f);
+  return b ^ ((uint32_t)((int32_t)b >> 31) | 0x80000000u);
 }
 // Inverse of order_key for keys of numbers (>= 2).
 __device__ __forceinline__ float key_value(uint32_t key) {
@@ -207,7 +207,7 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), 2)
           // to 0 and saturates large ones
           if (bins)
             sbins[tl * bpitch + e] =
-                (uint16_t)(v >= 0.f ? min((int)(v * (float)LMOE_NBINS), LMOE_NBINS - 1) : 0);
+                (uint16_t)min(__float2uint_rz(v * (float)LMOE_NBINS), (unsigned)(LMOE_NBINS - 1));
         } else {
           key[j] = 0u;
         }
@@ -551,10 +551,23 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), 2)
     if (c) atomicAdd(&ccopy[e], c);
   }
   if (bins) {
-    // expert-major store: one warp writes 32 tokens (64 bytes) of one expert per step
     const int nt = min(kTokBlock, ntok - t0);
-    for (int e = warp; e < E; e += W)
-      if (lane < nt) bins[(size_t)e * ld_bins + t0 + lane] = sbins[lane * bpitch + e];
+    if (nt == kTokBlock) {
+      // expert-major store, 16 bytes a thread: 8 tokens of one expert (4 threads per expert row of
+      // the block's 32 tokens; the row starts 64-byte aligned, ld_bins being a multiple of 32)
+      for (int i = threadIdx.x; i < E * 4; i += blockDim.x) {
+        const int e = i >> 2, c = (i & 3) * 8;
+        const uint16_t* col = sbins + c * bpitch + e;
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) w[q] = (uint32_t)col[2 * q * bpitch] | ((uint32_t)col[(2 * q + 1) * bpitch] << 16);
+        *reinterpret_cast<uint4*>(bins + (size_t)e * ld_bins + t0 + c) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    } else {
+      // the last, partial block: one token a lane
+      for (int e = warp; e < E; e += W)
+        if (lane < nt) bins[(size_t)e * ld_bins + t0 + lane] = sbins[lane * bpitch + e];
+    }
   }
 }
 
