@@ -213,14 +213,15 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), 2)
         }
       }
       int my_sel = -1;
-      // k rounds of selection.  With the exact decision enabled, near-ties among the chosen and
-      // with the best unchosen expert (a warp max of the remaining keys) mark the token, and
-      // only then do further rounds collect the experts within tau of the k-th (at most
-      // kRefineExtra)
+      // k rounds of selection (lane i keeps the i-th choice and its key).  With the exact decision
+      // enabled, near-ties among the chosen and with the best unchosen expert (a warp max of the
+      // remaining keys) then mark the token, and only a marked token takes further rounds, which
+      // collect the experts within tau of the k-th (at most kRefineExtra)
       const int kmax = rf.x ? min(min(k + kRefineExtra, 32), E) : k;
-      float u_prev = 0.f, u_k1 = 0.f, my_u = 0.f;
+      float u_k1 = 0.f, my_u = 0.f;
       bool amb = false, odd = false;  // odd: a candidate without a numeric score
-      int nc = 0, lim = k;
+      int nc = k;
+      uint32_t my_key = 0u;
       // each lane keeps its best remaining key h1 (slot j1) and, while hv, the next one h2 (slot
       // j2); a round takes the warp's best h1 (ties to the lower expert), and the lane it came from
       // moves up its second, re-scanning its keys (minus the taken ones, bits of tk) only when the
@@ -248,12 +249,8 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), 2)
         }
         hv = true;
       };
-      best_two();
-      for (int i = 0; i < lim; ++i) {
-        const uint32_t wmax = __reduce_max_sync(kFull, h1);
-        if (i >= k) {  // an extra candidate: only within tau of the k-th, and only a number
-          if (wmax < 2u || !(key_value(wmax) >= u_k1 - rf.tau)) break;
-        }
+      // one round: the warp's best remaining key wmax (> 0) goes to lane i
+      auto take = [&](int i, uint32_t wmax) {
         const uint32_t emin = __reduce_min_sync(kFull, h1 == wmax ? (uint32_t)(j1 * 32 + lane) : 0xffffffffu);
         if ((emin & 31u) == (uint32_t)lane) {  // this lane's best was taken
           tk |= 1u << j1;
@@ -265,21 +262,32 @@ __global__ void __launch_bounds__(32 * topk_warps(NJ), 2)
             best_two();
           }
         }
-        if (lane == i) my_sel = (int)emin;
-        if (rf.x) {
-          const float ui = wmax >= 2u ? key_value(wmax) : 0.f;
-          if (wmax < 2u) odd = true;
-          if (lane == i) my_u = ui;
-          if (i > 0 && wmax >= 2u && u_prev - ui < rf.tau) amb = true;
-          if (i == k - 1) {
-            u_k1 = ui;
-            const uint32_t nk = __reduce_max_sync(kFull, h1);  // best remaining key
-            if (nk >= 2u && ui - key_value(nk) < rf.tau) amb = true;
-            if (amb) lim = kmax;
-          }
-          u_prev = ui;
+        if (lane == i) {
+          my_sel = (int)emin;
+          my_key = wmax;
         }
-        nc = i + 1;
+      };
+      best_two();
+      for (int i = 0; i < k; ++i) take(i, __reduce_max_sync(kFull, h1));
+      if (rf.x) {
+        // the chosen in order: u_i (0 for a key without a number), a near-tie between neighbours
+        const bool num = my_key >= 2u;
+        my_u = num ? key_value(my_key) : 0.f;
+        odd = __any_sync(kFull, lane < k && !num);
+        const float u_up = __shfl_up_sync(kFull, my_u, 1);
+        amb = __any_sync(kFull, lane > 0 && lane < k && num && u_up - my_u < rf.tau);
+        u_k1 = __shfl_sync(kFull, my_u, k - 1);
+        const uint32_t nk = __reduce_max_sync(kFull, h1);  // best remaining key
+        if (nk >= 2u && u_k1 - key_value(nk) < rf.tau) amb = true;
+        if (amb) {  // warp-uniform: extra candidates, numbers within tau of the k-th only
+          for (int i = k; i < kmax; ++i) {
+            const uint32_t wmax = __reduce_max_sync(kFull, h1);
+            if (wmax < 2u || !(key_value(wmax) >= u_k1 - rf.tau)) break;
+            take(i, wmax);
+            if (lane == i) my_u = key_value(wmax);
+            nc = i + 1;
+          }
+        }
       }
       if (amb) {  // warp-uniform: decided by the whole block after the token loop
         int slot = 0;
